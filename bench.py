@@ -1,0 +1,548 @@
+"""Benchmark of the FP8 block-scaled GEMM library on B200.
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+for the default workload ("decode"), the six decode-shaped dense GEMMs of the
+DeepGEMM pages' DeepSeek-V3/R1 inference shapes, M in {64, 128} x (N, K) in
+{(2112, 7168), (32768, 512), (7168, 2048)}, each with its own E4M3 operands and
+power-of-two block scales, every step through the library's public call.
+The metric for M <= 128 is HBM bandwidth: algorithmic bytes (A, B, their
+scales, and D) per second.  The other workloads ("smoke", "prefill",
+"contiguous", "masked") report TFLOPS and are for profiling and study.
+
+Timing: inputs sit in HBM, R copies of them at different addresses are rotated
+so that the bytes touched between two visits of one copy exceed the 126 MB L2;
+each step is a captured CUDA graph of its GEMM launches; a barrier and a device
+synchronisation bracket exactly K timed steps, timed with CUDA events; the
+result is the maximum over ranks.  A second timed pass records CUDA events
+around every launch for the per-kernel duration behind the roofline fraction.
+
+Under torchrun every rank runs the same per-rank workload on its own GPU (no
+data-path collective: the GEMMs of a step are independent problems), so the
+scaling is weak and ``value`` counts the bytes of all ranks.
+
+``--impl reference`` times the CPU oracle instead, on the host cores, on a
+bounded sample of the same step (the oracle is test infrastructure; this leg
+and the ``cpu_baseline`` object are the only product uses of it).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------- workloads --
+
+def build_workload(name: str, seed: int = 0):
+    """List of (kind, problem) making up one step."""
+    if name == "decode":
+        return [("dense", workloads.dense_problem(m, n, k, seed=seed + i))
+                for i, (m, n, k) in enumerate(workloads.DECODE_SHAPES)]
+    if name == "smoke":
+        m, n, k = workloads.SMOKE_SHAPE
+        return [("dense", workloads.dense_problem(m, n, k, seed=seed))]
+    if name == "prefill":
+        return [("dense", workloads.dense_problem(m, n, k, seed=seed + i))
+                for i, (m, n, k) in enumerate(workloads.PREFILL_SHAPES)]
+    if name == "contiguous":
+        return [("contiguous", workloads.contiguous_problem(**workloads.CONTIGUOUS_MOE, seed=seed))]
+    if name == "masked":
+        return [("masked", workloads.masked_problem(**workloads.MASKED_MOE, seed=seed))]
+    raise ValueError(name)
+
+
+def workload_meta(name: str):
+    """(metric, unit, bound) for a workload."""
+    if name in ("decode", "smoke"):
+        return "FP8 GEMM HBM bandwidth (M<=128)", "GB/s", "hbm"
+    return "FP8 GEMM TFLOPS", "TFLOP/s", "tensor"
+
+
+def step_units(items, unit: str) -> float:
+    """Algorithmic bytes (GB/s metric) or FLOPs (TFLOP/s metric) of one step."""
+    if unit == "GB/s":
+        return float(sum(p.bytes() for _, p in items))
+    return float(sum(p.flops() for _, p in items))
+
+
+def scale_units(x: float, unit: str, seconds: float) -> float:
+    return x / seconds / (1e9 if unit == "GB/s" else 1e12)
+
+
+# --------------------------------------------------------------- helpers --
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return json.load(f), "measured"
+    except OSError:
+        return dict(PEAKS_FALLBACK), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "moe_grouped_gemm_09_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary, or None if absent or taken on other kernel sources."""
+    path = os.path.join(ROOT, "profiles", f"traffic_{workload}.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if rec.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except OSError:
+            self.proc = None
+        time.sleep(0.2)
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[4:8]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- GPU arm --
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    import moe_grouped_gemm_09_b200 as dg
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", device_id=torch.device("cuda", local_rank),
+                                timeout=__import__("datetime").timedelta(seconds=120))
+    dev = torch.device("cuda", local_rank if world > 1 else torch.cuda.current_device())
+    torch.cuda.set_device(dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    items = build_workload(args.workload, seed=args.seed)
+    metric, unit, bound = workload_meta(args.workload)
+    units = step_units(items, unit)
+    set_bytes = sum(p.a.nbytes + p.b.nbytes + p.sfa.nbytes + p.sfb.nbytes for _, p in items)
+    R = max(2, math.ceil(3 * L2_BYTES / max(set_bytes, 1)))
+    if args.workload in ("prefill", "contiguous", "masked"):
+        R = max(2, min(R, 4))
+    flush_note = f"inputs rotated over {R} copies ({R * set_bytes / 2**20:.0f} MiB > 3x L2)"
+
+    # device copies: R rotation sets of the inputs, one output per GEMM
+    def to_dev(x):
+        return torch.from_numpy(np.ascontiguousarray(x)).to(dev)
+
+    sets = []
+    for r in range(R):
+        one = []
+        for kind, p in items:
+            t = {"a": to_dev(p.a), "sfa": to_dev(p.sfa), "b": to_dev(p.b), "sfb": to_dev(p.sfb)}
+            if kind == "contiguous":
+                t["m_indices"] = to_dev(p.m_indices)
+            if kind == "masked":
+                t["masked_m"] = to_dev(p.masked_m)
+            one.append(t)
+        sets.append(one)
+    outs = []
+    for kind, p in items:
+        if kind == "dense":
+            outs.append(torch.empty((p.M, p.N), dtype=torch.bfloat16, device=dev))
+        elif kind == "contiguous":
+            outs.append(torch.empty((p.M_sum, p.N), dtype=torch.bfloat16, device=dev))
+        else:
+            outs.append(torch.empty((p.G, p.max_m, p.N), dtype=torch.bfloat16, device=dev))
+
+    def launch_step(r, events=None):
+        for j, ((kind, p), t, d) in enumerate(zip(items, sets[r], outs)):
+            if events is not None:
+                events[j][0].record()
+            if kind == "dense":
+                dg.fp8_gemm_nt(t["a"], t["sfa"], t["b"], t["sfb"], d)
+            elif kind == "contiguous":
+                dg.m_grouped_fp8_gemm_nt_contiguous(t["a"], t["sfa"], t["b"], t["sfb"],
+                                                    t["m_indices"], d)
+            else:
+                dg.m_grouped_fp8_gemm_nt_masked(t["a"], t["sfa"], t["b"], t["sfb"],
+                                                t["masked_m"], p.expected_m, d)
+            if events is not None:
+                events[j][1].record()
+
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.synchronize(dev)
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):          # eager warm-up (also sizes the workspace)
+            launch_step(i % R)
+    torch.cuda.synchronize(dev)
+    if dg.get_last_device_error() != 0:
+        raise RuntimeError("device error during warm-up")
+
+    # one graph per rotation set, and one with per-launch events
+    graphs, ev_graphs, ev_sets = [], [], []
+    for r in range(R):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            launch_step(r)
+        graphs.append(g)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in items]
+        ge = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(ge, stream=stream):
+            launch_step(r, evs)
+        ev_graphs.append(ge)
+        ev_sets.append(evs)
+    with torch.cuda.stream(stream):
+        for i in range(2 * R):
+            graphs[i % R].replay()
+    torch.cuda.synchronize(dev)
+
+    # ---- timed region: exactly K steps ----
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index) as clocks:
+        with torch.cuda.stream(stream):
+            start.record(stream)
+            for i in range(args.steps):
+                graphs[i % R].replay()
+            end.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier()
+    ms = start.elapsed_time(end) / args.steps
+    ms = max_over_ranks(ms)
+    if dg.get_last_device_error() != 0:
+        raise RuntimeError("device error during the timed steps")
+
+    # ---- per-launch durations (second timed pass, events around each launch) ----
+    n_ev = max(R, min(args.steps, 200))
+    per_launch = [[] for _ in items]
+    torch.cuda.synchronize(dev)
+    for i in range(n_ev):
+        r = i % R
+        with torch.cuda.stream(stream):
+            ev_graphs[r].replay()
+        torch.cuda.synchronize(dev)
+        for j in range(len(items)):
+            per_launch[j].append(ev_sets[r][j][0].elapsed_time(ev_sets[r][j][1]))
+    kernel_ms = [statistics.mean(v) for v in per_launch]
+    kernel_units = [step_units([it], unit) for it in items]
+    achieved = scale_units(sum(kernel_units), unit, sum(kernel_ms) / 1e3)
+
+    # ---- end to end: host buffers, copies inside the timed region ----
+    pinned = []
+    for kind, p in items:
+        t = {"a": torch.from_numpy(p.a).pin_memory(), "sfa": torch.from_numpy(p.sfa).pin_memory(),
+             "b": torch.from_numpy(p.b).pin_memory(), "sfb": torch.from_numpy(p.sfb).pin_memory()}
+        if kind == "contiguous":
+            t["m_indices"] = torch.from_numpy(p.m_indices).pin_memory()
+        if kind == "masked":
+            t["masked_m"] = torch.from_numpy(p.masked_m).pin_memory()
+        pinned.append(t)
+    host_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
+    h2d = sum(v.numel() * v.element_size() for t in pinned for v in t.values())
+    d2h = sum(o.numel() * o.element_size() for o in outs)
+    e2e_steps = max(3, min(args.steps, args.e2e_steps))
+
+    def e2e_step():
+        for t_h, t_d in zip(pinned, sets[0]):
+            for k in t_h:
+                t_d[k].copy_(t_h[k], non_blocking=True)
+        launch_step(0)
+        for o_h, o_d in zip(host_out, outs):
+            o_h.copy_(o_d, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            e2e_step()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps)
+
+    # ---- CPU baseline (rank 0, single-GPU run only) ----
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = run_oracle_sample(items, unit, budget_s=args.cpu_budget_s)
+
+    peaks, peak_kind = load_peaks()
+    if bound == "hbm":
+        peak = float(peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"]))
+    else:
+        # E4M3 dense peak = 2x the measured BF16 figure (nominal FP8:BF16 ratio 4.5:2.25)
+        peak = 2.0 * float(peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"]))
+    value = scale_units(units * world, unit, ms / 1e3)
+    launches_per_step = len(items)
+    res = {
+        "metric": metric,
+        "value": round(value, 3),
+        "unit": unit,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms, 6),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "e4m3",
+        "data": "synthetic",
+        "config": {
+            "workload": args.workload,
+            "gemms": [dict(kind=k, **_shape(p)) for k, p in items],
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": flush_note,
+            "graph": "one CUDA graph per step",
+        },
+        "e2e": {"value": round(scale_units(units * world, unit, e2e_ms / 1e3), 3), "unit": unit,
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+        "gpu_launches": int(args.steps * launches_per_step),
+        "roofline": {
+            "bound": bound,
+            "achieved": round(achieved, 3),
+            "peak": peak,
+            "unit": unit,
+            "frac": round(achieved / peak, 4),
+            "traffic": profiled_traffic(args.workload),
+            "peak_source": f"{peak_kind} ({'hbm_gbs copy' if bound == 'hbm' else '2 x bf16_tflops'})",
+            "kernel_ms": [round(x, 5) for x in kernel_ms],
+        },
+        "clocks": clocks.summary(),
+    }
+    if cpu is not None:
+        res["cpu_baseline"] = cpu
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        del graphs, ev_graphs
+        dist.destroy_process_group()
+
+
+def _shape(p):
+    if isinstance(p, workloads.DenseProblem):
+        return {"M": p.M, "N": p.N, "K": p.K}
+    if isinstance(p, workloads.ContiguousProblem):
+        return {"M_sum": p.M_sum, "N": p.N, "K": p.K, "G": p.G, "valid_rows": p.valid_rows()}
+    return {"G": p.G, "max_m": p.max_m, "N": p.N, "K": p.K, "valid_rows": p.valid_rows(),
+            "expected_m": p.expected_m}
+
+
+# ------------------------------------------------------ CPU oracle timing --
+
+def _row_units(items, unit):
+    """Total rows per GEMM, for scaling a row sample up to the full step."""
+    out = []
+    for kind, p in items:
+        if kind == "dense":
+            out.append(p.M)
+        else:
+            out.append(p.valid_rows())
+    return out
+
+
+def _oracle_rows(o, kind, p, rows: np.ndarray):
+    if kind == "dense":
+        o.gemm_nt(p.a[rows], p.sfa[rows], p.b, p.sfb, want_acc=False)
+    elif kind == "contiguous":
+        valid = np.nonzero(p.m_indices >= 0)[0][rows]
+        o.grouped_contiguous(p.a[valid], p.sfa[valid], p.b, p.sfb, p.m_indices[valid])
+    else:
+        pairs = [(g, m) for g in range(p.G) for m in range(min(max(int(p.masked_m[g]), 0), p.max_m))]
+        sel = [pairs[i] for i in rows]
+        for g, m in sel:
+            o.gemm_nt(p.a[g, m:m + 1], p.sfa[g, m:m + 1], p.b[g], p.sfb[g], want_acc=False)
+
+
+def run_oracle_sample(items, unit, budget_s: float):
+    """Time the oracle on a bounded row sample of the step and scale to the
+    full step by rows (its cost is linear in output rows)."""
+    import oracle
+    o = oracle.default()
+    rows_total = _row_units(items, unit)
+    units = step_units(items, unit)
+    # rows per GEMM: grow until the sample takes about budget_s
+    frac = 1.0 / 64
+    while True:
+        t0 = time.perf_counter()
+        done_frac = []
+        for (kind, p), tot in zip(items, rows_total):
+            n = max(1, int(round(tot * frac)))
+            _oracle_rows(o, kind, p, np.arange(n))
+            done_frac.append(n / tot)
+        dt = time.perf_counter() - t0
+        if dt > budget_s / 4 or frac >= 1.0:
+            break
+        frac = min(1.0, frac * max(2.0, budget_s / 2 / max(dt, 1e-3)))
+    full_s = dt / (sum(done_frac) / len(done_frac))
+    return {"value": round(scale_units(units, unit, full_s), 4), "unit": unit,
+            "cores": o.num_threads(), "kind": "oracle",
+            "sample": f"first {100 * min(done_frac):.2f}%..{100 * max(done_frac):.2f}% of the output "
+                      f"rows of every GEMM of one step ({dt:.1f} s), scaled to the full step by rows"}
+
+
+def run_reference(args):
+    """The oracle as the reference arm: K timed steps, each a bounded sample."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    o = oracle.default()
+    items = build_workload(args.workload, seed=args.seed)
+    metric, unit, _ = workload_meta(args.workload)
+    units = step_units(items, unit)
+    rows_total = _row_units(items, unit)
+    # each step: one output row per host thread, of one GEMM (round robin over
+    # the GEMMs, walking down their rows); scaled to the full step by rows
+    per = max(1, o.num_threads())
+    cursor = [0] * len(items)
+
+    def one_step(i):
+        j = i % len(items)
+        n = min(per, rows_total[j])
+        rows = (cursor[j] + np.arange(n)) % rows_total[j]
+        cursor[j] = int((cursor[j] + n) % rows_total[j])
+        _oracle_rows(o, items[j][0], items[j][1], rows)
+        return n / rows_total[j] / len(items)
+
+    for i in range(args.warmup):
+        one_step(i)
+    full_equiv = 0.0
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        full_equiv += one_step(i)
+    dt = time.perf_counter() - t0
+    full_s = dt / full_equiv
+    value = scale_units(units, unit, full_s)
+    res = {
+        "impl": "reference",
+        "metric": metric, "value": round(value, 4), "unit": unit, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * full_s, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "gemms": [dict(kind=k, **_shape(p)) for k, p in items]},
+        "cpu_baseline": {"value": round(value, 4), "unit": unit, "cores": o.num_threads(),
+                         "kind": "oracle",
+                         "sample": f"{args.steps} timed steps of {per} output rows each (one GEMM per "
+                                   f"step, round robin), {dt:.1f} s, scaled to full steps by rows"},
+        "e2e": {"value": round(value, 4), "unit": unit, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(res), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default="decode",
+                    choices=("decode", "smoke", "prefill", "contiguous", "masked"))
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--cpu-budget-s", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

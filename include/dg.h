@@ -1,0 +1,155 @@
+/*
+ * dg.h -- C ABI of the B200 (sm_100a) FP8 block-scaled GEMM library.
+ *
+ * The library computes D = A * B^T with A and B in FP8 E4M3 ("fn" variant,
+ * max 448), fine-grained power-of-two FP32 scales, FP32 accumulation and a
+ * BF16 output, in three forms:
+ *
+ *   dense                 D[M,N]        = A[M,K] B[N,K]^T
+ *   M-grouped contiguous  D[r,:]        = A[r,:] B[m_indices[r]]^T  for every row r
+ *   M-grouped masked      D[g,m,:]      = A[g,m,:] B[g]^T           for m < masked_m[g]
+ *
+ * Sources: the operation and its fine-grained scaling and FP32 promotion are
+ * described in the DeepGEMM release article (deepseek.csdn.net), part 1.2
+ * "precision safeguards"; the call names fp8_gemm_nt and
+ * m_grouped_fp8_gemm_nt_contiguous in the DeepGEMM project card
+ * (aiproducthub.cn), sections "quick start" and "technical implementation"
+ * (M-axis grouping with N and K fixed, contiguous layout); the masked grouped
+ * call (m_grouped_gemm_fp8_masked) and set_num_sms in the release article,
+ * part 4.2 "advanced tuning"; the dense + contiguous + masked set in the
+ * youleyou.com article "DeepGEMM -- an efficient FP8 GEMM library", section
+ * on performance.
+ *
+ * Conventions shared by every GEMM entry point
+ * --------------------------------------------
+ *  - Every pointer argument is a DEVICE pointer into memory owned by the
+ *    caller.  The library never frees, retains or reallocates it.
+ *  - Operands (row-major, densely packed, no strides):
+ *      a    E4M3 bytes, K contiguous ("K-major");
+ *      b    E4M3 bytes [.., N, K], K contiguous;
+ *      sfa  float32 [rows of A, K/128]: scale of A row r for K block kb is
+ *           sfa[r * (K/128) + kb];
+ *      sfb  float32 [.., ceil(N/128), K/128]: scale of the 128 x 128 block
+ *           (n/128, kb) of B;
+ *      d    bfloat16 [rows of A, N], overwritten (no C / beta input).
+ *    The scales must be positive normal powers of two (2^-126 .. 2^127), as
+ *    produced by scale = 2^ceil(log2(amax/448)); the kernel uses the exponent
+ *    field only.
+ *  - Requirements (checked on the host, DG_ERR_INVALID_ARG otherwise):
+ *    K > 0 and K % 128 == 0; N > 0 and N % 16 == 0; a, b and d 16-byte
+ *    aligned, sfa/sfb 4-byte aligned, m_indices/masked_m 4-byte aligned.
+ *    A zero-row problem (M == 0, M_sum == 0, G == 0 or max_m == 0) is a
+ *    no-op returning DG_OK.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy
+ *    default stream) and return once the work is enqueued.  The device the
+ *    pointers live on must be the calling thread's current CUDA device.
+ *  - Errors: argument errors return before anything is launched; launch
+ *    errors return DG_ERR_CUDA.  A kernel that finds an inconsistency on the
+ *    device (a wait that runs out of time, an m_indices block naming two
+ *    experts, an expert index >= G) records a code that
+ *    dg_get_last_device_error() reports after the stream is synchronised.
+ *  - Results are deterministic: the same inputs give bit-identical outputs
+ *    on every run (no floating-point atomics; split-K partial sums are added
+ *    in a fixed order).
+ *  - Thread-safe: the per-device caches are guarded by a mutex.  Calls that
+ *    use split-K share one per-device workspace, so such calls must not run
+ *    concurrently on different streams of the same device.
+ */
+#ifndef DG_H_
+#define DG_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* dg_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+  DG_OK = 0,
+  DG_ERR_INVALID_ARG = 1,    /* bad size, null or misaligned pointer */
+  DG_ERR_UNSUPPORTED = 2,    /* legal but not supported (e.g. too many groups) */
+  DG_ERR_CUDA = 3,           /* a CUDA runtime / driver call failed */
+  DG_ERR_ARCH = 4,           /* the current device is not sm_100 */
+  DG_ERR_DEVICE = 5          /* a device-side error was recorded (see below) */
+} dg_status;
+
+/* Dense NT GEMM: D[M,N] = A[M,K] * B[N,K]^T.
+ * a [M,K] E4M3, sfa [M, K/128], b [N,K] E4M3, sfb [ceil(N/128), K/128],
+ * d [M,N] BF16.  M >= 0. */
+dg_status dg_fp8_gemm_nt(const void* a, const float* sfa, const void* b, const float* sfb,
+                         void* d, int M, int N, int K, dg_stream_t stream);
+
+/* M-grouped GEMM, contiguous layout (MoE experts' tokens concatenated along M).
+ * a [M_sum,K], sfa [M_sum,K/128], b [G,N,K], sfb [G,ceil(N/128),K/128],
+ * d [M_sum,N], m_indices int32 [M_sum] (device): the expert of row r, or -1
+ * for a padding row, whose row of D is left untouched.  M_sum % 128 == 0, and
+ * every aligned block of 128 rows holds rows of at most one expert (plus
+ * padding): each expert's segment starts at a multiple of 128.  Rows whose
+ * index is another expert than their block's, or >= G, are not written and
+ * set a device error. */
+dg_status dg_m_grouped_fp8_gemm_nt_contiguous(const void* a, const float* sfa, const void* b,
+                                              const float* sfb, void* d, const int* m_indices,
+                                              int M_sum, int N, int K, int G, dg_stream_t stream);
+
+/* M-grouped GEMM, masked layout (decode: token counts known only on the device).
+ * a [G,max_m,K], sfa [G,max_m,K/128], b [G,N,K], sfb [G,ceil(N/128),K/128],
+ * d [G,max_m,N], masked_m int32 [G] (device): rows m >= masked_m[g] of group g
+ * (clamped to [0, max_m]) are never written.  expected_m is a host-side hint
+ * of the typical masked_m used only to pick a configuration; results do not
+ * depend on it.  G <= 1024. */
+dg_status dg_m_grouped_fp8_gemm_nt_masked(const void* a, const float* sfa, const void* b,
+                                          const float* sfb, void* d, const int* masked_m, int G,
+                                          int max_m, int N, int K, int expected_m,
+                                          dg_stream_t stream);
+
+/* Cap on the number of SMs the GEMMs use (release article, part 4.2:
+ * set_num_sms).  n <= 0 restores the default (all SMs of the device).
+ * Applies to later calls from every thread. */
+dg_status dg_set_num_sms(int n);
+/* The cap in force for the current device (its SM count when no cap is set),
+ * or -1 if no CUDA device is usable. */
+int dg_get_num_sms(void);
+
+/* Reads and clears the device error word of the current device.  *code is 0
+ * when no device-side error was recorded since the last call.  Synchronises
+ * the device.  Returns DG_ERR_CUDA if the device cannot be queried.  Clearing
+ * also resets the split-K arrival counters, which a failed kernel may have
+ * left non-zero. */
+dg_status dg_get_last_device_error(int* code);
+
+/* Per-launch time limit of every wait inside the kernels, in milliseconds
+ * (default 1000).  A wait that runs out records a device error and the kernel
+ * returns instead of hanging. */
+dg_status dg_set_wait_timeout_ms(int ms);
+
+/* Human-readable name of a status code.  Never NULL. */
+const char* dg_status_string(dg_status s);
+
+/* Configuration the picker chooses for a problem, without launching anything
+ * and without a GPU (num_sms is given explicitly).  kind: 0 dense, 1
+ * contiguous, 2 masked; rows: M, M_sum or max_m; expected_m only for masked.
+ * Fills block_n, stages, split_k, grid (CTAs launched for the given rows). */
+typedef struct {
+  int block_m;
+  int block_n;
+  int stages;
+  int num_acc;
+  int split_k;
+  int grid;
+  int smem_bytes;
+  int tmem_cols;
+} dg_config;
+
+dg_status dg_query_config(int kind, int rows, int N, int K, int G, int expected_m, int num_sms,
+                          dg_config* out);
+
+/* Library version, "major.minor.patch". */
+const char* dg_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DG_H_ */

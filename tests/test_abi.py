@@ -1,0 +1,127 @@
+"""The C ABI without a GPU: the library loads, exports every entry point that
+include/dg.h declares, rejects bad arguments before touching a device, and its
+configuration picker (host code) makes sane choices."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dg.h")
+
+
+@pytest.fixture(scope="module")
+def dg():
+    from moe_grouped_gemm_09_b200 import build
+    build.build()
+    import moe_grouped_gemm_09_b200 as lib
+    return lib
+
+
+def declared_functions() -> list[str]:
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"\b(dg_\w+)\s*\(", text)
+    return sorted(set(n for n in names if n not in ("dg_status", "dg_stream_t", "dg_config")))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("dg_fp8_gemm_nt", "dg_m_grouped_fp8_gemm_nt_contiguous",
+                     "dg_m_grouped_fp8_gemm_nt_masked", "dg_set_num_sms"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(dg):
+    lib = ctypes.CDLL(dg.LIB_PATH)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+    assert set(dg.EXPORTED_SYMBOLS) == set(declared_functions())
+
+
+def test_version_and_status_strings(dg):
+    assert re.fullmatch(r"\d+\.\d+\.\d+", dg.version())
+    assert dg.status_string(0) == "DG_OK"
+    assert dg.status_string(1) == "DG_ERR_INVALID_ARG"
+    assert dg.status_string(99) == "DG_ERR_UNKNOWN"
+
+
+FAKE = 0x10000  # never dereferenced: the checks below fail before any device work
+
+
+@pytest.mark.parametrize("M,N,K", [(4, 15, 128), (4, 16, 100), (4, 16, 0), (-1, 16, 128), (4, 0, 128)])
+def test_dense_bad_sizes_rejected(dg, M, N, K):
+    rc = dg._gemm_nt(FAKE, FAKE, FAKE, FAKE, FAKE, M, N, K, None)
+    assert rc == 1  # DG_ERR_INVALID_ARG
+
+
+def test_dense_null_and_misaligned_rejected(dg):
+    assert dg._gemm_nt(FAKE, FAKE, None, FAKE, FAKE, 4, 16, 128, None) == 1
+    assert dg._gemm_nt(FAKE + 8, FAKE, FAKE, FAKE, FAKE, 4, 16, 128, None) == 1
+    assert dg._gemm_nt(FAKE, FAKE + 2, FAKE, FAKE, FAKE, 4, 16, 128, None) == 1
+
+
+def test_zero_rows_is_a_noop(dg):
+    # no device is touched for an empty problem, even with null pointers
+    assert dg._gemm_nt(None, None, None, None, None, 0, 16, 128, None) == 0
+    assert dg._gemm_masked(None, None, None, None, None, None, 0, 64, 16, 128, 1, None) == 0
+
+
+def test_grouped_bad_arguments_rejected(dg):
+    # contiguous: M_sum not a multiple of 128, missing m_indices
+    assert dg._gemm_contig(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 100, 16, 128, 2, None) == 1
+    assert dg._gemm_contig(FAKE, FAKE, FAKE, FAKE, FAKE, None, 128, 16, 128, 2, None) == 1
+    # masked: missing masked_m; too many groups
+    assert dg._gemm_masked(FAKE, FAKE, FAKE, FAKE, FAKE, None, 2, 64, 16, 128, 1, None) == 1
+    assert dg._gemm_masked(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 5000, 64, 16, 128, 1, None) == 2
+
+
+def test_timeout_setter(dg):
+    with pytest.raises(dg.DgError):
+        dg.set_wait_timeout_ms(0)
+    dg.set_wait_timeout_ms(1000)
+
+
+# ------------------------------------------------------------- the picker --
+
+def test_decode_shapes_split_k_to_one_wave(dg):
+    for (m, n, k) in [(64, 2112, 7168), (128, 2112, 7168), (64, 7168, 2048)]:
+        c = dg.query_config(0, m, n, k, num_sms=148)
+        n_tiles = -(-n // c["block_n"])
+        assert c["split_k"] >= 2
+        assert n_tiles * c["split_k"] <= 148
+        assert c["grid"] == n_tiles * c["split_k"]
+        assert (k // 128) // c["split_k"] >= 2
+
+
+def test_wide_decode_needs_no_split(dg):
+    c = dg.query_config(0, 64, 32768, 512, num_sms=148)
+    assert c["split_k"] == 1 and c["grid"] == 148
+
+
+def test_prefill_is_persistent(dg):
+    for (m, n, k) in [(4096, 2112, 7168), (4096, 24576, 1536), (4096, 7168, 16384)]:
+        c = dg.query_config(0, m, n, k, num_sms=148)
+        assert c["split_k"] == 1 and c["grid"] == 148
+        assert c["smem_bytes"] <= 232448 and c["tmem_cols"] <= 512
+
+
+def test_sm_cap_bounds_the_grid(dg):
+    for kind, rows, g in ((0, 4096, 1), (1, 10112, 32), (2, 256, 32)):
+        c = dg.query_config(kind, rows, 4096, 7168, G=g, expected_m=128, num_sms=48)
+        assert c["grid"] <= 48
+
+
+def test_small_problem_grid_is_its_tile_count(dg):
+    c = dg.query_config(0, 300, 96, 128, num_sms=148)
+    assert c["grid"] == (-(-300 // 128)) * (-(-96 // c["block_n"]))
+
+
+def test_query_rejects_bad_input(dg):
+    with pytest.raises(dg.DgError):
+        dg.query_config(3, 64, 128, 128)
+    with pytest.raises(dg.DgError):
+        dg.query_config(0, 64, 100, 128)

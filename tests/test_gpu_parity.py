@@ -1,0 +1,221 @@
+"""GPU parity: the CUDA library, called through its C ABI (via the Python
+binding), against the CPU oracle on the same seeded inputs.
+
+Small shapes are compared element by element over the whole output; the
+full-size workloads (the pages' DeepSeek-V3/R1-shaped decode and prefill GEMMs
+and the two MoE layouts) are compared on every row where the oracle finishes in
+seconds, else on sampled rows that cover every 128-row tile boundary.  Rows the
+method must leave untouched (contiguous padding, masked rows) are checked to
+still hold the sentinel bit pattern.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from parity import (check_close, d_bits, dev, oracle_contiguous_rows, oracle_dense_rows,
+                    oracle_masked_rows, sample_rows, sentinel_like)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dg():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import moe_grouped_gemm_09_b200 as lib
+    lib.set_num_sms(0)
+    assert lib.get_last_device_error() == 0
+    return lib
+
+
+def run_dense(dg, p: workloads.DenseProblem):
+    d = sentinel_like((p.M, p.N))
+    dg.fp8_gemm_nt(dev(p.a), dev(p.sfa), dev(p.b), dev(p.sfb), d)
+    torch.cuda.synchronize()
+    assert dg.get_last_device_error() == 0
+    return d_bits(d)
+
+
+SMALL_DENSE = [
+    (1, 16, 128), (64, 512, 1024), (127, 144, 256), (128, 128, 128), (129, 272, 384),
+    (200, 2112, 512), (256, 256, 640), (300, 96, 128), (64, 48, 896), (16, 4112, 256),
+]
+
+
+@pytest.mark.parametrize("M,N,K", SMALL_DENSE)
+def test_dense_small(dg, M, N, K):
+    p = workloads.dense_problem(M, N, K, seed=1)
+    got = run_dense(dg, p)
+    ref, _ = oracle.default().gemm_nt(p.a, p.sfa, p.b, p.sfb, want_acc=False)
+    check_close(got, ref, f"dense {M}x{N}x{K}")
+
+
+def test_dense_integer_exact(dg):
+    """Values in {-1, 0, 1} with unit scales: every output is an integer of
+    magnitude <= K = 256, exact in FP32 and BF16, so the result is bit-exact."""
+    rng = np.random.default_rng(5)
+    M, N, K = 200, 272, 256
+    enc = np.array([0xB8, 0x00, 0x38], np.uint8)
+    ia, ib = rng.integers(-1, 2, (M, K)), rng.integers(-1, 2, (N, K))
+    p = workloads.DenseProblem(enc[ia + 1], np.ones((M, 2), np.float32), enc[ib + 1],
+                               np.ones((3, 2), np.float32), M, N, K)
+    got = run_dense(dg, p)
+    want = torch.from_numpy((ia @ ib.T).astype(np.float32)).to(torch.bfloat16)
+    assert np.array_equal(got, want.view(torch.int16).numpy().view(np.uint16))
+
+
+def test_dense_scale_layout(dg):
+    """Every row of A and every 128x128 block of B gets its own power-of-two
+    scale, so a scale read from the wrong row, column block or K block shows."""
+    rng = np.random.default_rng(6)
+    M, N, K = 256, 384, 512
+    p = workloads.dense_problem(M, N, K, seed=2)
+    p.sfa = np.ldexp(1.0, rng.integers(-12, 4, p.sfa.shape)).astype(np.float32)
+    p.sfb = np.ldexp(1.0, rng.integers(-12, 4, p.sfb.shape)).astype(np.float32)
+    got = run_dense(dg, p)
+    ref, _ = oracle.default().gemm_nt(p.a, p.sfa, p.b, p.sfb, want_acc=False)
+    check_close(got, ref, "scale layout")
+
+
+@pytest.mark.parametrize("M,N,K", workloads.DECODE_SHAPES)
+def test_dense_decode_full(dg, M, N, K):
+    """The decode-shaped workloads, whole output (split-K path)."""
+    p = workloads.dense_problem(M, N, K, seed=0)
+    got = run_dense(dg, p)
+    ref, _ = oracle.default().gemm_nt(p.a, p.sfa, p.b, p.sfb, want_acc=False)
+    check_close(got, ref, f"decode {M}x{N}x{K}")
+
+
+@pytest.mark.parametrize("M,N,K", workloads.PREFILL_SHAPES)
+def test_dense_prefill_sampled(dg, M, N, K):
+    p = workloads.dense_problem(M, N, K, seed=0)
+    got = run_dense(dg, p)
+    rows = sample_rows(M, 48, seed=M + N)
+    check_close(got[rows], oracle_dense_rows(p, rows), f"prefill {M}x{N}x{K}")
+
+
+def test_dense_deterministic(dg):
+    p = workloads.dense_problem(64, 2112, 7168, seed=3)   # split-K path
+    a, b = run_dense(dg, p), run_dense(dg, p)
+    assert np.array_equal(a, b)
+
+
+def test_dense_zero_rows(dg):
+    dg.fp8_gemm_nt(torch.empty((0, 128), dtype=torch.uint8, device="cuda"),
+                   torch.empty((0, 1), device="cuda"),
+                   torch.zeros((16, 128), dtype=torch.uint8, device="cuda"),
+                   torch.ones((1, 1), device="cuda"))
+    torch.cuda.synchronize()
+
+
+def test_num_sms_cap(dg):
+    p = workloads.dense_problem(300, 1024, 512, seed=4)
+    ref = run_dense(dg, p)
+    try:
+        dg.set_num_sms(7)
+        assert dg.get_num_sms() == 7
+        got = run_dense(dg, p)
+    finally:
+        dg.set_num_sms(0)
+    assert np.array_equal(got, ref)
+
+
+# --------------------------------------------------------------- contiguous --
+
+def run_contiguous(dg, p: workloads.ContiguousProblem):
+    d = sentinel_like((p.M_sum, p.N))
+    dg.m_grouped_fp8_gemm_nt_contiguous(dev(p.a), dev(p.sfa), dev(p.b), dev(p.sfb),
+                                        dev(p.m_indices), d)
+    torch.cuda.synchronize()
+    return d_bits(d)
+
+
+def test_contiguous_small(dg):
+    p = workloads.contiguous_problem(G=4, N=144, K=256, seed=1, counts=np.array([3, 0, 130, 1]))
+    got = run_contiguous(dg, p)
+    assert dg.get_last_device_error() == 0
+    ref = np.full((p.M_sum, p.N), workloads.SENTINEL_BF16, np.uint16)
+    oracle.default().grouped_contiguous(p.a, p.sfa, p.b, p.sfb, p.m_indices, d=ref)
+    pad = p.m_indices < 0
+    assert np.all(got[pad] == workloads.SENTINEL_BF16), "padding rows were written"
+    check_close(got[~pad], ref[~pad], "contiguous small")
+
+
+def test_contiguous_full_sampled(dg):
+    p = workloads.contiguous_problem(**workloads.CONTIGUOUS_MOE, seed=0)
+    got = run_contiguous(dg, p)
+    assert dg.get_last_device_error() == 0
+    pad = p.m_indices < 0
+    assert np.all(got[pad] == workloads.SENTINEL_BF16), "padding rows were written"
+    valid = np.nonzero(~pad)[0]
+    rows = valid[sample_rows(len(valid), 64, seed=9)]
+    check_close(got[rows], oracle_contiguous_rows(p, rows), "contiguous full")
+
+
+def test_contiguous_mixed_block_reports(dg):
+    """A 128-row block naming two experts: the block belongs to the largest
+    index in it, rows naming another expert stay untouched, and the device
+    error word says why."""
+    p = workloads.contiguous_problem(G=3, N=128, K=128, seed=2, counts=np.array([100, 128, 0]))
+    p.m_indices[200] = 0  # inside expert 1's block
+    got = run_contiguous(dg, p)
+    assert dg.get_last_device_error() == 0x201
+    assert np.all(got[200] == workloads.SENTINEL_BF16)
+    block_expert = np.repeat(p.m_indices.reshape(-1, 128).max(axis=1), 128)
+    ok = np.nonzero((p.m_indices >= 0) & (p.m_indices == block_expert))[0]
+    check_close(got[ok], oracle_contiguous_rows(p, ok), "mixed block, other rows")
+
+
+# ------------------------------------------------------------------- masked --
+
+def run_masked(dg, p: workloads.MaskedProblem):
+    d = sentinel_like((p.G, p.max_m, p.N))
+    dg.m_grouped_fp8_gemm_nt_masked(dev(p.a), dev(p.sfa), dev(p.b), dev(p.sfb),
+                                    dev(p.masked_m), p.expected_m, d)
+    torch.cuda.synchronize()
+    return d_bits(d)
+
+
+def test_masked_small(dg):
+    p = workloads.masked_problem(G=5, max_m=200, N=144, K=256, seed=1,
+                                 masked_m=np.array([0, 200, 3, 129, 250]))
+    got = run_masked(dg, p)
+    assert dg.get_last_device_error() == 0
+    ref = np.full((p.G, p.max_m, p.N), workloads.SENTINEL_BF16, np.uint16)
+    oracle.default().grouped_masked(p.a, p.sfa, p.b, p.sfb, p.masked_m, d=ref)
+    for g in range(p.G):
+        v = min(max(int(p.masked_m[g]), 0), p.max_m)
+        assert np.all(got[g, v:] == workloads.SENTINEL_BF16), f"group {g}: masked rows written"
+        if v:
+            check_close(got[g, :v], ref[g, :v], f"masked group {g}")
+
+
+def test_masked_full_sampled(dg):
+    p = workloads.masked_problem(**workloads.MASKED_MOE, seed=0)
+    got = run_masked(dg, p)
+    assert dg.get_last_device_error() == 0
+    rng = np.random.default_rng(4)
+    pairs = []
+    for g in range(p.G):
+        v = int(p.masked_m[g])
+        assert np.all(got[g, v:] == workloads.SENTINEL_BF16), f"group {g}: masked rows written"
+        for m in sorted(set([0, v - 1] + rng.integers(0, max(v, 1), 2).tolist())):
+            if 0 <= m < v:
+                pairs.append((g, m))
+    ref = oracle_masked_rows(p, pairs)
+    got_rows = np.stack([got[g, m] for g, m in pairs])
+    check_close(got_rows, ref, "masked full")
+
+
+def test_masked_expected_m_does_not_change_results(dg):
+    p = workloads.masked_problem(G=4, max_m=256, N=256, K=256, seed=3)
+    a = run_masked(dg, p)
+    p.expected_m = 1
+    b = run_masked(dg, p)
+    p.expected_m = 256
+    c = run_masked(dg, p)
+    assert np.array_equal(a, b) and np.array_equal(a, c)
