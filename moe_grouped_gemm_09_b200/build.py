@@ -1,6 +1,7 @@
 """Build the CUDA library ``libdg.so`` in-tree with nvcc for sm_100a.
 
-Run ``python -m moe_grouped_gemm_09_b200.build`` (or call ``build()``).  The
+Run ``python moe_grouped_gemm_09_b200/build.py`` (or call ``build()``; load this
+file by path, since importing the package loads the library it builds).  The
 shared library is written next to this file so that it ships with the source
 tree; it links the CUDA runtime statically and reaches the driver's tensor-map
 encoder through ``cudaGetDriverEntryPoint``, so loading it needs no GPU.

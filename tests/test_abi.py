@@ -15,8 +15,8 @@ HEADER = os.path.join(ROOT, "include", "dg.h")
 
 @pytest.fixture(scope="module")
 def dg():
-    from moe_grouped_gemm_09_b200 import build
-    build.build()
+    from conftest import ensure_library_built
+    ensure_library_built()
     import moe_grouped_gemm_09_b200 as lib
     return lib
 
