@@ -145,6 +145,32 @@ typedef struct {
 dg_status dg_query_config(int kind, int rows, int N, int K, int G, int expected_m, int num_sms,
                           dg_config* out);
 
+/* Dense NT GEMM that allocates no device memory, for callers that cannot call
+ * cudaMalloc -- e.g. code running under a caching allocator or a memory pool
+ * that owns all device memory, or a host that must not grow its footprint
+ * after start-up.  The pages have no counterpart of this call.
+ *
+ * Same operands, layouts and requirements as dg_fp8_gemm_nt.  The scratch it
+ * needs (split-K partial sums, split-K arrival counters, a device error word)
+ * is a fixed 12.27 MiB __device__ array inside the library, which every GPU
+ * that loads the library holds until the process exits.  Problems whose
+ * split-K partial sums would not fit in its 12 MiB return DG_ERR_UNSUPPORTED
+ * (on a 148-SM B200 every shape fits: the partials are at most one 64 KiB tile
+ * per SM).  It calls no cudaMalloc, cudaFree or allocating library routine.
+ *
+ * The first call on a device sets that device up (architecture check and the
+ * device address of the array through cudaGetSymbolAddress); make that first
+ * call before any stream capture.  Every call shares the one array and each
+ * call clears the counters it uses on `stream` before its kernel, so calls
+ * whose kernels overlap on the GPU (different streams, or several threads)
+ * race and may return wrong results: serialise them.  The SM cap of
+ * dg_set_num_sms does not apply here (all SMs are used), and device-side
+ * error codes of this call stay in the array: dg_get_last_device_error does
+ * not report them.  Waits inside the kernel are bounded as in every call. */
+dg_status dg_fp8_gemm_nt_noalloc(const void* a, const float* sfa, const void* b,
+                                 const float* sfb, void* d, int M, int N, int K,
+                                 dg_stream_t stream);
+
 /* Library version, "major.minor.patch". */
 const char* dg_version(void);
 

@@ -6,7 +6,7 @@ This module is a thin binding over the C ABI of ``libdg.so`` (declared in
 pointers, sizes and the current CUDA stream, and raises on a non-zero status.
 Every step of the computation runs in the library's CUDA kernels; there is no
 Python or CPU fallback, and importing this package fails if the library has not
-been built (``python -m moe_grouped_gemm_09_b200.build``).
+been built (``python moe_grouped_gemm_09_b200/build.py``).
 
 The calls mirror the DeepGEMM API named on the pages (``fp8_gemm_nt``,
 ``m_grouped_fp8_gemm_nt_contiguous``, a masked grouped call and
@@ -25,7 +25,7 @@ LIB_PATH = os.path.join(_HERE, "libdg.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with "
-                      "`python -m moe_grouped_gemm_09_b200.build` (nvcc, sm_100a)")
+                      "`python moe_grouped_gemm_09_b200/build.py` (nvcc, sm_100a)")
 
 _lib = ctypes.CDLL(LIB_PATH)
 
@@ -47,6 +47,7 @@ _set_num_sms = _decl("dg_set_num_sms", [_I])
 _get_num_sms = _decl("dg_get_num_sms", [])
 _get_last_err = _decl("dg_get_last_device_error", [ctypes.POINTER(ctypes.c_int)])
 _set_timeout = _decl("dg_set_wait_timeout_ms", [_I])
+_gemm_nt_noalloc = _decl("dg_fp8_gemm_nt_noalloc", [_P, _P, _P, _P, _P, _I, _I, _I, _P])
 _status_string = _decl("dg_status_string", [_I], ctypes.c_char_p)
 _version = _decl("dg_version", [], ctypes.c_char_p)
 
@@ -61,7 +62,7 @@ _query = _decl("dg_query_config", [_I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(Dg
 EXPORTED_SYMBOLS = ("dg_fp8_gemm_nt", "dg_m_grouped_fp8_gemm_nt_contiguous",
                     "dg_m_grouped_fp8_gemm_nt_masked", "dg_set_num_sms", "dg_get_num_sms",
                     "dg_get_last_device_error", "dg_set_wait_timeout_ms", "dg_status_string",
-                    "dg_query_config", "dg_version")
+                    "dg_query_config", "dg_version", "dg_fp8_gemm_nt_noalloc")
 
 DEVICE_ERRORS = {
     0x101: "wait timeout in the TMA producer",
@@ -133,6 +134,26 @@ def fp8_gemm_nt(a: torch.Tensor, sfa: torch.Tensor, b: torch.Tensor, sfb: torch.
     with torch.cuda.device(dev):
         _check(_gemm_nt(a.data_ptr(), sfa.data_ptr(), b.data_ptr(), sfb.data_ptr(), d.data_ptr(),
                         M, N, K, _stream_ptr(dev)), "dg_fp8_gemm_nt")
+    return d
+
+
+def fp8_gemm_nt_noalloc(a: torch.Tensor, sfa: torch.Tensor, b: torch.Tensor, sfb: torch.Tensor,
+                        d: torch.Tensor) -> torch.Tensor:
+    """Dense GEMM through the entry point that allocates no device memory (its
+    scratch is a fixed array inside the library), for callers that cannot
+    allocate.  ``d`` must be given.  Calls must not overlap on the GPU."""
+    _fp8_bytes(a, "a"); _fp8_bytes(b, "b")
+    M, K = a.shape
+    N = b.shape[0]
+    dev = a.device
+    _need(a, "a", None, (M, K), dev)
+    _need(b, "b", None, (N, K), dev)
+    _need(sfa, "sfa", torch.float32, (M, K // 128), dev)
+    _need(sfb, "sfb", torch.float32, ((N + 127) // 128, K // 128), dev)
+    _need(d, "d", torch.bfloat16, (M, N), dev)
+    with torch.cuda.device(dev):
+        _check(_gemm_nt_noalloc(a.data_ptr(), sfa.data_ptr(), b.data_ptr(), sfb.data_ptr(),
+                                d.data_ptr(), M, N, K, _stream_ptr(dev)), "dg_fp8_gemm_nt_noalloc")
     return d
 
 
