@@ -107,17 +107,26 @@ def kernel_source_hash() -> str:
 
 
 def profiled_traffic(workload: str):
-    """DRAM bytes per launch of the dominant kernel from the committed ncu
-    summary, or None if absent or taken on other kernel sources."""
-    path = os.path.join(ROOT, "profiles", f"traffic_{workload}.json")
+    """DRAM bytes per launch of the dominant kernel, from the committed ncu
+    summary ``profiles/fp8_gemm_<workload>_traffic.md`` (its lines
+    ``traffic_bytes_per_launch:`` and ``kernel_source_hash:``), or None if the
+    summary is absent or was taken on other kernel sources."""
+    path = os.path.join(ROOT, "profiles", f"fp8_gemm_{workload}_traffic.md")
+    rec = {}
     try:
         with open(path) as f:
-            rec = json.load(f)
-    except (OSError, ValueError):
+            for line in f:
+                if ":" in line and not line.startswith((" ", "#", "|")):
+                    k, v = line.split(":", 1)
+                    rec[k.strip().strip("`")] = v.strip().strip("`")
+    except OSError:
         return None
     if rec.get("kernel_source_hash") != kernel_source_hash():
         return None
-    return rec.get("dram_bytes_per_launch")
+    try:
+        return int(float(rec["traffic_bytes_per_launch"]))
+    except (KeyError, ValueError):
+        return None
 
 
 class ClockSampler:

@@ -51,9 +51,9 @@
  *  - Results are deterministic: the same inputs give bit-identical outputs
  *    on every run (no floating-point atomics; split-K partial sums are added
  *    in a fixed order).
- *  - Thread-safe: the per-device caches are guarded by a mutex.  Calls that
- *    use split-K share one per-device workspace, so such calls must not run
- *    concurrently on different streams of the same device.
+ *  - Thread-safe: the per-device caches are guarded by a mutex.  No call
+ *    uses global scratch memory beyond the device error word, so calls may
+ *    run concurrently on different streams.
  */
 #ifndef DG_H_
 #define DG_H_
@@ -114,9 +114,7 @@ int dg_get_num_sms(void);
 
 /* Reads and clears the device error word of the current device.  *code is 0
  * when no device-side error was recorded since the last call.  Synchronises
- * the device.  Returns DG_ERR_CUDA if the device cannot be queried.  Clearing
- * also resets the split-K arrival counters, which a failed kernel may have
- * left non-zero. */
+ * the device.  Returns DG_ERR_CUDA if the device cannot be queried. */
 dg_status dg_get_last_device_error(int* code);
 
 /* Per-launch time limit of every wait inside the kernels, in milliseconds
@@ -130,16 +128,18 @@ const char* dg_status_string(dg_status s);
 /* Configuration the picker chooses for a problem, without launching anything
  * and without a GPU (num_sms is given explicitly).  kind: 0 dense, 1
  * contiguous, 2 masked; rows: M, M_sum or max_m; expected_m only for masked.
- * Fills block_n, stages, split_k, grid (CTAs launched for the given rows). */
+ * For the masked form the grid is an upper bound (the real tile count is
+ * read from masked_m on the device). */
 typedef struct {
-  int block_m;
-  int block_n;
-  int stages;
-  int num_acc;
-  int split_k;
-  int grid;
-  int smem_bytes;
-  int tmem_cols;
+  int block_m;     /* rows of A per tile (128) */
+  int block_n;     /* rows of B (columns of D) per tile */
+  int stages;      /* depth of the shared-memory operand ring */
+  int num_acc;     /* TMEM accumulator buffers */
+  int split_k;     /* K slices per output tile (> 1: one CTA cluster per tile) */
+  int grid;        /* CTAs launched */
+  int smem_bytes;  /* dynamic shared memory per CTA */
+  int tmem_cols;   /* TMEM columns allocated per CTA */
+  int kps;         /* 128-wide K blocks per ring stage */
 } dg_config;
 
 dg_status dg_query_config(int kind, int rows, int N, int K, int G, int expected_m, int num_sms,
@@ -150,23 +150,23 @@ dg_status dg_query_config(int kind, int rows, int N, int K, int G, int expected_
  * that owns all device memory, or a host that must not grow its footprint
  * after start-up.  The pages have no counterpart of this call.
  *
- * Same operands, layouts and requirements as dg_fp8_gemm_nt.  The scratch it
- * needs (split-K partial sums, split-K arrival counters, a device error word)
- * is a fixed 12.27 MiB __device__ array inside the library, which every GPU
- * that loads the library holds until the process exits.  Problems whose
- * split-K partial sums would not fit in its 12 MiB return DG_ERR_UNSUPPORTED
- * (on a 148-SM B200 every shape fits: the partials are at most one 64 KiB tile
- * per SM).  It calls no cudaMalloc, cudaFree or allocating library routine.
+ * Same operands, layouts and requirements as dg_fp8_gemm_nt.  The only
+ * scratch it needs, the device error word that the kernel's bounded waits
+ * report into, is a fixed 256-byte __device__ array inside the library,
+ * which every GPU that loads the library holds until the process exits
+ * (split-K partial sums stay in on-chip shared memory, so no problem size
+ * needs more).  It calls no cudaMalloc, cudaFree or allocating library
+ * routine.
  *
- * The first call on a device sets that device up (architecture check and the
- * device address of the array through cudaGetSymbolAddress); make that first
- * call before any stream capture.  Every call shares the one array and each
- * call clears the counters it uses on `stream` before its kernel, so calls
- * whose kernels overlap on the GPU (different streams, or several threads)
- * race and may return wrong results: serialise them.  The SM cap of
- * dg_set_num_sms does not apply here (all SMs are used), and device-side
- * error codes of this call stay in the array: dg_get_last_device_error does
- * not report them.  Waits inside the kernel are bounded as in every call. */
+ * The first call on a device sets that device up (architecture check,
+ * cluster-occupancy query and the device address of the array through
+ * cudaGetSymbolAddress); make that first call before any stream capture.
+ * Every call shares the one array, which keeps the last call's contents;
+ * calls whose kernels overlap on the GPU (different streams, or several
+ * threads) share it too.  The SM cap of dg_set_num_sms does not apply here
+ * (all SMs are used), and device-side error codes of this call stay in the
+ * array: dg_get_last_device_error does not report them.  Waits inside the
+ * kernel are bounded as in every call. */
 dg_status dg_fp8_gemm_nt_noalloc(const void* a, const float* sfa, const void* b,
                                  const float* sfb, void* d, int M, int N, int K,
                                  dg_stream_t stream);

@@ -54,7 +54,8 @@ _version = _decl("dg_version", [], ctypes.c_char_p)
 
 class DgConfig(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in
-                ("block_m", "block_n", "stages", "num_acc", "split_k", "grid", "smem_bytes", "tmem_cols")]
+                ("block_m", "block_n", "stages", "num_acc", "split_k", "grid", "smem_bytes", "tmem_cols",
+                 "kps")]
 
 
 _query = _decl("dg_query_config", [_I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(DgConfig)])

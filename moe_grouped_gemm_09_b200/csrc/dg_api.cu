@@ -8,6 +8,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "../../include/dg.h"
 #include "dg_config.h"
@@ -17,16 +18,14 @@ namespace dg {
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kCounterSlots = 1 << 16;
 
 struct DeviceState {
   bool ready = false;
   int num_sms = 0;
   int* error_word = nullptr;      // one int, device memory
-  float* workspace = nullptr;     // split-K partials
-  size_t workspace_bytes = 0;
-  int* counters = nullptr;        // split-K arrival counters
   bool smem_attr_set[3][kNumVariants] = {};
+  bool limits_known = false;
+  ClusterLimits limits = {};      // co-resident split-K clusters per variant and size
 };
 
 std::mutex g_mutex;
@@ -79,8 +78,6 @@ dg_status device_state(DeviceState** out, int* dev_out) {
     st.num_sms = prop.multiProcessorCount;
     if (cudaMalloc(&st.error_word, sizeof(int)) != cudaSuccess) return DG_ERR_CUDA;
     if (cudaMemset(st.error_word, 0, sizeof(int)) != cudaSuccess) return DG_ERR_CUDA;
-    if (cudaMalloc(&st.counters, kCounterSlots * sizeof(int)) != cudaSuccess) return DG_ERR_CUDA;
-    if (cudaMemset(st.counters, 0, kCounterSlots * sizeof(int)) != cudaSuccess) return DG_ERR_CUDA;
     if (cudaDeviceSynchronize() != cudaSuccess) return DG_ERR_CUDA;
     st.ready = true;
   }
@@ -89,21 +86,54 @@ dg_status device_state(DeviceState** out, int* dev_out) {
   return DG_OK;
 }
 
-// Grow the split-K workspace of a device to at least `bytes`.  The workspace
-// is only ever grown (never freed) so that earlier launches stay valid.
-dg_status ensure_workspace(DeviceState& st, size_t bytes) {
-  if (bytes <= st.workspace_bytes) return DG_OK;
-  size_t want = bytes < (size_t(16) << 20) ? (size_t(16) << 20) : bytes;
-  if (st.workspace) {
-    // A larger workspace replaces the old one once the device is idle.
-    if (cudaDeviceSynchronize() != cudaSuccess) return DG_ERR_CUDA;
-    cudaFree(st.workspace);
-    st.workspace = nullptr;
-    st.workspace_bytes = 0;
+// Rows per TMA box of A: a dense A shorter than one 128-row block is fetched
+// with a box of its own (16-row rounded) height, so the SM moves no padding.
+int a_box_rows(int kind, int rows) {
+  if (kind != kDense || rows >= kBlockM) return kBlockM;
+  return ((rows + 15) / 16) * 16;
+}
+
+// DG_FORCE_CONFIG="<block_n>:<split_k>[:<kps>:<a_rows>]" overrides the picker
+// (tuning sweeps); without kps/a_rows a general (one K block per stage) variant.
+// Ignored unless the variant exists and, for split_k > 1, the problem is a
+// dense one with a single 128-row block.
+void forced_config(int kind, int rows, int N, int K, int G, int sms, PickedConfig* pc) {
+  const char* e = std::getenv("DG_FORCE_CONFIG");
+  if (!e || !e[0]) return;
+  int bn = 0, sk = 1;
+  if (std::sscanf(e, "%d:%d", &bn, &sk) < 1) return;
+  int kps = 0, ar = 0;
+  std::sscanf(e, "%*d:%*d:%d:%d", &kps, &ar);
+  int v = -1;
+  for (int i = 0; i < kNumVariants; ++i) {
+    const Variant& x = kVariants[i];
+    if (x.block_n != bn) continue;
+    if (kps ? (x.kps != kps || (ar && x.a_rows != ar)) : x.decode) continue;
+    if (x.decode && kind != kDense) continue;
+    if (a_box_rows(kind, rows) > x.a_rows) continue;
+    v = i;
   }
-  if (cudaMalloc(&st.workspace, want) != cudaSuccess) return DG_ERR_CUDA;
-  st.workspace_bytes = want;
-  return DG_OK;
+  const int KB = K / kBlockK;
+  if (v < 0 || sk < 1 || sk > kMaxSplitK || sk > KB) return;
+  if (sk > 1 && (kind != kDense || rows > kBlockM)) return;
+  if ((sk - 1) * ceil_div(KB, sk) >= KB) return;
+  const long long groups = (kind == kMasked) ? G : 1;
+  const long long tiles = groups * ceil_div(rows, kBlockM) * ceil_div(N, bn);
+  pc->variant = v;
+  pc->split_k = sk;
+  pc->out_tiles = static_cast<int>(tiles);
+  pc->grid = sk > 1 ? static_cast<int>(tiles) * sk : static_cast<int>(tiles < sms ? tiles : sms);
+}
+
+// L2 prefetch of the first tile before the dependency wait; DG_NO_PREFETCH=1
+// turns it off (for measurements).
+int prefetch_enabled() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = std::getenv("DG_NO_PREFETCH");
+    v = (e && e[0] && e[0] != '0') ? 0 : 1;
+  }
+  return v;
 }
 
 int effective_sms(const DeviceState& st) {
@@ -114,57 +144,143 @@ int effective_sms(const DeviceState& st) {
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-// 3-D tensor map over E4M3 bytes [d2][d1][d0] (d0 = K contiguous) with a
-// box of box1 rows x 128 bytes and the 128-byte swizzle.
-dg_status make_map(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
-                   uint32_t box1) {
-  cuuint64_t dims[3] = {d0, d1, d2};
-  cuuint64_t strides[2] = {d0, d0 * d1};  // bytes, for dims 1 and 2
-  cuuint32_t box[3] = {128, box1, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims,
+// 4-D tensor map over E4M3 bytes [groups][rows][K] viewed as
+// {128 bytes of K, rows, K/128 blocks, groups} with strides {K, 128, rows*K}:
+// a box of {128, box_rows, kps, 1} brings kps K blocks of box_rows rows, laid
+// out in shared memory as kps consecutive [box_rows][128 B] tiles with the
+// 128-byte swizzle.
+dg_status make_map(CUtensorMap* map, const void* base, uint64_t K, uint64_t rows, uint64_t groups,
+                   uint32_t box_rows, uint32_t kps) {
+  cuuint64_t dims[4] = {128, rows, K / 128, groups};
+  cuuint64_t strides[3] = {K, 128, K * rows};  // bytes, for dims 1..3
+  cuuint32_t box[4] = {128, box_rows, kps, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims,
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? DG_OK : DG_ERR_CUDA;
 }
 
+template <int V>
+using ShapeOf = KernelShape<kVariants[V].block_n, kVariants[V].stages, kVariants[V].num_acc,
+                            kVariants[V].kps, kVariants[V].a_rows>;
+
+// Kernels are instantiated only for the (form, variant) pairs that exist:
+// the decode variants serve the dense form only.
+template <int KIND, int V>
+constexpr bool kBuilt = KIND == kDense || !kVariants[V].decode;
+
+template <int KIND, int V>
+auto kernel_of() {
+  constexpr Variant var = kVariants[V];
+  return fp8_gemm_kernel<KIND, var.block_n, var.stages, var.num_acc, var.kps, var.a_rows>;
+}
+
+template <int KIND, int V>
+dg_status set_smem_attr(DeviceState& st) {
+  if constexpr (!kBuilt<KIND, V>) {
+    return DG_ERR_UNSUPPORTED;
+  } else {
+    if (!st.smem_attr_set[KIND][V]) {
+      if (cudaFuncSetAttribute(kernel_of<KIND, V>(), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               ShapeOf<V>::kSmemBytes) != cudaSuccess)
+        return DG_ERR_CUDA;
+      st.smem_attr_set[KIND][V] = true;
+    }
+    return DG_OK;
+  }
+}
+
+// How many split-K clusters of each size the device co-schedules, per decode
+// variant of the dense kernel (a cluster must fit in one GPC).
+template <int V>
+dg_status query_cluster_limits(DeviceState& st) {
+  if constexpr (kVariants[V].decode) {
+    dg_status s = set_smem_attr<kDense, V>(st);
+    if (s != DG_OK) return s;
+    for (int c = 1; c <= kMaxSplitK; ++c) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(c, 1, 1);
+      cfg.blockDim = dim3(kThreads, 1, 1);
+      cfg.dynamicSmemBytes = ShapeOf<V>::kSmemBytes;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = c;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kernel_of<kDense, V>(), &cfg) != cudaSuccess) {
+        cudaGetLastError();  // clear; treat as "not known"
+        n = 0;
+      }
+      st.limits.max_clusters[V][c] = n;
+    }
+  }
+  return DG_OK;
+}
+
+template <int... V>
+dg_status query_all_cluster_limits(DeviceState& st, std::integer_sequence<int, V...>) {
+  dg_status s = DG_OK;
+  ((s = (s == DG_OK ? query_cluster_limits<V>(st) : s)), ...);
+  return s;
+}
+
+dg_status ensure_cluster_limits(DeviceState& st) {
+  if (st.limits_known) return DG_OK;
+  dg_status s = query_all_cluster_limits(st, std::make_integer_sequence<int, kNumVariants>{});
+  if (s != DG_OK) return s;
+  st.limits_known = true;
+  return DG_OK;
+}
+
 template <int KIND, int V>
 dg_status launch_variant(DeviceState& st, const CUtensorMap& ta, const CUtensorMap& tb,
                          const GemmArgs& args, int grid, cudaStream_t stream) {
-  constexpr Variant var = kVariants[V];
-  using Shape = KernelShape<var.block_n, var.stages, var.num_acc>;
-  auto kern = fp8_gemm_kernel<KIND, var.block_n, var.stages, var.num_acc>;
-  if (!st.smem_attr_set[KIND][V]) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Shape::kSmemBytes) != cudaSuccess)
-      return DG_ERR_CUDA;
-    st.smem_attr_set[KIND][V] = true;
+  if constexpr (!kBuilt<KIND, V>) {
+    return DG_ERR_UNSUPPORTED;
+  } else {
+    dg_status s = set_smem_attr<KIND, V>(st);
+    if (s != DG_OK) return s;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = ShapeOf<V>::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    int n_attr = 1;
+    if (args.split_k > 1) {  // the CTAs of one output tile form a cluster
+      attr[1].id = cudaLaunchAttributeClusterDimension;
+      attr[1].val.clusterDim.x = args.split_k;
+      attr[1].val.clusterDim.y = 1;
+      attr[1].val.clusterDim.z = 1;
+      n_attr = 2;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = n_attr;
+    return from_cuda(cudaLaunchKernelEx(&cfg, kernel_of<KIND, V>(), ta, tb, args));
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid, 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = Shape::kSmemBytes;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ta, tb, args);
-  return from_cuda(e);
+}
+
+template <int KIND, int... V>
+dg_status launch_dispatch(DeviceState& st, int variant, const CUtensorMap& ta,
+                          const CUtensorMap& tb, const GemmArgs& args, int grid,
+                          cudaStream_t stream, std::integer_sequence<int, V...>) {
+  dg_status s = DG_ERR_UNSUPPORTED;
+  ((variant == V ? (s = launch_variant<KIND, V>(st, ta, tb, args, grid, stream), 0) : 0), ...);
+  return s;
 }
 
 template <int KIND>
 dg_status launch(DeviceState& st, int variant, const CUtensorMap& ta, const CUtensorMap& tb,
                  const GemmArgs& args, int grid, cudaStream_t stream) {
-  switch (variant) {
-    case 0: return launch_variant<KIND, 0>(st, ta, tb, args, grid, stream);
-    case 1: return launch_variant<KIND, 1>(st, ta, tb, args, grid, stream);
-    case 2: return launch_variant<KIND, 2>(st, ta, tb, args, grid, stream);
-    case 3: return launch_variant<KIND, 3>(st, ta, tb, args, grid, stream);
-    default: return DG_ERR_UNSUPPORTED;
-  }
+  return launch_dispatch<KIND>(st, variant, ta, tb, args, grid, stream,
+                               std::make_integer_sequence<int, kNumVariants>{});
 }
 
 // Shared path of the three GEMM forms.
@@ -193,7 +309,12 @@ dg_status run(int kind, const void* a, const float* sfa, const void* b, const fl
   dg_status s = device_state(&st, nullptr);
   if (s != DG_OK) return s;
   const int sms = effective_sms(*st);
-  const PickedConfig pc = pick_config(kind, rows, N, K, G, expected_m, sms);
+  if (kind == kDense && rows <= 128) {
+    s = ensure_cluster_limits(*st);
+    if (s != DG_OK) return s;
+  }
+  PickedConfig pc = pick_config(kind, rows, N, K, G, expected_m, sms, &st->limits);
+  forced_config(kind, rows, N, K, G, sms, &pc);
   const Variant var = kVariants[pc.variant];
 
   GemmArgs args = {};
@@ -214,21 +335,20 @@ dg_status run(int kind, const void* a, const float* sfa, const void* b, const fl
   args.masked_m = masked_m;
   args.error_word = st->error_word;
   args.timeout_ns = g_timeout_ns;
-  args.counters = st->counters;
-  if (pc.split_k > 1) {
-    if (pc.out_tiles > kCounterSlots) return DG_ERR_UNSUPPORTED;
-    const size_t ws = static_cast<size_t>(pc.out_tiles) * pc.split_k * kBlockM * var.block_n *
-                      sizeof(float);
-    s = ensure_workspace(*st, ws);
-    if (s != DG_OK) return s;
-  }
-  args.workspace = st->workspace;
+  args.a_box_rows = a_box_rows(kind, rows);
+  if (args.a_box_rows > var.a_rows) return DG_ERR_UNSUPPORTED;
+  args.prefetch = prefetch_enabled();
+  // split-K runs one tile per CTA, one cluster per output tile
+  if (pc.split_k > 1 &&
+      (kind != kDense || pc.grid != args.num_m_blocks * args.num_n_blocks * pc.split_k ||
+       rows > kBlockM || !split_fits(var, rows, pc.split_k)))
+    return DG_ERR_UNSUPPORTED;
 
   CUtensorMap ta, tb;
   const int b_groups = (kind == kDense) ? 1 : G;
-  s = make_map(&ta, a, K, rows, kind == kMasked ? G : 1, kBlockM);
+  s = make_map(&ta, a, K, rows, kind == kMasked ? G : 1, args.a_box_rows, var.kps);
   if (s != DG_OK) return s;
-  s = make_map(&tb, b, K, N, b_groups, var.block_n);
+  s = make_map(&tb, b, K, N, b_groups, var.block_n, var.kps);
   if (s != DG_OK) return s;
 
   if (print_configs())
@@ -300,8 +420,6 @@ dg_status dg_get_last_device_error(int* code) {
   *code = v;
   if (v != 0) {
     if (cudaMemset(st->error_word, 0, sizeof(int)) != cudaSuccess) return DG_ERR_CUDA;
-    if (cudaMemset(st->counters, 0, kCounterSlots * sizeof(int)) != cudaSuccess)
-      return DG_ERR_CUDA;
     if (cudaDeviceSynchronize() != cudaSuccess) return DG_ERR_CUDA;
   }
   return DG_OK;
@@ -340,12 +458,18 @@ dg_status dg_query_config(int kind, int rows, int N, int K, int G, int expected_
   out->num_acc = v.num_acc;
   out->split_k = pc.split_k;
   out->grid = pc.grid;
-  switch (pc.variant) {
-    case 0: out->smem_bytes = KernelShape<256, 4, 1>::kSmemBytes; out->tmem_cols = KernelShape<256, 4, 1>::kTmemCols; break;
-    case 1: out->smem_bytes = KernelShape<128, 6, 2>::kSmemBytes; out->tmem_cols = KernelShape<128, 6, 2>::kTmemCols; break;
-    case 2: out->smem_bytes = KernelShape<64, 8, 2>::kSmemBytes; out->tmem_cols = KernelShape<64, 8, 2>::kTmemCols; break;
-    default: out->smem_bytes = KernelShape<32, 9, 2>::kSmemBytes; out->tmem_cols = KernelShape<32, 9, 2>::kTmemCols; break;
-  }
+  constexpr int smem[] = {ShapeOf<0>::kSmemBytes, ShapeOf<1>::kSmemBytes, ShapeOf<2>::kSmemBytes,
+                          ShapeOf<3>::kSmemBytes, ShapeOf<4>::kSmemBytes, ShapeOf<5>::kSmemBytes,
+                          ShapeOf<6>::kSmemBytes, ShapeOf<7>::kSmemBytes, ShapeOf<8>::kSmemBytes,
+                          ShapeOf<9>::kSmemBytes};
+  constexpr int tmem[] = {ShapeOf<0>::kTmemCols, ShapeOf<1>::kTmemCols, ShapeOf<2>::kTmemCols,
+                          ShapeOf<3>::kTmemCols, ShapeOf<4>::kTmemCols, ShapeOf<5>::kTmemCols,
+                          ShapeOf<6>::kTmemCols, ShapeOf<7>::kTmemCols, ShapeOf<8>::kTmemCols,
+                          ShapeOf<9>::kTmemCols};
+  static_assert(sizeof(smem) / sizeof(smem[0]) == kNumVariants, "one entry per variant");
+  out->smem_bytes = smem[pc.variant];
+  out->tmem_cols = tmem[pc.variant];
+  out->kps = v.kps;
   return DG_OK;
 }
 

@@ -14,32 +14,113 @@ struct Variant {
   int block_n;
   int stages;
   int num_acc;
+  int kps;      // 128-wide K blocks per ring stage (one TMA box of each operand)
+  int a_rows;   // rows of A a stage holds (64: dense A of at most 64 rows)
+  bool decode;  // built for dense problems of at most one 128-row block
 };
 
-// The compiled variants, largest tile first.
+// The compiled variants: general ones first (every form), then the
+// decode-shaped dense ones, whose stages are several K blocks deep so that
+// each TMA box moves 32-64 KB.
 constexpr Variant kVariants[] = {
-    {256, 4, 1},
-    {128, 6, 2},
-    {64, 8, 2},
-    {32, 9, 2},
+    {256, 4, 1, 1, 128, false},
+    {128, 6, 2, 1, 128, false},
+    {64, 8, 2, 1, 128, false},
+    {32, 9, 2, 1, 128, false},
+    {128, 2, 1, 4, 64, true},
+    {64, 3, 2, 4, 64, true},
+    {256, 2, 1, 2, 64, true},
+    {128, 3, 1, 2, 128, true},
+    {64, 4, 2, 2, 128, true},
+    {256, 2, 1, 2, 128, true},
 };
 constexpr int kNumVariants = sizeof(kVariants) / sizeof(kVariants[0]);
+constexpr int kMaxSplitK = 8;  // portable cluster size
 
 struct PickedConfig {
   int variant;   // index into kVariants
-  int split_k;   // K slices per output tile
+  int split_k;   // K slices per output tile (> 1: one cluster of split_k CTAs per tile)
   int grid;      // CTAs to launch
   int out_tiles; // output tiles (upper bound for masked)
 };
 
 inline int ceil_div(long long a, long long b) { return static_cast<int>((a + b - 1) / b); }
 
+// How many clusters of `cluster` CTAs of variant `variant` the device can run
+// at once.  max_clusters[v][s] for s in 1..kMaxSplitK; a value <= 0 means
+// "not known": then the SM count divided by the cluster size is assumed.
+struct ClusterLimits {
+  int max_clusters[kNumVariants][kMaxSplitK + 1];
+};
+
+inline int cluster_limit(const ClusterLimits* lim, int v, int s, int num_sms) {
+  int n = lim ? lim->max_clusters[v][s] : 0;
+  return n > 0 ? n : num_sms / s;
+}
+
+// Split-K parks each CTA's FP32 partial and the slices the other CTAs push to
+// it in the (then idle) operand ring: (2 * rows + split) rows of BLOCK_N + 4
+// floats must fit.
+inline bool split_fits(const Variant& var, int rows, int split) {
+  const long long ring = static_cast<long long>(var.stages) * var.kps * (var.a_rows + var.block_n) * 128;
+  const long long need = static_cast<long long>(2 * rows + split) * (var.block_n + 4) * 4;
+  return need <= ring;
+}
+
+// Decode-shaped dense problems (at most one 128-row block): HBM-bound.  Pick
+// the variant and K split (one cluster of `split` CTAs per output tile, all in
+// one wave) that minimise an estimate of the time: the larger of the whole
+// kernel's HBM time and the busiest CTA's streaming time, plus the pipeline
+// ramp and the reduction.  A CTA's streaming rate grows with the TMA box size
+// (about 37 GB/s per SM for 16 KB boxes, up to about 120 GB/s for 64 KB boxes,
+// measured on B200).  Returns false if no one-wave configuration exists.
+inline bool pick_decode(int rows, int N, int K, int num_sms, const ClusterLimits* lim,
+                        PickedConfig* out) {
+  const int KB = K / 128;
+  const double hbm_bytes_per_us = 5.8e6;  // whole GPU, streaming with large boxes
+  double best = 1e30;
+  bool found = false;
+  for (int v = 0; v < kNumVariants; ++v) {
+    const Variant& var = kVariants[v];
+    if (!var.decode || rows > var.a_rows) continue;
+    const int bn = var.block_n;
+    const int nt = ceil_div(N, bn);
+    const double box_kb = var.kps * bn * 128 / 1024.0;
+    double r_cta = 37.0 * box_kb / 16.0;  // GB/s = KB per microsecond
+    if (r_cta > 120.0) r_cta = 120.0;
+    for (int s = 1; s <= kMaxSplitK && s <= KB; ++s) {
+      if (nt * s > num_sms) break;
+      const int per = ceil_div(KB, s);
+      if ((s - 1) * per >= KB) continue;          // an empty slice
+      if (s > 1 && cluster_limit(lim, v, s, num_sms) < nt) continue;
+      if (s > 1 && !split_fits(var, rows, s)) continue;
+      const double b_cta = static_cast<double>(bn) * per * 128 / 1024.0;     // KB
+      const double a_cta = static_cast<double>(rows) * per * 128 / 1024.0;   // KB
+      const double t_cta = (b_cta + a_cta) / r_cta;                         // us
+      const double t_hbm = static_cast<double>(N) * K / hbm_bytes_per_us;  // us
+      const double t = (t_cta > t_hbm ? t_cta : t_hbm) + 1.5 + (s > 1 ? 0.8 : 0.0);
+      if (t < best - 1e-9) {
+        best = t;
+        found = true;
+        out->variant = v;
+        out->split_k = s;
+        out->out_tiles = nt;
+        out->grid = nt * s;
+      }
+    }
+  }
+  return found;
+}
+
 // kind: 0 dense, 1 contiguous, 2 masked.  rows: M, M_sum or max_m.
 inline PickedConfig pick_config(int kind, int rows, int N, int K, int G, int expected_m,
-                                int num_sms) {
+                                int num_sms, const ClusterLimits* lim = nullptr) {
   PickedConfig best{1, 1, 1, 1};
-  const int KB = K / 128;
-  // Rows that will actually carry tokens, per group, for the estimate.
+  if (kind == 0 && rows <= 128 && pick_decode(rows, N, K, num_sms, lim, &best)) return best;
+
+  // Everything else: persistent CTAs, no split.  Choose the tile width that
+  // minimises (waves x tile width), a proxy for the busiest SM's time,
+  // preferring wider tiles on ties.
   int eff_rows = rows;
   int groups = 1;
   if (kind == 2) {
@@ -47,33 +128,9 @@ inline PickedConfig pick_config(int kind, int rows, int N, int K, int G, int exp
     groups = G;
   }
   const int m_blocks = groups * ceil_div(eff_rows > 0 ? eff_rows : 1, 128);
-
-  // Decode-shaped dense problems (one 128-row block): memory-bound.  Keep a
-  // 128-wide tile and split K until the tiles fill the SMs in one wave.
-  if (kind == 0 && rows <= 128) {
-    const int v = 1;  // BLOCK_N = 128
-    const int n_tiles = ceil_div(N, kVariants[v].block_n);
-    int split = 1;
-    for (int s = 2; s <= KB && n_tiles * s <= num_sms; ++s) {
-      if (KB / s < 2) break;  // keep at least two K blocks per slice
-      split = s;
-    }
-    // prefer a split that divides the K blocks evenly, if one nearly as large exists
-    for (int s = split; s >= 2 && s * 4 >= split * 3; --s) {
-      if (KB % s == 0) { split = s; break; }
-    }
-    best.variant = v;
-    best.split_k = split;
-    best.out_tiles = n_tiles;
-    const int tiles = n_tiles * split;
-    best.grid = tiles < num_sms ? tiles : num_sms;
-    return best;
-  }
-
-  // Everything else: choose the tile width minimising (waves x tile width),
-  // a proxy for the time of the busiest SM, preferring wider tiles on ties.
   double best_cost = 1e30;
   for (int v = 0; v < kNumVariants; ++v) {
+    if (kVariants[v].decode) continue;
     const int bn = kVariants[v].block_n;
     if (bn > 128 && N <= 128) continue;
     const int n_tiles = ceil_div(N, bn);

@@ -1,12 +1,14 @@
 // dg_fp8_gemm_nt_noalloc: the dense GEMM for callers that cannot allocate
-// device memory.  Its scratch (split-K partial sums, split-K arrival counters
-// and the device error word) lives in one file-scope __device__ array of fixed
-// size instead of memory the library would otherwise cudaMalloc on first use.
-// The declaration and the contract are in include/dg.h.
+// device memory.  Its scratch -- the device error word the kernel's bounded
+// waits report into -- lives in one file-scope __device__ array of fixed size
+// instead of memory the library would otherwise cudaMalloc on first use.
+// (Split-K reduces through distributed shared memory and needs no global
+// scratch.)  The declaration and the contract are in include/dg.h.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
+#include <utility>
 
 #include "../../include/dg.h"
 #include "dg_config.h"
@@ -15,12 +17,8 @@
 namespace dg {
 namespace {
 
-// Layout of the static scratch: [error word | pad][counters][split-K partials]
-constexpr size_t kNaErrorBytes = 256;
-constexpr int kNaCounters = 4096;
-constexpr size_t kNaCounterBytes = kNaCounters * sizeof(int);
-constexpr size_t kNaWorkspaceBytes = size_t(12) << 20;  // 12 MiB of FP32 partial sums
-constexpr size_t kNaScratchBytes = kNaErrorBytes + kNaCounterBytes + kNaWorkspaceBytes;
+// Layout of the static scratch: [error word | pad to 256 bytes]
+constexpr size_t kNaScratchBytes = 256;
 
 // Every GPU that loads the library holds this array until the process exits.
 // In host code `g_noalloc_scratch` is only a host-side stand-in for the
@@ -34,6 +32,7 @@ struct NaDevice {
   int num_sms = 0;
   unsigned char* scratch = nullptr;  // device address of g_noalloc_scratch
   bool smem_attr_set[kNumVariants] = {};
+  ClusterLimits limits = {};         // co-resident split-K clusters (0: not known)
 };
 
 std::mutex g_na_mutex;
@@ -44,6 +43,63 @@ using NaEncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, v
                                 const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                 CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 NaEncodeFn g_na_encode = nullptr;
+
+template <int V>
+using NaShape = KernelShape<kVariants[V].block_n, kVariants[V].stages, kVariants[V].num_acc,
+                            kVariants[V].kps, kVariants[V].a_rows>;
+
+template <int V>
+auto na_kernel() {
+  constexpr Variant var = kVariants[V];
+  return fp8_gemm_kernel<kDense, var.block_n, var.stages, var.num_acc, var.kps, var.a_rows>;
+}
+
+template <int V>
+dg_status na_smem_attr(NaDevice& st) {
+  if (!st.smem_attr_set[V]) {
+    if (cudaFuncSetAttribute(na_kernel<V>(), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             NaShape<V>::kSmemBytes) != cudaSuccess)
+      return DG_ERR_CUDA;
+    st.smem_attr_set[V] = true;
+  }
+  return DG_OK;
+}
+
+// Split-K clusters of each size the device co-schedules for decode variant V.
+template <int V>
+dg_status na_cluster_limits(NaDevice& st) {
+  if constexpr (kVariants[V].decode) {
+    dg_status s = na_smem_attr<V>(st);
+    if (s != DG_OK) return s;
+    for (int c = 1; c <= kMaxSplitK; ++c) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(c, 1, 1);
+      cfg.blockDim = dim3(kThreads, 1, 1);
+      cfg.dynamicSmemBytes = NaShape<V>::kSmemBytes;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = c;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, na_kernel<V>(), &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        n = 0;
+      }
+      st.limits.max_clusters[V][c] = n;
+    }
+  }
+  return DG_OK;
+}
+
+template <int... V>
+dg_status na_all_cluster_limits(NaDevice& st, std::integer_sequence<int, V...>) {
+  dg_status s = DG_OK;
+  ((s = (s == DG_OK ? na_cluster_limits<V>(st) : s)), ...);
+  return s;
+}
 
 // Once per device, with that device current: check the architecture, find the
 // tensor-map encoder and the device address of the static scratch.  Nothing
@@ -74,18 +130,22 @@ dg_status na_setup(NaDevice** out) {
       return DG_ERR_CUDA;
     st.scratch = static_cast<unsigned char*>(ptr);
     st.num_sms = sms;
+    dg_status s = na_all_cluster_limits(st, std::make_integer_sequence<int, kNumVariants>{});
+    if (s != DG_OK) return s;
     st.ready = true;
   }
   *out = &st;
   return DG_OK;
 }
 
-dg_status na_map(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint32_t box1) {
-  cuuint64_t dims[3] = {d0, d1, 1};
-  cuuint64_t strides[2] = {d0, d0 * d1};
-  cuuint32_t box[3] = {128, box1, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = g_na_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims,
+// Same 4-D view of an E4M3 [rows][K] matrix as the regular entry points use.
+dg_status na_map(CUtensorMap* map, const void* base, uint64_t K, uint64_t rows, uint32_t box_rows,
+                 uint32_t kps) {
+  cuuint64_t dims[4] = {128, rows, K / 128, 1};
+  cuuint64_t strides[3] = {K, 128, K * rows};
+  cuuint32_t box[4] = {128, box_rows, kps, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = g_na_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims,
                            strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -95,21 +155,33 @@ dg_status na_map(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, u
 template <int V>
 dg_status na_launch(NaDevice& st, const CUtensorMap& ta, const CUtensorMap& tb,
                     const GemmArgs& args, int grid, cudaStream_t stream) {
-  constexpr Variant var = kVariants[V];
-  using Shape = KernelShape<var.block_n, var.stages, var.num_acc>;
-  auto kern = fp8_gemm_kernel<kDense, var.block_n, var.stages, var.num_acc>;
-  if (!st.smem_attr_set[V]) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Shape::kSmemBytes) != cudaSuccess)
-      return DG_ERR_CUDA;
-    st.smem_attr_set[V] = true;
-  }
+  dg_status s = na_smem_attr<V>(st);
+  if (s != DG_OK) return s;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = Shape::kSmemBytes;
+  cfg.dynamicSmemBytes = NaShape<V>::kSmemBytes;
   cfg.stream = stream;
-  return cudaLaunchKernelEx(&cfg, kern, ta, tb, args) == cudaSuccess ? DG_OK : DG_ERR_CUDA;
+  cudaLaunchAttribute attr[1];
+  if (args.split_k > 1) {  // the CTAs of one output tile form a cluster
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = args.split_k;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  return cudaLaunchKernelEx(&cfg, na_kernel<V>(), ta, tb, args) == cudaSuccess ? DG_OK
+                                                                               : DG_ERR_CUDA;
+}
+
+template <int... V>
+dg_status na_dispatch(NaDevice& st, int variant, const CUtensorMap& ta, const CUtensorMap& tb,
+                      const GemmArgs& args, int grid, cudaStream_t stream,
+                      std::integer_sequence<int, V...>) {
+  dg_status s = DG_ERR_UNSUPPORTED;
+  ((variant == V ? (s = na_launch<V>(st, ta, tb, args, grid, stream), 0) : 0), ...);
+  return s;
 }
 
 }  // namespace
@@ -134,7 +206,7 @@ extern "C" dg_status dg_fp8_gemm_nt_noalloc(const void* a, const float* sfa, con
   dg_status s = na_setup(&st);
   if (s != DG_OK) return s;
 
-  const PickedConfig pc = pick_config(kDense, M, N, K, 1, 0, st->num_sms);
+  const PickedConfig pc = pick_config(kDense, M, N, K, 1, 0, st->num_sms, &st->limits);
   const Variant var = kVariants[pc.variant];
   GemmArgs args = {};
   args.rows = M;
@@ -151,28 +223,19 @@ extern "C" dg_status dg_fp8_gemm_nt_noalloc(const void* a, const float* sfa, con
   args.sfb = sfb;
   args.d = static_cast<__nv_bfloat16*>(d);
   args.error_word = reinterpret_cast<int*>(st->scratch);
-  args.counters = reinterpret_cast<int*>(st->scratch + kNaErrorBytes);
-  args.workspace = reinterpret_cast<float*>(st->scratch + kNaErrorBytes + kNaCounterBytes);
   args.timeout_ns = 1000ull * 1000 * 1000;
-  if (pc.split_k > 1) {
-    const size_t ws = static_cast<size_t>(pc.out_tiles) * pc.split_k * kBlockM * var.block_n *
-                      sizeof(float);
-    if (ws > kNaWorkspaceBytes || pc.out_tiles > kNaCounters) return DG_ERR_UNSUPPORTED;
-    // the arrival counters must start at zero; the array keeps the last call's contents
-    if (cudaMemsetAsync(args.counters, 0, pc.out_tiles * sizeof(int), stream) != cudaSuccess)
-      return DG_ERR_CUDA;
-  }
+  args.a_box_rows = M >= kBlockM ? kBlockM : ((M + 15) / 16) * 16;
+  args.prefetch = 1;
+  if (args.a_box_rows > var.a_rows) return DG_ERR_UNSUPPORTED;
+  if (pc.split_k > 1 && (pc.grid != args.num_m_blocks * args.num_n_blocks * pc.split_k ||
+                         M > kBlockM || !split_fits(var, M, pc.split_k)))
+    return DG_ERR_UNSUPPORTED;
 
   CUtensorMap ta, tb;
-  s = na_map(&ta, a, K, M, kBlockM);
+  s = na_map(&ta, a, K, M, args.a_box_rows, var.kps);
   if (s != DG_OK) return s;
-  s = na_map(&tb, b, K, N, var.block_n);
+  s = na_map(&tb, b, K, N, var.block_n, var.kps);
   if (s != DG_OK) return s;
-  switch (pc.variant) {
-    case 0: return na_launch<0>(*st, ta, tb, args, pc.grid, stream);
-    case 1: return na_launch<1>(*st, ta, tb, args, pc.grid, stream);
-    case 2: return na_launch<2>(*st, ta, tb, args, pc.grid, stream);
-    case 3: return na_launch<3>(*st, ta, tb, args, pc.grid, stream);
-    default: return DG_ERR_UNSUPPORTED;
-  }
+  return na_dispatch(*st, pc.variant, ta, tb, args, pc.grid, stream,
+                     std::make_integer_sequence<int, kNumVariants>{});
 }

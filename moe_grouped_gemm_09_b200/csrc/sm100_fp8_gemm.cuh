@@ -21,10 +21,18 @@
 //  * Warp roles in a 256-thread CTA: warp 0 issues TMA loads of A and B tiles
 //    (128-byte swizzle) into a multi-stage shared-memory ring; warp 1 owns the
 //    TMEM allocation and issues tcgen05.cp (scales) + tcgen05.mma; warp 2
-//    turns the FP32 scales of each stage into the UE8M0 layout that tcgen05.cp
-//    expects; warps 4..7 drain the TMEM accumulator (tcgen05.ld), convert to
-//    BF16 and store, or, for split-K, write FP32 partials and let the last CTA
-//    of the tile reduce them in a fixed order (deterministic).
+//    turns the FP32 scales into the UE8M0 layout that tcgen05.cp expects,
+//    loading them several stages ahead so that their latency stays hidden;
+//    warps 4..7 drain the TMEM accumulator (tcgen05.ld), convert to BF16 and
+//    store.
+//  * Split-K (decode shapes, too few output tiles for the SMs): the CTAs that
+//    share an output tile form one thread-block cluster, each computes the
+//    partial sum of its K slice, parks it in its own shared memory, and after
+//    a cluster barrier every CTA reduces a slice of the rows by reading the
+//    partials of all CTAs through distributed shared memory, in a fixed
+//    order (deterministic), then stores BF16.  No global scratch is used.
+//  * Before waiting on the previous kernel (programmatic dependent launch),
+//    the producer asks TMA to prefetch its first tile's operands into L2.
 //  * Persistent CTAs walk a static tile sequence.  For the grouped layouts the
 //    sequence is group-aware: contiguous tiles read their expert from
 //    m_indices and skip all-padding blocks; masked tiles are enumerated over
@@ -58,7 +66,8 @@ struct GemmArgs {
   int num_m_blocks;  // m-blocks per group: ceil(rows / 128)
   int num_n_blocks;  // ceil(N / BLOCK_N)
   int k_blocks;      // K / 128
-  int split_k;       // number of K slices per output tile (>= 1)
+  int split_k;       // K slices per output tile; > 1: cluster of split_k CTAs per tile,
+                     // launched with exactly one tile per CTA
   int kb_per_split;  // ceil(k_blocks / split_k)
   int nb128;         // ceil(N / 128): B scale blocks along N
   const float* sfa;  // [G * rows, k_blocks]   (dense/contiguous: G = 1 row space)
@@ -66,16 +75,17 @@ struct GemmArgs {
   __nv_bfloat16* d;  // [G * rows, N]
   const int* m_indices;  // contiguous: [rows]
   const int* masked_m;   // masked: [G]
-  float* workspace;      // split-K partials
-  int* counters;         // split-K arrival counters, one per output tile, zero between launches
   int* error_word;
   unsigned long long timeout_ns;
+  int a_box_rows;    // rows of A one TMA box brings (128, or fewer for a short dense A)
+  int prefetch;      // 1: warm L2 with the first tile before waiting on the previous kernel
 };
 
 constexpr int kBlockM = 128;
 constexpr int kBlockK = 128;
 constexpr int kThreads = 256;
 constexpr int kMaxMaskedGroups = 1024;
+constexpr int kMaxSplit = 8;  // CTAs per split-K cluster (portable cluster size)
 
 __host__ __device__ constexpr int pow2_ceil(int x) {
   int p = 32;
@@ -83,22 +93,43 @@ __host__ __device__ constexpr int pow2_ceil(int x) {
   return p;
 }
 
-template <int BLOCK_N, int STAGES, int NUM_ACC>
+// Compile-time geometry of one kernel variant.
+//   BLOCK_N  output columns (rows of B) per tile
+//   STAGES   depth of the shared-memory operand ring
+//   NUM_ACC  TMEM accumulator buffers (2: the epilogue of a tile overlaps the
+//            next tile's main loop)
+//   KPS      128-wide K blocks per ring stage: every stage is one TMA box of A
+//            and one of B, each KPS K blocks deep (bigger boxes stream faster)
+//   A_ROWS   rows of A a stage holds room for (64 for a dense A of at most 64
+//            rows, else 128)
+template <int BLOCK_N, int STAGES, int NUM_ACC, int KPS = 1, int A_ROWS = 128>
 struct KernelShape {
-  static constexpr int kABytes = kBlockM * kBlockK;  // one E4M3 byte per element
-  static constexpr int kBBytes = BLOCK_N * kBlockK;
+  static constexpr int kABytes = KPS * A_ROWS * kBlockK;  // one E4M3 byte per element
+  static constexpr int kBBytes = KPS * BLOCK_N * kBlockK;
   static constexpr int kSfbChunks = (BLOCK_N + 127) / 128;
   static constexpr int kSfBytes = 512 * (1 + kSfbChunks);  // SFA 512 B + SFB 512 B per 128 rows
   static constexpr int kSfCols = 4 * (1 + kSfbChunks);     // TMEM columns per stage
   static constexpr int kAccCols = NUM_ACC * BLOCK_N;
   static constexpr int kTmemCols = pow2_ceil(kAccCols + STAGES * kSfCols);
-  static constexpr int kBarBytes = 8 * (2 * STAGES + 2 * NUM_ACC + 1);
-  static constexpr int kMiscBytes = 16 + 4 * (kMaxMaskedGroups + 1);
+  static constexpr int kBarBytes = 8 * (2 * STAGES + 2 * NUM_ACC + 2);
+  // epilogue: each of the 4 epilogue warps transposes 32 rows x kEpiCols
+  // BF16 columns through shared memory so that its global stores are whole
+  // 128-byte row segments
+  static constexpr int kEpiCols = BLOCK_N >= 64 ? 64 : 32;
+  static constexpr int kEpiPitch = kEpiCols * 2 + 16;  // bytes per staged row (bank spread)
+  static constexpr int kEpiBytes = 4 * 32 * kEpiPitch;
+  static constexpr int kMiscBytes = 16 + 4 * (kMaxMaskedGroups + 1);  // tmem slot, flags, prefix
+  // A short A tile is read by the 128-row MMA past its end (rows that only
+  // feed never-stored accumulator rows); the B ring follows the A ring, so
+  // that read stays inside this CTA's shared memory.
   static constexpr int kSmemBytes = 1024 /* alignment slack */ + STAGES * (kABytes + kBBytes) +
-                                    STAGES * kSfBytes + kBarBytes + kMiscBytes;
+                                    STAGES * kSfBytes + kEpiBytes + kBarBytes + kMiscBytes;
+  static_assert(kSmemBytes <= 232448, "shared memory budget (227 KB) exceeded");
   static_assert(kTmemCols <= 512, "TMEM budget exceeded");
   static_assert(BLOCK_N % 32 == 0 && BLOCK_N >= 32 && BLOCK_N <= 256, "BLOCK_N");
-  static_assert(kBBytes % 1024 == 0, "B tile must keep 1024-byte alignment");
+  static_assert(KPS >= 1 && KPS <= 4, "up to four K blocks share one scale-factor word");
+  static_assert(A_ROWS == 64 || A_ROWS == 128, "A_ROWS");
+  static_assert((BLOCK_N * kBlockK) % 1024 == 0, "B sub-tiles must keep 1024-byte alignment");
 };
 
 struct Tile {
@@ -106,12 +137,9 @@ struct Tile {
   bool skip;
 };
 
-__device__ __forceinline__ uint32_t ue8m0_x4(float v) {
-  // A positive power-of-two FP32 value is 2^(e-127) with e its exponent
-  // field; UE8M0 encodes 2^(e-127) as the byte e.  Replicated into 4 bytes.
-  uint32_t e = (__float_as_uint(v) >> 23) & 0xFFu;
-  return e * 0x01010101u;
-}
+// A positive power-of-two FP32 value is 2^(e-127) with e its exponent field;
+// UE8M0 encodes 2^(e-127) as the byte e.
+__device__ __forceinline__ uint32_t ue8m0(float v) { return (__float_as_uint(v) >> 23) & 0xFFu; }
 
 // Expert of a 128-row block in the contiguous layout: the largest m_indices
 // entry of the block (padding rows are -1).  Warp-collective.
@@ -187,11 +215,62 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-template <int KIND, int BLOCK_N, int STAGES, int NUM_ACC>
+// Walks the tiles one CTA owns (t = first, first + stride, ...), skipping
+// tiles with no work.  Warp-collective for the contiguous layout.
+template <int KIND>
+struct TileWalker {
+  int t, stride, total;
+  Tile ti;
+  bool valid;
+
+  __device__ __forceinline__ void seek(const GemmArgs& p, const int* s_prefix, int lane) {
+    valid = false;
+    while (t < total) {
+      ti = get_tile<KIND>(t, p, s_prefix, lane);
+      if (!ti.skip) { valid = true; return; }
+      t += stride;
+    }
+  }
+  __device__ __forceinline__ void start(int first, int stride_, int total_, const GemmArgs& p,
+                                        const int* s_prefix, int lane) {
+    t = first; stride = stride_; total = total_;
+    seek(p, s_prefix, lane);
+  }
+  __device__ __forceinline__ void next(const GemmArgs& p, const int* s_prefix, int lane) {
+    t += stride;
+    seek(p, s_prefix, lane);
+  }
+};
+
+// Walks (tile, stage) pairs in the order the pipeline consumes them; a stage
+// starts at K block `kb` and covers up to STEP K blocks.
+template <int KIND, int STEP>
+struct StageWalker {
+  TileWalker<KIND> w;
+  int kb;
+  bool done;
+
+  __device__ __forceinline__ void start(int first, int stride, int total, const GemmArgs& p,
+                                        const int* s_prefix, int lane) {
+    w.start(first, stride, total, p, s_prefix, lane);
+    done = !w.valid;
+    kb = done ? 0 : w.ti.kb_begin;
+  }
+  __device__ __forceinline__ void next(const GemmArgs& p, const int* s_prefix, int lane) {
+    kb += STEP;
+    if (kb >= w.ti.kb_end) {
+      w.next(p, s_prefix, lane);
+      done = !w.valid;
+      kb = done ? 0 : w.ti.kb_begin;
+    }
+  }
+};
+
+template <int KIND, int BLOCK_N, int STAGES, int NUM_ACC, int KPS, int A_ROWS>
 __global__ void __launch_bounds__(kThreads, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     const __grid_constant__ CUtensorMap tmap_b, const GemmArgs p) {
-  using Shape = KernelShape<BLOCK_N, STAGES, NUM_ACC>;
+  using Shape = KernelShape<BLOCK_N, STAGES, NUM_ACC, KPS, A_ROWS>;
   constexpr int A_BYTES = Shape::kABytes;
   constexpr int B_BYTES = Shape::kBBytes;
   constexpr int SF_BYTES = Shape::kSfBytes;
@@ -199,6 +278,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int SFB_CHUNKS = Shape::kSfbChunks;
   constexpr int ACC_COLS = Shape::kAccCols;
   constexpr int TMEM_COLS = Shape::kTmemCols;
+  constexpr int RED_PITCH = BLOCK_N + 4;  // floats per row of a parked split-K partial
+  // split-K: parked partial (valid rows) plus incoming slices (at most
+  // valid rows + split more) live in the idle operand ring; the host only
+  // picks a split for which (2 * valid rows + split) rows fit.
+  static_assert(kBlockM * RED_PITCH * 4 <= STAGES * (A_BYTES + B_BYTES),
+                "split-K partial must fit in the operand ring");
+  static_assert(KPS == 1 || KIND == kDense, "multi-K-block stages are built for the dense form");
 
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment for the 128-byte-swizzled operand tiles
@@ -207,18 +293,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sA = smem;
   uint8_t* sB = sA + STAGES * A_BYTES;
   uint8_t* sSF = sB + STAGES * B_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sSF + STAGES * SF_BYTES);
+  uint8_t* sEpi = sSF + STAGES * SF_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sEpi + Shape::kEpiBytes);
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;
   uint64_t* acc_empty = acc_full + NUM_ACC;
   uint64_t* drain = acc_empty + NUM_ACC;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* recv_bar = drain + 1;  // split-K: partial slices pushed by the other CTAs
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(recv_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  volatile int* s_is_last = abort_flag + 1;
-  int* s_prefix = const_cast<int*>(s_is_last + 2);
+  int* s_prefix = const_cast<int*>(abort_flag + 3);
+  // split-K: this CTA's FP32 partial, parked over the (by then idle) operand ring
+  float* red = reinterpret_cast<float*>(sA);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
+  const bool split = p.split_k > 1;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -230,6 +320,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::mbar_init(&acc_empty[a], 128);  // every epilogue thread
     }
     ptx::mbar_init(drain, 1);
+    ptx::mbar_init(recv_bar, 1);
     *abort_flag = 0;
     ptx::fence_mbar_init();
     ptx::prefetch_tensormap(&tmap_a);
@@ -239,9 +330,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::tmem_alloc(tmem_slot, TMEM_COLS);
     ptx::tmem_relinquish();
   }
-  // Everything above touches no input; wait for the preceding kernel (if it
-  // was launched as a programmatic dependency) only now.
+  if (KIND == kDense && p.prefetch && warp == 0 && lane == 0 &&
+      blockIdx.x < p.num_m_blocks * p.num_n_blocks * p.split_k) {
+    // Warm L2 with this CTA's first tile while the previous kernel finishes
+    // (the tile order of the dense form does not depend on device data).
+    const Tile ti = get_tile<kDense>(blockIdx.x, p, nullptr, lane);
+    const int kb_end = min(ti.kb_end, ti.kb_begin + STAGES * KPS);
+    for (int kb = ti.kb_begin; kb < kb_end; kb += KPS) {
+      ptx::tma_prefetch_l2_4d(&tmap_b, 0, ti.n_blk * BLOCK_N, kb, 0);
+      ptx::tma_prefetch_l2_4d(&tmap_a, 0, ti.m_blk * kBlockM, kb, 0);
+    }
+  }
+  // Everything above reads no input; from here on the inputs may be the
+  // previous kernel's outputs, so wait for it (a no-op without programmatic
+  // dependent launch), and let the next kernel start its own prologue.
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (KIND == kMasked && threadIdx.x == 96) {
     int acc = 0;
     for (int g = 0; g < p.G; ++g) {
@@ -269,16 +373,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ti.skip) continue;
       const int a_row = ti.m_blk * kBlockM;
       const int a_grp = (KIND == kMasked) ? ti.group : 0;
-      for (int kb = ti.kb_begin; kb < ti.kb_end; ++kb, ++it) {
+      for (int kb = ti.kb_begin; kb < ti.kb_end; kb += KPS, ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
         if (lane == 0) {
           ok = ptx::mbar_wait(&empty[s], ph ^ 1, ctl, kDevTimeoutProducer);
           if (ok) {
-            ptx::mbar_arrive_expect_tx(&full[s], A_BYTES + B_BYTES);
-            ptx::tma_load_3d(sA + s * A_BYTES, &tmap_a, &full[s], kb * kBlockK, a_row, a_grp);
-            ptx::tma_load_3d(sB + s * B_BYTES, &tmap_b, &full[s], kb * kBlockK,
-                             ti.n_blk * BLOCK_N, ti.group);
+            // One box of A and one of B, each KPS K blocks deep (blocks past K
+            // are zero-filled and still counted).  A short dense A (fewer
+            // than 128 rows) is fetched with a box of only its rows; the
+            // 128-row MMA then reads stale shared memory for the other rows,
+            // which only feeds accumulator rows that are never stored.
+            ptx::mbar_arrive_expect_tx(&full[s], KPS * (p.a_box_rows + BLOCK_N) * kBlockK);
+            ptx::tma_load_4d(sA + s * A_BYTES, &tmap_a, &full[s], 0, a_row, kb, a_grp);
+            ptx::tma_load_4d(sB + s * B_BYTES, &tmap_b, &full[s], 0, ti.n_blk * BLOCK_N, kb,
+                             ti.group);
           }
         }
         ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
@@ -305,7 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       ptx::tc_fence_after_sync();
       const uint32_t d_tmem = tmem_base + a * BLOCK_N;
-      for (int kb = ti.kb_begin; kb < ti.kb_end; ++kb, ++it) {
+      for (int kb = ti.kb_begin; kb < ti.kb_end; kb += KPS, ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
         if (lane == 0) ok = ptx::mbar_wait(&full[s], ph, ctl, kDevTimeoutMma);
@@ -320,12 +429,23 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int h = 0; h < SFB_CHUNKS; ++h)
             ptx::tc_cp_32x128b_warpx4(sfb_tmem + 4 * h, ptx::sdesc_sf_32x16(sf_smem + 512 * (1 + h)));
-          const uint64_t da = ptx::sdesc_kmajor_sw128(ptx::smem_addr(sA + s * A_BYTES));
-          const uint64_t db = ptx::sdesc_kmajor_sw128(ptx::smem_addr(sB + s * B_BYTES));
+          const uint32_t a_base = ptx::smem_addr(sA + s * A_BYTES);
+          const uint32_t b_base = ptx::smem_addr(sB + s * B_BYTES);
 #pragma unroll
-          for (int ks = 0; ks < kBlockK / 32; ++ks)
-            ptx::tc_mma_mxf8_block_scale(d_tmem, da + 2 * ks, db + 2 * ks, idesc, sfa_tmem,
-                                         sfb_tmem, kb > ti.kb_begin || ks > 0);
+          for (int j = 0; j < KPS; ++j) {
+            if (kb + j >= ti.kb_end) break;
+            // K block j of the stage: its scale factors are byte j of every
+            // TMEM scale word (selected by the scale-factor id)
+            const uint64_t da = ptx::sdesc_kmajor_sw128(a_base + j * p.a_box_rows * kBlockK);
+            const uint64_t db = ptx::sdesc_kmajor_sw128(b_base + j * BLOCK_N * kBlockK);
+            const uint32_t id = idesc | (static_cast<uint32_t>(j) << 29) | (static_cast<uint32_t>(j) << 4);
+            const uint32_t byte_sel = static_cast<uint32_t>(j) << 30;
+#pragma unroll
+            for (int ks = 0; ks < kBlockK / 32; ++ks)
+              ptx::tc_mma_mxf8_block_scale(d_tmem, da + 2 * ks, db + 2 * ks, id,
+                                           sfa_tmem | byte_sel, sfb_tmem | byte_sel,
+                                           kb + j > ti.kb_begin || ks > 0);
+          }
           ptx::tc_commit(&empty[s]);
         }
         __syncwarp();
@@ -343,16 +463,53 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == 2) {
     // --------------------------------------------- scale-factor producer --
+    // The FP32 scales of a stage are loaded PF stages before they are
+    // written, so the global-load latency overlaps several pipeline stages.
+    // Scale words pack the stage's K blocks: byte j belongs to K block j.
+    constexpr int PF = (8 + KPS - 1) / KPS;
     const int KB = p.k_blocks;
-    int it = 0;
-    bool ok = true;
-    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-      const Tile ti = get_tile<KIND>(t, p, s_prefix, lane);
-      if (ti.skip) continue;
+    float va[PF][4][KPS];
+    float vb[PF][SFB_CHUNKS][KPS];
+    StageWalker<KIND, KPS> ld, wr;
+    ld.start(blockIdx.x, gridDim.x, total, p, s_prefix, lane);
+    wr.start(blockIdx.x, gridDim.x, total, p, s_prefix, lane);
+
+    auto issue = [&](float (&a)[4][KPS], float (&b)[SFB_CHUNKS][KPS]) {
+      const Tile& ti = ld.w.ti;
       const int row_base = (KIND == kMasked ? ti.group * p.rows : 0) + ti.m_blk * kBlockM;
       const int rows_left = p.rows - ti.m_blk * kBlockM;  // rows of this block that exist
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int r = 32 * c + lane;
+#pragma unroll
+        for (int j = 0; j < KPS; ++j)
+          a[c][j] = (r < rows_left && ld.kb + j < ti.kb_end)
+                        ? __ldg(p.sfa + (size_t)(row_base + r) * KB + ld.kb + j)
+                        : 1.0f;
+      }
+      // B scale blocks are 128 rows; every tile width divides or is a
+      // multiple of 128, so one value covers each 128-row chunk of the tile.
       const float* sfb_g = p.sfb + (size_t)ti.group * p.nb128 * KB;
-      for (int kb = ti.kb_begin; kb < ti.kb_end; ++kb, ++it) {
+#pragma unroll
+      for (int h = 0; h < SFB_CHUNKS; ++h) {
+        const int nb = min((ti.n_blk * BLOCK_N + 128 * h) / 128, p.nb128 - 1);
+#pragma unroll
+        for (int j = 0; j < KPS; ++j)
+          b[h][j] = (ld.kb + j < ti.kb_end) ? __ldg(sfb_g + (size_t)nb * KB + ld.kb + j) : 1.0f;
+      }
+      ld.next(p, s_prefix, lane);
+    };
+
+#pragma unroll
+    for (int j = 0; j < PF; ++j)
+      if (!ld.done) issue(va[j], vb[j]);
+
+    int it = 0;
+    bool ok = true;
+    while (!wr.done && ok) {
+#pragma unroll
+      for (int slot = 0; slot < PF; ++slot) {
+        if (wr.done || !ok) break;
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
         if (lane == 0) ok = ptx::mbar_wait(&empty[s], ph ^ 1, ctl, kDevTimeoutScales);
@@ -360,31 +517,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         uint8_t* sf = sSF + s * SF_BYTES;
         // A scales: TMEM lane l, column c holds row 32c + l of the tile.
-        uint4 wa;
-        uint32_t* wa_ = reinterpret_cast<uint32_t*>(&wa);
+        uint32_t w[4];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          const int r = 32 * c + lane;
-          const float v = (r < rows_left) ? __ldg(p.sfa + (size_t)(row_base + r) * KB + kb) : 1.0f;
-          wa_[c] = ue8m0_x4(v);
+          uint32_t x = 0x7F7F7F7Fu;  // unused bytes: scale 1
+#pragma unroll
+          for (int j = 0; j < KPS; ++j)
+            x = (x & ~(0xFFu << (8 * j))) | (ue8m0(va[slot][c][j]) << (8 * j));
+          w[c] = x;
         }
-        *reinterpret_cast<uint4*>(sf + 16 * lane) = wa;
-        // B scales: one per 128 rows of B, replicated over the rows of the tile.
+        *reinterpret_cast<uint4*>(sf + 16 * lane) = make_uint4(w[0], w[1], w[2], w[3]);
 #pragma unroll
         for (int h = 0; h < SFB_CHUNKS; ++h) {
-          uint4 wb;
-          uint32_t* wb_ = reinterpret_cast<uint32_t*>(&wb);
+          uint32_t x = 0x7F7F7F7Fu;
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const int n = ti.n_blk * BLOCK_N + 128 * h + 32 * c + lane;
-            const int nb = min(n / 128, p.nb128 - 1);
-            wb_[c] = ue8m0_x4(__ldg(sfb_g + (size_t)nb * KB + kb));
-          }
-          *reinterpret_cast<uint4*>(sf + 512 * (1 + h) + 16 * lane) = wb;
+          for (int j = 0; j < KPS; ++j)
+            x = (x & ~(0xFFu << (8 * j))) | (ue8m0(vb[slot][h][j]) << (8 * j));
+          *reinterpret_cast<uint4*>(sf + 512 * (1 + h) + 16 * lane) = make_uint4(x, x, x, x);
         }
         ptx::fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&full[s]);
+        if (!ld.done) issue(va[slot], vb[slot]);
+        wr.next(p, s_prefix, lane);
+        ++it;
       }
     }
   } else if (warp >= 4) {
@@ -399,14 +555,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ti.skip) {
         if (KIND == kContiguous && ti.group >= p.G && ep_tid == 0)
           atomicCAS(p.error_word, 0, kDevExpertRange);
+        if (split) {
+          // an empty K slice still contributes (zeros) to the cluster's sum
+          const int valid_rows = min(p.rows - ti.m_blk * kBlockM, kBlockM);
+          if (row_local < valid_rows)
+            for (int c = 0; c < BLOCK_N; c += 4)
+              *reinterpret_cast<float4*>(red + row_local * RED_PITCH + c) = make_float4(0, 0, 0, 0);
+          ptx::fence_proxy_async_smem();  // parked rows are read by bulk copies
+        }
         continue;
       }
       const int a = acc_it % NUM_ACC;
       const uint32_t aph = (acc_it / NUM_ACC) & 1;
       if (lane == 0) ok = ptx::mbar_wait(&acc_full[a], aph, ctl, kDevTimeoutEpilogue);
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-      // all four epilogue warps take the same branch, so the named barriers
-      // below are always reached by all 128 threads
+      // all four epilogue warps take the same branch
       ok = named_bar_and(2, 128, ok);
       if (!ok) break;
       ptx::tc_fence_after_sync();
@@ -431,94 +594,136 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + a * BLOCK_N;
       const int n0 = ti.n_blk * BLOCK_N;
 
-      if (p.split_k == 1) {
+      // A warp whose 32 rows are all outside the output (a short dense A, a
+      // masked group) skips the TMEM reads; it still releases the buffer.
+      if (__any_sync(0xFFFFFFFFu, valid)) {
+        constexpr int CH = Shape::kEpiCols;  // columns per TMEM wait
+        uint8_t* stage = sEpi + q * 32 * Shape::kEpiPitch;
 #pragma unroll 1
-        for (int c0 = 0; c0 < BLOCK_N; c0 += 32) {
-          uint32_t r[32];
-          ptx::tc_ld_32x32b_x32(t_row + c0, r);
+        for (int c0 = 0; c0 < BLOCK_N; c0 += CH) {
+          uint32_t r[CH];
+          ptx::tc_ld_32x32b_x32(t_row + c0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+          if (CH == 64)
+            ptx::tc_ld_32x32b_x32(t_row + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[CH - 32]));
           ptx::tc_wait_ld();
-          if (valid) {
-            __nv_bfloat16* drow = p.d + grow * p.N;
+          if (split) {
+            // park the FP32 partial; the cluster reduces it below
+            if (valid) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const int n = n0 + c0 + 8 * j;
-              if (n < p.N) {
-                uint4 v;
-                v.x = pack_bf16x2(__uint_as_float(r[8 * j + 0]), __uint_as_float(r[8 * j + 1]));
-                v.y = pack_bf16x2(__uint_as_float(r[8 * j + 2]), __uint_as_float(r[8 * j + 3]));
-                v.z = pack_bf16x2(__uint_as_float(r[8 * j + 4]), __uint_as_float(r[8 * j + 5]));
-                v.w = pack_bf16x2(__uint_as_float(r[8 * j + 6]), __uint_as_float(r[8 * j + 7]));
-                *reinterpret_cast<uint4*>(drow + n) = v;
-              }
+              for (int j = 0; j < CH / 4; ++j)
+                *reinterpret_cast<float4*>(red + row_local * RED_PITCH + c0 + 4 * j) =
+                    make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+            }
+            continue;
+          }
+          // BF16 row of this lane into the warp's staging tile ...
+#pragma unroll
+          for (int j = 0; j < CH / 8; ++j) {
+            uint4 v;
+            v.x = pack_bf16x2(__uint_as_float(r[8 * j + 0]), __uint_as_float(r[8 * j + 1]));
+            v.y = pack_bf16x2(__uint_as_float(r[8 * j + 2]), __uint_as_float(r[8 * j + 3]));
+            v.z = pack_bf16x2(__uint_as_float(r[8 * j + 4]), __uint_as_float(r[8 * j + 5]));
+            v.w = pack_bf16x2(__uint_as_float(r[8 * j + 6]), __uint_as_float(r[8 * j + 7]));
+            *reinterpret_cast<uint4*>(stage + lane * Shape::kEpiPitch + 16 * j) = v;
+          }
+          __syncwarp();
+          // ... then whole row segments: a store instruction covers 32 / (CH / 8)
+          // rows, CH / 8 lanes per row, 16 bytes a lane.
+          constexpr int LPR = CH / 8;    // lanes per row
+          constexpr int RPI = 32 / LPR;  // rows per instruction
+          const int sub = lane % LPR;
+#pragma unroll
+          for (int i = 0; i < 32 / RPI; ++i) {
+            const int rr = RPI * i + lane / LPR;  // row within the warp's 32
+            const bool row_ok = __shfl_sync(0xFFFFFFFFu, valid, rr);
+            const int n = n0 + c0 + 8 * sub;
+            if (row_ok && n < p.N) {
+              const size_t g_row = grow - lane + rr;  // the rows of a warp are consecutive
+              *reinterpret_cast<uint4*>(p.d + g_row * p.N + n) =
+                  *reinterpret_cast<const uint4*>(stage + rr * Shape::kEpiPitch + 16 * sub);
             }
           }
+          __syncwarp();
         }
-        ptx::tc_fence_before_sync();
-        ptx::mbar_arrive(&acc_empty[a]);
-      } else {
-        // Split-K: FP32 partial of this K slice to the workspace, laid out as
-        // [column/4][row][4] so that a warp's stores are contiguous.
-        const int S = p.split_k;
-        float4* ws_tile = reinterpret_cast<float4*>(p.workspace) +
-                          (size_t)ti.out_tile * S * (kBlockM * BLOCK_N / 4);
-        float4* mine = ws_tile + (size_t)ti.split * (kBlockM * BLOCK_N / 4);
-#pragma unroll 1
-        for (int c0 = 0; c0 < BLOCK_N; c0 += 32) {
-          uint32_t r[32];
-          ptx::tc_ld_32x32b_x32(t_row + c0, r);
-          ptx::tc_wait_ld();
-          if (valid) {
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-              __stcg(mine + (size_t)(c0 / 4 + j) * kBlockM + row_local,
-                     make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
-                                 __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3])));
-          }
-        }
-        ptx::tc_fence_before_sync();
-        ptx::mbar_arrive(&acc_empty[a]);
-        __threadfence();
-        named_bar_sync(1, 128);
-        if (ep_tid == 0) {
-          const int old = atomicAdd(p.counters + ti.out_tile, 1);
-          *s_is_last = (old == S - 1);
-        }
-        named_bar_sync(1, 128);
-        if (*s_is_last) {
-          __threadfence();
-          if (valid) {
-            __nv_bfloat16* drow = p.d + grow * p.N;
-#pragma unroll 1
-            for (int c8 = 0; c8 < BLOCK_N / 8; ++c8) {
-              const int n = n0 + 8 * c8;
-              if (n >= p.N) break;
-              float4 lo = __ldcg(ws_tile + (size_t)(2 * c8) * kBlockM + row_local);
-              float4 hi = __ldcg(ws_tile + (size_t)(2 * c8 + 1) * kBlockM + row_local);
-              for (int sp = 1; sp < S; ++sp) {  // fixed order: deterministic
-                const float4* part = ws_tile + (size_t)sp * (kBlockM * BLOCK_N / 4);
-                const float4 l2 = __ldcg(part + (size_t)(2 * c8) * kBlockM + row_local);
-                const float4 h2 = __ldcg(part + (size_t)(2 * c8 + 1) * kBlockM + row_local);
-                lo.x += l2.x; lo.y += l2.y; lo.z += l2.z; lo.w += l2.w;
-                hi.x += h2.x; hi.y += h2.y; hi.z += h2.z; hi.w += h2.w;
-              }
-              uint4 v;
-              v.x = pack_bf16x2(lo.x, lo.y);
-              v.y = pack_bf16x2(lo.z, lo.w);
-              v.z = pack_bf16x2(hi.x, hi.y);
-              v.w = pack_bf16x2(hi.z, hi.w);
-              *reinterpret_cast<uint4*>(drow + n) = v;
-            }
-          }
-          if (ep_tid == 0) p.counters[ti.out_tile] = 0;  // ready for the next launch
-        }
-        named_bar_sync(1, 128);  // s_is_last is reused by the next tile
+        if (split) ptx::fence_proxy_async_smem();  // parked rows are read by bulk copies
       }
+      ptx::tc_fence_before_sync();
+      ptx::mbar_arrive(&acc_empty[a]);
       ++acc_it;
     }
   }
 
-  // Let a dependent kernel (programmatic launch) start its prologue.
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (split) {
+    // ---------------------------------------- split-K cluster reduction --
+    // One output tile per cluster, one K slice per CTA (rank = slice).  The
+    // tile's valid rows are cut into one slice per CTA; every CTA pushes the
+    // rows of each other CTA's slice of its parked partial to that CTA with
+    // one bulk copy (distributed shared memory), then sums the partials of
+    // its own slice in rank order and stores BF16.
+    const int S = p.split_k;
+    const uint32_t rank = ptx::cluster_ctarank();
+    const Tile ti = get_tile<KIND>(blockIdx.x, p, s_prefix, lane);
+    const int valid_rows = min(p.rows - ti.m_blk * kBlockM, kBlockM);
+    const int rows_per = (valid_rows + S - 1) / S;
+    auto slice_rows = [&](int r) { return max(0, min(valid_rows, (r + 1) * rows_per) - r * rows_per); };
+    // incoming slices land after the parked rows: slot `src` holds CTA src's rows
+    float* recv = red + valid_rows * RED_PITCH;
+    static_assert(RED_PITCH % 4 == 0, "16-byte rows");
+    __syncwarp();
+    ptx::cluster_sync();  // every CTA has parked its partial and is done with its ring
+    if (threadIdx.x == 0) {
+      const uint32_t mine = static_cast<uint32_t>(slice_rows(rank) * RED_PITCH * 4);
+      ptx::mbar_arrive_expect_tx(recv_bar, (S - 1) * mine);
+      const uint32_t bar_local = ptx::smem_addr(recv_bar);
+      const uint32_t slot_local = ptx::smem_addr(recv + rank * rows_per * RED_PITCH);
+      for (int dst = 0; dst < S; ++dst) {
+        const int n_rows = slice_rows(dst);
+        if (dst == static_cast<int>(rank) || n_rows == 0) continue;
+        ptx::bulk_copy_to_peer(ptx::map_shared_rank(slot_local, dst),
+                               red + dst * rows_per * RED_PITCH,
+                               static_cast<uint32_t>(n_rows * RED_PITCH * 4),
+                               ptx::map_shared_rank(bar_local, dst));
+      }
+      ptx::bulk_commit_group();
+    }
+    if (warp >= 4) {
+      const int ep_tid = threadIdx.x - 128;
+      bool ok = true;
+      if (lane == 0) ok = ptx::mbar_wait(recv_bar, 0, ctl, kDevTimeoutEpilogue);
+      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+      const int r0 = rank * rows_per;
+      constexpr int C8 = BLOCK_N / 8;
+      const int items = ok ? slice_rows(rank) * C8 : 0;
+      const int n0 = ti.n_blk * BLOCK_N;
+      for (int item = ep_tid; item < items; item += 128) {
+        const int lr = item / C8;  // row within the slice
+        const int c = 8 * (item % C8);
+        if (n0 + c >= p.N) continue;
+        float4 lo = make_float4(0, 0, 0, 0), hi = make_float4(0, 0, 0, 0);
+        for (int src = 0; src < S; ++src) {  // fixed order: deterministic
+          const float* part = (src == static_cast<int>(rank))
+                                  ? red + (r0 + lr) * RED_PITCH + c
+                                  : recv + (src * rows_per + lr) * RED_PITCH + c;
+          const float4 x = *reinterpret_cast<const float4*>(part);
+          const float4 y = *reinterpret_cast<const float4*>(part + 4);
+          lo.x += x.x; lo.y += x.y; lo.z += x.z; lo.w += x.w;
+          hi.x += y.x; hi.y += y.y; hi.z += y.z; hi.w += y.w;
+        }
+        uint4 v;
+        v.x = pack_bf16x2(lo.x, lo.y);
+        v.y = pack_bf16x2(lo.z, lo.w);
+        v.z = pack_bf16x2(hi.x, hi.y);
+        v.w = pack_bf16x2(hi.z, hi.w);
+        const size_t grow = (size_t)ti.m_blk * kBlockM + r0 + lr;
+        *reinterpret_cast<uint4*>(p.d + grow * p.N + n0 + c) = v;
+      }
+    }
+    if (threadIdx.x == 0) ptx::bulk_wait_group_read0();  // outgoing copies done reading
+    __syncwarp();
+    ptx::cluster_sync();  // no CTA leaves while a copy into it may still land
+  }
+
   ptx::tc_fence_before_sync();
   __syncthreads();
   if (warp == 1) {

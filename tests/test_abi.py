@@ -87,19 +87,26 @@ def test_timeout_setter(dg):
 
 # ------------------------------------------------------------- the picker --
 
-def test_decode_shapes_split_k_to_one_wave(dg):
-    for (m, n, k) in [(64, 2112, 7168), (128, 2112, 7168), (64, 7168, 2048)]:
+def test_decode_shapes_run_in_one_wave_of_deep_stages(dg):
+    """Decode-shaped dense problems use a decode variant (several K blocks per
+    stage) and exactly one wave of CTAs; split-K tiles are whole clusters."""
+    for (m, n, k) in [(64, 2112, 7168), (128, 2112, 7168), (64, 7168, 2048), (128, 7168, 2048),
+                      (64, 32768, 512), (128, 32768, 512), (64, 512, 1024)]:
         c = dg.query_config(0, m, n, k, num_sms=148)
         n_tiles = -(-n // c["block_n"])
-        assert c["split_k"] >= 2
-        assert n_tiles * c["split_k"] <= 148
-        assert c["grid"] == n_tiles * c["split_k"]
-        assert (k // 128) // c["split_k"] >= 2
+        assert c["kps"] >= 2, (m, n, k, c)
+        assert c["grid"] == n_tiles * c["split_k"] <= 148, (m, n, k, c)
+        kb = k // 128
+        per = -(-kb // c["split_k"])
+        assert (c["split_k"] - 1) * per < kb            # no empty K slice
+        assert c["smem_bytes"] <= 232448 and c["tmem_cols"] <= 512
 
 
-def test_wide_decode_needs_no_split(dg):
-    c = dg.query_config(0, 64, 32768, 512, num_sms=148)
-    assert c["split_k"] == 1 and c["grid"] == 148
+def test_decode_split_is_a_portable_cluster(dg):
+    for n in (512, 2112, 4096, 7168):
+        for k in (512, 1024, 2048, 7168, 16384):
+            c = dg.query_config(0, 64, n, k, num_sms=148)
+            assert 1 <= c["split_k"] <= 8
 
 
 def test_prefill_is_persistent(dg):
