@@ -7,6 +7,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <array>
 #include <mutex>
 #include <utility>
 
@@ -93,8 +94,9 @@ int a_box_rows(int kind, int rows) {
   return ((rows + 15) / 16) * 16;
 }
 
-// DG_FORCE_CONFIG="<block_n>:<split_k>[:<kps>:<a_rows>]" overrides the picker
-// (tuning sweeps); without kps/a_rows a general (one K block per stage) variant.
+// DG_FORCE_CONFIG="<block_n>:<split_k>[:<kps>:<a_rows>[:<small>]]" overrides
+// the picker (tuning sweeps); without kps/a_rows a general (one K block per
+// stage) variant.
 // Ignored unless the variant exists and, for split_k > 1, the problem is a
 // dense one with a single 128-row block.
 void forced_config(int kind, int rows, int N, int K, int G, int sms, PickedConfig* pc) {
@@ -102,13 +104,14 @@ void forced_config(int kind, int rows, int N, int K, int G, int sms, PickedConfi
   if (!e || !e[0]) return;
   int bn = 0, sk = 1;
   if (std::sscanf(e, "%d:%d", &bn, &sk) < 1) return;
-  int kps = 0, ar = 0;
-  std::sscanf(e, "%*d:%*d:%d:%d", &kps, &ar);
+  int kps = 0, ar = 0, sm = -1;
+  std::sscanf(e, "%*d:%*d:%d:%d:%d", &kps, &ar, &sm);
   int v = -1;
   for (int i = 0; i < kNumVariants; ++i) {
     const Variant& x = kVariants[i];
     if (x.block_n != bn) continue;
     if (kps ? (x.kps != kps || (ar && x.a_rows != ar)) : x.decode) continue;
+    if (sm >= 0 && x.small != (sm != 0)) continue;
     if (x.decode && kind != kDense) continue;
     if (a_box_rows(kind, rows) > x.a_rows) continue;
     v = i;
@@ -162,19 +165,39 @@ dg_status make_map(CUtensorMap* map, const void* base, uint64_t K, uint64_t rows
   return r == CUDA_SUCCESS ? DG_OK : DG_ERR_CUDA;
 }
 
+// 2-D tensor map over the BF16 output D [rows][N] with a box of 32 rows x
+// 64 columns and the 128-byte swizzle (the epilogue's staging layout).
+dg_status make_d_map(CUtensorMap* map, void* base, uint64_t N, uint64_t rows) {
+  cuuint64_t dims[2] = {N, rows};
+  cuuint64_t strides[1] = {N * 2};
+  cuuint32_t box[2] = {64, 32};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? DG_OK : DG_ERR_CUDA;
+}
+
 template <int V>
 using ShapeOf = KernelShape<kVariants[V].block_n, kVariants[V].stages, kVariants[V].num_acc,
-                            kVariants[V].kps, kVariants[V].a_rows>;
+                            kVariants[V].kps, kVariants[V].a_rows, kVariants[V].small>;
 
 // Kernels are instantiated only for the (form, variant) pairs that exist:
 // the decode variants serve the dense form only.
+// Per-variant shared-memory bytes (what = 0) or TMEM columns (what = 1).
+template <int what, int... V>
+constexpr std::array<int, sizeof...(V)> variant_table(std::integer_sequence<int, V...>) {
+  return {(what == 0 ? ShapeOf<V>::kSmemBytes : ShapeOf<V>::kTmemCols)...};
+}
+
 template <int KIND, int V>
 constexpr bool kBuilt = KIND == kDense || !kVariants[V].decode;
 
 template <int KIND, int V>
 auto kernel_of() {
   constexpr Variant var = kVariants[V];
-  return fp8_gemm_kernel<KIND, var.block_n, var.stages, var.num_acc, var.kps, var.a_rows>;
+  return fp8_gemm_kernel<KIND, var.block_n, var.stages, var.num_acc, var.kps, var.a_rows,
+                         var.small>;
 }
 
 template <int KIND, int V>
@@ -239,7 +262,8 @@ dg_status ensure_cluster_limits(DeviceState& st) {
 
 template <int KIND, int V>
 dg_status launch_variant(DeviceState& st, const CUtensorMap& ta, const CUtensorMap& tb,
-                         const GemmArgs& args, int grid, cudaStream_t stream) {
+                         const CUtensorMap& td, const GemmArgs& args, int grid,
+                         cudaStream_t stream) {
   if constexpr (!kBuilt<KIND, V>) {
     return DG_ERR_UNSUPPORTED;
   } else {
@@ -263,23 +287,24 @@ dg_status launch_variant(DeviceState& st, const CUtensorMap& ta, const CUtensorM
     }
     cfg.attrs = attr;
     cfg.numAttrs = n_attr;
-    return from_cuda(cudaLaunchKernelEx(&cfg, kernel_of<KIND, V>(), ta, tb, args));
+    return from_cuda(cudaLaunchKernelEx(&cfg, kernel_of<KIND, V>(), ta, tb, td, args));
   }
 }
 
 template <int KIND, int... V>
 dg_status launch_dispatch(DeviceState& st, int variant, const CUtensorMap& ta,
-                          const CUtensorMap& tb, const GemmArgs& args, int grid,
-                          cudaStream_t stream, std::integer_sequence<int, V...>) {
+                          const CUtensorMap& tb, const CUtensorMap& td, const GemmArgs& args,
+                          int grid, cudaStream_t stream, std::integer_sequence<int, V...>) {
   dg_status s = DG_ERR_UNSUPPORTED;
-  ((variant == V ? (s = launch_variant<KIND, V>(st, ta, tb, args, grid, stream), 0) : 0), ...);
+  ((variant == V ? (s = launch_variant<KIND, V>(st, ta, tb, td, args, grid, stream), 0) : 0),
+   ...);
   return s;
 }
 
 template <int KIND>
 dg_status launch(DeviceState& st, int variant, const CUtensorMap& ta, const CUtensorMap& tb,
-                 const GemmArgs& args, int grid, cudaStream_t stream) {
-  return launch_dispatch<KIND>(st, variant, ta, tb, args, grid, stream,
+                 const CUtensorMap& td, const GemmArgs& args, int grid, cudaStream_t stream) {
+  return launch_dispatch<KIND>(st, variant, ta, tb, td, args, grid, stream,
                                std::make_integer_sequence<int, kNumVariants>{});
 }
 
@@ -338,6 +363,9 @@ dg_status run(int kind, const void* a, const float* sfa, const void* b, const fl
   args.a_box_rows = a_box_rows(kind, rows);
   if (args.a_box_rows > var.a_rows) return DG_ERR_UNSUPPORTED;
   args.prefetch = prefetch_enabled();
+  // a small variant runs one tile per CTA (its epilogue reuses the ring)
+  if (var.small && (kind != kDense || pc.grid != args.num_m_blocks * args.num_n_blocks * pc.split_k))
+    return DG_ERR_UNSUPPORTED;
   // split-K runs one tile per CTA, one cluster per output tile
   if (pc.split_k > 1 &&
       (kind != kDense || pc.grid != args.num_m_blocks * args.num_n_blocks * pc.split_k ||
@@ -350,6 +378,9 @@ dg_status run(int kind, const void* a, const float* sfa, const void* b, const fl
   if (s != DG_OK) return s;
   s = make_map(&tb, b, K, N, b_groups, var.block_n, var.kps);
   if (s != DG_OK) return s;
+  CUtensorMap td;
+  s = make_d_map(&td, d, N, static_cast<uint64_t>(a_rows));
+  if (s != DG_OK) return s;
 
   if (print_configs())
     std::fprintf(stderr,
@@ -359,9 +390,10 @@ dg_status run(int kind, const void* a, const float* sfa, const void* b, const fl
                  pc.split_k, pc.grid);
 
   switch (kind) {
-    case kDense: return launch<kDense>(*st, pc.variant, ta, tb, args, pc.grid, stream);
-    case kContiguous: return launch<kContiguous>(*st, pc.variant, ta, tb, args, pc.grid, stream);
-    default: return launch<kMasked>(*st, pc.variant, ta, tb, args, pc.grid, stream);
+    case kDense: return launch<kDense>(*st, pc.variant, ta, tb, td, args, pc.grid, stream);
+    case kContiguous:
+      return launch<kContiguous>(*st, pc.variant, ta, tb, td, args, pc.grid, stream);
+    default: return launch<kMasked>(*st, pc.variant, ta, tb, td, args, pc.grid, stream);
   }
 }
 
@@ -458,15 +490,8 @@ dg_status dg_query_config(int kind, int rows, int N, int K, int G, int expected_
   out->num_acc = v.num_acc;
   out->split_k = pc.split_k;
   out->grid = pc.grid;
-  constexpr int smem[] = {ShapeOf<0>::kSmemBytes, ShapeOf<1>::kSmemBytes, ShapeOf<2>::kSmemBytes,
-                          ShapeOf<3>::kSmemBytes, ShapeOf<4>::kSmemBytes, ShapeOf<5>::kSmemBytes,
-                          ShapeOf<6>::kSmemBytes, ShapeOf<7>::kSmemBytes, ShapeOf<8>::kSmemBytes,
-                          ShapeOf<9>::kSmemBytes};
-  constexpr int tmem[] = {ShapeOf<0>::kTmemCols, ShapeOf<1>::kTmemCols, ShapeOf<2>::kTmemCols,
-                          ShapeOf<3>::kTmemCols, ShapeOf<4>::kTmemCols, ShapeOf<5>::kTmemCols,
-                          ShapeOf<6>::kTmemCols, ShapeOf<7>::kTmemCols, ShapeOf<8>::kTmemCols,
-                          ShapeOf<9>::kTmemCols};
-  static_assert(sizeof(smem) / sizeof(smem[0]) == kNumVariants, "one entry per variant");
+  constexpr auto smem = variant_table<0>(std::make_integer_sequence<int, kNumVariants>{});
+  constexpr auto tmem = variant_table<1>(std::make_integer_sequence<int, kNumVariants>{});
   out->smem_bytes = smem[pc.variant];
   out->tmem_cols = tmem[pc.variant];
   out->kps = v.kps;

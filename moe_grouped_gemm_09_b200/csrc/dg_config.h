@@ -17,22 +17,29 @@ struct Variant {
   int kps;      // 128-wide K blocks per ring stage (one TMA box of each operand)
   int a_rows;   // rows of A a stage holds (64: dense A of at most 64 rows)
   bool decode;  // built for dense problems of at most one 128-row block
+  bool small;   // two CTAs fit per SM; one tile per CTA
 };
 
 // The compiled variants: general ones first (every form), then the
 // decode-shaped dense ones, whose stages are several K blocks deep so that
-// each TMA box moves 32-64 KB.
+// each TMA box moves 32-64 KB, then the small decode ones (at most ~100 KB of
+// shared memory and 256 TMEM columns, so that the next kernel's CTAs can be
+// resident and warm L2 with their weights while this kernel drains).
 constexpr Variant kVariants[] = {
-    {256, 4, 1, 1, 128, false},
-    {128, 6, 2, 1, 128, false},
-    {64, 8, 2, 1, 128, false},
-    {32, 9, 2, 1, 128, false},
-    {128, 2, 1, 4, 64, true},
-    {64, 3, 2, 4, 64, true},
-    {256, 2, 1, 2, 64, true},
-    {128, 3, 1, 2, 128, true},
-    {64, 4, 2, 2, 128, true},
-    {256, 2, 1, 2, 128, true},
+    {256, 4, 1, 1, 128, false, false},
+    {128, 6, 2, 1, 128, false, false},
+    {64, 8, 2, 1, 128, false, false},
+    {32, 9, 2, 1, 128, false, false},
+    {128, 2, 1, 4, 64, true, false},
+    {64, 3, 2, 4, 64, true, false},
+    {256, 2, 1, 2, 64, true, false},
+    {128, 3, 1, 2, 128, true, false},
+    {64, 4, 2, 2, 128, true, false},
+    {256, 2, 1, 2, 128, true, false},
+    {128, 2, 1, 2, 64, true, true},
+    {64, 3, 1, 2, 64, true, true},
+    {128, 3, 1, 1, 128, true, true},
+    {64, 2, 1, 2, 128, true, true},
 };
 constexpr int kNumVariants = sizeof(kVariants) / sizeof(kVariants[0]);
 constexpr int kMaxSplitK = 8;  // portable cluster size
@@ -69,36 +76,43 @@ inline bool split_fits(const Variant& var, int rows, int split) {
 
 // Decode-shaped dense problems (at most one 128-row block): HBM-bound.  Pick
 // the variant and K split (one cluster of `split` CTAs per output tile, all in
-// one wave) that minimise an estimate of the time: the larger of the whole
-// kernel's HBM time and the busiest CTA's streaming time, plus the pipeline
-// ramp and the reduction.  A CTA's streaming rate grows with the TMA box size
-// (about 37 GB/s per SM for 16 KB boxes, up to about 120 GB/s for 64 KB boxes,
-// measured on B200).  Returns false if no one-wave configuration exists.
+// one wave) that minimise an estimate of the time:
+//   fixed cost + max(HBM time of B, busiest CTA's streaming time) + split tail
+// where a CTA streams its B slice plus (at a discount: it is read from L2) its
+// A slice at a rate that grows with the TMA box size.  The constants were
+// fitted to a sweep of every (variant, split) on the six decode-shaped
+// workloads on B200 (the fit picks within 4% of the best measured
+// configuration for each).  Returns false if no one-wave configuration exists.
 inline bool pick_decode(int rows, int N, int K, int num_sms, const ClusterLimits* lim,
                         PickedConfig* out) {
   const int KB = K / 128;
-  const double hbm_bytes_per_us = 5.8e6;  // whole GPU, streaming with large boxes
+  constexpr double kHbmBytesPerUs = 4.5e6;  // effective, whole GPU
+  constexpr double kRate16KB = 50.0;        // KB per microsecond per CTA, 16 KB boxes
+  constexpr double kRateCap = 90.0;         // KB per microsecond per CTA, large boxes
+  constexpr double kAWeight = 0.35;         // A slices come from L2
+  constexpr double kFixedUs = 6.0;
+  constexpr double kSplitUs = 3.0;          // cluster barriers, pushes, reduction
   double best = 1e30;
   bool found = false;
   for (int v = 0; v < kNumVariants; ++v) {
     const Variant& var = kVariants[v];
-    if (!var.decode || rows > var.a_rows) continue;
+    if (!var.decode || var.small || rows > var.a_rows) continue;
     const int bn = var.block_n;
     const int nt = ceil_div(N, bn);
     const double box_kb = var.kps * bn * 128 / 1024.0;
-    double r_cta = 37.0 * box_kb / 16.0;  // GB/s = KB per microsecond
-    if (r_cta > 120.0) r_cta = 120.0;
+    double r_cta = kRate16KB * box_kb / 16.0;
+    if (r_cta > kRateCap) r_cta = kRateCap;
     for (int s = 1; s <= kMaxSplitK && s <= KB; ++s) {
       if (nt * s > num_sms) break;
       const int per = ceil_div(KB, s);
       if ((s - 1) * per >= KB) continue;          // an empty slice
       if (s > 1 && cluster_limit(lim, v, s, num_sms) < nt) continue;
       if (s > 1 && !split_fits(var, rows, s)) continue;
-      const double b_cta = static_cast<double>(bn) * per * 128 / 1024.0;     // KB
-      const double a_cta = static_cast<double>(rows) * per * 128 / 1024.0;   // KB
-      const double t_cta = (b_cta + a_cta) / r_cta;                         // us
-      const double t_hbm = static_cast<double>(N) * K / hbm_bytes_per_us;  // us
-      const double t = (t_cta > t_hbm ? t_cta : t_hbm) + 1.5 + (s > 1 ? 0.8 : 0.0);
+      const double b_cta = static_cast<double>(bn) * per * 128 / 1024.0;    // KB
+      const double a_cta = static_cast<double>(rows) * per * 128 / 1024.0;  // KB
+      const double t_cta = (b_cta + kAWeight * a_cta) / r_cta;             // us
+      const double t_hbm = static_cast<double>(N) * K / kHbmBytesPerUs;     // us
+      const double t = kFixedUs + (t_cta > t_hbm ? t_cta : t_hbm) + (s > 1 ? kSplitUs : 0.0);
       if (t < best - 1e-9) {
         best = t;
         found = true;
@@ -118,9 +132,12 @@ inline PickedConfig pick_config(int kind, int rows, int N, int K, int G, int exp
   PickedConfig best{1, 1, 1, 1};
   if (kind == 0 && rows <= 128 && pick_decode(rows, N, K, num_sms, lim, &best)) return best;
 
-  // Everything else: persistent CTAs, no split.  Choose the tile width that
-  // minimises (waves x tile width), a proxy for the busiest SM's time,
-  // preferring wider tiles on ties.
+  // Everything else: persistent CTAs, no split.  Tile time is set by the
+  // bytes the SM must pull through TMA per K block (A 16 KB + B BLOCK_N x
+  // 128 B; measured on B200 to bound these compute-bound tiles), so choose
+  // the variant minimising waves x bytes per K block.  For the dense form a
+  // variant with two K blocks per stage (bigger boxes) also competes; it pays
+  // off for short K.
   int eff_rows = rows;
   int groups = 1;
   if (kind == 2) {
@@ -130,13 +147,16 @@ inline PickedConfig pick_config(int kind, int rows, int N, int K, int G, int exp
   const int m_blocks = groups * ceil_div(eff_rows > 0 ? eff_rows : 1, 128);
   double best_cost = 1e30;
   for (int v = 0; v < kNumVariants; ++v) {
-    if (kVariants[v].decode) continue;
-    const int bn = kVariants[v].block_n;
+    const Variant& var = kVariants[v];
+    if (var.small || var.a_rows != 128) continue;
+    if (var.decode && (kind != 0 || var.kps != 2 || var.block_n != 256)) continue;
+    const int bn = var.block_n;
     if (bn > 128 && N <= 128) continue;
     const int n_tiles = ceil_div(N, bn);
     const long long tiles = static_cast<long long>(m_blocks) * n_tiles;
     const int waves = ceil_div(tiles, num_sms);
-    const double cost = waves * (bn + 32.0);
+    double cost = waves * (16.0 + bn / 8.0);
+    if (var.kps == 2) cost *= (K <= 2048 ? 0.85 : 1.02);
     if (cost < best_cost - 1e-9) {
       best_cost = cost;
       best.variant = v;

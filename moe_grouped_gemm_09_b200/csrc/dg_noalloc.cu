@@ -46,12 +46,13 @@ NaEncodeFn g_na_encode = nullptr;
 
 template <int V>
 using NaShape = KernelShape<kVariants[V].block_n, kVariants[V].stages, kVariants[V].num_acc,
-                            kVariants[V].kps, kVariants[V].a_rows>;
+                            kVariants[V].kps, kVariants[V].a_rows, kVariants[V].small>;
 
 template <int V>
 auto na_kernel() {
   constexpr Variant var = kVariants[V];
-  return fp8_gemm_kernel<kDense, var.block_n, var.stages, var.num_acc, var.kps, var.a_rows>;
+  return fp8_gemm_kernel<kDense, var.block_n, var.stages, var.num_acc, var.kps, var.a_rows,
+                         var.small>;
 }
 
 template <int V>
@@ -152,9 +153,20 @@ dg_status na_map(CUtensorMap* map, const void* base, uint64_t K, uint64_t rows, 
   return r == CUDA_SUCCESS ? DG_OK : DG_ERR_CUDA;
 }
 
+dg_status na_d_map(CUtensorMap* map, void* base, uint64_t N, uint64_t rows) {
+  cuuint64_t dims[2] = {N, rows};
+  cuuint64_t strides[1] = {N * 2};
+  cuuint32_t box[2] = {64, 32};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_na_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? DG_OK : DG_ERR_CUDA;
+}
+
 template <int V>
 dg_status na_launch(NaDevice& st, const CUtensorMap& ta, const CUtensorMap& tb,
-                    const GemmArgs& args, int grid, cudaStream_t stream) {
+                    const CUtensorMap& td, const GemmArgs& args, int grid, cudaStream_t stream) {
   dg_status s = na_smem_attr<V>(st);
   if (s != DG_OK) return s;
   cudaLaunchConfig_t cfg = {};
@@ -171,16 +183,16 @@ dg_status na_launch(NaDevice& st, const CUtensorMap& ta, const CUtensorMap& tb,
     cfg.attrs = attr;
     cfg.numAttrs = 1;
   }
-  return cudaLaunchKernelEx(&cfg, na_kernel<V>(), ta, tb, args) == cudaSuccess ? DG_OK
-                                                                               : DG_ERR_CUDA;
+  return cudaLaunchKernelEx(&cfg, na_kernel<V>(), ta, tb, td, args) == cudaSuccess ? DG_OK
+                                                                                   : DG_ERR_CUDA;
 }
 
 template <int... V>
 dg_status na_dispatch(NaDevice& st, int variant, const CUtensorMap& ta, const CUtensorMap& tb,
-                      const GemmArgs& args, int grid, cudaStream_t stream,
+                      const CUtensorMap& td, const GemmArgs& args, int grid, cudaStream_t stream,
                       std::integer_sequence<int, V...>) {
   dg_status s = DG_ERR_UNSUPPORTED;
-  ((variant == V ? (s = na_launch<V>(st, ta, tb, args, grid, stream), 0) : 0), ...);
+  ((variant == V ? (s = na_launch<V>(st, ta, tb, td, args, grid, stream), 0) : 0), ...);
   return s;
 }
 
@@ -227,6 +239,8 @@ extern "C" dg_status dg_fp8_gemm_nt_noalloc(const void* a, const float* sfa, con
   args.a_box_rows = M >= kBlockM ? kBlockM : ((M + 15) / 16) * 16;
   args.prefetch = 1;
   if (args.a_box_rows > var.a_rows) return DG_ERR_UNSUPPORTED;
+  if (var.small && pc.grid != args.num_m_blocks * args.num_n_blocks * pc.split_k)
+    return DG_ERR_UNSUPPORTED;
   if (pc.split_k > 1 && (pc.grid != args.num_m_blocks * args.num_n_blocks * pc.split_k ||
                          M > kBlockM || !split_fits(var, M, pc.split_k)))
     return DG_ERR_UNSUPPORTED;
@@ -236,6 +250,9 @@ extern "C" dg_status dg_fp8_gemm_nt_noalloc(const void* a, const float* sfa, con
   if (s != DG_OK) return s;
   s = na_map(&tb, b, K, N, var.block_n, var.kps);
   if (s != DG_OK) return s;
-  return na_dispatch(*st, pc.variant, ta, tb, args, pc.grid, stream,
+  CUtensorMap td;
+  s = na_d_map(&td, d, N, M);
+  if (s != DG_OK) return s;
+  return na_dispatch(*st, pc.variant, ta, tb, td, args, pc.grid, stream,
                      std::make_integer_sequence<int, kNumVariants>{});
 }

@@ -102,7 +102,11 @@ __host__ __device__ constexpr int pow2_ceil(int x) {
 //            and one of B, each KPS K blocks deep (bigger boxes stream faster)
 //   A_ROWS   rows of A a stage holds room for (64 for a dense A of at most 64
 //            rows, else 128)
-template <int BLOCK_N, int STAGES, int NUM_ACC, int KPS = 1, int A_ROWS = 128>
+//   SMALL    a decode variant small enough (shared memory and TMEM) for two
+//            CTAs per SM, so that the next kernel's CTAs can start (and warm
+//            L2) while this kernel drains; it runs one tile per CTA and
+//            stages its epilogue in the then idle operand ring
+template <int BLOCK_N, int STAGES, int NUM_ACC, int KPS = 1, int A_ROWS = 128, bool SMALL = false>
 struct KernelShape {
   static constexpr int kABytes = KPS * A_ROWS * kBlockK;  // one E4M3 byte per element
   static constexpr int kBBytes = KPS * BLOCK_N * kBlockK;
@@ -112,19 +116,25 @@ struct KernelShape {
   static constexpr int kAccCols = NUM_ACC * BLOCK_N;
   static constexpr int kTmemCols = pow2_ceil(kAccCols + STAGES * kSfCols);
   static constexpr int kBarBytes = 8 * (2 * STAGES + 2 * NUM_ACC + 2);
-  // epilogue: each of the 4 epilogue warps transposes 32 rows x kEpiCols
-  // BF16 columns through shared memory so that its global stores are whole
-  // 128-byte row segments
+  // epilogue: each of the 4 epilogue warps stages 32 rows x kEpiCols BF16
+  // columns in shared memory (16-byte chunks XOR-swizzled by row, the layout
+  // of the 128-byte TMA swizzle), then stores them with one TMA box or with
+  // whole row segments
   static constexpr int kEpiCols = BLOCK_N >= 64 ? 64 : 32;
-  static constexpr int kEpiPitch = kEpiCols * 2 + 16;  // bytes per staged row (bank spread)
-  static constexpr int kEpiBytes = 4 * 32 * kEpiPitch;
-  static constexpr int kMiscBytes = 16 + 4 * (kMaxMaskedGroups + 1);  // tmem slot, flags, prefix
+  static constexpr int kEpiPitch = kEpiCols * 2;        // bytes per staged row
+  static constexpr int kEpiBytes = SMALL ? 0 : 4 * 32 * kEpiPitch;
+  // tmem slot, flags, and (grouped forms) the masked prefix
+  static constexpr int kMiscBytes = 16 + (SMALL ? 0 : 4 * (kMaxMaskedGroups + 1));
   // A short A tile is read by the 128-row MMA past its end (rows that only
   // feed never-stored accumulator rows); the B ring follows the A ring, so
   // that read stays inside this CTA's shared memory.
   static constexpr int kSmemBytes = 1024 /* alignment slack */ + STAGES * (kABytes + kBBytes) +
                                     STAGES * kSfBytes + kEpiBytes + kBarBytes + kMiscBytes;
   static_assert(kSmemBytes <= 232448, "shared memory budget (227 KB) exceeded");
+  static_assert(!SMALL || (kSmemBytes <= 115712 && kTmemCols <= 256),
+                "a small variant must leave room for a second CTA on its SM");
+  static_assert(STAGES * (kABytes + kBBytes) >= 4 * BLOCK_N * 64,
+                "a single-tile CTA stages its whole output tile in the ring");
   static_assert(kTmemCols <= 512, "TMEM budget exceeded");
   static_assert(BLOCK_N % 32 == 0 && BLOCK_N >= 32 && BLOCK_N <= 256, "BLOCK_N");
   static_assert(KPS >= 1 && KPS <= 4, "up to four K blocks share one scale-factor word");
@@ -266,11 +276,12 @@ struct StageWalker {
   }
 };
 
-template <int KIND, int BLOCK_N, int STAGES, int NUM_ACC, int KPS, int A_ROWS>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int KIND, int BLOCK_N, int STAGES, int NUM_ACC, int KPS, int A_ROWS, bool SMALL>
+__global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
-                    const __grid_constant__ CUtensorMap tmap_b, const GemmArgs p) {
-  using Shape = KernelShape<BLOCK_N, STAGES, NUM_ACC, KPS, A_ROWS>;
+                    const __grid_constant__ CUtensorMap tmap_b,
+                    const __grid_constant__ CUtensorMap tmap_d, const GemmArgs p) {
+  using Shape = KernelShape<BLOCK_N, STAGES, NUM_ACC, KPS, A_ROWS, SMALL>;
   constexpr int A_BYTES = Shape::kABytes;
   constexpr int B_BYTES = Shape::kBBytes;
   constexpr int SF_BYTES = Shape::kSfBytes;
@@ -284,7 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // picks a split for which (2 * valid rows + split) rows fit.
   static_assert(kBlockM * RED_PITCH * 4 <= STAGES * (A_BYTES + B_BYTES),
                 "split-K partial must fit in the operand ring");
-  static_assert(KPS == 1 || KIND == kDense, "multi-K-block stages are built for the dense form");
+  static_assert((KPS == 1 && !SMALL) || KIND == kDense, "decode variants serve the dense form");
 
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment for the 128-byte-swizzled operand tiles
@@ -292,9 +303,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
   uint8_t* sA = smem;
   uint8_t* sB = sA + STAGES * A_BYTES;
-  uint8_t* sSF = sB + STAGES * B_BYTES;
-  uint8_t* sEpi = sSF + STAGES * SF_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sEpi + Shape::kEpiBytes);
+  // epilogue staging tiles (1024-aligned, swizzled): their own region, or,
+  // when every CTA has a single tile (always for a small variant), the operand
+  // ring, idle once that tile's MMAs are done, with one tile per warp and chunk
+  const int n_tiles_total = (KIND == kMasked ? -1 : p.num_m_blocks * p.num_n_blocks * p.split_k);
+  const bool one_tile = SMALL || (n_tiles_total >= 0 && n_tiles_total <= static_cast<int>(gridDim.x));
+  uint8_t* sEpi = one_tile ? sA : sB + STAGES * B_BYTES;
+  uint8_t* sSF = sB + STAGES * B_BYTES + Shape::kEpiBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sSF + STAGES * SF_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;
   uint64_t* acc_empty = acc_full + NUM_ACC;
@@ -302,7 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* recv_bar = drain + 1;  // split-K: partial slices pushed by the other CTAs
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(recv_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int* s_prefix = const_cast<int*>(abort_flag + 3);
+  int* s_prefix = const_cast<int*>(abort_flag + 3);  // masked form only
   // split-K: this CTA's FP32 partial, parked over the (by then idle) operand ring
   float* red = reinterpret_cast<float*>(sA);
 
@@ -325,6 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::fence_mbar_init();
     ptx::prefetch_tensormap(&tmap_a);
     ptx::prefetch_tensormap(&tmap_b);
+    ptx::prefetch_tensormap(&tmap_d);
   }
   if (warp == 1) {
     ptx::tmem_alloc(tmem_slot, TMEM_COLS);
@@ -334,11 +351,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       blockIdx.x < p.num_m_blocks * p.num_n_blocks * p.split_k) {
     // Warm L2 with this CTA's first tile while the previous kernel finishes
     // (the tile order of the dense form does not depend on device data).
+    // (A small variant prefetches the whole K range of B, the weights it
+    // streams; the others the first stages of both operands.)
     const Tile ti = get_tile<kDense>(blockIdx.x, p, nullptr, lane);
-    const int kb_end = min(ti.kb_end, ti.kb_begin + STAGES * KPS);
+    const int kb_end = SMALL ? ti.kb_end : min(ti.kb_end, ti.kb_begin + STAGES * KPS);
     for (int kb = ti.kb_begin; kb < kb_end; kb += KPS) {
       ptx::tma_prefetch_l2_4d(&tmap_b, 0, ti.n_blk * BLOCK_N, kb, 0);
-      ptx::tma_prefetch_l2_4d(&tmap_a, 0, ti.m_blk * kBlockM, kb, 0);
+      if (!SMALL) ptx::tma_prefetch_l2_4d(&tmap_a, 0, ti.m_blk * kBlockM, kb, 0);
     }
   }
   // Everything above reads no input; from here on the inputs may be the
@@ -598,7 +617,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       // masked group) skips the TMEM reads; it still releases the buffer.
       if (__any_sync(0xFFFFFFFFu, valid)) {
         constexpr int CH = Shape::kEpiCols;  // columns per TMEM wait
-        uint8_t* stage = sEpi + q * 32 * Shape::kEpiPitch;
+        constexpr int NCH = BLOCK_N / CH;    // chunks per tile
+        // one staging tile per warp; a small variant has one per warp and chunk
+        uint8_t* stage0 = sEpi + q * (one_tile ? NCH : 1) * 32 * Shape::kEpiPitch;
+        // TMA store of whole 32-row boxes: the dense form always (rows past M
+        // are clipped); the grouped forms only when all 32 rows are written.
+        const bool tma_store = CH == 64 && !split &&
+                               (KIND == kDense || __all_sync(0xFFFFFFFFu, valid));
 #pragma unroll 1
         for (int c0 = 0; c0 < BLOCK_N; c0 += CH) {
           uint32_t r[CH];
@@ -606,6 +631,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (CH == 64)
             ptx::tc_ld_32x32b_x32(t_row + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[CH - 32]));
           ptx::tc_wait_ld();
+          uint8_t* stage = one_tile ? stage0 + (c0 / CH) * 32 * Shape::kEpiPitch : stage0;
           if (split) {
             // park the FP32 partial; the cluster reduces it below
             if (valid) {
@@ -617,31 +643,45 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             continue;
           }
-          // BF16 row of this lane into the warp's staging tile ...
+          // BF16 row of this lane into the warp's staging tile (chunk j of row
+          // `lane` at chunk position j ^ (lane % 8): the 128-byte swizzle) ...
+          constexpr int CPR = CH / 8;  // 16-byte chunks per row
 #pragma unroll
-          for (int j = 0; j < CH / 8; ++j) {
+          for (int j = 0; j < CPR; ++j) {
             uint4 v;
             v.x = pack_bf16x2(__uint_as_float(r[8 * j + 0]), __uint_as_float(r[8 * j + 1]));
             v.y = pack_bf16x2(__uint_as_float(r[8 * j + 2]), __uint_as_float(r[8 * j + 3]));
             v.z = pack_bf16x2(__uint_as_float(r[8 * j + 4]), __uint_as_float(r[8 * j + 5]));
             v.w = pack_bf16x2(__uint_as_float(r[8 * j + 6]), __uint_as_float(r[8 * j + 7]));
-            *reinterpret_cast<uint4*>(stage + lane * Shape::kEpiPitch + 16 * j) = v;
+            *reinterpret_cast<uint4*>(stage + lane * Shape::kEpiPitch + 16 * (j ^ (lane % CPR))) = v;
+          }
+          if (tma_store) {
+            // ... then one TMA box of 32 rows x 64 columns (rows past the
+            // tensor's end and columns past N are clipped by the TMA unit)
+            ptx::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              ptx::tma_store_2d(&tmap_d, stage, n0 + c0, static_cast<int>(grow - lane));
+              ptx::bulk_commit_group();
+              if (!one_tile) ptx::bulk_wait_group_read0();  // staging tile free again
+            }
+            __syncwarp();
+            continue;
           }
           __syncwarp();
-          // ... then whole row segments: a store instruction covers 32 / (CH / 8)
-          // rows, CH / 8 lanes per row, 16 bytes a lane.
-          constexpr int LPR = CH / 8;    // lanes per row
-          constexpr int RPI = 32 / LPR;  // rows per instruction
-          const int sub = lane % LPR;
+          // ... or whole row segments: a store instruction covers 32 / CPR
+          // rows, CPR lanes per row, 16 bytes a lane.
+          constexpr int RPI = 32 / CPR;  // rows per instruction
+          const int sub = lane % CPR;
 #pragma unroll
           for (int i = 0; i < 32 / RPI; ++i) {
-            const int rr = RPI * i + lane / LPR;  // row within the warp's 32
+            const int rr = RPI * i + lane / CPR;  // row within the warp's 32
             const bool row_ok = __shfl_sync(0xFFFFFFFFu, valid, rr);
             const int n = n0 + c0 + 8 * sub;
             if (row_ok && n < p.N) {
               const size_t g_row = grow - lane + rr;  // the rows of a warp are consecutive
-              *reinterpret_cast<uint4*>(p.d + g_row * p.N + n) =
-                  *reinterpret_cast<const uint4*>(stage + rr * Shape::kEpiPitch + 16 * sub);
+              *reinterpret_cast<uint4*>(p.d + g_row * p.N + n) = *reinterpret_cast<const uint4*>(
+                  stage + rr * Shape::kEpiPitch + 16 * (sub ^ (rr % CPR)));
             }
           }
           __syncwarp();
@@ -652,6 +692,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::mbar_arrive(&acc_empty[a]);
       ++acc_it;
     }
+    if (lane == 0) ptx::bulk_wait_group0();  // this warp's TMA stores have landed
   }
 
   if (split) {

@@ -183,6 +183,21 @@ __device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, const vo
       : "memory");
 }
 
+// 2-D tiled store of one box from shared memory to global memory (bulk group).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int c0,
+                                             int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(smem_addr(src)), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+// Wait until every bulk group of this thread has completed (writes done).
+__device__ __forceinline__ void bulk_wait_group0() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
 // Close the current group of bulk copies issued by this thread, and wait until
 // every group has finished reading its source.
 __device__ __forceinline__ void bulk_commit_group() {
