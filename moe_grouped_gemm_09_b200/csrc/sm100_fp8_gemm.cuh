@@ -133,7 +133,7 @@ struct KernelShape {
   static_assert(kSmemBytes <= 232448, "shared memory budget (227 KB) exceeded");
   static_assert(!SMALL || (kSmemBytes <= 115712 && kTmemCols <= 256),
                 "a small variant must leave room for a second CTA on its SM");
-  static_assert(STAGES * (kABytes + kBBytes) >= 4 * BLOCK_N * 64,
+  static_assert(STAGES * (kABytes + kBBytes) >= 8 * BLOCK_N * 64,
                 "a single-tile CTA stages its whole output tile in the ring");
   static_assert(kTmemCols <= 512, "TMEM budget exceeded");
   static_assert(BLOCK_N % 32 == 0 && BLOCK_N >= 32 && BLOCK_N <= 256, "BLOCK_N");
@@ -383,6 +383,111 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
   const int total = (KIND == kMasked ? s_prefix[p.G]
                                      : p.num_m_blocks * p.num_n_blocks) * p.split_k;
 
+  // Drains TMEM accumulator buffer `a` of tile `ti`, lane quarter q (rows
+  // 32q..32q+31), columns [c_begin, c_end): BF16 through the staging tiles
+  // at stage0 to D, or (split-K) FP32 into the parked partial.
+  constexpr int NCH_ALL = BLOCK_N / Shape::kEpiCols;
+  const CUtensorMap* dmap = &tmap_d;
+  auto drain_acc = [&](const Tile& ti, int a, int q, int c_begin, int c_end, uint8_t* stage0,
+                       bool report) {
+    // which output row this thread owns, and whether it may be written
+    const int row_local = 32 * q + lane;  // accumulator row = TMEM lane
+    const int m_in_group = ti.m_blk * kBlockM + row_local;
+    bool valid;
+    size_t grow;
+    if (KIND == kMasked) {
+      const int mm = min(max(__ldg(p.masked_m + ti.group), 0), p.rows);
+      valid = m_in_group < mm;
+      grow = (size_t)ti.group * p.rows + m_in_group;
+    } else {
+      valid = m_in_group < p.rows;
+      grow = m_in_group;
+      if (KIND == kContiguous && valid) {
+        const int e = __ldg(p.m_indices + m_in_group);
+        if (report && e >= 0 && e != ti.group) atomicCAS(p.error_word, 0, kDevMixedExperts);
+        valid = (e == ti.group);
+      }
+    }
+    const uint32_t t_row = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + a * BLOCK_N;
+    const int n0 = ti.n_blk * BLOCK_N;
+
+    // A warp whose 32 rows are all outside the output (a short dense A, a
+    // masked group) skips the TMEM reads; it still releases the buffer.
+    if (__any_sync(0xFFFFFFFFu, valid)) {
+      constexpr int CH = Shape::kEpiCols;  // columns per TMEM wait
+      // TMA store of whole 32-row boxes: the dense form always (rows past M
+      // are clipped); the grouped forms only when all 32 rows are written.
+      const bool tma_store = CH == 64 && !split &&
+                             (KIND == kDense || __all_sync(0xFFFFFFFFu, valid));
+#pragma unroll 1
+      for (int c0 = c_begin; c0 < c_end; c0 += CH) {
+        uint32_t r[CH];
+        ptx::tc_ld_32x32b_x32(t_row + c0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+        if (CH == 64)
+          ptx::tc_ld_32x32b_x32(t_row + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[CH - 32]));
+        ptx::tc_wait_ld();
+        uint8_t* stage = one_tile ? stage0 + ((c0 - c_begin) / CH) * 32 * Shape::kEpiPitch : stage0;
+        if (split) {
+          // park the FP32 partial; the cluster reduces it below
+          if (valid) {
+#pragma unroll
+            for (int j = 0; j < CH / 4; ++j)
+              *reinterpret_cast<float4*>(red + row_local * RED_PITCH + c0 + 4 * j) =
+                  make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                              __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+          }
+          continue;
+        }
+        // BF16 row of this lane into the warp's staging tile (chunk j of row
+        // `lane` at chunk position j ^ (lane % 8): the 128-byte swizzle) ...
+        constexpr int CPR = CH / 8;  // 16-byte chunks per row
+#pragma unroll
+        for (int j = 0; j < CPR; ++j) {
+          uint4 v;
+          v.x = pack_bf16x2(__uint_as_float(r[8 * j + 0]), __uint_as_float(r[8 * j + 1]));
+          v.y = pack_bf16x2(__uint_as_float(r[8 * j + 2]), __uint_as_float(r[8 * j + 3]));
+          v.z = pack_bf16x2(__uint_as_float(r[8 * j + 4]), __uint_as_float(r[8 * j + 5]));
+          v.w = pack_bf16x2(__uint_as_float(r[8 * j + 6]), __uint_as_float(r[8 * j + 7]));
+          *reinterpret_cast<uint4*>(stage + lane * Shape::kEpiPitch + 16 * (j ^ (lane % CPR))) = v;
+        }
+        if (tma_store) {
+          // ... then one TMA box of 32 rows x 64 columns (rows past the
+          // tensor's end and columns past N are clipped by the TMA unit)
+          ptx::fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            ptx::tma_store_2d(dmap, stage, n0 + c0, static_cast<int>(grow - lane));
+            ptx::bulk_commit_group();
+            if (!one_tile) ptx::bulk_wait_group_read0();  // staging tile free again
+          }
+          __syncwarp();
+          continue;
+        }
+        __syncwarp();
+        // ... or whole row segments: a store instruction covers 32 / CPR
+        // rows, CPR lanes per row, 16 bytes a lane.
+        constexpr int RPI = 32 / CPR;  // rows per instruction
+        const int sub = lane % CPR;
+#pragma unroll
+        for (int i = 0; i < 32 / RPI; ++i) {
+          const int rr = RPI * i + lane / CPR;  // row within the warp's 32
+          const bool row_ok = __shfl_sync(0xFFFFFFFFu, valid, rr);
+          const int n = n0 + c0 + 8 * sub;
+          if (row_ok && n < p.N) {
+            const size_t g_row = grow - lane + rr;  // the rows of a warp are consecutive
+            *reinterpret_cast<uint4*>(p.d + g_row * p.N + n) = *reinterpret_cast<const uint4*>(
+                stage + rr * Shape::kEpiPitch + 16 * (sub ^ (rr % CPR)));
+          }
+        }
+        __syncwarp();
+      }
+      if (split) ptx::fence_proxy_async_smem();  // parked rows are read by bulk copies
+    }
+  };
+  // A single-tile CTA's warps 0-3 are idle once their roles end: they drain
+  // the upper half of the columns while warps 4-7 drain the lower half.
+  const bool helpers = one_tile && !split && KIND != kMasked && BLOCK_N >= 2 * Shape::kEpiCols;
+
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer --
     int it = 0;
@@ -593,104 +698,30 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
       if (!ok) break;
       ptx::tc_fence_after_sync();
 
-      // which output row this thread owns, and whether it may be written
-      const int m_in_group = ti.m_blk * kBlockM + row_local;
-      bool valid;
-      size_t grow;
-      if (KIND == kMasked) {
-        const int mm = min(max(__ldg(p.masked_m + ti.group), 0), p.rows);
-        valid = m_in_group < mm;
-        grow = (size_t)ti.group * p.rows + m_in_group;
-      } else {
-        valid = m_in_group < p.rows;
-        grow = m_in_group;
-        if (KIND == kContiguous && valid) {
-          const int e = __ldg(p.m_indices + m_in_group);
-          if (e >= 0 && e != ti.group) atomicCAS(p.error_word, 0, kDevMixedExperts);
-          valid = (e == ti.group);
-        }
-      }
-      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + a * BLOCK_N;
-      const int n0 = ti.n_blk * BLOCK_N;
-
-      // A warp whose 32 rows are all outside the output (a short dense A, a
-      // masked group) skips the TMEM reads; it still releases the buffer.
-      if (__any_sync(0xFFFFFFFFu, valid)) {
-        constexpr int CH = Shape::kEpiCols;  // columns per TMEM wait
-        constexpr int NCH = BLOCK_N / CH;    // chunks per tile
-        // one staging tile per warp; a small variant has one per warp and chunk
-        uint8_t* stage0 = sEpi + q * (one_tile ? NCH : 1) * 32 * Shape::kEpiPitch;
-        // TMA store of whole 32-row boxes: the dense form always (rows past M
-        // are clipped); the grouped forms only when all 32 rows are written.
-        const bool tma_store = CH == 64 && !split &&
-                               (KIND == kDense || __all_sync(0xFFFFFFFFu, valid));
-#pragma unroll 1
-        for (int c0 = 0; c0 < BLOCK_N; c0 += CH) {
-          uint32_t r[CH];
-          ptx::tc_ld_32x32b_x32(t_row + c0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-          if (CH == 64)
-            ptx::tc_ld_32x32b_x32(t_row + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[CH - 32]));
-          ptx::tc_wait_ld();
-          uint8_t* stage = one_tile ? stage0 + (c0 / CH) * 32 * Shape::kEpiPitch : stage0;
-          if (split) {
-            // park the FP32 partial; the cluster reduces it below
-            if (valid) {
-#pragma unroll
-              for (int j = 0; j < CH / 4; ++j)
-                *reinterpret_cast<float4*>(red + row_local * RED_PITCH + c0 + 4 * j) =
-                    make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
-                                __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
-            }
-            continue;
-          }
-          // BF16 row of this lane into the warp's staging tile (chunk j of row
-          // `lane` at chunk position j ^ (lane % 8): the 128-byte swizzle) ...
-          constexpr int CPR = CH / 8;  // 16-byte chunks per row
-#pragma unroll
-          for (int j = 0; j < CPR; ++j) {
-            uint4 v;
-            v.x = pack_bf16x2(__uint_as_float(r[8 * j + 0]), __uint_as_float(r[8 * j + 1]));
-            v.y = pack_bf16x2(__uint_as_float(r[8 * j + 2]), __uint_as_float(r[8 * j + 3]));
-            v.z = pack_bf16x2(__uint_as_float(r[8 * j + 4]), __uint_as_float(r[8 * j + 5]));
-            v.w = pack_bf16x2(__uint_as_float(r[8 * j + 6]), __uint_as_float(r[8 * j + 7]));
-            *reinterpret_cast<uint4*>(stage + lane * Shape::kEpiPitch + 16 * (j ^ (lane % CPR))) = v;
-          }
-          if (tma_store) {
-            // ... then one TMA box of 32 rows x 64 columns (rows past the
-            // tensor's end and columns past N are clipped by the TMA unit)
-            ptx::fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-              ptx::tma_store_2d(&tmap_d, stage, n0 + c0, static_cast<int>(grow - lane));
-              ptx::bulk_commit_group();
-              if (!one_tile) ptx::bulk_wait_group_read0();  // staging tile free again
-            }
-            __syncwarp();
-            continue;
-          }
-          __syncwarp();
-          // ... or whole row segments: a store instruction covers 32 / CPR
-          // rows, CPR lanes per row, 16 bytes a lane.
-          constexpr int RPI = 32 / CPR;  // rows per instruction
-          const int sub = lane % CPR;
-#pragma unroll
-          for (int i = 0; i < 32 / RPI; ++i) {
-            const int rr = RPI * i + lane / CPR;  // row within the warp's 32
-            const bool row_ok = __shfl_sync(0xFFFFFFFFu, valid, rr);
-            const int n = n0 + c0 + 8 * sub;
-            if (row_ok && n < p.N) {
-              const size_t g_row = grow - lane + rr;  // the rows of a warp are consecutive
-              *reinterpret_cast<uint4*>(p.d + g_row * p.N + n) = *reinterpret_cast<const uint4*>(
-                  stage + rr * Shape::kEpiPitch + 16 * (sub ^ (rr % CPR)));
-            }
-          }
-          __syncwarp();
-        }
-        if (split) ptx::fence_proxy_async_smem();  // parked rows are read by bulk copies
-      }
+      const int split_col = helpers ? BLOCK_N / 2 : BLOCK_N;
+      // staging: in one_tile mode warp w owns tiles [w * NCH_ALL, (w + 1) * NCH_ALL)
+      drain_acc(ti, a, q, 0, split_col,
+                sEpi + (one_tile ? warp * NCH_ALL : q) * 32 * Shape::kEpiPitch, true);
       ptx::tc_fence_before_sync();
       ptx::mbar_arrive(&acc_empty[a]);
       ++acc_it;
+    }
+    if (lane == 0) ptx::bulk_wait_group0();  // this warp's TMA stores have landed
+  }
+
+  if (helpers && warp < 4 && !*abort_flag) {
+    if (static_cast<int>(blockIdx.x) < total) {
+      const Tile ti = get_tile<KIND>(blockIdx.x, p, s_prefix, lane);
+      if (!ti.skip) {
+        bool ok = true;
+        if (lane == 0) ok = ptx::mbar_wait(&acc_full[0], 0, ctl, kDevTimeoutEpilogue);
+        ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+        if (ok) {
+          ptx::tc_fence_after_sync();
+          drain_acc(ti, 0, warp, BLOCK_N / 2, BLOCK_N,
+                    sEpi + (warp * NCH_ALL + NCH_ALL / 2) * 32 * Shape::kEpiPitch, false);
+        }
+      }
     }
     if (lane == 0) ptx::bulk_wait_group0();  // this warp's TMA stores have landed
   }
