@@ -11,7 +11,7 @@ scales, and D) per second.  The other workloads ("smoke", "prefill",
 
 Timing: inputs sit in HBM, R copies of them at different addresses are rotated
 so that the bytes touched between two visits of one copy exceed the 126 MB L2;
-each step is a captured CUDA graph of its GEMM launches; a barrier and a device
+the steps of one rotation cycle are one captured CUDA graph; a barrier and a device
 synchronisation bracket exactly K timed steps, timed with CUDA events; the
 result is the maximum over ranks.  A second timed pass records CUDA events
 around every launch for the per-kernel duration behind the roofline fraction.
@@ -288,13 +288,22 @@ def run_gpu(args):
     if dg.get_last_device_error() != 0:
         raise RuntimeError("device error during warm-up")
 
-    # one graph per rotation set, and one with per-launch events
-    graphs, ev_graphs, ev_sets = [], [], []
-    for r in range(R):
+    # One graph holds a whole rotation cycle (steps on sets 0..R-1, so that
+    # consecutive launches overlap through programmatic dependent launch
+    # across step boundaries too), one the first `K mod R` steps of a cycle;
+    # one graph per set adds events around each launch.
+    def capture(n_steps):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
-            launch_step(r)
-        graphs.append(g)
+            for r in range(n_steps):
+                launch_step(r)
+        return g
+
+    cycle = capture(R)
+    rem = args.steps % R
+    tail = capture(rem) if rem else None
+    ev_graphs, ev_sets = [], []
+    for r in range(R):
         # external events: recorded as real event nodes inside the graph
         evs = [(torch.cuda.Event(enable_timing=True, external=True),
                 torch.cuda.Event(enable_timing=True, external=True)) for _ in items]
@@ -304,8 +313,8 @@ def run_gpu(args):
         ev_graphs.append(ge)
         ev_sets.append(evs)
     with torch.cuda.stream(stream):
-        for i in range(2 * R):
-            graphs[i % R].replay()
+        cycle.replay()
+        cycle.replay()
     torch.cuda.synchronize(dev)
 
     # ---- timed region: exactly K steps ----
@@ -315,8 +324,10 @@ def run_gpu(args):
     with ClockSampler(dev.index) as clocks:
         with torch.cuda.stream(stream):
             start.record(stream)
-            for i in range(args.steps):
-                graphs[i % R].replay()
+            for _ in range(args.steps // R):   # exactly args.steps steps in all
+                cycle.replay()
+            if tail is not None:
+                tail.replay()
             end.record(stream)
         torch.cuda.synchronize(dev)
     barrier()
@@ -432,7 +443,7 @@ def run_gpu(args):
     if rank == 0:
         print(json.dumps(res), flush=True)
     if world > 1:
-        del graphs, ev_graphs
+        del cycle, tail, ev_graphs
         dist.destroy_process_group()
 
 

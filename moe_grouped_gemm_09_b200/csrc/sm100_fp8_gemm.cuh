@@ -347,17 +347,19 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
     ptx::tmem_alloc(tmem_slot, TMEM_COLS);
     ptx::tmem_relinquish();
   }
-  if (KIND == kDense && p.prefetch && warp == 0 && lane == 0 &&
+  if (KIND == kDense && p.prefetch && warp == 0 &&
       blockIdx.x < p.num_m_blocks * p.num_n_blocks * p.split_k) {
     // Warm L2 with this CTA's first tile while the previous kernel finishes
     // (the tile order of the dense form does not depend on device data).
-    // (A small variant prefetches the whole K range of B, the weights it
-    // streams; the others the first stages of both operands.)
+    // A small variant prefetches the whole K range of B, the weights it
+    // streams; the others the first stages of both operands.
     const Tile ti = get_tile<kDense>(blockIdx.x, p, nullptr, lane);
-    const int kb_end = SMALL ? ti.kb_end : min(ti.kb_end, ti.kb_begin + STAGES * KPS);
-    for (int kb = ti.kb_begin; kb < kb_end; kb += KPS) {
-      ptx::tma_prefetch_l2_4d(&tmap_b, 0, ti.n_blk * BLOCK_N, kb, 0);
-      if (!SMALL) ptx::tma_prefetch_l2_4d(&tmap_a, 0, ti.m_blk * kBlockM, kb, 0);
+    if (lane == 0) {
+      const int kb_end = SMALL ? ti.kb_end : min(ti.kb_end, ti.kb_begin + STAGES * KPS);
+      for (int kb = ti.kb_begin; kb < kb_end; kb += KPS) {
+        ptx::tma_prefetch_l2_4d(&tmap_b, 0, ti.n_blk * BLOCK_N, kb, 0);
+        if (!SMALL) ptx::tma_prefetch_l2_4d(&tmap_a, 0, ti.m_blk * kBlockM, kb, 0);
+      }
     }
   }
   // Everything above reads no input; from here on the inputs may be the
@@ -706,7 +708,9 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
       ptx::mbar_arrive(&acc_empty[a]);
       ++acc_it;
     }
-    if (lane == 0) ptx::bulk_wait_group0();  // this warp's TMA stores have landed
+    // this warp's TMA stores have read their staging tiles (the writes
+    // themselves are part of the grid's completion)
+    if (lane == 0) ptx::bulk_wait_group_read0();
   }
 
   if (helpers && warp < 4 && !*abort_flag) {
@@ -723,7 +727,9 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
         }
       }
     }
-    if (lane == 0) ptx::bulk_wait_group0();  // this warp's TMA stores have landed
+    // this warp's TMA stores have read their staging tiles (the writes
+    // themselves are part of the grid's completion)
+    if (lane == 0) ptx::bulk_wait_group_read0();
   }
 
   if (split) {
@@ -759,21 +765,26 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
       }
       ptx::bulk_commit_group();
     }
-    if (warp >= 4) {
-      const int ep_tid = threadIdx.x - 128;
+    {
+      __syncwarp();
       bool ok = true;
       if (lane == 0) ok = ptx::mbar_wait(recv_bar, 0, ctl, kDevTimeoutEpilogue);
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+      // every copy into this CTA has landed: the cluster barrier that keeps
+      // CTAs alive for incoming copies can complete while this CTA reduces
+      ptx::cluster_arrive_relaxed();
       const int r0 = rank * rows_per;
       constexpr int C8 = BLOCK_N / 8;
       const int items = ok ? slice_rows(rank) * C8 : 0;
       const int n0 = ti.n_blk * BLOCK_N;
-      for (int item = ep_tid; item < items; item += 128) {
+      for (int item = threadIdx.x; item < items; item += kThreads) {
         const int lr = item / C8;  // row within the slice
         const int c = 8 * (item % C8);
         if (n0 + c >= p.N) continue;
         float4 lo = make_float4(0, 0, 0, 0), hi = make_float4(0, 0, 0, 0);
-        for (int src = 0; src < S; ++src) {  // fixed order: deterministic
+#pragma unroll
+        for (int src = 0; src < kMaxSplit; ++src) {  // fixed order: deterministic
+          if (src >= S) break;
           const float* part = (src == static_cast<int>(rank))
                                   ? red + (r0 + lr) * RED_PITCH + c
                                   : recv + (src * rows_per + lr) * RED_PITCH + c;
@@ -793,7 +804,7 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
     }
     if (threadIdx.x == 0) ptx::bulk_wait_group_read0();  // outgoing copies done reading
     __syncwarp();
-    ptx::cluster_sync();  // no CTA leaves while a copy into it may still land
+    ptx::cluster_wait();  // no CTA leaves while a copy into it may still land
   }
 
   ptx::tc_fence_before_sync();
