@@ -13,8 +13,10 @@ Timing: inputs sit in HBM, R copies of them at different addresses are rotated
 so that the bytes touched between two visits of one copy exceed the 126 MB L2;
 the steps of one rotation cycle are one captured CUDA graph; a barrier and a device
 synchronisation bracket exactly K timed steps, timed with CUDA events; the
-result is the maximum over ranks.  A second timed pass records CUDA events
-around every launch for the per-kernel duration behind the roofline fraction.
+result is the maximum over ranks.  The library's kernel is the only kernel in
+the timed region, so the roofline's achieved rate is the step's algorithmic
+units over that time; a second timed pass replays, per GEMM of the step, a
+graph of back-to-back launches of that GEMM alone (``per_gemm_us``).
 
 Under torchrun every rank runs the same per-rank workload on its own GPU (no
 data-path collective: the GEMMs of a step are independent problems), so the
@@ -264,20 +266,20 @@ def run_gpu(args):
         else:
             outs.append(torch.empty((p.G, p.max_m, p.N), dtype=torch.bfloat16, device=dev))
 
-    def launch_step(r, events=None):
-        for j, ((kind, p), t, d) in enumerate(zip(items, sets[r], outs)):
-            if events is not None:
-                events[j][0].record()
-            if kind == "dense":
-                dg.fp8_gemm_nt(t["a"], t["sfa"], t["b"], t["sfb"], d)
-            elif kind == "contiguous":
-                dg.m_grouped_fp8_gemm_nt_contiguous(t["a"], t["sfa"], t["b"], t["sfb"],
-                                                    t["m_indices"], d)
-            else:
-                dg.m_grouped_fp8_gemm_nt_masked(t["a"], t["sfa"], t["b"], t["sfb"],
-                                                t["masked_m"], p.expected_m, d)
-            if events is not None:
-                events[j][1].record()
+    def launch_one(j, r):
+        (kind, p), t, d = items[j], sets[r][j], outs[j]
+        if kind == "dense":
+            dg.fp8_gemm_nt(t["a"], t["sfa"], t["b"], t["sfb"], d)
+        elif kind == "contiguous":
+            dg.m_grouped_fp8_gemm_nt_contiguous(t["a"], t["sfa"], t["b"], t["sfb"],
+                                                t["m_indices"], d)
+        else:
+            dg.m_grouped_fp8_gemm_nt_masked(t["a"], t["sfa"], t["b"], t["sfb"],
+                                            t["masked_m"], p.expected_m, d)
+
+    def launch_step(r):
+        for j in range(len(items)):
+            launch_one(j, r)
 
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.synchronize(dev)
@@ -302,16 +304,14 @@ def run_gpu(args):
     cycle = capture(R)
     rem = args.steps % R
     tail = capture(rem) if rem else None
-    ev_graphs, ev_sets = [], []
-    for r in range(R):
-        # external events: recorded as real event nodes inside the graph
-        evs = [(torch.cuda.Event(enable_timing=True, external=True),
-                torch.cuda.Event(enable_timing=True, external=True)) for _ in items]
-        ge = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(ge, stream=stream):
-            launch_step(r, evs)
-        ev_graphs.append(ge)
-        ev_sets.append(evs)
+    # per GEMM of the step: one graph of its launches on every rotation set
+    per_gemm_graphs = []
+    for j in range(len(items)):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for r in range(R):
+                launch_one(j, r)
+        per_gemm_graphs.append(g)
     with torch.cuda.stream(stream):
         cycle.replay()
         cycle.replay()
@@ -336,20 +336,24 @@ def run_gpu(args):
     if dg.get_last_device_error() != 0:
         raise RuntimeError("device error during the timed steps")
 
-    # ---- per-launch durations (second timed pass, events around each launch) ----
-    n_ev = max(R, min(args.steps, 200))
-    per_launch = [[] for _ in items]
-    torch.cuda.synchronize(dev)
-    for i in range(n_ev):
-        r = i % R
+    # The one kernel of the step is the dominant kernel: its average launch
+    # duration over the timed region is ms / launches and its algorithmic
+    # bytes (or FLOPs) per launch are the step's / launches, so the achieved
+    # rate is the step's units over the timed time.
+    achieved = scale_units(units, unit, ms / 1e3)
+
+    # ---- per GEMM (second timed pass): R back-to-back launches of one shape ----
+    kernel_ms = []
+    for j, g in enumerate(per_gemm_graphs):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         with torch.cuda.stream(stream):
-            ev_graphs[r].replay()
+            g.replay()
+            e0.record(stream)
+            for _ in range(args.per_gemm_reps):
+                g.replay()
+            e1.record(stream)
         torch.cuda.synchronize(dev)
-        for j in range(len(items)):
-            per_launch[j].append(ev_sets[r][j][0].elapsed_time(ev_sets[r][j][1]))
-    kernel_ms = [statistics.mean(v) for v in per_launch]
-    kernel_units = [step_units([it], unit) for it in items]
-    achieved = scale_units(sum(kernel_units), unit, sum(kernel_ms) / 1e3)
+        kernel_ms.append(e0.elapsed_time(e1) / (args.per_gemm_reps * R))
 
     # ---- end to end: host buffers, copies inside the timed region ----
     pinned = []
@@ -421,7 +425,7 @@ def run_gpu(args):
             "gemms": [dict(kind=k, **_shape(p)) for k, p in items],
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
             "l2": flush_note,
-            "graph": "one CUDA graph per step",
+            "graph": f"one CUDA graph per rotation cycle of {R} steps",
         },
         "e2e": {"value": round(whole_job_value(units, world, e2e_ms, unit), 3), "unit": unit,
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
@@ -434,7 +438,8 @@ def run_gpu(args):
             "frac": round(achieved / peak, 4),
             "traffic": profiled_traffic(args.workload),
             "peak_source": f"{peak_kind} ({'hbm_gbs copy' if bound == 'hbm' else '2 x bf16_tflops'})",
-            "kernel_ms": [round(x, 5) for x in kernel_ms],
+            "launch_avg_us": round(ms * 1e3 / launches_per_step, 3),
+            "per_gemm_us": [round(x * 1e3, 3) for x in kernel_ms],
         },
         "clocks": clocks.summary(),
     }
@@ -443,7 +448,7 @@ def run_gpu(args):
     if rank == 0:
         print(json.dumps(res), flush=True)
     if world > 1:
-        del cycle, tail, ev_graphs
+        del cycle, tail, per_gemm_graphs
         dist.destroy_process_group()
 
 
@@ -502,11 +507,22 @@ def run_oracle_sample(items, unit, budget_s: float):
         if dt > budget_s / 4 or frac >= 1.0:
             break
         frac = min(1.0, frac * max(2.0, budget_s / 2 / max(dt, 1e-3)))
-    full_s = dt / (sum(done_frac) / len(done_frac))
+    if frac >= 1.0 and dt < budget_s / 2:
+        # the whole step is cheap: time whole steps back to back instead
+        reps = max(2, int(budget_s / 2 / max(dt, 1e-3)))
+        t0 = time.perf_counter()
+        for _ in range(reps):
+            for kind, p in items:
+                _oracle_rows(o, kind, p, np.arange(_row_units([(kind, p)], unit)[0]))
+        dt = time.perf_counter() - t0
+        full_s = dt / reps
+        sample = f"{reps} whole steps back to back ({dt:.1f} s)"
+    else:
+        full_s = dt / (sum(done_frac) / len(done_frac))
+        sample = (f"first {100 * min(done_frac):.2f}%..{100 * max(done_frac):.2f}% of the output "
+                  f"rows of every GEMM of one step ({dt:.1f} s), scaled to the full step by rows")
     return {"value": round(scale_units(units, unit, full_s), 4), "unit": unit,
-            "cores": o.num_threads(), "kind": "oracle",
-            "sample": f"first {100 * min(done_frac):.2f}%..{100 * max(done_frac):.2f}% of the output "
-                      f"rows of every GEMM of one step ({dt:.1f} s), scaled to the full step by rows"}
+            "cores": o.num_threads(), "kind": "oracle", "sample": sample}
 
 
 def run_reference(args):
@@ -569,7 +585,9 @@ def main():
                     choices=("decode", "smoke", "prefill", "contiguous", "masked"))
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=50)
-    ap.add_argument("--cpu-budget-s", type=float, default=12.0)
+    ap.add_argument("--per-gemm-reps", type=int, default=20,
+                    help="replays of each single-GEMM graph behind per_gemm_us")
+    ap.add_argument("--cpu-budget-s", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:

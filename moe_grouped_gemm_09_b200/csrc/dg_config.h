@@ -8,6 +8,8 @@
 // them: BLOCK_N, pipeline depth, accumulator buffers, split-K and grid size.
 #pragma once
 
+#include <cmath>
+
 namespace dg {
 
 struct Variant {
@@ -77,21 +79,23 @@ inline bool split_fits(const Variant& var, int rows, int split) {
 // Decode-shaped dense problems (at most one 128-row block): HBM-bound.  Pick
 // the variant and K split (one cluster of `split` CTAs per output tile, all in
 // one wave) that minimise an estimate of the time:
-//   fixed cost + max(HBM time of B, busiest CTA's streaming time) + split tail
+//   fixed cost + smooth max(HBM time of B, busiest CTA's streaming time)
+//   + split tail
 // where a CTA streams its B slice plus (at a discount: it is read from L2) its
-// A slice at a rate that grows with the TMA box size.  The constants were
-// fitted to a sweep of every (variant, split) on the six decode-shaped
-// workloads on B200 (the fit picks within 4% of the best measured
-// configuration for each).  Returns false if no one-wave configuration exists.
+// A slice at a rate that grows with the bytes one ring stage moves (both
+// boxes).  The constants were fitted to a sweep of every (variant, split) on
+// the six decode-shaped workloads on B200: the pick is the fastest measured
+// configuration, or within 0.25 us of it, for each.  Returns false if no
+// one-wave configuration exists.
 inline bool pick_decode(int rows, int N, int K, int num_sms, const ClusterLimits* lim,
                         PickedConfig* out) {
   const int KB = K / 128;
   constexpr double kHbmBytesPerUs = 4.5e6;  // effective, whole GPU
-  constexpr double kRate16KB = 50.0;        // KB per microsecond per CTA, 16 KB boxes
-  constexpr double kRateCap = 90.0;         // KB per microsecond per CTA, large boxes
-  constexpr double kAWeight = 0.35;         // A slices come from L2
+  constexpr double kRate16KB = 20.0;        // KB per microsecond per CTA, 16 KB stages
+  constexpr double kRateCap = 70.0;         // KB per microsecond per CTA, large stages
+  constexpr double kAWeight = 0.2;          // A slices come from L2
   constexpr double kFixedUs = 6.0;
-  constexpr double kSplitUs = 3.0;          // cluster barriers, pushes, reduction
+  constexpr double kSplitUs = 1.5;          // cluster barriers, pushes, reduction
   double best = 1e30;
   bool found = false;
   for (int v = 0; v < kNumVariants; ++v) {
@@ -99,8 +103,8 @@ inline bool pick_decode(int rows, int N, int K, int num_sms, const ClusterLimits
     if (!var.decode || var.small || rows > var.a_rows) continue;
     const int bn = var.block_n;
     const int nt = ceil_div(N, bn);
-    const double box_kb = var.kps * bn * 128 / 1024.0;
-    double r_cta = kRate16KB * box_kb / 16.0;
+    const double stage_kb = var.kps * (bn + var.a_rows) * 128 / 1024.0;
+    double r_cta = kRate16KB * stage_kb / 16.0;
     if (r_cta > kRateCap) r_cta = kRateCap;
     for (int s = 1; s <= kMaxSplitK && s <= KB; ++s) {
       if (nt * s > num_sms) break;
@@ -112,7 +116,8 @@ inline bool pick_decode(int rows, int N, int K, int num_sms, const ClusterLimits
       const double a_cta = static_cast<double>(rows) * per * 128 / 1024.0;  // KB
       const double t_cta = (b_cta + kAWeight * a_cta) / r_cta;             // us
       const double t_hbm = static_cast<double>(N) * K / kHbmBytesPerUs;     // us
-      const double t = kFixedUs + (t_cta > t_hbm ? t_cta : t_hbm) + (s > 1 ? kSplitUs : 0.0);
+      const double t_stream = std::pow(std::pow(t_cta, 8.0) + std::pow(t_hbm, 8.0), 0.125);
+      const double t = kFixedUs + t_stream + (s > 1 ? kSplitUs : 0.0);
       if (t < best - 1e-9) {
         best = t;
         found = true;
