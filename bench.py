@@ -88,6 +88,24 @@ def scale_units(x: float, unit: str, seconds: float) -> float:
     return x / seconds / (1e9 if unit == "GB/s" else 1e12)
 
 
+SPEC_HBM_GBS = 8000.0     # B200 HBM3e, vendor figure
+SPEC_FP8_TFLOPS = 4500.0  # B200 dense E4M3, vendor figure
+
+
+def roofline_terms(items, ms: float, hbm_gbs: float, fp8_tflops: float) -> dict:
+    """Roofline of one step: every GEMM's time bound is the larger of its
+    FLOPs at the FP8 peak and its algorithmic bytes at the HBM bandwidth; the
+    step's bound is the sum.  ``bound`` names the term that dominates the sum."""
+    def t_roof(hbm, fp8):
+        return sum(max(p.flops() / (fp8 * 1e12), p.bytes() / (hbm * 1e9)) for _, p in items)
+    t_flop = sum(p.flops() for _, p in items) / (fp8_tflops * 1e12)
+    t_byte = sum(p.bytes() for _, p in items) / (hbm_gbs * 1e9)
+    t = t_roof(hbm_gbs, fp8_tflops)
+    return {"bound": "tensor" if t_flop >= t_byte else "hbm", "t_roof_s": t,
+            "frac_time": t / (ms / 1e3),
+            "frac_time_spec": t_roof(SPEC_HBM_GBS, SPEC_FP8_TFLOPS) / (ms / 1e3)}
+
+
 # --------------------------------------------------------------- helpers --
 
 def load_peaks():
@@ -234,7 +252,7 @@ def run_gpu(args):
         return reduce_max(x, world, dev)
 
     items = build_workload(args.workload, seed=args.seed)
-    metric, unit, bound = workload_meta(args.workload)
+    metric, unit, _ = workload_meta(args.workload)
     units = step_units(items, unit)
     set_bytes = sum(p.a.nbytes + p.b.nbytes + p.sfa.nbytes + p.sfb.nbytes for _, p in items)
     R = max(2, math.ceil(3 * L2_BYTES / max(set_bytes, 1)))
@@ -339,8 +357,7 @@ def run_gpu(args):
     # The one kernel of the step is the dominant kernel: its average launch
     # duration over the timed region is ms / launches and its algorithmic
     # bytes (or FLOPs) per launch are the step's / launches, so the achieved
-    # rate is the step's units over the timed time.
-    achieved = scale_units(units, unit, ms / 1e3)
+    # rate (below) is the step's units over the timed time.
 
     # ---- per GEMM (second timed pass): R back-to-back launches of one shape ----
     kernel_ms = []
@@ -400,11 +417,14 @@ def run_gpu(args):
         cpu = run_oracle_sample(items, unit, budget_s=args.cpu_budget_s)
 
     peaks, peak_kind = load_peaks()
-    if bound == "hbm":
-        peak = float(peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"]))
-    else:
-        # E4M3 dense peak = 2x the measured BF16 figure (nominal FP8:BF16 ratio 4.5:2.25)
-        peak = 2.0 * float(peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"]))
+    hbm_peak = float(peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"]))
+    # E4M3 dense peak = 2x the measured BF16 figure (nominal FP8:BF16 ratio 4.5:2.25)
+    fp8_peak = 2.0 * float(peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"]))
+    roof = roofline_terms(items, ms, hbm_peak, fp8_peak)
+    bound = roof["bound"]
+    r_unit = "GB/s" if bound == "hbm" else "TFLOP/s"
+    peak = hbm_peak if bound == "hbm" else fp8_peak
+    achieved = scale_units(step_units(items, r_unit), r_unit, ms / 1e3)
     value = whole_job_value(units, world, ms, unit)
     launches_per_step = len(items)
     res = {
@@ -434,10 +454,13 @@ def run_gpu(args):
             "bound": bound,
             "achieved": round(achieved, 3),
             "peak": peak,
-            "unit": unit,
+            "unit": r_unit,
             "frac": round(achieved / peak, 4),
             "traffic": profiled_traffic(args.workload),
             "peak_source": f"{peak_kind} ({'hbm_gbs copy' if bound == 'hbm' else '2 x bf16_tflops'})",
+            "roofline_time_us": round(roof["t_roof_s"] * 1e6, 3),
+            "frac_time": round(roof["frac_time"], 4),
+            "frac_time_spec": round(roof["frac_time_spec"], 4),
             "launch_avg_us": round(ms * 1e3 / launches_per_step, 3),
             "per_gemm_us": [round(x * 1e3, 3) for x in kernel_ms],
         },
@@ -482,9 +505,18 @@ def _oracle_rows(o, kind, p, rows: np.ndarray):
         o.grouped_contiguous(p.a[valid], p.sfa[valid], p.b, p.sfb, p.m_indices[valid])
     else:
         pairs = [(g, m) for g in range(p.G) for m in range(min(max(int(p.masked_m[g]), 0), p.max_m))]
-        sel = [pairs[i] for i in rows]
-        for g, m in sel:
-            o.gemm_nt(p.a[g, m:m + 1], p.sfa[g, m:m + 1], p.b[g], p.sfb[g], want_acc=False)
+        sel = sorted(pairs[i] for i in rows)
+        # one oracle call per run of consecutive rows of one group (the oracle
+        # spreads the rows of a call over its threads)
+        i = 0
+        while i < len(sel):
+            g, m0 = sel[i]
+            j = i + 1
+            while j < len(sel) and sel[j] == (g, m0 + (j - i)):
+                j += 1
+            o.gemm_nt(p.a[g, m0:m0 + (j - i)], p.sfa[g, m0:m0 + (j - i)], p.b[g], p.sfb[g],
+                      want_acc=False)
+            i = j
 
 
 def run_oracle_sample(items, unit, budget_s: float):

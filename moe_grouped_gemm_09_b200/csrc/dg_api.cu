@@ -87,9 +87,11 @@ dg_status device_state(DeviceState** out, int* dev_out) {
   return DG_OK;
 }
 
-// Rows per TMA box of A: a dense A shorter than one 128-row block is fetched
+// Rows per TMA box of A: a whole tile (128 rows, or 256 for a two-half
+// variant), except that a dense A shorter than one 128-row block is fetched
 // with a box of its own (16-row rounded) height, so the SM moves no padding.
-int a_box_rows(int kind, int rows) {
+int a_box_rows(int kind, int rows, const Variant& var) {
+  if (var.a_rows == 256) return 256;
   if (kind != kDense || rows >= kBlockM) return kBlockM;
   return ((rows + 15) / 16) * 16;
 }
@@ -112,8 +114,9 @@ void forced_config(int kind, int rows, int N, int K, int G, int sms, PickedConfi
     if (x.block_n != bn) continue;
     if (kps ? (x.kps != kps || (ar && x.a_rows != ar)) : x.decode) continue;
     if (sm >= 0 && x.small != (sm != 0)) continue;
-    if (x.decode && kind != kDense) continue;
-    if (a_box_rows(kind, rows) > x.a_rows) continue;
+    if ((x.decode || x.a_rows == 256) && kind != kDense) continue;
+    if (x.a_rows == 256 && rows < 256) continue;
+    if (a_box_rows(kind, rows, x) > x.a_rows) continue;
     v = i;
   }
   const int KB = K / kBlockK;
@@ -121,7 +124,7 @@ void forced_config(int kind, int rows, int N, int K, int G, int sms, PickedConfi
   if (sk > 1 && (kind != kDense || rows > kBlockM)) return;
   if ((sk - 1) * ceil_div(KB, sk) >= KB) return;
   const long long groups = (kind == kMasked) ? G : 1;
-  const long long tiles = groups * ceil_div(rows, kBlockM) * ceil_div(N, bn);
+  const long long tiles = groups * ceil_div(rows, tile_rows(kVariants[v])) * ceil_div(N, bn);
   pc->variant = v;
   pc->split_k = sk;
   pc->out_tiles = static_cast<int>(tiles);
@@ -183,7 +186,7 @@ using ShapeOf = KernelShape<kVariants[V].block_n, kVariants[V].stages, kVariants
                             kVariants[V].kps, kVariants[V].a_rows, kVariants[V].small>;
 
 // Kernels are instantiated only for the (form, variant) pairs that exist:
-// the decode variants serve the dense form only.
+// the decode variants and the 256-row variants serve the dense form only.
 // Per-variant shared-memory bytes (what = 0) or TMEM columns (what = 1).
 template <int what, int... V>
 constexpr std::array<int, sizeof...(V)> variant_table(std::integer_sequence<int, V...>) {
@@ -191,7 +194,7 @@ constexpr std::array<int, sizeof...(V)> variant_table(std::integer_sequence<int,
 }
 
 template <int KIND, int V>
-constexpr bool kBuilt = KIND == kDense || !kVariants[V].decode;
+constexpr bool kBuilt = KIND == kDense || (!kVariants[V].decode && kVariants[V].a_rows != 256);
 
 template <int KIND, int V>
 auto kernel_of() {
@@ -347,7 +350,7 @@ dg_status run(int kind, const void* a, const float* sfa, const void* b, const fl
   args.N = N;
   args.K = K;
   args.G = (kind == kDense) ? 1 : G;
-  args.num_m_blocks = ceil_div(rows, kBlockM);
+  args.num_m_blocks = ceil_div(rows, tile_rows(var));
   args.num_n_blocks = ceil_div(N, var.block_n);
   args.k_blocks = K / kBlockK;
   args.split_k = pc.split_k;
@@ -360,8 +363,9 @@ dg_status run(int kind, const void* a, const float* sfa, const void* b, const fl
   args.masked_m = masked_m;
   args.error_word = st->error_word;
   args.timeout_ns = g_timeout_ns;
-  args.a_box_rows = a_box_rows(kind, rows);
+  args.a_box_rows = a_box_rows(kind, rows, var);
   if (args.a_box_rows > var.a_rows) return DG_ERR_UNSUPPORTED;
+  if (var.a_rows == 256 && (kind != kDense || pc.split_k > 1)) return DG_ERR_UNSUPPORTED;
   args.prefetch = prefetch_enabled();
   // a small variant runs one tile per CTA (its epilogue reuses the ring)
   if (var.small && (kind != kDense || pc.grid != args.num_m_blocks * args.num_n_blocks * pc.split_k))
@@ -484,7 +488,7 @@ dg_status dg_query_config(int kind, int rows, int N, int K, int G, int expected_
     return DG_ERR_INVALID_ARG;
   const PickedConfig pc = pick_config(kind, rows, N, K, G, expected_m, num_sms);
   const Variant v = kVariants[pc.variant];
-  out->block_m = kBlockM;
+  out->block_m = tile_rows(v);
   out->block_n = v.block_n;
   out->stages = v.stages;
   out->num_acc = v.num_acc;

@@ -17,12 +17,14 @@ struct Variant {
   int stages;
   int num_acc;
   int kps;      // 128-wide K blocks per ring stage (one TMA box of each operand)
-  int a_rows;   // rows of A a stage holds (64: dense A of at most 64 rows)
+  int a_rows;   // rows of A a stage holds (64: dense A of at most 64 rows;
+                // 256: a tile of two 128-row halves sharing each B tile)
   bool decode;  // built for dense problems of at most one 128-row block
   bool small;   // two CTAs fit per SM; one tile per CTA
 };
 
-// The compiled variants: general ones first (every form), then the
+// The compiled variants: general ones first (every form; the 256-row one
+// serves the dense form only, and only when forced), then the
 // decode-shaped dense ones, whose stages are several K blocks deep so that
 // each TMA box moves 32-64 KB, then the small decode ones (at most ~100 KB of
 // shared memory and 256 TMEM columns, so that the next kernel's CTAs can be
@@ -32,6 +34,7 @@ constexpr Variant kVariants[] = {
     {128, 6, 2, 1, 128, false, false},
     {64, 8, 2, 1, 128, false, false},
     {32, 9, 2, 1, 128, false, false},
+    {192, 3, 1, 1, 256, false, false},
     {128, 2, 1, 4, 64, true, false},
     {64, 3, 2, 4, 64, true, false},
     {256, 2, 1, 2, 64, true, false},
@@ -54,6 +57,9 @@ struct PickedConfig {
 };
 
 inline int ceil_div(long long a, long long b) { return static_cast<int>((a + b - 1) / b); }
+
+// Output rows of one tile of a variant.
+inline int tile_rows(const Variant& v) { return v.a_rows == 256 ? 256 : 128; }
 
 // How many clusters of `cluster` CTAs of variant `variant` the device can run
 // at once.  max_clusters[v][s] for s in 1..kMaxSplitK; a value <= 0 means
@@ -149,18 +155,23 @@ inline PickedConfig pick_config(int kind, int rows, int N, int K, int G, int exp
     eff_rows = expected_m > 0 ? (expected_m < rows ? expected_m : rows) : rows;
     groups = G;
   }
-  const int m_blocks = groups * ceil_div(eff_rows > 0 ? eff_rows : 1, 128);
   double best_cost = 1e30;
   for (int v = 0; v < kNumVariants; ++v) {
     const Variant& var = kVariants[v];
-    if (var.small || var.a_rows != 128) continue;
+    if (var.small || var.a_rows < 128) continue;
     if (var.decode && (kind != 0 || var.kps != 2 || var.block_n != 256)) continue;
+    // The 256-row variant (fewer operand bytes per FLOP) measured no faster
+    // than the 128 x 256 tiles on B200: the ring is bound by the latency of
+    // the bytes in flight, not by their count.  It is taken only when forced.
+    if (var.a_rows == 256) continue;
     const int bn = var.block_n;
     if (bn > 128 && N <= 128) continue;
+    const int tm = tile_rows(var);
+    const int m_blocks = groups * ceil_div(eff_rows > 0 ? eff_rows : 1, tm);
     const int n_tiles = ceil_div(N, bn);
     const long long tiles = static_cast<long long>(m_blocks) * n_tiles;
     const int waves = ceil_div(tiles, num_sms);
-    double cost = waves * (16.0 + bn / 8.0);
+    double cost = waves * (tm / 8.0 + bn / 8.0);
     if (var.kps == 2) cost *= (K <= 2048 ? 0.85 : 1.02);
     if (cost < best_cost - 1e-9) {
       best_cost = cost;
@@ -168,12 +179,13 @@ inline PickedConfig pick_config(int kind, int rows, int N, int K, int G, int exp
     }
   }
   const int bn = kVariants[best.variant].block_n;
+  const int tm = tile_rows(kVariants[best.variant]);
   const int n_tiles = ceil_div(N, bn);
   long long tiles;
   if (kind == 2) {
-    tiles = static_cast<long long>(G) * ceil_div(rows, 128) * n_tiles;  // upper bound
+    tiles = static_cast<long long>(G) * ceil_div(rows, tm) * n_tiles;  // upper bound
   } else {
-    tiles = static_cast<long long>(ceil_div(rows, 128)) * n_tiles;
+    tiles = static_cast<long long>(ceil_div(rows, tm)) * n_tiles;
   }
   best.split_k = 1;
   best.out_tiles = tiles > 0x7fffffff ? 0x7fffffff : static_cast<int>(tiles);

@@ -225,7 +225,7 @@ extern "C" dg_status dg_fp8_gemm_nt_noalloc(const void* a, const float* sfa, con
   args.N = N;
   args.K = K;
   args.G = 1;
-  args.num_m_blocks = ceil_div(M, kBlockM);
+  args.num_m_blocks = ceil_div(M, tile_rows(var));
   args.num_n_blocks = ceil_div(N, var.block_n);
   args.k_blocks = K / kBlockK;
   args.split_k = pc.split_k;
@@ -236,7 +236,7 @@ extern "C" dg_status dg_fp8_gemm_nt_noalloc(const void* a, const float* sfa, con
   args.d = static_cast<__nv_bfloat16*>(d);
   args.error_word = reinterpret_cast<int*>(st->scratch);
   args.timeout_ns = 1000ull * 1000 * 1000;
-  args.a_box_rows = M >= kBlockM ? kBlockM : ((M + 15) / 16) * 16;
+  args.a_box_rows = var.a_rows == 256 ? 256 : M >= kBlockM ? kBlockM : ((M + 15) / 16) * 16;
   args.prefetch = 1;
   if (args.a_box_rows > var.a_rows) return DG_ERR_UNSUPPORTED;
   if (var.small && pc.grid != args.num_m_blocks * args.num_n_blocks * pc.split_k)

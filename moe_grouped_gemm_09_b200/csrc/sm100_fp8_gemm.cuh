@@ -101,26 +101,33 @@ __host__ __device__ constexpr int pow2_ceil(int x) {
 //   KPS      128-wide K blocks per ring stage: every stage is one TMA box of A
 //            and one of B, each KPS K blocks deep (bigger boxes stream faster)
 //   A_ROWS   rows of A a stage holds room for (64 for a dense A of at most 64
-//            rows, else 128)
+//            rows, 128, or 256 for a tile of two 128-row MMA halves that
+//            share every B tile: fewer operand bytes per FLOP)
 //   SMALL    a decode variant small enough (shared memory and TMEM) for two
 //            CTAs per SM, so that the next kernel's CTAs can start (and warm
 //            L2) while this kernel drains; it runs one tile per CTA and
 //            stages its epilogue in the then idle operand ring
 template <int BLOCK_N, int STAGES, int NUM_ACC, int KPS = 1, int A_ROWS = 128, bool SMALL = false>
 struct KernelShape {
+  static constexpr int kHalves = A_ROWS == 256 ? 2 : 1;  // 128-row MMA halves of a tile
+  static constexpr int kTileM = kBlockM * kHalves;        // output rows of a tile
   static constexpr int kABytes = KPS * A_ROWS * kBlockK;  // one E4M3 byte per element
   static constexpr int kBBytes = KPS * BLOCK_N * kBlockK;
   static constexpr int kSfbChunks = (BLOCK_N + 127) / 128;
-  static constexpr int kSfBytes = 512 * (1 + kSfbChunks);  // SFA 512 B + SFB 512 B per 128 rows
-  static constexpr int kSfCols = 4 * (1 + kSfbChunks);     // TMEM columns per stage
-  static constexpr int kAccCols = NUM_ACC * BLOCK_N;
+  // 128-row scale blocks of B one tile can touch (a tile that is not aligned
+  // to 128 rows straddles one more)
+  static constexpr int kSfbBlocks = kSfbChunks + (BLOCK_N % 128 != 0 && 128 % BLOCK_N != 0 ? 1 : 0);
+  // SFA 512 B per 128 rows of A + SFB 512 B per 128 rows of B
+  static constexpr int kSfBytes = 512 * (kHalves + kSfbChunks);
+  static constexpr int kSfCols = 4 * (kHalves + kSfbChunks);  // TMEM columns per stage
+  static constexpr int kAccCols = NUM_ACC * kHalves * BLOCK_N;
   static constexpr int kTmemCols = pow2_ceil(kAccCols + STAGES * kSfCols);
   static constexpr int kBarBytes = 8 * (2 * STAGES + 2 * NUM_ACC + 2);
   // epilogue: each of the 4 epilogue warps stages 32 rows x kEpiCols BF16
   // columns in shared memory (16-byte chunks XOR-swizzled by row, the layout
   // of the 128-byte TMA swizzle), then stores them with one TMA box or with
   // whole row segments
-  static constexpr int kEpiCols = BLOCK_N >= 64 ? 64 : 32;
+  static constexpr int kEpiCols = BLOCK_N % 64 == 0 ? 64 : 32;
   static constexpr int kEpiPitch = kEpiCols * 2;        // bytes per staged row
   static constexpr int kEpiBytes = SMALL ? 0 : 4 * 32 * kEpiPitch;
   // tmem slot, flags, and (grouped forms) the masked prefix
@@ -138,7 +145,8 @@ struct KernelShape {
   static_assert(kTmemCols <= 512, "TMEM budget exceeded");
   static_assert(BLOCK_N % 32 == 0 && BLOCK_N >= 32 && BLOCK_N <= 256, "BLOCK_N");
   static_assert(KPS >= 1 && KPS <= 4, "up to four K blocks share one scale-factor word");
-  static_assert(A_ROWS == 64 || A_ROWS == 128, "A_ROWS");
+  static_assert(A_ROWS == 64 || A_ROWS == 128 || A_ROWS == 256, "A_ROWS");
+  static_assert(A_ROWS != 256 || (!SMALL && KPS == 1), "two-half tiles are general variants");
   static_assert((BLOCK_N * kBlockK) % 1024 == 0, "B sub-tiles must keep 1024-byte alignment");
 };
 
@@ -185,15 +193,20 @@ __device__ __forceinline__ Tile get_tile(int t, const GemmArgs& p, const int* s_
     ti.group = lo;
     ti.n_blk = local / mb;
     ti.m_blk = local % mb;
-  } else {
+  } else if (KIND == kDense) {
+    // column-major over tiles: the CTAs of one wave share a few B column
+    // tiles and read every A row block
     ti.m_blk = u % p.num_m_blocks;
     ti.n_blk = u / p.num_m_blocks;
     ti.group = 0;
-    if (KIND == kContiguous) {
-      int e = block_expert(p.m_indices, ti.m_blk * kBlockM, p.rows, lane);
-      ti.group = e;
-      ti.skip = (e < 0) || (e >= p.G);
-    }
+  } else {
+    // row-major over tiles: the CTAs of one wave cover a few consecutive
+    // 128-row blocks (one or a few experts) and all their column tiles, so
+    // each expert's B streams from HBM about once and is reused from L2
+    ti.m_blk = u / p.num_n_blocks;
+    ti.n_blk = u % p.num_n_blocks;
+    ti.group = block_expert(p.m_indices, ti.m_blk * kBlockM, p.rows, lane);
+    ti.skip = (ti.group < 0) || (ti.group >= p.G);
   }
   ti.kb_begin = ti.split * p.kb_per_split;
   ti.kb_end = min(p.k_blocks, ti.kb_begin + p.kb_per_split);
@@ -287,6 +300,9 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
   constexpr int SF_BYTES = Shape::kSfBytes;
   constexpr int SF_COLS = Shape::kSfCols;
   constexpr int SFB_CHUNKS = Shape::kSfbChunks;
+  constexpr int SFB_BLOCKS = Shape::kSfbBlocks;
+  constexpr int HALVES = Shape::kHalves;
+  constexpr int TILE_M = Shape::kTileM;
   constexpr int ACC_COLS = Shape::kAccCols;
   constexpr int TMEM_COLS = Shape::kTmemCols;
   constexpr int RED_PITCH = BLOCK_N + 4;  // floats per row of a parked split-K partial
@@ -296,6 +312,7 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
   static_assert(kBlockM * RED_PITCH * 4 <= STAGES * (A_BYTES + B_BYTES),
                 "split-K partial must fit in the operand ring");
   static_assert((KPS == 1 && !SMALL) || KIND == kDense, "decode variants serve the dense form");
+  static_assert(HALVES == 1 || KIND == kDense, "a 256-row tile could straddle two groups");
 
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment for the 128-byte-swizzled operand tiles
@@ -307,7 +324,8 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
   // when every CTA has a single tile (always for a small variant), the operand
   // ring, idle once that tile's MMAs are done, with one tile per warp and chunk
   const int n_tiles_total = (KIND == kMasked ? -1 : p.num_m_blocks * p.num_n_blocks * p.split_k);
-  const bool one_tile = SMALL || (n_tiles_total >= 0 && n_tiles_total <= static_cast<int>(gridDim.x));
+  const bool one_tile = HALVES == 1 && (SMALL || (n_tiles_total >= 0 &&
+                                                  n_tiles_total <= static_cast<int>(gridDim.x)));
   uint8_t* sEpi = one_tile ? sA : sB + STAGES * B_BYTES;
   uint8_t* sSF = sB + STAGES * B_BYTES + Shape::kEpiBytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(sSF + STAGES * SF_BYTES);
@@ -358,28 +376,35 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
       const int kb_end = SMALL ? ti.kb_end : min(ti.kb_end, ti.kb_begin + STAGES * KPS);
       for (int kb = ti.kb_begin; kb < kb_end; kb += KPS) {
         ptx::tma_prefetch_l2_4d(&tmap_b, 0, ti.n_blk * BLOCK_N, kb, 0);
-        if (!SMALL) ptx::tma_prefetch_l2_4d(&tmap_a, 0, ti.m_blk * kBlockM, kb, 0);
+        if (!SMALL) ptx::tma_prefetch_l2_4d(&tmap_a, 0, ti.m_blk * TILE_M, kb, 0);
       }
     }
   }
-  // Everything above reads no input; from here on the inputs may be the
-  // previous kernel's outputs, so wait for it (a no-op without programmatic
-  // dependent launch), and let the next kernel start its own prologue.
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  if (KIND == kMasked && threadIdx.x == 96) {
-    int acc = 0;
-    for (int g = 0; g < p.G; ++g) {
-      s_prefix[g] = acc;
-      int mm = min(max(p.masked_m[g], 0), p.rows);
-      acc += ((mm + kBlockM - 1) / kBlockM) * p.num_n_blocks;
-    }
-    s_prefix[p.G] = acc;
-  }
+  // Barriers, the abort flag and the TMEM base are published before waiting
+  // on the previous kernel, so that every role starts right after the wait.
   ptx::tc_fence_before_sync();
   __syncthreads();
   ptx::tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
+  // Let the next kernel start its own prologue (once every CTA of this grid
+  // got here), then, since everything above reads no input and from here on
+  // the inputs may be the previous kernel's outputs, wait for that kernel (a
+  // no-op without programmatic dependent launch).
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (KIND == kMasked) {
+    // the tile sequence of the masked form depends on masked_m (device data)
+    if (threadIdx.x == 96) {
+      int acc = 0;
+      for (int g = 0; g < p.G; ++g) {
+        s_prefix[g] = acc;
+        int mm = min(max(p.masked_m[g], 0), p.rows);
+        acc += ((mm + kBlockM - 1) / kBlockM) * p.num_n_blocks;
+      }
+      s_prefix[p.G] = acc;
+    }
+    __syncthreads();
+  }
 
   ptx::WaitCtl ctl{abort_flag, p.error_word, p.timeout_ns};
   const int total = (KIND == kMasked ? s_prefix[p.G]
@@ -390,11 +415,11 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
   // at stage0 to D, or (split-K) FP32 into the parked partial.
   constexpr int NCH_ALL = BLOCK_N / Shape::kEpiCols;
   const CUtensorMap* dmap = &tmap_d;
-  auto drain_acc = [&](const Tile& ti, int a, int q, int c_begin, int c_end, uint8_t* stage0,
-                       bool report) {
+  auto drain_acc = [&](const Tile& ti, int a, int h, int q, int c_begin, int c_end,
+                       uint8_t* stage0, bool report) {
     // which output row this thread owns, and whether it may be written
     const int row_local = 32 * q + lane;  // accumulator row = TMEM lane
-    const int m_in_group = ti.m_blk * kBlockM + row_local;
+    const int m_in_group = ti.m_blk * TILE_M + kBlockM * h + row_local;
     bool valid;
     size_t grow;
     if (KIND == kMasked) {
@@ -410,7 +435,8 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
         valid = (e == ti.group);
       }
     }
-    const uint32_t t_row = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + a * BLOCK_N;
+    const uint32_t t_row =
+        tmem_base + (static_cast<uint32_t>(32 * q) << 16) + (a * HALVES + h) * BLOCK_N;
     const int n0 = ti.n_blk * BLOCK_N;
 
     // A warp whose 32 rows are all outside the output (a short dense A, a
@@ -497,7 +523,7 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
       const Tile ti = get_tile<KIND>(t, p, s_prefix, lane);
       if (ti.skip) continue;
-      const int a_row = ti.m_blk * kBlockM;
+      const int a_row = ti.m_blk * TILE_M;
       const int a_grp = (KIND == kMasked) ? ti.group : 0;
       for (int kb = ti.kb_begin; kb < ti.kb_end; kb += KPS, ++it) {
         const int s = it % STAGES;
@@ -539,7 +565,7 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
       if (!ok) break;
       ptx::tc_fence_after_sync();
-      const uint32_t d_tmem = tmem_base + a * BLOCK_N;
+      const uint32_t d_tmem = tmem_base + a * HALVES * BLOCK_N;
       for (int kb = ti.kb_begin; kb < ti.kb_end; kb += KPS, ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
@@ -548,13 +574,18 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
         if (!ok) break;
         ptx::tc_fence_after_sync();
         if (lane == 0) {
+          // per stage: SFA words of each 128-row half, then SFB words of
+          // each 128-row chunk of the tile's B rows
           const uint32_t sfa_tmem = tmem_base + ACC_COLS + s * SF_COLS;
-          const uint32_t sfb_tmem = sfa_tmem + 4;
+          const uint32_t sfb_tmem = sfa_tmem + 4 * HALVES;
           const uint32_t sf_smem = ptx::smem_addr(sSF + s * SF_BYTES);
-          ptx::tc_cp_32x128b_warpx4(sfa_tmem, ptx::sdesc_sf_32x16(sf_smem));
+#pragma unroll
+          for (int h = 0; h < HALVES; ++h)
+            ptx::tc_cp_32x128b_warpx4(sfa_tmem + 4 * h, ptx::sdesc_sf_32x16(sf_smem + 512 * h));
 #pragma unroll
           for (int h = 0; h < SFB_CHUNKS; ++h)
-            ptx::tc_cp_32x128b_warpx4(sfb_tmem + 4 * h, ptx::sdesc_sf_32x16(sf_smem + 512 * (1 + h)));
+            ptx::tc_cp_32x128b_warpx4(sfb_tmem + 4 * h,
+                                      ptx::sdesc_sf_32x16(sf_smem + 512 * (HALVES + h)));
           const uint32_t a_base = ptx::smem_addr(sA + s * A_BYTES);
           const uint32_t b_base = ptx::smem_addr(sB + s * B_BYTES);
 #pragma unroll
@@ -562,15 +593,20 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
             if (kb + j >= ti.kb_end) break;
             // K block j of the stage: its scale factors are byte j of every
             // TMEM scale word (selected by the scale-factor id)
-            const uint64_t da = ptx::sdesc_kmajor_sw128(a_base + j * p.a_box_rows * kBlockK);
             const uint64_t db = ptx::sdesc_kmajor_sw128(b_base + j * BLOCK_N * kBlockK);
             const uint32_t id = idesc | (static_cast<uint32_t>(j) << 29) | (static_cast<uint32_t>(j) << 4);
             const uint32_t byte_sel = static_cast<uint32_t>(j) << 30;
 #pragma unroll
-            for (int ks = 0; ks < kBlockK / 32; ++ks)
-              ptx::tc_mma_mxf8_block_scale(d_tmem, da + 2 * ks, db + 2 * ks, id,
-                                           sfa_tmem | byte_sel, sfb_tmem | byte_sel,
-                                           kb + j > ti.kb_begin || ks > 0);
+            for (int h = 0; h < HALVES; ++h) {
+              // half h: A rows 128h.. of the stage's tile, its own accumulator
+              const uint64_t da = ptx::sdesc_kmajor_sw128(a_base + j * p.a_box_rows * kBlockK +
+                                                          h * kBlockM * kBlockK);
+#pragma unroll
+              for (int ks = 0; ks < kBlockK / 32; ++ks)
+                ptx::tc_mma_mxf8_block_scale(d_tmem + h * BLOCK_N, da + 2 * ks, db + 2 * ks, id,
+                                             (sfa_tmem + 4 * h) | byte_sel, sfb_tmem | byte_sel,
+                                             kb + j > ti.kb_begin || ks > 0);
+            }
           }
           ptx::tc_commit(&empty[s]);
         }
@@ -594,34 +630,38 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
     // Scale words pack the stage's K blocks: byte j belongs to K block j.
     constexpr int PF = (8 + KPS - 1) / KPS;
     const int KB = p.k_blocks;
-    float va[PF][4][KPS];
-    float vb[PF][SFB_CHUNKS][KPS];
+    float va[PF][HALVES][4][KPS];
+    float vb[PF][SFB_BLOCKS][KPS];
     StageWalker<KIND, KPS> ld, wr;
     ld.start(blockIdx.x, gridDim.x, total, p, s_prefix, lane);
     wr.start(blockIdx.x, gridDim.x, total, p, s_prefix, lane);
 
-    auto issue = [&](float (&a)[4][KPS], float (&b)[SFB_CHUNKS][KPS]) {
+    auto issue = [&](float (&a)[HALVES][4][KPS], float (&b)[SFB_BLOCKS][KPS]) {
       const Tile& ti = ld.w.ti;
-      const int row_base = (KIND == kMasked ? ti.group * p.rows : 0) + ti.m_blk * kBlockM;
-      const int rows_left = p.rows - ti.m_blk * kBlockM;  // rows of this block that exist
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int r = 32 * c + lane;
+      for (int h = 0; h < HALVES; ++h) {
+        const int m0 = ti.m_blk * TILE_M + kBlockM * h;  // first row of this half
+        const int row_base = (KIND == kMasked ? ti.group * p.rows : 0) + m0;
+        const int rows_left = p.rows - m0;  // rows of this half that exist
 #pragma unroll
-        for (int j = 0; j < KPS; ++j)
-          a[c][j] = (r < rows_left && ld.kb + j < ti.kb_end)
-                        ? __ldg(p.sfa + (size_t)(row_base + r) * KB + ld.kb + j)
-                        : 1.0f;
+        for (int c = 0; c < 4; ++c) {
+          const int r = 32 * c + lane;
+#pragma unroll
+          for (int j = 0; j < KPS; ++j)
+            a[h][c][j] = (r < rows_left && ld.kb + j < ti.kb_end)
+                             ? __ldg(p.sfa + (size_t)(row_base + r) * KB + ld.kb + j)
+                             : 1.0f;
+        }
       }
-      // B scale blocks are 128 rows; every tile width divides or is a
-      // multiple of 128, so one value covers each 128-row chunk of the tile.
+      // B scale blocks are 128 rows: the tile's rows touch blocks b0, b0 + 1, ...
       const float* sfb_g = p.sfb + (size_t)ti.group * p.nb128 * KB;
+      const int b0 = ti.n_blk * BLOCK_N / 128;
 #pragma unroll
-      for (int h = 0; h < SFB_CHUNKS; ++h) {
-        const int nb = min((ti.n_blk * BLOCK_N + 128 * h) / 128, p.nb128 - 1);
+      for (int i = 0; i < SFB_BLOCKS; ++i) {
+        const int nb = min(b0 + i, p.nb128 - 1);
 #pragma unroll
         for (int j = 0; j < KPS; ++j)
-          b[h][j] = (ld.kb + j < ti.kb_end) ? __ldg(sfb_g + (size_t)nb * KB + ld.kb + j) : 1.0f;
+          b[i][j] = (ld.kb + j < ti.kb_end) ? __ldg(sfb_g + (size_t)nb * KB + ld.kb + j) : 1.0f;
       }
       ld.next(p, s_prefix, lane);
     };
@@ -642,24 +682,42 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
         ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
         if (!ok) break;
         uint8_t* sf = sSF + s * SF_BYTES;
-        // A scales: TMEM lane l, column c holds row 32c + l of the tile.
-        uint32_t w[4];
+        // A scales: TMEM lane l, column c holds row 32c + l of the half.
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t x = 0x7F7F7F7Fu;  // unused bytes: scale 1
+        for (int h = 0; h < HALVES; ++h) {
+          uint32_t w[4];
 #pragma unroll
-          for (int j = 0; j < KPS; ++j)
-            x = (x & ~(0xFFu << (8 * j))) | (ue8m0(va[slot][c][j]) << (8 * j));
-          w[c] = x;
+          for (int c = 0; c < 4; ++c) {
+            uint32_t x = 0x7F7F7F7Fu;  // unused bytes: scale 1
+#pragma unroll
+            for (int j = 0; j < KPS; ++j)
+              x = (x & ~(0xFFu << (8 * j))) | (ue8m0(va[slot][h][c][j]) << (8 * j));
+            w[c] = x;
+          }
+          *reinterpret_cast<uint4*>(sf + 512 * h + 16 * lane) = make_uint4(w[0], w[1], w[2], w[3]);
         }
-        *reinterpret_cast<uint4*>(sf + 16 * lane) = make_uint4(w[0], w[1], w[2], w[3]);
+        // B scales, same layout per 128-row chunk of the tile's B rows: row
+        // r of the tile takes the scale of its own 128-row block of B
+        const int n_off = (wr.w.ti.n_blk * BLOCK_N) % 128;  // tile start within its block
 #pragma unroll
         for (int h = 0; h < SFB_CHUNKS; ++h) {
-          uint32_t x = 0x7F7F7F7Fu;
+          uint32_t w[4];
 #pragma unroll
-          for (int j = 0; j < KPS; ++j)
-            x = (x & ~(0xFFu << (8 * j))) | (ue8m0(vb[slot][h][j]) << (8 * j));
-          *reinterpret_cast<uint4*>(sf + 512 * (1 + h) + 16 * lane) = make_uint4(x, x, x, x);
+          for (int c = 0; c < 4; ++c) {
+            const int idx = min((n_off + 128 * h + 32 * c + lane) / 128, SFB_BLOCKS - 1);
+            uint32_t x = 0x7F7F7F7Fu;
+#pragma unroll
+            for (int j = 0; j < KPS; ++j) {
+              float v = vb[slot][0][j];
+#pragma unroll
+              for (int i = 1; i < SFB_BLOCKS; ++i)
+                if (idx == i) v = vb[slot][i][j];
+              x = (x & ~(0xFFu << (8 * j))) | (ue8m0(v) << (8 * j));
+            }
+            w[c] = x;
+          }
+          *reinterpret_cast<uint4*>(sf + 512 * (HALVES + h) + 16 * lane) =
+              make_uint4(w[0], w[1], w[2], w[3]);
         }
         ptx::fence_proxy_async_smem();
         __syncwarp();
@@ -702,8 +760,10 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
 
       const int split_col = helpers ? BLOCK_N / 2 : BLOCK_N;
       // staging: in one_tile mode warp w owns tiles [w * NCH_ALL, (w + 1) * NCH_ALL)
-      drain_acc(ti, a, q, 0, split_col,
-                sEpi + (one_tile ? warp * NCH_ALL : q) * 32 * Shape::kEpiPitch, true);
+#pragma unroll
+      for (int h = 0; h < HALVES; ++h)
+        drain_acc(ti, a, h, q, 0, split_col,
+                  sEpi + (one_tile ? warp * NCH_ALL : q) * 32 * Shape::kEpiPitch, true);
       ptx::tc_fence_before_sync();
       ptx::mbar_arrive(&acc_empty[a]);
       ++acc_it;
@@ -722,7 +782,7 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
         ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
         if (ok) {
           ptx::tc_fence_after_sync();
-          drain_acc(ti, 0, warp, BLOCK_N / 2, BLOCK_N,
+          drain_acc(ti, 0, 0, warp, BLOCK_N / 2, BLOCK_N,
                     sEpi + (warp * NCH_ALL + NCH_ALL / 2) * 32 * Shape::kEpiPitch, false);
         }
       }

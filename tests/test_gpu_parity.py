@@ -81,6 +81,26 @@ def test_dense_scale_layout(dg):
     check_close(got, ref, "scale layout")
 
 
+# Every general variant, forced, on one ragged shape with a random power-of-two
+# scale per A row and per B block (the picker would choose only some of them
+# for this shape).  "192:1:1:256:0" is the two-half 256-row tile; its 192-wide
+# column tiles straddle the 128-row scale blocks of B.
+FORCED_GENERAL = ["256:1", "128:1", "64:1", "32:1", "192:1:1:256:0"]
+
+
+@pytest.mark.parametrize("cfg", FORCED_GENERAL)
+def test_dense_forced_variant(dg, cfg, monkeypatch):
+    rng = np.random.default_rng(11)
+    M, N, K = 300, 400, 384
+    p = workloads.dense_problem(M, N, K, seed=7)
+    p.sfa = np.ldexp(1.0, rng.integers(-10, 4, p.sfa.shape)).astype(np.float32)
+    p.sfb = np.ldexp(1.0, rng.integers(-10, 4, p.sfb.shape)).astype(np.float32)
+    monkeypatch.setenv("DG_FORCE_CONFIG", cfg)
+    got = run_dense(dg, p)
+    ref, _ = oracle.default().gemm_nt(p.a, p.sfa, p.b, p.sfb, want_acc=False)
+    check_close(got, ref, f"forced {cfg}")
+
+
 @pytest.mark.parametrize("M,N,K", workloads.DECODE_SHAPES)
 def test_dense_decode_full(dg, M, N, K):
     """The decode-shaped workloads, whole output (split-K path)."""
