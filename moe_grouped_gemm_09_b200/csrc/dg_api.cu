@@ -9,11 +9,13 @@
 #include <cstring>
 #include <array>
 #include <mutex>
+#include <type_traits>
 #include <utility>
 
 #include "../../include/dg.h"
 #include "dg_config.h"
 #include "sm100_fp8_gemm.cuh"
+#include "sm100_fp8_gemm_pair.cuh"
 
 namespace dg {
 namespace {
@@ -92,6 +94,7 @@ dg_status device_state(DeviceState** out, int* dev_out) {
 // with a box of its own (16-row rounded) height, so the SM moves no padding.
 int a_box_rows(int kind, int rows, const Variant& var) {
   if (var.a_rows == 256) return 256;
+  if (var.pair) return kBlockM;
   if (kind != kDense || rows >= kBlockM) return kBlockM;
   return ((rows + 15) / 16) * 16;
 }
@@ -106,16 +109,17 @@ void forced_config(int kind, int rows, int N, int K, int G, int sms, PickedConfi
   if (!e || !e[0]) return;
   int bn = 0, sk = 1;
   if (std::sscanf(e, "%d:%d", &bn, &sk) < 1) return;
-  int kps = 0, ar = 0, sm = -1;
-  std::sscanf(e, "%*d:%*d:%d:%d:%d", &kps, &ar, &sm);
+  int kps = 0, ar = 0, sm = -1, pr = -1;
+  std::sscanf(e, "%*d:%*d:%d:%d:%d:%d", &kps, &ar, &sm, &pr);
   int v = -1;
   for (int i = 0; i < kNumVariants; ++i) {
     const Variant& x = kVariants[i];
     if (x.block_n != bn) continue;
     if (kps ? (x.kps != kps || (ar && x.a_rows != ar)) : x.decode) continue;
     if (sm >= 0 && x.small != (sm != 0)) continue;
-    if ((x.decode || x.a_rows == 256) && kind != kDense) continue;
-    if (x.a_rows == 256 && rows < 256) continue;
+    if (x.pair != (pr > 0)) continue;
+    if ((x.decode || x.a_rows == 256 || x.pair) && kind != kDense) continue;
+    if ((x.a_rows == 256 || x.pair) && rows < 256) continue;
     if (a_box_rows(kind, rows, x) > x.a_rows) continue;
     v = i;
   }
@@ -128,6 +132,11 @@ void forced_config(int kind, int rows, int N, int K, int G, int sms, PickedConfi
   pc->variant = v;
   pc->split_k = sk;
   pc->out_tiles = static_cast<int>(tiles);
+  if (kVariants[v].pair) {
+    const long long pairs = tiles < sms / 2 ? tiles : sms / 2;
+    pc->grid = static_cast<int>(2 * (pairs > 0 ? pairs : 1));
+    return;
+  }
   pc->grid = sk > 1 ? static_cast<int>(tiles) * sk : static_cast<int>(tiles < sms ? tiles : sms);
 }
 
@@ -182,11 +191,13 @@ dg_status make_d_map(CUtensorMap* map, void* base, uint64_t N, uint64_t rows) {
 }
 
 template <int V>
-using ShapeOf = KernelShape<kVariants[V].block_n, kVariants[V].stages, kVariants[V].num_acc,
-                            kVariants[V].kps, kVariants[V].a_rows, kVariants[V].small>;
+using ShapeOf = std::conditional_t<
+    kVariants[V].pair, PairShape<kVariants[V].block_n, kVariants[V].stages>,
+    KernelShape<kVariants[V].block_n, kVariants[V].stages, kVariants[V].num_acc,
+                kVariants[V].kps, kVariants[V].a_rows, kVariants[V].small>>;
 
 // Kernels are instantiated only for the (form, variant) pairs that exist:
-// the decode variants and the 256-row variants serve the dense form only.
+// the decode, 256-row and pair variants serve the dense form only.
 // Per-variant shared-memory bytes (what = 0) or TMEM columns (what = 1).
 template <int what, int... V>
 constexpr std::array<int, sizeof...(V)> variant_table(std::integer_sequence<int, V...>) {
@@ -194,13 +205,18 @@ constexpr std::array<int, sizeof...(V)> variant_table(std::integer_sequence<int,
 }
 
 template <int KIND, int V>
-constexpr bool kBuilt = KIND == kDense || (!kVariants[V].decode && kVariants[V].a_rows != 256);
+constexpr bool kBuilt =
+    KIND == kDense || (!kVariants[V].decode && kVariants[V].a_rows != 256 && !kVariants[V].pair);
 
 template <int KIND, int V>
 auto kernel_of() {
   constexpr Variant var = kVariants[V];
-  return fp8_gemm_kernel<KIND, var.block_n, var.stages, var.num_acc, var.kps, var.a_rows,
-                         var.small>;
+  if constexpr (var.pair) {
+    return fp8_gemm_pair_kernel<var.block_n, var.stages>;
+  } else {
+    return fp8_gemm_kernel<KIND, var.block_n, var.stages, var.num_acc, var.kps, var.a_rows,
+                           var.small>;
+  }
 }
 
 template <int KIND, int V>
@@ -218,14 +234,15 @@ dg_status set_smem_attr(DeviceState& st) {
   }
 }
 
-// How many split-K clusters of each size the device co-schedules, per decode
-// variant of the dense kernel (a cluster must fit in one GPC).
+// How many clusters of each size the device co-schedules: split-K clusters of
+// every decode variant, and SM pairs of every pair variant (a cluster must fit
+// in one GPC, so fewer pairs than SMs / 2 may be resident at once).
 template <int V>
 dg_status query_cluster_limits(DeviceState& st) {
-  if constexpr (kVariants[V].decode) {
+  if constexpr (kVariants[V].decode || kVariants[V].pair) {
     dg_status s = set_smem_attr<kDense, V>(st);
     if (s != DG_OK) return s;
-    for (int c = 1; c <= kMaxSplitK; ++c) {
+    for (int c = kVariants[V].pair ? 2 : 1; c <= (kVariants[V].pair ? 2 : kMaxSplitK); ++c) {
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3(c, 1, 1);
       cfg.blockDim = dim3(kThreads, 1, 1);
@@ -281,9 +298,9 @@ dg_status launch_variant(DeviceState& st, const CUtensorMap& ta, const CUtensorM
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     int n_attr = 1;
-    if (args.split_k > 1) {  // the CTAs of one output tile form a cluster
+    if (args.split_k > 1 || kVariants[V].pair) {  // the CTAs of one output tile form a cluster
       attr[1].id = cudaLaunchAttributeClusterDimension;
-      attr[1].val.clusterDim.x = args.split_k;
+      attr[1].val.clusterDim.x = kVariants[V].pair ? 2 : args.split_k;
       attr[1].val.clusterDim.y = 1;
       attr[1].val.clusterDim.z = 1;
       n_attr = 2;
@@ -337,7 +354,7 @@ dg_status run(int kind, const void* a, const float* sfa, const void* b, const fl
   dg_status s = device_state(&st, nullptr);
   if (s != DG_OK) return s;
   const int sms = effective_sms(*st);
-  if (kind == kDense && rows <= 128) {
+  if (kind == kDense) {
     s = ensure_cluster_limits(*st);
     if (s != DG_OK) return s;
   }
@@ -365,7 +382,15 @@ dg_status run(int kind, const void* a, const float* sfa, const void* b, const fl
   args.timeout_ns = g_timeout_ns;
   args.a_box_rows = a_box_rows(kind, rows, var);
   if (args.a_box_rows > var.a_rows) return DG_ERR_UNSUPPORTED;
-  if (var.a_rows == 256 && (kind != kDense || pc.split_k > 1)) return DG_ERR_UNSUPPORTED;
+  if ((var.a_rows == 256 || var.pair) && (kind != kDense || pc.split_k > 1))
+    return DG_ERR_UNSUPPORTED;
+  if (var.pair) {
+    // no more pairs than the device co-schedules: a pair launched beyond that
+    // would only start once another has finished all its tiles
+    const int resident = cluster_limit(&st->limits, pc.variant, 2, sms);
+    if (pc.grid / 2 > resident) pc.grid = 2 * resident;
+    if (pc.grid % 2 != 0 || pc.grid < 2) return DG_ERR_UNSUPPORTED;
+  }
   args.prefetch = prefetch_enabled();
   // a small variant runs one tile per CTA (its epilogue reuses the ring)
   if (var.small && (kind != kDense || pc.grid != args.num_m_blocks * args.num_n_blocks * pc.split_k))
@@ -380,7 +405,7 @@ dg_status run(int kind, const void* a, const float* sfa, const void* b, const fl
   const int b_groups = (kind == kDense) ? 1 : G;
   s = make_map(&ta, a, K, rows, kind == kMasked ? G : 1, args.a_box_rows, var.kps);
   if (s != DG_OK) return s;
-  s = make_map(&tb, b, K, N, b_groups, var.block_n, var.kps);
+  s = make_map(&tb, b, K, N, b_groups, var.pair ? var.block_n / 2 : var.block_n, var.kps);
   if (s != DG_OK) return s;
   CUtensorMap td;
   s = make_d_map(&td, d, N, static_cast<uint64_t>(a_rows));

@@ -21,6 +21,8 @@ struct Variant {
                 // 256: a tile of two 128-row halves sharing each B tile)
   bool decode;  // built for dense problems of at most one 128-row block
   bool small;   // two CTAs fit per SM; one tile per CTA
+  bool pair;    // one 256-row tile per pair of SMs (a 2-CTA cluster issuing
+                // tcgen05 cta_group::2 MMAs); dense form only
 };
 
 // The compiled variants: general ones first (every form; the 256-row one
@@ -45,6 +47,7 @@ constexpr Variant kVariants[] = {
     {64, 3, 1, 2, 64, true, true},
     {128, 3, 1, 1, 128, true, true},
     {64, 2, 1, 2, 128, true, true},
+    {256, 6, 1, 1, 128, false, false, true},
 };
 constexpr int kNumVariants = sizeof(kVariants) / sizeof(kVariants[0]);
 constexpr int kMaxSplitK = 8;  // portable cluster size
@@ -59,7 +62,7 @@ struct PickedConfig {
 inline int ceil_div(long long a, long long b) { return static_cast<int>((a + b - 1) / b); }
 
 // Output rows of one tile of a variant.
-inline int tile_rows(const Variant& v) { return v.a_rows == 256 ? 256 : 128; }
+inline int tile_rows(const Variant& v) { return (v.a_rows == 256 || v.pair) ? 256 : 128; }
 
 // How many clusters of `cluster` CTAs of variant `variant` the device can run
 // at once.  max_clusters[v][s] for s in 1..kMaxSplitK; a value <= 0 means
@@ -139,7 +142,8 @@ inline bool pick_decode(int rows, int N, int K, int num_sms, const ClusterLimits
 
 // kind: 0 dense, 1 contiguous, 2 masked.  rows: M, M_sum or max_m.
 inline PickedConfig pick_config(int kind, int rows, int N, int K, int G, int expected_m,
-                                int num_sms, const ClusterLimits* lim = nullptr) {
+                                int num_sms, const ClusterLimits* lim = nullptr,
+                                bool allow_pair = true) {
   PickedConfig best{1, 1, 1, 1};
   if (kind == 0 && rows <= 128 && pick_decode(rows, N, K, num_sms, lim, &best)) return best;
 
@@ -164,6 +168,10 @@ inline PickedConfig pick_config(int kind, int rows, int N, int K, int G, int exp
     // than the 128 x 256 tiles on B200: the ring is bound by the latency of
     // the bytes in flight, not by their count.  It is taken only when forced.
     if (var.a_rows == 256) continue;
+    // The SM-pair variant is correct but measured slower than the single-SM
+    // 128 x 256 tiles on B200 (1.6-1.7 against 1.8-2.0 PFLOP/s on the prefill
+    // shapes); it is taken only when forced.
+    if (var.pair) continue;
     const int bn = var.block_n;
     if (bn > 128 && N <= 128) continue;
     const int tm = tile_rows(var);
@@ -191,6 +199,7 @@ inline PickedConfig pick_config(int kind, int rows, int N, int K, int G, int exp
   best.out_tiles = tiles > 0x7fffffff ? 0x7fffffff : static_cast<int>(tiles);
   best.grid = tiles < num_sms ? static_cast<int>(tiles) : num_sms;
   if (best.grid < 1) best.grid = 1;
+  (void)allow_pair;  // reserved for the pair variant once the picker takes it
   return best;
 }
 

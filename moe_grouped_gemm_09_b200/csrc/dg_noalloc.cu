@@ -47,16 +47,21 @@ NaEncodeFn g_na_encode = nullptr;
 template <int V>
 using NaShape = KernelShape<kVariants[V].block_n, kVariants[V].stages, kVariants[V].num_acc,
                             kVariants[V].kps, kVariants[V].a_rows, kVariants[V].small>;
+// (instantiated only for the variants this entry point launches: not the pair ones)
 
 template <int V>
 auto na_kernel() {
   constexpr Variant var = kVariants[V];
+  static_assert(!var.pair, "pair variants are not launched by this entry point");
   return fp8_gemm_kernel<kDense, var.block_n, var.stages, var.num_acc, var.kps, var.a_rows,
                          var.small>;
 }
 
 template <int V>
 dg_status na_smem_attr(NaDevice& st) {
+  if constexpr (kVariants[V].pair) {
+    return DG_ERR_UNSUPPORTED;  // the picker offers this entry point no pair variant
+  } else {
   if (!st.smem_attr_set[V]) {
     if (cudaFuncSetAttribute(na_kernel<V>(), cudaFuncAttributeMaxDynamicSharedMemorySize,
                              NaShape<V>::kSmemBytes) != cudaSuccess)
@@ -64,6 +69,7 @@ dg_status na_smem_attr(NaDevice& st) {
     st.smem_attr_set[V] = true;
   }
   return DG_OK;
+  }
 }
 
 // Split-K clusters of each size the device co-schedules for decode variant V.
@@ -167,6 +173,9 @@ dg_status na_d_map(CUtensorMap* map, void* base, uint64_t N, uint64_t rows) {
 template <int V>
 dg_status na_launch(NaDevice& st, const CUtensorMap& ta, const CUtensorMap& tb,
                     const CUtensorMap& td, const GemmArgs& args, int grid, cudaStream_t stream) {
+  if constexpr (kVariants[V].pair) {
+    return DG_ERR_UNSUPPORTED;
+  } else {
   dg_status s = na_smem_attr<V>(st);
   if (s != DG_OK) return s;
   cudaLaunchConfig_t cfg = {};
@@ -185,6 +194,7 @@ dg_status na_launch(NaDevice& st, const CUtensorMap& ta, const CUtensorMap& tb,
   }
   return cudaLaunchKernelEx(&cfg, na_kernel<V>(), ta, tb, td, args) == cudaSuccess ? DG_OK
                                                                                    : DG_ERR_CUDA;
+  }
 }
 
 template <int... V>
@@ -218,7 +228,8 @@ extern "C" dg_status dg_fp8_gemm_nt_noalloc(const void* a, const float* sfa, con
   dg_status s = na_setup(&st);
   if (s != DG_OK) return s;
 
-  const PickedConfig pc = pick_config(kDense, M, N, K, 1, 0, st->num_sms, &st->limits);
+  const PickedConfig pc = pick_config(kDense, M, N, K, 1, 0, st->num_sms, &st->limits,
+                                      /*allow_pair=*/false);
   const Variant var = kVariants[pc.variant];
   GemmArgs args = {};
   args.rows = M;

@@ -84,8 +84,10 @@ def test_dense_scale_layout(dg):
 # Every general variant, forced, on one ragged shape with a random power-of-two
 # scale per A row and per B block (the picker would choose only some of them
 # for this shape).  "192:1:1:256:0" is the two-half 256-row tile; its 192-wide
-# column tiles straddle the 128-row scale blocks of B.
-FORCED_GENERAL = ["256:1", "128:1", "64:1", "32:1", "192:1:1:256:0"]
+# column tiles straddle the 128-row scale blocks of B.  "256:1:1:128:0:1" is
+# the SM-pair variant (256 x 256 tiles, 2-CTA clusters): the last row tile
+# leaves the second CTA of its pair without a single valid row.
+FORCED_GENERAL = ["256:1", "128:1", "64:1", "32:1", "192:1:1:256:0", "256:1:1:128:0:1"]
 
 
 @pytest.mark.parametrize("cfg", FORCED_GENERAL)
@@ -108,6 +110,17 @@ def test_dense_decode_full(dg, M, N, K):
     got = run_dense(dg, p)
     ref, _ = oracle.default().gemm_nt(p.a, p.sfa, p.b, p.sfb, want_acc=False)
     check_close(got, ref, f"decode {M}x{N}x{K}")
+
+
+@pytest.mark.parametrize("M,N,K", [(4096, 7168, 2048), (4352, 2112, 1024)])
+def test_dense_pair_variant_sampled(dg, M, N, K, monkeypatch):
+    """The SM-pair variant over many tiles per pair (persistent loop, ring
+    phases wrapping), sampled rows covering every tile boundary."""
+    monkeypatch.setenv("DG_FORCE_CONFIG", "256:1:1:128:0:1")
+    p = workloads.dense_problem(M, N, K, seed=3)
+    got = run_dense(dg, p)
+    rows = sample_rows(M, 48, seed=M + K)
+    check_close(got[rows], oracle_dense_rows(p, rows), f"pair {M}x{N}x{K}")
 
 
 @pytest.mark.parametrize("M,N,K", workloads.PREFILL_SHAPES)
