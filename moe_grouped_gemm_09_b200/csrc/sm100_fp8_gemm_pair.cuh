@@ -23,10 +23,11 @@
 // shared-memory offsets in both CTAs):
 //  * full[s] (leader's only): the leader's producer arrives with the whole
 //    stage's transaction bytes (both CTAs), both CTAs' TMA loads complete on
-//    it (cta_group::2 form, no multicast), and both CTAs' scale warps arrive
+//    it (cta_group::2 form; each CTA loads its own boxes), and both CTAs'
+//    scale warps arrive
 //    after writing their UE8M0 words (the peer remotely);
-//  * empty[s] (both): the leader's MMA commit arrives on both (multicast);
-//  * acc_full (both): the leader's commit at the end of a tile, on both;
+//  * empty[s] (both): the leader's MMA warp commits once to each CTA's;
+//  * acc_full (both): the leader's commits at the end of a tile, one each;
 //  * acc_empty (leader's): one arrive per epilogue warp of both CTAs.
 // Scale factors: each CTA's scale warp writes the SFA words of its 128 rows
 // and the SFB words of all 256 B rows of the tile; the leader's
@@ -80,7 +81,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int TMEM_COLS = Shape::kTmemCols;
   constexpr int B_HALF = Shape::kBHalf;
   constexpr int TILE_M = Shape::kTileM;
-  constexpr uint16_t kPairMask = 0x3;
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = ptx::smem_addr(smem_raw);
@@ -139,6 +139,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   };
   // the leader's copy of a barrier, as a cluster address
   auto leader_bar = [&](uint64_t* bar) { return ptx::map_shared_rank(ptx::smem_addr(bar), 0); };
+  // MMA completion, signalled on the barrier at this offset in both CTAs
+  auto commit_both = [&](uint64_t* bar) {
+    ptx::tc_commit_pair(ptx::map_shared_rank(ptx::smem_addr(bar), 0));
+    ptx::tc_commit_pair(ptx::map_shared_rank(ptx::smem_addr(bar), 1));
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer --
@@ -199,17 +204,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int ks = 0; ks < kBlockK / 32; ++ks)
               ptx::tc_mma_pair_mxf8_block_scale(tmem_base, da + 2 * ks, db + 2 * ks, idesc,
                                                 sfa_tmem, sfb_tmem, kb > 0 || ks > 0);
-            ptx::tc_commit_pair_mc(&empty[s], kPairMask);
+            commit_both(&empty[s]);
           }
           __syncwarp();
         }
         if (!ok) break;
-        if (lane == 0) ptx::tc_commit_pair_mc(acc_full, kPairMask);
+        if (lane == 0) commit_both(acc_full);
         __syncwarp();
       }
       // every MMA this thread issued has completed once `drain` flips
       if (lane == 0) {
-        ptx::tc_commit_pair_mc(drain, 0x1);
+        ptx::tc_commit_pair(ptx::map_shared_rank(ptx::smem_addr(drain), 0));
         ptx::mbar_wait_drain(drain, 0, 50000000ull);
       }
       __syncwarp();

@@ -143,7 +143,8 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, u
 // The same load issued by each CTA of an MMA pair (tcgen05 cta_group::2): the
 // box lands in this CTA's shared memory and completes on `bar_cluster`, an
 // mbarrier of either CTA of the pair (map_shared_rank), so that the pair's
-// leader sees both halves of a stage on one barrier.  No multicast.
+// leader sees both halves of a stage on one barrier.  Each CTA loads only its
+// own box.
 __device__ __forceinline__ void tma_load_4d_pair(void* dst, const CUtensorMap* map,
                                                  uint32_t bar_cluster, int c0, int c1, int c2,
                                                  int c3) {
@@ -315,14 +316,12 @@ __device__ __forceinline__ void tc_commit(uint64_t* bar) {
 }
 
 // Pair form of tc_commit, issued by the pair's leader: arrive on the mbarrier
-// at this shared-memory offset in every CTA of `cta_mask` once all tcgen05
-// operations issued so far have completed.
-__device__ __forceinline__ void tc_commit_pair_mc(uint64_t* bar, uint16_t cta_mask) {
-  asm volatile(
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
-      " [%0], %1;" ::"r"(smem_addr(bar)),
-      "h"(cta_mask)
-      : "memory");
+// at cluster address `bar_cluster` (this CTA's or the peer's, from
+// map_shared_rank) once all tcgen05 operations issued so far have completed.
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar_cluster) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar_cluster)
+               : "memory");
 }
 
 // Pair form of tc_cp_32x128b_warpx4, issued by the leader: each CTA of the
