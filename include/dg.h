@@ -81,6 +81,25 @@ typedef enum {
 dg_status dg_fp8_gemm_nt(const void* a, const float* sfa, const void* b, const float* sfb,
                          void* d, int M, int N, int K, dg_stream_t stream);
 
+/* The dense GEMM with other operand layouts (DeepGEMM project card,
+ * aiproducthub.cn, "core features": NT / TN / NN / TT layouts on SM100).  The
+ * first letter is A's layout, the second B's; "n" for A and "t" for B are
+ * the K-major layouts of dg_fp8_gemm_nt:
+ *   nn: a [M,K] (K-major),  b [K,N] (N-major: the element of row n and
+ *       column k of B at b[k*N + n])
+ *   tn: a [K,M] (M-major: a[k*M + m]),  b [K,N] (N-major)
+ *   tt: a [K,M] (M-major),  b [N,K] (K-major)
+ * D[M,N] = A * B^T in every case, with the scales, D and all other rules of
+ * dg_fp8_gemm_nt (sfa [M, K/128], sfb [ceil(N/128), K/128], d [M,N] BF16).
+ * An M-major A needs M % 16 == 0 (its rows of M bytes are 16-byte units);
+ * otherwise DG_ERR_INVALID_ARG. */
+dg_status dg_fp8_gemm_nn(const void* a, const float* sfa, const void* b, const float* sfb,
+                         void* d, int M, int N, int K, dg_stream_t stream);
+dg_status dg_fp8_gemm_tn(const void* a, const float* sfa, const void* b, const float* sfb,
+                         void* d, int M, int N, int K, dg_stream_t stream);
+dg_status dg_fp8_gemm_tt(const void* a, const float* sfa, const void* b, const float* sfb,
+                         void* d, int M, int N, int K, dg_stream_t stream);
+
 /* M-grouped GEMM, contiguous layout (MoE experts' tokens concatenated along M).
  * a [M_sum,K], sfa [M_sum,K/128], b [G,N,K], sfb [G,ceil(N/128),K/128],
  * d [M_sum,N], m_indices int32 [M_sum] (device): the expert of row r, or -1

@@ -41,6 +41,9 @@ def _decl(name, args, res=ctypes.c_int):
 
 
 _gemm_nt = _decl("dg_fp8_gemm_nt", [_P, _P, _P, _P, _P, _I, _I, _I, _P])
+_gemm_nn = _decl("dg_fp8_gemm_nn", [_P, _P, _P, _P, _P, _I, _I, _I, _P])
+_gemm_tn = _decl("dg_fp8_gemm_tn", [_P, _P, _P, _P, _P, _I, _I, _I, _P])
+_gemm_tt = _decl("dg_fp8_gemm_tt", [_P, _P, _P, _P, _P, _I, _I, _I, _P])
 _gemm_contig = _decl("dg_m_grouped_fp8_gemm_nt_contiguous", [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P])
 _gemm_masked = _decl("dg_m_grouped_fp8_gemm_nt_masked", [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P])
 _set_num_sms = _decl("dg_set_num_sms", [_I])
@@ -63,7 +66,8 @@ _query = _decl("dg_query_config", [_I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(Dg
 EXPORTED_SYMBOLS = ("dg_fp8_gemm_nt", "dg_m_grouped_fp8_gemm_nt_contiguous",
                     "dg_m_grouped_fp8_gemm_nt_masked", "dg_set_num_sms", "dg_get_num_sms",
                     "dg_get_last_device_error", "dg_set_wait_timeout_ms", "dg_status_string",
-                    "dg_query_config", "dg_version", "dg_fp8_gemm_nt_noalloc")
+                    "dg_query_config", "dg_version", "dg_fp8_gemm_nt_noalloc", "dg_fp8_gemm_nn",
+                    "dg_fp8_gemm_tn", "dg_fp8_gemm_tt")
 
 DEVICE_ERRORS = {
     0x101: "wait timeout in the TMA producer",
@@ -136,6 +140,42 @@ def fp8_gemm_nt(a: torch.Tensor, sfa: torch.Tensor, b: torch.Tensor, sfb: torch.
         _check(_gemm_nt(a.data_ptr(), sfa.data_ptr(), b.data_ptr(), sfb.data_ptr(), d.data_ptr(),
                         M, N, K, _stream_ptr(dev)), "dg_fp8_gemm_nt")
     return d
+
+
+def _gemm_layout(name, fn, a_m_major: bool, b_n_major: bool, a, sfa, b, sfb, d):
+    _fp8_bytes(a, "a"); _fp8_bytes(b, "b")
+    K, M = a.shape if a_m_major else a.shape[::-1]
+    N = b.shape[1] if b_n_major else b.shape[0]
+    dev = a.device
+    _need(a, "a", None, (K, M) if a_m_major else (M, K), dev)
+    _need(b, "b", None, (K, N) if b_n_major else (N, K), dev)
+    _need(sfa, "sfa", torch.float32, (M, K // 128), dev)
+    _need(sfb, "sfb", torch.float32, ((N + 127) // 128, K // 128), dev)
+    if d is None:
+        d = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    _need(d, "d", torch.bfloat16, (M, N), dev)
+    with torch.cuda.device(dev):
+        _check(fn(a.data_ptr(), sfa.data_ptr(), b.data_ptr(), sfb.data_ptr(), d.data_ptr(),
+                  M, N, K, _stream_ptr(dev)), name)
+    return d
+
+
+def fp8_gemm_nn(a, sfa, b, sfb, d=None):
+    """``D[M,N] = A B^T`` with A ``[M, K]`` (K-major) and B given N-major as
+    ``b [K, N]``; scales and D as in :func:`fp8_gemm_nt`."""
+    return _gemm_layout("dg_fp8_gemm_nn", _gemm_nn, False, True, a, sfa, b, sfb, d)
+
+
+def fp8_gemm_tn(a, sfa, b, sfb, d=None):
+    """``D[M,N] = A B^T`` with A given M-major as ``a [K, M]`` (M % 16 == 0) and
+    B N-major as ``b [K, N]``."""
+    return _gemm_layout("dg_fp8_gemm_tn", _gemm_tn, True, True, a, sfa, b, sfb, d)
+
+
+def fp8_gemm_tt(a, sfa, b, sfb, d=None):
+    """``D[M,N] = A B^T`` with A given M-major as ``a [K, M]`` (M % 16 == 0) and
+    B ``[N, K]`` (K-major)."""
+    return _gemm_layout("dg_fp8_gemm_tt", _gemm_tt, True, False, a, sfa, b, sfb, d)
 
 
 def fp8_gemm_nt_noalloc(a: torch.Tensor, sfa: torch.Tensor, b: torch.Tensor, sfb: torch.Tensor,

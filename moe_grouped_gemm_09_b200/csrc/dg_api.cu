@@ -26,7 +26,7 @@ struct DeviceState {
   bool ready = false;
   int num_sms = 0;
   int* error_word = nullptr;      // one int, device memory
-  bool smem_attr_set[3][kNumVariants] = {};
+  bool smem_attr_set[6][kNumVariants] = {};  // per form (below) and variant
   bool limits_known = false;
   ClusterLimits limits = {};      // co-resident split-K clusters per variant and size
 };
@@ -190,6 +190,33 @@ dg_status make_d_map(CUtensorMap* map, void* base, uint64_t N, uint64_t rows) {
   return r == CUDA_SUCCESS ? DG_OK : DG_ERR_CUDA;
 }
 
+// Launch forms: the three GEMM forms, then the dense form with M-major A
+// and/or N-major B (the forms differ in their kernel instantiation).
+enum Form : int { kFormDense = 0, kFormContiguous = 1, kFormMasked = 2, kFormNN = 3, kFormTN = 4,
+                  kFormTT = 5 };
+constexpr int kind_of_form(int f) { return f < 3 ? f : kDense; }
+constexpr int layout_of_form(int f) {
+  return f == kFormNN ? kLayoutNN : f == kFormTN ? kLayoutTN : f == kFormTT ? kLayoutTT : kLayoutNT;
+}
+// Variants that serve M-/N-major operands: general ones with 128-column B boxes.
+constexpr bool mn_capable(const Variant& v) {
+  return !v.decode && !v.small && !v.pair && v.kps == 1 && v.a_rows == 128 && v.block_n % 128 == 0;
+}
+
+// 2-D tensor map over an M-/N-major operand stored as [K, mn] bytes (mn
+// contiguous), boxes of 128 mn bytes x 128 K rows with the 128-byte swizzle.
+dg_status make_map_mn(CUtensorMap* map, const void* base, uint64_t mn, uint64_t K) {
+  cuuint64_t dims[2] = {mn, K};
+  cuuint64_t strides[1] = {mn};
+  cuuint32_t box[2] = {128, 128};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? DG_OK : DG_ERR_CUDA;
+}
+
 template <int V>
 using ShapeOf = std::conditional_t<
     kVariants[V].pair, PairShape<kVariants[V].block_n, kVariants[V].stages>,
@@ -204,18 +231,21 @@ constexpr std::array<int, sizeof...(V)> variant_table(std::integer_sequence<int,
   return {(what == 0 ? ShapeOf<V>::kSmemBytes : ShapeOf<V>::kTmemCols)...};
 }
 
-template <int KIND, int V>
+template <int FORM, int V>
 constexpr bool kBuilt =
-    KIND == kDense || (!kVariants[V].decode && kVariants[V].a_rows != 256 && !kVariants[V].pair);
+    FORM == kFormDense ||
+    ((FORM == kFormContiguous || FORM == kFormMasked) && !kVariants[V].decode &&
+     kVariants[V].a_rows != 256 && !kVariants[V].pair) ||
+    (FORM >= kFormNN && mn_capable(kVariants[V]));
 
-template <int KIND, int V>
+template <int FORM, int V>
 auto kernel_of() {
   constexpr Variant var = kVariants[V];
   if constexpr (var.pair) {
     return fp8_gemm_pair_kernel<var.block_n, var.stages>;
   } else {
-    return fp8_gemm_kernel<KIND, var.block_n, var.stages, var.num_acc, var.kps, var.a_rows,
-                           var.small>;
+    return fp8_gemm_kernel<kind_of_form(FORM), var.block_n, var.stages, var.num_acc, var.kps,
+                           var.a_rows, var.small, layout_of_form(FORM)>;
   }
 }
 
@@ -329,9 +359,12 @@ dg_status launch(DeviceState& st, int variant, const CUtensorMap& ta, const CUte
 }
 
 // Shared path of the three GEMM forms.
-dg_status run(int kind, const void* a, const float* sfa, const void* b, const float* sfb,
+dg_status run(int form, const void* a, const float* sfa, const void* b, const float* sfb,
               void* d, const int* m_indices, const int* masked_m, int rows, int N, int K, int G,
               int expected_m, cudaStream_t stream) {
+  const int kind = kind_of_form(form);
+  const int layout = layout_of_form(form);
+  const bool a_mn = (layout & 1) != 0, b_mn = (layout & 2) != 0;
   // ---- argument checks (no device work) ----
   if (rows < 0 || G < 0) return DG_ERR_INVALID_ARG;
   if (K <= 0 || K % 128 != 0 || N <= 0 || N % 16 != 0) return DG_ERR_INVALID_ARG;
@@ -342,6 +375,7 @@ dg_status run(int kind, const void* a, const float* sfa, const void* b, const fl
     return DG_ERR_INVALID_ARG;
   if (kind == kContiguous && (!m_indices || !aligned(m_indices, 4) || rows % 128 != 0))
     return DG_ERR_INVALID_ARG;
+  if (a_mn && rows % 16 != 0) return DG_ERR_INVALID_ARG;  // [K, M] rows of whole 16-byte units
   if (kind == kMasked && (!masked_m || !aligned(masked_m, 4))) return DG_ERR_INVALID_ARG;
   if (kind == kMasked && G > kMaxMaskedGroups) return DG_ERR_UNSUPPORTED;
   const long long a_rows = (kind == kMasked) ? static_cast<long long>(G) * rows : rows;
@@ -358,9 +392,11 @@ dg_status run(int kind, const void* a, const float* sfa, const void* b, const fl
     s = ensure_cluster_limits(*st);
     if (s != DG_OK) return s;
   }
-  PickedConfig pc = pick_config(kind, rows, N, K, G, expected_m, sms, &st->limits);
+  PickedConfig pc = pick_config(kind, rows, N, K, G, expected_m, sms, &st->limits,
+                                /*allow_pair=*/true, /*mn_operands=*/layout != kLayoutNT);
   forced_config(kind, rows, N, K, G, sms, &pc);
   const Variant var = kVariants[pc.variant];
+  if (layout != kLayoutNT && (!mn_capable(var) || pc.split_k > 1)) return DG_ERR_UNSUPPORTED;
 
   GemmArgs args = {};
   args.rows = rows;
@@ -380,7 +416,7 @@ dg_status run(int kind, const void* a, const float* sfa, const void* b, const fl
   args.masked_m = masked_m;
   args.error_word = st->error_word;
   args.timeout_ns = g_timeout_ns;
-  args.a_box_rows = a_box_rows(kind, rows, var);
+  args.a_box_rows = a_mn ? kBlockM : a_box_rows(kind, rows, var);
   if (args.a_box_rows > var.a_rows) return DG_ERR_UNSUPPORTED;
   if ((var.a_rows == 256 || var.pair) && (kind != kDense || pc.split_k > 1))
     return DG_ERR_UNSUPPORTED;
@@ -403,9 +439,11 @@ dg_status run(int kind, const void* a, const float* sfa, const void* b, const fl
 
   CUtensorMap ta, tb;
   const int b_groups = (kind == kDense) ? 1 : G;
-  s = make_map(&ta, a, K, rows, kind == kMasked ? G : 1, args.a_box_rows, var.kps);
+  s = a_mn ? make_map_mn(&ta, a, rows, K)
+           : make_map(&ta, a, K, rows, kind == kMasked ? G : 1, args.a_box_rows, var.kps);
   if (s != DG_OK) return s;
-  s = make_map(&tb, b, K, N, b_groups, var.pair ? var.block_n / 2 : var.block_n, var.kps);
+  s = b_mn ? make_map_mn(&tb, b, N, K)
+           : make_map(&tb, b, K, N, b_groups, var.pair ? var.block_n / 2 : var.block_n, var.kps);
   if (s != DG_OK) return s;
   CUtensorMap td;
   s = make_d_map(&td, d, N, static_cast<uint64_t>(a_rows));
@@ -418,11 +456,15 @@ dg_status run(int kind, const void* a, const float* sfa, const void* b, const fl
                  kind, rows, N, K, G, expected_m, var.block_n, var.stages, var.num_acc,
                  pc.split_k, pc.grid);
 
-  switch (kind) {
-    case kDense: return launch<kDense>(*st, pc.variant, ta, tb, td, args, pc.grid, stream);
-    case kContiguous:
-      return launch<kContiguous>(*st, pc.variant, ta, tb, td, args, pc.grid, stream);
-    default: return launch<kMasked>(*st, pc.variant, ta, tb, td, args, pc.grid, stream);
+  switch (form) {
+    case kFormDense: return launch<kFormDense>(*st, pc.variant, ta, tb, td, args, pc.grid, stream);
+    case kFormContiguous:
+      return launch<kFormContiguous>(*st, pc.variant, ta, tb, td, args, pc.grid, stream);
+    case kFormMasked:
+      return launch<kFormMasked>(*st, pc.variant, ta, tb, td, args, pc.grid, stream);
+    case kFormNN: return launch<kFormNN>(*st, pc.variant, ta, tb, td, args, pc.grid, stream);
+    case kFormTN: return launch<kFormTN>(*st, pc.variant, ta, tb, td, args, pc.grid, stream);
+    default: return launch<kFormTT>(*st, pc.variant, ta, tb, td, args, pc.grid, stream);
   }
 }
 
@@ -435,7 +477,25 @@ extern "C" {
 
 dg_status dg_fp8_gemm_nt(const void* a, const float* sfa, const void* b, const float* sfb,
                          void* d, int M, int N, int K, dg_stream_t stream) {
-  return run(kDense, a, sfa, b, sfb, d, nullptr, nullptr, M, N, K, 1, 0,
+  return run(kFormDense, a, sfa, b, sfb, d, nullptr, nullptr, M, N, K, 1, 0,
+             reinterpret_cast<cudaStream_t>(stream));
+}
+
+dg_status dg_fp8_gemm_nn(const void* a, const float* sfa, const void* b, const float* sfb,
+                         void* d, int M, int N, int K, dg_stream_t stream) {
+  return run(kFormNN, a, sfa, b, sfb, d, nullptr, nullptr, M, N, K, 1, 0,
+             reinterpret_cast<cudaStream_t>(stream));
+}
+
+dg_status dg_fp8_gemm_tn(const void* a, const float* sfa, const void* b, const float* sfb,
+                         void* d, int M, int N, int K, dg_stream_t stream) {
+  return run(kFormTN, a, sfa, b, sfb, d, nullptr, nullptr, M, N, K, 1, 0,
+             reinterpret_cast<cudaStream_t>(stream));
+}
+
+dg_status dg_fp8_gemm_tt(const void* a, const float* sfa, const void* b, const float* sfb,
+                         void* d, int M, int N, int K, dg_stream_t stream) {
+  return run(kFormTT, a, sfa, b, sfb, d, nullptr, nullptr, M, N, K, 1, 0,
              reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -443,7 +503,7 @@ dg_status dg_m_grouped_fp8_gemm_nt_contiguous(const void* a, const float* sfa, c
                                               const float* sfb, void* d, const int* m_indices,
                                               int M_sum, int N, int K, int G,
                                               dg_stream_t stream) {
-  return run(kContiguous, a, sfa, b, sfb, d, m_indices, nullptr, M_sum, N, K, G, 0,
+  return run(kFormContiguous, a, sfa, b, sfb, d, m_indices, nullptr, M_sum, N, K, G, 0,
              reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -451,7 +511,7 @@ dg_status dg_m_grouped_fp8_gemm_nt_masked(const void* a, const float* sfa, const
                                           const float* sfb, void* d, const int* masked_m, int G,
                                           int max_m, int N, int K, int expected_m,
                                           dg_stream_t stream) {
-  return run(kMasked, a, sfa, b, sfb, d, nullptr, masked_m, max_m, N, K, G, expected_m,
+  return run(kFormMasked, a, sfa, b, sfb, d, nullptr, masked_m, max_m, N, K, G, expected_m,
              reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -143,9 +143,11 @@ inline bool pick_decode(int rows, int N, int K, int num_sms, const ClusterLimits
 // kind: 0 dense, 1 contiguous, 2 masked.  rows: M, M_sum or max_m.
 inline PickedConfig pick_config(int kind, int rows, int N, int K, int G, int expected_m,
                                 int num_sms, const ClusterLimits* lim = nullptr,
-                                bool allow_pair = true) {
+                                bool allow_pair = true, bool mn_operands = false) {
   PickedConfig best{1, 1, 1, 1};
-  if (kind == 0 && rows <= 128 && pick_decode(rows, N, K, num_sms, lim, &best)) return best;
+  if (kind == 0 && rows <= 128 && !mn_operands &&
+      pick_decode(rows, N, K, num_sms, lim, &best))
+    return best;
 
   // Everything else: persistent CTAs, no split.  Tile time is set by the
   // bytes the SM must pull through TMA per K block (A 16 KB + B BLOCK_N x
@@ -163,6 +165,8 @@ inline PickedConfig pick_config(int kind, int rows, int N, int K, int G, int exp
   for (int v = 0; v < kNumVariants; ++v) {
     const Variant& var = kVariants[v];
     if (var.small || var.a_rows < 128) continue;
+    // M-/N-major operands: one K block per stage and whole 128-column B boxes
+    if (mn_operands && (var.decode || var.kps != 1 || var.block_n % 128 != 0)) continue;
     if (var.decode && (kind != 0 || var.kps != 2 || var.block_n != 256)) continue;
     // The 256-row variant (fewer operand bytes per FLOP) measured no faster
     // than the 128 x 256 tiles on B200: the ring is bound by the latency of

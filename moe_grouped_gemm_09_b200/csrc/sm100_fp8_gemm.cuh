@@ -27,12 +27,14 @@
 //    store.
 //  * Split-K (decode shapes, too few output tiles for the SMs): the CTAs that
 //    share an output tile form one thread-block cluster, each computes the
-//    partial sum of its K slice, parks it in its own shared memory, and after
-//    a cluster barrier every CTA reduces a slice of the rows by reading the
-//    partials of all CTAs through distributed shared memory, in a fixed
-//    order (deterministic), then stores BF16.  No global scratch is used.
+//    partial sum of its K slice and parks it in its own shared memory; after
+//    a cluster barrier every CTA pushes the rows each other CTA owns to that
+//    CTA with one bulk copy (distributed shared memory), and every CTA sums
+//    the partials of its own rows in a fixed order (deterministic), then
+//    stores BF16.  No global scratch is used.
 //  * Before waiting on the previous kernel (programmatic dependent launch),
 //    the producer asks TMA to prefetch its first tile's operands into L2.
+//  * A single-tile CTA (decode) drains its accumulator with all eight warps.
 //  * Persistent CTAs walk a static tile sequence.  For the grouped layouts the
 //    sequence is group-aware: contiguous tiles read their expert from
 //    m_indices and skip all-padding blocks; masked tiles are enumerated over
@@ -48,6 +50,11 @@
 namespace dg {
 
 enum GemmKind : int { kDense = 0, kContiguous = 1, kMasked = 2 };
+
+// Operand layouts of the dense form (DeepGEMM project card, core features:
+// NT / NN / TN / TT on SM100).  Bit 0: A is M-major ([K, M] in memory);
+// bit 1: B is N-major ([K, N]).  NT, both K-major, is the grouped forms' only one.
+enum GemmLayout : int { kLayoutNT = 0, kLayoutTT = 1, kLayoutNN = 2, kLayoutTN = 3 };
 
 // Device error codes (also the values reported through the C ABI).
 enum DeviceError : int {
@@ -289,7 +296,8 @@ struct StageWalker {
   }
 };
 
-template <int KIND, int BLOCK_N, int STAGES, int NUM_ACC, int KPS, int A_ROWS, bool SMALL>
+template <int KIND, int BLOCK_N, int STAGES, int NUM_ACC, int KPS, int A_ROWS, bool SMALL,
+          int LAYOUT = kLayoutNT>
 __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     const __grid_constant__ CUtensorMap tmap_b,
@@ -313,6 +321,14 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
                 "split-K partial must fit in the operand ring");
   static_assert((KPS == 1 && !SMALL) || KIND == kDense, "decode variants serve the dense form");
   static_assert(HALVES == 1 || KIND == kDense, "a 256-row tile could straddle two groups");
+  // M-major A / N-major B: 2-D maps over [K, M] / [K, N] with boxes of 128
+  // MN bytes x 128 K rows; one K block per stage, whole 128-row A boxes, and B
+  // tiles made of whole 128-column boxes.
+  constexpr bool A_MN = (LAYOUT & 1) != 0;
+  constexpr bool B_MN = (LAYOUT & 2) != 0;
+  static_assert(LAYOUT == kLayoutNT ||
+                    (KIND == kDense && KPS == 1 && A_ROWS == 128 && !SMALL && BLOCK_N % 128 == 0),
+                "M-/N-major operands: dense form, general variants with 128-column B boxes");
 
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment for the 128-byte-swizzled operand tiles
@@ -375,8 +391,17 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
     if (lane == 0) {
       const int kb_end = SMALL ? ti.kb_end : min(ti.kb_end, ti.kb_begin + STAGES * KPS);
       for (int kb = ti.kb_begin; kb < kb_end; kb += KPS) {
-        ptx::tma_prefetch_l2_4d(&tmap_b, 0, ti.n_blk * BLOCK_N, kb, 0);
-        if (!SMALL) ptx::tma_prefetch_l2_4d(&tmap_a, 0, ti.m_blk * TILE_M, kb, 0);
+        if constexpr (B_MN) {
+          for (int h = 0; h < BLOCK_N / 128; ++h)
+            ptx::tma_prefetch_l2_2d(&tmap_b, ti.n_blk * BLOCK_N + 128 * h, kb * kBlockK);
+        } else {
+          ptx::tma_prefetch_l2_4d(&tmap_b, 0, ti.n_blk * BLOCK_N, kb, 0);
+        }
+        if constexpr (A_MN) {
+          ptx::tma_prefetch_l2_2d(&tmap_a, ti.m_blk * TILE_M, kb * kBlockK);
+        } else {
+          if (!SMALL) ptx::tma_prefetch_l2_4d(&tmap_a, 0, ti.m_blk * TILE_M, kb, 0);
+        }
       }
     }
   }
@@ -537,9 +562,21 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
             // 128-row MMA then reads stale shared memory for the other rows,
             // which only feeds accumulator rows that are never stored.
             ptx::mbar_arrive_expect_tx(&full[s], KPS * (p.a_box_rows + BLOCK_N) * kBlockK);
-            ptx::tma_load_4d(sA + s * A_BYTES, &tmap_a, &full[s], 0, a_row, kb, a_grp);
-            ptx::tma_load_4d(sB + s * B_BYTES, &tmap_b, &full[s], 0, ti.n_blk * BLOCK_N, kb,
-                             ti.group);
+            if constexpr (A_MN) {
+              ptx::tma_load_2d(sA + s * A_BYTES, &tmap_a, &full[s], a_row, kb * kBlockK);
+            } else {
+              ptx::tma_load_4d(sA + s * A_BYTES, &tmap_a, &full[s], 0, a_row, kb, a_grp);
+            }
+            if constexpr (B_MN) {
+              // 128-column blocks of the tile, 128 x 128 bytes each
+#pragma unroll
+              for (int h = 0; h < BLOCK_N / 128; ++h)
+                ptx::tma_load_2d(sB + s * B_BYTES + h * 128 * kBlockK, &tmap_b, &full[s],
+                                 ti.n_blk * BLOCK_N + 128 * h, kb * kBlockK);
+            } else {
+              ptx::tma_load_4d(sB + s * B_BYTES, &tmap_b, &full[s], 0, ti.n_blk * BLOCK_N, kb,
+                               ti.group);
+            }
           }
         }
         ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
@@ -553,7 +590,7 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer --
-    constexpr uint32_t idesc = ptx::idesc_mxf8_e4m3_ue8m0(kBlockM, BLOCK_N);
+    constexpr uint32_t idesc = ptx::idesc_mxf8_e4m3_ue8m0(kBlockM, BLOCK_N, A_MN, B_MN);
     int it = 0, acc_it = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
@@ -593,17 +630,26 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
             if (kb + j >= ti.kb_end) break;
             // K block j of the stage: its scale factors are byte j of every
             // TMEM scale word (selected by the scale-factor id)
-            const uint64_t db = ptx::sdesc_kmajor_sw128(b_base + j * BLOCK_N * kBlockK);
+            // a K step of 32 moves 32 bytes along a K-major row, or 4 swizzle
+            // atoms (4096 bytes) down an M-/N-major tile
+            constexpr uint32_t kStepA = A_MN ? 4096 >> 4 : 32 >> 4;
+            constexpr uint32_t kStepB = B_MN ? 4096 >> 4 : 32 >> 4;
+            const uint64_t db =
+                B_MN ? ptx::sdesc_mnmajor_sw128(b_base, 128 * kBlockK)
+                     : ptx::sdesc_kmajor_sw128(b_base + j * BLOCK_N * kBlockK);
             const uint32_t id = idesc | (static_cast<uint32_t>(j) << 29) | (static_cast<uint32_t>(j) << 4);
             const uint32_t byte_sel = static_cast<uint32_t>(j) << 30;
 #pragma unroll
             for (int h = 0; h < HALVES; ++h) {
               // half h: A rows 128h.. of the stage's tile, its own accumulator
-              const uint64_t da = ptx::sdesc_kmajor_sw128(a_base + j * p.a_box_rows * kBlockK +
-                                                          h * kBlockM * kBlockK);
+              const uint64_t da =
+                  A_MN ? ptx::sdesc_mnmajor_sw128(a_base, 128 * kBlockK)
+                       : ptx::sdesc_kmajor_sw128(a_base + j * p.a_box_rows * kBlockK +
+                                                 h * kBlockM * kBlockK);
 #pragma unroll
               for (int ks = 0; ks < kBlockK / 32; ++ks)
-                ptx::tc_mma_mxf8_block_scale(d_tmem + h * BLOCK_N, da + 2 * ks, db + 2 * ks, id,
+                ptx::tc_mma_mxf8_block_scale(d_tmem + h * BLOCK_N, da + kStepA * ks,
+                                             db + kStepB * ks, id,
                                              (sfa_tmem + 4 * h) | byte_sel, sfb_tmem | byte_sel,
                                              kb + j > ti.kb_begin || ks > 0);
             }

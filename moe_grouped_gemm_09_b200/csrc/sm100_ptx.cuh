@@ -121,6 +121,16 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
 }
 
 // 3-D tiled load of one box into shared memory, completing on `bar`.
+// 2-D tiled load of one box into shared memory, completing on `bar`.
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(c0), "r"(c1)
+      : "memory");
+}
+
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
                                             int c0, int c1, int c2) {
   asm volatile(
@@ -167,6 +177,13 @@ __device__ __forceinline__ void tma_prefetch_l2_4d(const CUtensorMap* map, int c
 // Ask the TMA unit to bring one box of a tensor into L2 (no shared memory
 // involved, no completion to wait for).  Always safe: L2 is the point of
 // coherence, so a later load sees any write made after the prefetch.
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* map, int c0, int c1) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1)
+               : "memory");
+}
+
 __device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* map, int c0, int c1,
                                                    int c2) {
   asm volatile(
@@ -407,6 +424,21 @@ __device__ __forceinline__ uint64_t sdesc_kmajor_sw128(uint32_t saddr) {
   return d;
 }
 
+// Shared-memory matrix descriptor for an MN-major operand tile stored with the
+// 128-byte swizzle, as a TMA box of {128 bytes of M (or N), K rows} lands it:
+// one row of 128 MN elements per K index, 8-row swizzle atoms 1024 bytes
+// apart along K, and further 128-wide MN blocks `mn_block_bytes` apart.  A
+// K step of 32 inside the tile adds 4 atoms (4096 bytes) to the start.
+__device__ __forceinline__ uint64_t sdesc_mnmajor_sw128(uint32_t saddr, uint32_t mn_block_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);          // start address
+  d |= static_cast<uint64_t>((mn_block_bytes >> 4) & 0x3FFFu) << 16;  // leading byte offset
+  d |= static_cast<uint64_t>(1024u >> 4) << 32;                 // stride byte offset
+  d |= static_cast<uint64_t>(1u) << 46;                         // descriptor version (sm_100)
+  d |= static_cast<uint64_t>(2u) << 61;                         // 128-byte swizzle
+  return d;
+}
+
 // Descriptor for the unswizzled 32-row x 16-byte source of tcgen05.cp.32x128b:
 // row r at byte 16*r (8-row core matrices 128 bytes apart).
 __device__ __forceinline__ uint64_t sdesc_sf_32x16(uint32_t saddr) {
@@ -419,13 +451,15 @@ __device__ __forceinline__ uint64_t sdesc_sf_32x16(uint32_t saddr) {
 }
 
 // Instruction descriptor of tcgen05.mma.kind::mxf8f6f4.block_scale for
-// E4M3 x E4M3 operands, both K-major, UE8M0 scale factors, FP32 accumulation,
+// E4M3 x E4M3 operands (K-major unless a_mn / b_mn), UE8M0 scale factors, FP32 accumulation,
 // M = 128, N = n (multiple of 8 up to 256).
-__host__ __device__ constexpr uint32_t idesc_mxf8_e4m3_ue8m0(int m, int n) {
+__host__ __device__ constexpr uint32_t idesc_mxf8_e4m3_ue8m0(int m, int n, bool a_mn = false,
+                                                       bool b_mn = false) {
   return (0u << 4)                                // B scale-factor byte id
          | (0u << 7)                              // A format: E4M3
          | (0u << 10)                             // B format: E4M3
-         | (0u << 15) | (0u << 16)                // A, B K-major
+         | (static_cast<uint32_t>(a_mn) << 15)    // A: 0 K-major, 1 M-major
+         | (static_cast<uint32_t>(b_mn) << 16)    // B: 0 K-major, 1 N-major
          | (static_cast<uint32_t>(n >> 3) << 17)  // N / 8
          | (1u << 23)                             // scale format: UE8M0
          | (static_cast<uint32_t>(m >> 4) << 24)  // M / 16

@@ -64,6 +64,17 @@ def test_dense_null_and_misaligned_rejected(dg):
     assert dg._gemm_nt(FAKE, FAKE + 2, FAKE, FAKE, FAKE, 4, 16, 128, None) == 1
 
 
+def test_layout_forms_reject_bad_arguments(dg):
+    # an M-major A needs M % 16 == 0; all three forms share the dense checks
+    assert dg._gemm_tn(FAKE, FAKE, FAKE, FAKE, FAKE, 20, 16, 128, None) == 1
+    assert dg._gemm_tt(FAKE, FAKE, FAKE, FAKE, FAKE, 20, 16, 128, None) == 1
+    for fn in (dg._gemm_nn, dg._gemm_tn, dg._gemm_tt):
+        assert fn(FAKE, FAKE, FAKE, FAKE, FAKE, 32, 15, 128, None) == 1
+        assert fn(FAKE, FAKE, FAKE, FAKE, FAKE, 32, 16, 100, None) == 1
+        assert fn(FAKE + 8, FAKE, FAKE, FAKE, FAKE, 32, 16, 128, None) == 1
+        assert fn(None, None, None, None, None, 0, 16, 128, None) == 0
+
+
 def test_zero_rows_is_a_noop(dg):
     # no device is touched for an empty problem, even with null pointers
     assert dg._gemm_nt(None, None, None, None, None, 0, 16, 128, None) == 0

@@ -103,6 +103,43 @@ def test_dense_forced_variant(dg, cfg, monkeypatch):
     check_close(got, ref, f"forced {cfg}")
 
 
+# The other operand layouts: the same problem handed over with A M-major
+# ([K, M]) and/or B N-major ([K, N]); random power-of-two scales per A row and
+# per B block; ragged N and several tiles.
+LAYOUT_CASES = [(256, 384, 512), (208, 272, 384), (64, 256, 1024), (512, 640, 256)]
+
+
+@pytest.mark.parametrize("layout", ["nn", "tn", "tt"])
+@pytest.mark.parametrize("M,N,K", LAYOUT_CASES)
+def test_dense_operand_layouts(dg, layout, M, N, K):
+    rng = np.random.default_rng(M + N + K)
+    p = workloads.dense_problem(M, N, K, seed=8)
+    p.sfa = np.ldexp(1.0, rng.integers(-10, 4, p.sfa.shape)).astype(np.float32)
+    p.sfb = np.ldexp(1.0, rng.integers(-10, 4, p.sfb.shape)).astype(np.float32)
+    a = dev(np.ascontiguousarray(p.a.T) if layout[0] == "t" else p.a)
+    b = dev(np.ascontiguousarray(p.b.T) if layout[1] == "n" else p.b)
+    d = sentinel_like((M, N))
+    getattr(dg, f"fp8_gemm_{layout}")(a, dev(p.sfa), b, dev(p.sfb), d)
+    torch.cuda.synchronize()
+    assert dg.get_last_device_error() == 0
+    ref, _ = oracle.default().gemm_nt(p.a, p.sfa, p.b, p.sfb, want_acc=False)
+    check_close(d_bits(d), ref, f"{layout} {M}x{N}x{K}")
+
+
+@pytest.mark.parametrize("layout", ["nn", "tn", "tt"])
+def test_dense_operand_layouts_prefill_sampled(dg, layout):
+    M, N, K = 4096, 2112, 7168
+    p = workloads.dense_problem(M, N, K, seed=9)
+    a = dev(np.ascontiguousarray(p.a.T) if layout[0] == "t" else p.a)
+    b = dev(np.ascontiguousarray(p.b.T) if layout[1] == "n" else p.b)
+    d = sentinel_like((M, N))
+    getattr(dg, f"fp8_gemm_{layout}")(a, dev(p.sfa), b, dev(p.sfb), d)
+    torch.cuda.synchronize()
+    got = d_bits(d)
+    rows = sample_rows(M, 24, seed=K)
+    check_close(got[rows], oracle_dense_rows(p, rows), f"{layout} prefill")
+
+
 @pytest.mark.parametrize("M,N,K", workloads.DECODE_SHAPES)
 def test_dense_decode_full(dg, M, N, K):
     """The decode-shaped workloads, whole output (split-K path)."""
