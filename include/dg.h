@@ -100,6 +100,16 @@ dg_status dg_fp8_gemm_tn(const void* a, const float* sfa, const void* b, const f
 dg_status dg_fp8_gemm_tt(const void* a, const float* sfa, const void* b, const float* sfb,
                          void* d, int M, int N, int K, dg_stream_t stream);
 
+/* Dense NT GEMM with FP32 output and an optional FP32 addend (the `c`
+ * argument of the DeepGEMM project card's "quick start" call
+ * fp8_gemm_nt(a, b, c, a_sf, b_sf)):
+ *   D[M,N] = A[M,K] * B[N,K]^T + C[M,N]     (C == NULL: D = A * B^T)
+ * a, sfa, b, sfb as in dg_fp8_gemm_nt; c and d float32 [M,N], row-major,
+ * 16-byte aligned; c may equal d (accumulate in place).  The FP32
+ * accumulator is added to C and stored without rounding to BF16. */
+dg_status dg_fp8_gemm_nt_f32(const void* a, const float* sfa, const void* b, const float* sfb,
+                             const float* c, float* d, int M, int N, int K, dg_stream_t stream);
+
 /* M-grouped GEMM, contiguous layout (MoE experts' tokens concatenated along M).
  * a [M_sum,K], sfa [M_sum,K/128], b [G,N,K], sfb [G,ceil(N/128),K/128],
  * d [M_sum,N], m_indices int32 [M_sum] (device): the expert of row r, or -1

@@ -44,6 +44,7 @@ _gemm_nt = _decl("dg_fp8_gemm_nt", [_P, _P, _P, _P, _P, _I, _I, _I, _P])
 _gemm_nn = _decl("dg_fp8_gemm_nn", [_P, _P, _P, _P, _P, _I, _I, _I, _P])
 _gemm_tn = _decl("dg_fp8_gemm_tn", [_P, _P, _P, _P, _P, _I, _I, _I, _P])
 _gemm_tt = _decl("dg_fp8_gemm_tt", [_P, _P, _P, _P, _P, _I, _I, _I, _P])
+_gemm_nt_f32 = _decl("dg_fp8_gemm_nt_f32", [_P, _P, _P, _P, _P, _P, _I, _I, _I, _P])
 _gemm_contig = _decl("dg_m_grouped_fp8_gemm_nt_contiguous", [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P])
 _gemm_masked = _decl("dg_m_grouped_fp8_gemm_nt_masked", [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P])
 _set_num_sms = _decl("dg_set_num_sms", [_I])
@@ -67,7 +68,7 @@ EXPORTED_SYMBOLS = ("dg_fp8_gemm_nt", "dg_m_grouped_fp8_gemm_nt_contiguous",
                     "dg_m_grouped_fp8_gemm_nt_masked", "dg_set_num_sms", "dg_get_num_sms",
                     "dg_get_last_device_error", "dg_set_wait_timeout_ms", "dg_status_string",
                     "dg_query_config", "dg_version", "dg_fp8_gemm_nt_noalloc", "dg_fp8_gemm_nn",
-                    "dg_fp8_gemm_tn", "dg_fp8_gemm_tt")
+                    "dg_fp8_gemm_tn", "dg_fp8_gemm_tt", "dg_fp8_gemm_nt_f32")
 
 DEVICE_ERRORS = {
     0x101: "wait timeout in the TMA producer",
@@ -176,6 +177,31 @@ def fp8_gemm_tt(a, sfa, b, sfb, d=None):
     """``D[M,N] = A B^T`` with A given M-major as ``a [K, M]`` (M % 16 == 0) and
     B ``[N, K]`` (K-major)."""
     return _gemm_layout("dg_fp8_gemm_tt", _gemm_tt, True, False, a, sfa, b, sfb, d)
+
+
+def fp8_gemm_nt_f32(a: torch.Tensor, sfa: torch.Tensor, b: torch.Tensor, sfb: torch.Tensor,
+                    c: Optional[torch.Tensor] = None,
+                    d: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """``D = A B^T + C`` in float32 (``C`` optional; ``c`` may be ``d`` itself to
+    accumulate in place); A, B, scales as in :func:`fp8_gemm_nt`."""
+    _fp8_bytes(a, "a"); _fp8_bytes(b, "b")
+    M, K = a.shape
+    N = b.shape[0]
+    dev = a.device
+    _need(a, "a", None, (M, K), dev)
+    _need(b, "b", None, (N, K), dev)
+    _need(sfa, "sfa", torch.float32, (M, K // 128), dev)
+    _need(sfb, "sfb", torch.float32, ((N + 127) // 128, K // 128), dev)
+    if c is not None:
+        _need(c, "c", torch.float32, (M, N), dev)
+    if d is None:
+        d = torch.empty((M, N), dtype=torch.float32, device=dev)
+    _need(d, "d", torch.float32, (M, N), dev)
+    with torch.cuda.device(dev):
+        _check(_gemm_nt_f32(a.data_ptr(), sfa.data_ptr(), b.data_ptr(), sfb.data_ptr(),
+                            None if c is None else c.data_ptr(), d.data_ptr(), M, N, K,
+                            _stream_ptr(dev)), "dg_fp8_gemm_nt_f32")
+    return d
 
 
 def fp8_gemm_nt_noalloc(a: torch.Tensor, sfa: torch.Tensor, b: torch.Tensor, sfb: torch.Tensor,

@@ -26,7 +26,7 @@ struct DeviceState {
   bool ready = false;
   int num_sms = 0;
   int* error_word = nullptr;      // one int, device memory
-  bool smem_attr_set[6][kNumVariants] = {};  // per form (below) and variant
+  bool smem_attr_set[7][kNumVariants] = {};  // per form (below) and variant
   bool limits_known = false;
   ClusterLimits limits = {};      // co-resident split-K clusters per variant and size
 };
@@ -191,14 +191,16 @@ dg_status make_d_map(CUtensorMap* map, void* base, uint64_t N, uint64_t rows) {
 }
 
 // Launch forms: the three GEMM forms, then the dense form with M-major A
-// and/or N-major B (the forms differ in their kernel instantiation).
+// and/or N-major B, then the dense form with FP32 output (D = A B^T + C); the
+// forms differ in their kernel instantiation.
 enum Form : int { kFormDense = 0, kFormContiguous = 1, kFormMasked = 2, kFormNN = 3, kFormTN = 4,
-                  kFormTT = 5 };
+                  kFormTT = 5, kFormF32 = 6 };
 constexpr int kind_of_form(int f) { return f < 3 ? f : kDense; }
 constexpr int layout_of_form(int f) {
   return f == kFormNN ? kLayoutNN : f == kFormTN ? kLayoutTN : f == kFormTT ? kLayoutTT : kLayoutNT;
 }
-// Variants that serve M-/N-major operands: general ones with 128-column B boxes.
+// Variants that serve M-/N-major operands and the FP32 output form: general
+// ones with 128-column B boxes.
 constexpr bool mn_capable(const Variant& v) {
   return !v.decode && !v.small && !v.pair && v.kps == 1 && v.a_rows == 128 && v.block_n % 128 == 0;
 }
@@ -245,7 +247,7 @@ auto kernel_of() {
     return fp8_gemm_pair_kernel<var.block_n, var.stages>;
   } else {
     return fp8_gemm_kernel<kind_of_form(FORM), var.block_n, var.stages, var.num_acc, var.kps,
-                           var.a_rows, var.small, layout_of_form(FORM)>;
+                           var.a_rows, var.small, layout_of_form(FORM), FORM == kFormF32>;
   }
 }
 
@@ -361,7 +363,7 @@ dg_status launch(DeviceState& st, int variant, const CUtensorMap& ta, const CUte
 // Shared path of the three GEMM forms.
 dg_status run(int form, const void* a, const float* sfa, const void* b, const float* sfb,
               void* d, const int* m_indices, const int* masked_m, int rows, int N, int K, int G,
-              int expected_m, cudaStream_t stream) {
+              int expected_m, cudaStream_t stream, const float* c = nullptr) {
   const int kind = kind_of_form(form);
   const int layout = layout_of_form(form);
   const bool a_mn = (layout & 1) != 0, b_mn = (layout & 2) != 0;
@@ -376,6 +378,7 @@ dg_status run(int form, const void* a, const float* sfa, const void* b, const fl
   if (kind == kContiguous && (!m_indices || !aligned(m_indices, 4) || rows % 128 != 0))
     return DG_ERR_INVALID_ARG;
   if (a_mn && rows % 16 != 0) return DG_ERR_INVALID_ARG;  // [K, M] rows of whole 16-byte units
+  if (form == kFormF32 && c && !aligned(c, 16)) return DG_ERR_INVALID_ARG;
   if (kind == kMasked && (!masked_m || !aligned(masked_m, 4))) return DG_ERR_INVALID_ARG;
   if (kind == kMasked && G > kMaxMaskedGroups) return DG_ERR_UNSUPPORTED;
   const long long a_rows = (kind == kMasked) ? static_cast<long long>(G) * rows : rows;
@@ -393,10 +396,12 @@ dg_status run(int form, const void* a, const float* sfa, const void* b, const fl
     if (s != DG_OK) return s;
   }
   PickedConfig pc = pick_config(kind, rows, N, K, G, expected_m, sms, &st->limits,
-                                /*allow_pair=*/true, /*mn_operands=*/layout != kLayoutNT);
+                                /*allow_pair=*/true,
+                                /*mn_operands=*/layout != kLayoutNT || form == kFormF32);
   forced_config(kind, rows, N, K, G, sms, &pc);
   const Variant var = kVariants[pc.variant];
-  if (layout != kLayoutNT && (!mn_capable(var) || pc.split_k > 1)) return DG_ERR_UNSUPPORTED;
+  if ((layout != kLayoutNT || form == kFormF32) && (!mn_capable(var) || pc.split_k > 1))
+    return DG_ERR_UNSUPPORTED;
 
   GemmArgs args = {};
   args.rows = rows;
@@ -412,6 +417,8 @@ dg_status run(int form, const void* a, const float* sfa, const void* b, const fl
   args.sfa = sfa;
   args.sfb = sfb;
   args.d = static_cast<__nv_bfloat16*>(d);
+  args.d_f32 = form == kFormF32 ? static_cast<float*>(d) : nullptr;
+  args.c_f32 = form == kFormF32 ? c : nullptr;
   args.m_indices = m_indices;
   args.masked_m = masked_m;
   args.error_word = st->error_word;
@@ -464,7 +471,8 @@ dg_status run(int form, const void* a, const float* sfa, const void* b, const fl
       return launch<kFormMasked>(*st, pc.variant, ta, tb, td, args, pc.grid, stream);
     case kFormNN: return launch<kFormNN>(*st, pc.variant, ta, tb, td, args, pc.grid, stream);
     case kFormTN: return launch<kFormTN>(*st, pc.variant, ta, tb, td, args, pc.grid, stream);
-    default: return launch<kFormTT>(*st, pc.variant, ta, tb, td, args, pc.grid, stream);
+    case kFormTT: return launch<kFormTT>(*st, pc.variant, ta, tb, td, args, pc.grid, stream);
+    default: return launch<kFormF32>(*st, pc.variant, ta, tb, td, args, pc.grid, stream);
   }
 }
 
@@ -497,6 +505,12 @@ dg_status dg_fp8_gemm_tt(const void* a, const float* sfa, const void* b, const f
                          void* d, int M, int N, int K, dg_stream_t stream) {
   return run(kFormTT, a, sfa, b, sfb, d, nullptr, nullptr, M, N, K, 1, 0,
              reinterpret_cast<cudaStream_t>(stream));
+}
+
+dg_status dg_fp8_gemm_nt_f32(const void* a, const float* sfa, const void* b, const float* sfb,
+                             const float* c, float* d, int M, int N, int K, dg_stream_t stream) {
+  return run(kFormF32, a, sfa, b, sfb, d, nullptr, nullptr, M, N, K, 1, 0,
+             reinterpret_cast<cudaStream_t>(stream), c);
 }
 
 dg_status dg_m_grouped_fp8_gemm_nt_contiguous(const void* a, const float* sfa, const void* b,

@@ -80,6 +80,8 @@ struct GemmArgs {
   const float* sfa;  // [G * rows, k_blocks]   (dense/contiguous: G = 1 row space)
   const float* sfb;  // [G, nb128, k_blocks]
   __nv_bfloat16* d;  // [G * rows, N]
+  float* d_f32;      // FP32 output form: D [rows, N] (d unused)
+  const float* c_f32;  // FP32 output form: C [rows, N] added to the product, or null
   const int* m_indices;  // contiguous: [rows]
   const int* masked_m;   // masked: [G]
   int* error_word;
@@ -297,7 +299,7 @@ struct StageWalker {
 };
 
 template <int KIND, int BLOCK_N, int STAGES, int NUM_ACC, int KPS, int A_ROWS, bool SMALL,
-          int LAYOUT = kLayoutNT>
+          int LAYOUT = kLayoutNT, bool OUT_F32 = false>
 __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     const __grid_constant__ CUtensorMap tmap_b,
@@ -326,6 +328,8 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
   // tiles made of whole 128-column boxes.
   constexpr bool A_MN = (LAYOUT & 1) != 0;
   constexpr bool B_MN = (LAYOUT & 2) != 0;
+  // FP32 output (D = A B^T + C): the dense form, no split-K (host-checked)
+  static_assert(!OUT_F32 || (KIND == kDense && A_ROWS == 128 && !SMALL), "FP32 output form");
   static_assert(LAYOUT == kLayoutNT ||
                     (KIND == kDense && KPS == 1 && A_ROWS == 128 && !SMALL && BLOCK_N % 128 == 0),
                 "M-/N-major operands: dense form, general variants with 128-column B boxes");
@@ -479,6 +483,26 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
         if (CH == 64)
           ptx::tc_ld_32x32b_x32(t_row + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[CH - 32]));
         ptx::tc_wait_ld();
+        if constexpr (OUT_F32) {
+          // FP32 output: each lane writes its own row's CH floats (whole
+          // 128-byte lines), adding C's if given (C may be D itself: every
+          // element is read and written by the same thread)
+          if (valid) {
+            const size_t off = grow * p.N + n0 + c0;
+#pragma unroll
+            for (int j = 0; j < CH / 4; ++j) {
+              if (n0 + c0 + 4 * j >= p.N) break;
+              float4 v = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                     __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+              if (p.c_f32) {
+                const float4 cv = *reinterpret_cast<const float4*>(p.c_f32 + off + 4 * j);
+                v.x += cv.x; v.y += cv.y; v.z += cv.z; v.w += cv.w;
+              }
+              *reinterpret_cast<float4*>(p.d_f32 + off + 4 * j) = v;
+            }
+          }
+          continue;
+        }
         uint8_t* stage = one_tile ? stage0 + ((c0 - c_begin) / CH) * 32 * Shape::kEpiPitch : stage0;
         if (split) {
           // park the FP32 partial; the cluster reduces it below

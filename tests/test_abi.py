@@ -75,6 +75,13 @@ def test_layout_forms_reject_bad_arguments(dg):
         assert fn(None, None, None, None, None, 0, 16, 128, None) == 0
 
 
+def test_f32_form_rejects_bad_arguments(dg):
+    assert dg._gemm_nt_f32(FAKE, FAKE, FAKE, FAKE, FAKE + 4, FAKE, 32, 16, 128, None) == 1  # c
+    assert dg._gemm_nt_f32(FAKE, FAKE, FAKE, FAKE, None, FAKE + 4, 32, 16, 128, None) == 1  # d
+    assert dg._gemm_nt_f32(FAKE, FAKE, FAKE, FAKE, None, FAKE, 32, 15, 128, None) == 1
+    assert dg._gemm_nt_f32(None, None, None, None, None, None, 0, 16, 128, None) == 0
+
+
 def test_zero_rows_is_a_noop(dg):
     # no device is touched for an empty problem, even with null pointers
     assert dg._gemm_nt(None, None, None, None, None, 0, 16, 128, None) == 0

@@ -140,6 +140,40 @@ def test_dense_operand_layouts_prefill_sampled(dg, layout):
     check_close(got[rows], oracle_dense_rows(p, rows), f"{layout} prefill")
 
 
+# FP32 output, D = A B^T + C.  The FP32 tensor-core accumulation against the
+# oracle's exact double sum plus C: per element within 1e-4 of
+# |ref| + rms(ref) (K/32 FP32 additions of exact products), and the global
+# 1 - 2 sum(xy) / sum(x^2 + y^2) within 1e-9.
+@pytest.mark.parametrize("mode", ["none", "c", "in_place"])
+@pytest.mark.parametrize("M,N,K", [(300, 400, 384), (64, 2112, 1024), (512, 256, 2048)])
+def test_dense_f32_output(dg, mode, M, N, K):
+    rng = np.random.default_rng(M * 3 + N + K)
+    p = workloads.dense_problem(M, N, K, seed=10)
+    _, acc = oracle.default().gemm_nt(p.a, p.sfa, p.b, p.sfb, want_acc=True)
+    c_host = rng.standard_normal((M, N)).astype(np.float32) * 8
+    a, sfa, b, sfb = dev(p.a), dev(p.sfa), dev(p.b), dev(p.sfb)
+    if mode == "none":
+        d = dg.fp8_gemm_nt_f32(a, sfa, b, sfb)
+        ref = acc
+    elif mode == "c":
+        c = dev(c_host)
+        d = dg.fp8_gemm_nt_f32(a, sfa, b, sfb, c=c)
+        assert np.array_equal(c.cpu().numpy(), c_host)  # C is read only
+        ref = acc + c_host.astype(np.float64)
+    else:
+        d = dev(c_host)
+        dg.fp8_gemm_nt_f32(a, sfa, b, sfb, c=d, d=d)
+        ref = acc + c_host.astype(np.float64)
+    torch.cuda.synchronize()
+    assert dg.get_last_device_error() == 0
+    got = d.cpu().numpy().astype(np.float64)
+    rms = np.sqrt(np.mean(ref * ref))
+    viol = np.abs(got - ref) / (1e-4 * (np.abs(ref) + rms))
+    assert viol.max() <= 1.0, f"f32 {mode} {M}x{N}x{K}: worst {viol.max():.3f}"
+    diff = 1 - 2 * np.sum(got * ref) / np.sum(got * got + ref * ref)
+    assert diff <= 1e-9, diff
+
+
 @pytest.mark.parametrize("M,N,K", workloads.DECODE_SHAPES)
 def test_dense_decode_full(dg, M, N, K):
     """The decode-shaped workloads, whole output (split-K path)."""
