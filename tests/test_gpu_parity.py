@@ -174,6 +174,38 @@ def test_dense_f32_output(dg, mode, M, N, K):
     assert diff <= 1e-9, diff
 
 
+@pytest.mark.parametrize("M,N,K", [(64, 2112, 1024), (512, 384, 512)])
+def test_dependent_launches_in_a_graph(dg, M, N, K):
+    """Four launches captured back to back in one CUDA graph, each adding
+    A B^T to the FP32 D the previous one wrote (programmatic dependent launch
+    lets a launch start before the previous one ends; it must not read D
+    before that one has finished writing it): D = 4 A B^T exactly as four
+    separate accumulations."""
+    p = workloads.dense_problem(M, N, K, seed=12)
+    _, acc = oracle.default().gemm_nt(p.a, p.sfa, p.b, p.sfb, want_acc=True)
+    a, sfa, b, sfb = dev(p.a), dev(p.sfa), dev(p.b), dev(p.sfb)
+    d = torch.zeros((M, N), dtype=torch.float32, device="cuda")
+    dg.fp8_gemm_nt_f32(a, sfa, b, sfb, c=d, d=d)  # eager warm-up (device set-up)
+    torch.cuda.synchronize()
+    stream = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for _ in range(4):
+            dg.fp8_gemm_nt_f32(a, sfa, b, sfb, c=d, d=d)
+    for rep in range(3):
+        d.zero_()
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            g.replay()
+        torch.cuda.synchronize()
+        assert dg.get_last_device_error() == 0
+        got = d.cpu().numpy().astype(np.float64)
+        ref = 4 * acc
+        rms = np.sqrt(np.mean(ref * ref))
+        viol = np.abs(got - ref) / (1e-4 * (np.abs(ref) + rms))
+        assert viol.max() <= 1.0, f"replay {rep}: worst {viol.max():.3f}"
+
+
 @pytest.mark.parametrize("M,N,K", workloads.DECODE_SHAPES)
 def test_dense_decode_full(dg, M, N, K):
     """The decode-shaped workloads, whole output (split-K path)."""
