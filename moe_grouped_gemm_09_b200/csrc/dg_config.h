@@ -89,22 +89,24 @@ inline bool split_fits(const Variant& var, int rows, int split) {
 // the variant and K split (one cluster of `split` CTAs per output tile, all in
 // one wave) that minimise an estimate of the time:
 //   fixed cost + smooth max(HBM time of B, busiest CTA's streaming time)
-//   + split tail
+//   + split tail (growing with the CTAs of a cluster)
 // where a CTA streams its B slice plus (at a discount: it is read from L2) its
 // A slice at a rate that grows with the bytes one ring stage moves (both
-// boxes).  The constants were fitted to a sweep of every (variant, split) on
-// the six decode-shaped workloads on B200: the pick is the fastest measured
-// configuration, or within 0.25 us of it, for each.  Returns false if no
-// one-wave configuration exists.
+// boxes).  The constants were fitted to three sweeps of every (variant,
+// split) on the six decode-shaped workloads, each on a different B200: in
+// every sweep the pick is the fastest measured configuration, or within
+// 0.35 us of it, for each shape.  Returns false if no one-wave configuration
+// exists.
 inline bool pick_decode(int rows, int N, int K, int num_sms, const ClusterLimits* lim,
                         PickedConfig* out) {
   const int KB = K / 128;
   constexpr double kHbmBytesPerUs = 4.5e6;  // effective, whole GPU
   constexpr double kRate16KB = 20.0;        // KB per microsecond per CTA, 16 KB stages
   constexpr double kRateCap = 70.0;         // KB per microsecond per CTA, large stages
-  constexpr double kAWeight = 0.2;          // A slices come from L2
+  constexpr double kAWeight = 0.35;         // A slices come from L2
   constexpr double kFixedUs = 6.0;
-  constexpr double kSplitUs = 1.5;          // cluster barriers, pushes, reduction
+  constexpr double kSplitUs = 1.0;          // cluster barriers, pushes, reduction ...
+  constexpr double kSplitPerCtaUs = 0.1;    // ... growing with the CTAs of a cluster
   double best = 1e30;
   bool found = false;
   for (int v = 0; v < kNumVariants; ++v) {
@@ -126,7 +128,7 @@ inline bool pick_decode(int rows, int N, int K, int num_sms, const ClusterLimits
       const double t_cta = (b_cta + kAWeight * a_cta) / r_cta;             // us
       const double t_hbm = static_cast<double>(N) * K / kHbmBytesPerUs;     // us
       const double t_stream = std::pow(std::pow(t_cta, 8.0) + std::pow(t_hbm, 8.0), 0.125);
-      const double t = kFixedUs + t_stream + (s > 1 ? kSplitUs : 0.0);
+      const double t = kFixedUs + t_stream + (s > 1 ? kSplitUs + kSplitPerCtaUs * s : 0.0);
       if (t < best - 1e-9) {
         best = t;
         found = true;

@@ -416,11 +416,16 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
   ptx::tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
   // Let the next kernel start its own prologue (once every CTA of this grid
-  // got here), then, since everything above reads no input and from here on
-  // the inputs may be the previous kernel's outputs, wait for that kernel (a
-  // no-op without programmatic dependent launch).
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  // got here).  Everything above reads no input; the inputs may be the
+  // previous kernel's outputs, so every thread waits for that kernel (a no-op
+  // without programmatic dependent launch) before it reads an input, writes
+  // D or starts a timed wait.  The dense form's tile sequence follows from
+  // the sizes alone, so each of its roles first sets up its first stage and
+  // waits only right before its first global access; the grouped forms'
+  // sequence depends on device data, so every thread waits here.
+  ptx::grid_launch_dependents();
+  constexpr bool kLateWait = (KIND == kDense);
+  if constexpr (!kLateWait) ptx::grid_dependency_wait();
   if (KIND == kMasked) {
     // the tile sequence of the masked form depends on masked_m (device data)
     if (threadIdx.x == 96) {
@@ -586,6 +591,7 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
             // 128-row MMA then reads stale shared memory for the other rows,
             // which only feeds accumulator rows that are never stored.
             ptx::mbar_arrive_expect_tx(&full[s], KPS * (p.a_box_rows + BLOCK_N) * kBlockK);
+            if (kLateWait && it == 0) ptx::grid_dependency_wait();
             if constexpr (A_MN) {
               ptx::tma_load_2d(sA + s * A_BYTES, &tmap_a, &full[s], a_row, kb * kBlockK);
             } else {
@@ -614,6 +620,7 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer --
+    if constexpr (kLateWait) ptx::grid_dependency_wait();
     constexpr uint32_t idesc = ptx::idesc_mxf8_e4m3_ue8m0(kBlockM, BLOCK_N, A_MN, B_MN);
     int it = 0, acc_it = 0;
     bool ok = true;
@@ -705,6 +712,7 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
     StageWalker<KIND, KPS> ld, wr;
     ld.start(blockIdx.x, gridDim.x, total, p, s_prefix, lane);
     wr.start(blockIdx.x, gridDim.x, total, p, s_prefix, lane);
+    if constexpr (kLateWait) ptx::grid_dependency_wait();
 
     auto issue = [&](float (&a)[HALVES][4][KPS], float (&b)[SFB_BLOCKS][KPS]) {
       const Tile& ti = ld.w.ti;
@@ -799,6 +807,7 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
     }
   } else if (warp >= 4) {
     // --------------------------------------------------------- epilogue --
+    if constexpr (kLateWait) ptx::grid_dependency_wait();
     const int q = warp & 3;                // TMEM lane quarter of this warp
     const int row_local = 32 * q + lane;   // accumulator row = TMEM lane
     const int ep_tid = threadIdx.x - 128;  // 0..127
@@ -842,6 +851,10 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
     // themselves are part of the grid's completion)
     if (lane == 0) ptx::bulk_wait_group_read0();
   }
+
+  // the threads that have not waited yet (the producer's other lanes, warp 3)
+  // do so before the helper drain and the split-K reduction write D
+  if constexpr (kLateWait) ptx::grid_dependency_wait();
 
   if (helpers && warp < 4 && !*abort_flag) {
     if (static_cast<int>(blockIdx.x) < total) {

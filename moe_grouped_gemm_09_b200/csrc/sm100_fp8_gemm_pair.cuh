@@ -128,8 +128,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   ptx::cluster_sync();
   ptx::tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  ptx::grid_launch_dependents();
+  ptx::grid_dependency_wait();
 
   ptx::WaitCtl ctl{abort_flag, p.error_word, p.timeout_ns};
   const int total = p.num_m_blocks * p.num_n_blocks;  // pair tiles

@@ -211,6 +211,16 @@ __device__ __forceinline__ void cluster_sync() {
 // The two halves of cluster_sync, for work that can overlap the barrier.  The
 // arrive is relaxed: it orders no memory accesses, it only says "this thread
 // got here".
+// Programmatic dependent launch: let the next kernel in the stream be
+// scheduled, and wait until the previous one has completed with its memory
+// visible (both no-ops for a launch without the programmatic attribute).
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 __device__ __forceinline__ void cluster_arrive_relaxed() {
   asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 }
