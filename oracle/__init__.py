@@ -1,6 +1,7 @@
 """CPU oracle for the FP8 block-scaled GEMM (dense, contiguous grouped, masked
-grouped): a plain, slow, obviously correct restatement of what the method
-computes, in double precision, rounded once to BF16.
+grouped) and for the same three forms with BF16 operands: a plain, slow,
+obviously correct restatement of what the method computes, in double
+precision, rounded once to BF16.
 
 TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
 CPU-baseline leg of ``bench.py`` may import this package.  It shares nothing with
@@ -59,6 +60,14 @@ def load(lib_path: str = _LIB_PATH):
     lib.oracle_grouped_contiguous.argtypes = [P, P, P, P, P, I64, I64, I64, I64, P, P]
     lib.oracle_grouped_masked.restype = ctypes.c_int
     lib.oracle_grouped_masked.argtypes = [P, P, P, P, P, I64, I64, I64, I64, P, P]
+    lib.oracle_bf16_decode.restype = ctypes.c_double
+    lib.oracle_bf16_decode.argtypes = [ctypes.c_uint16]
+    lib.oracle_bf16_gemm_nt.restype = ctypes.c_int
+    lib.oracle_bf16_gemm_nt.argtypes = [P, P, I64, I64, I64, P, P]
+    lib.oracle_bf16_grouped_contiguous.restype = ctypes.c_int
+    lib.oracle_bf16_grouped_contiguous.argtypes = [P, P, P, I64, I64, I64, I64, P, P]
+    lib.oracle_bf16_grouped_masked.restype = ctypes.c_int
+    lib.oracle_bf16_grouped_masked.argtypes = [P, P, P, I64, I64, I64, I64, P, P]
     lib.oracle_num_threads.restype = ctypes.c_int
     lib.oracle_num_threads.argtypes = []
     lib.oracle_set_num_threads.restype = None
@@ -156,6 +165,62 @@ class Oracle:
                                             _ptr(acc), _ptr(d))
         if rc != 0:
             raise ValueError(f"oracle_grouped_masked: bad arguments (rc={rc})")
+        return d, acc
+
+    # -- BF16 operands (no scales) --
+    def bf16_decode(self, bits: int) -> float:
+        return float(self.lib.oracle_bf16_decode(int(bits)))
+
+    def bf16_gemm_nt(self, a, b, want_acc: bool = True):
+        """Dense D = A B^T with BF16 operands given as uint16 bit patterns.
+        Returns ``(d uint16 [M,N], acc float64 [M,N] or None)``."""
+        a = _c(a, np.uint16); b = _c(b, np.uint16)
+        M, K = a.shape
+        N = b.shape[0]
+        assert b.shape[1] == K
+        d = np.empty((M, N), np.uint16)
+        acc = np.empty((M, N), np.float64) if want_acc else None
+        rc = self.lib.oracle_bf16_gemm_nt(_ptr(a), _ptr(b), M, N, K, _ptr(acc), _ptr(d))
+        if rc != 0:
+            raise ValueError(f"oracle_bf16_gemm_nt: failed (rc={rc})")
+        return d, acc
+
+    def bf16_grouped_contiguous(self, a, b, m_indices, d=None, acc=None):
+        """Contiguous grouped GEMM with BF16 operands; ``d``/``acc`` are
+        updated in place on valid rows only."""
+        a = _c(a, np.uint16); b = _c(b, np.uint16)
+        m_indices = _c(m_indices, np.int32)
+        M_sum, K = a.shape
+        G, N, _ = b.shape
+        assert b.shape[2] == K and m_indices.shape == (M_sum,)
+        if d is None:
+            d = np.zeros((M_sum, N), np.uint16)
+        assert d.dtype == np.uint16 and d.shape == (M_sum, N) and d.flags.c_contiguous
+        if acc is not None:
+            assert acc.dtype == np.float64 and acc.shape == (M_sum, N) and acc.flags.c_contiguous
+        rc = self.lib.oracle_bf16_grouped_contiguous(_ptr(a), _ptr(b), _ptr(m_indices),
+                                                     M_sum, N, K, G, _ptr(acc), _ptr(d))
+        if rc != 0:
+            raise ValueError(f"oracle_bf16_grouped_contiguous: failed (rc={rc})")
+        return d, acc
+
+    def bf16_grouped_masked(self, a, b, masked_m, d=None, acc=None):
+        """Masked grouped GEMM with BF16 operands; ``d``/``acc`` are updated in
+        place on rows ``m < masked_m[g]`` only."""
+        a = _c(a, np.uint16); b = _c(b, np.uint16)
+        masked_m = _c(masked_m, np.int32)
+        G, max_m, K = a.shape
+        N = b.shape[1]
+        assert b.shape == (G, N, K) and masked_m.shape == (G,)
+        if d is None:
+            d = np.zeros((G, max_m, N), np.uint16)
+        assert d.dtype == np.uint16 and d.shape == (G, max_m, N) and d.flags.c_contiguous
+        if acc is not None:
+            assert acc.dtype == np.float64 and acc.shape == (G, max_m, N)
+        rc = self.lib.oracle_bf16_grouped_masked(_ptr(a), _ptr(b), _ptr(masked_m),
+                                                 G, max_m, N, K, _ptr(acc), _ptr(d))
+        if rc != 0:
+            raise ValueError(f"oracle_bf16_grouped_masked: failed (rc={rc})")
         return d, acc
 
     def num_threads(self) -> int:

@@ -38,12 +38,23 @@
  *    features": grouped GEMM, contiguous and masked layouts).  masked_m is
  *    clamped to [0, max_m].
  *
+ * BF16 GEMM (same three forms, BF16 operands, no scales): the project card,
+ * section "core features", lists BF16 beside FP8 and FP4 in its unified
+ * dense GEMM family, and grouped GEMMs in contiguous and masked layouts for
+ * MoE.  The plainest reading, taken here: D = A B^T with A [M,K] and B [N,K]
+ * BF16 (K-major), every product exact in double, the sum in double, k
+ * ascending, one rounding to BF16; the grouped forms index rows and groups
+ * exactly as the FP8 ones do.  BF16 operands are decoded from the format
+ * definition (1 sign, 8 exponent bits with bias 127, 7 mantissa bits;
+ * exponent 0 is subnormal, 255 infinity or NaN) through a 65536-entry table.
+ *
  * Parallelism: OpenMP over output rows only; every element is computed by
  * the same sequential loop, so the result does not depend on the thread
  * count.
  */
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 #ifdef _OPENMP
 #include <omp.h>
@@ -213,6 +224,120 @@ int oracle_grouped_masked(const uint8_t *a, const float *sfa, const uint8_t *b,
                      acc ? acc + r * N : NULL, d ? d + r * N : NULL);
         }
     }
+    return 0;
+}
+
+/* ---- BF16 operands -------------------------------------------------------- */
+
+double oracle_bf16_decode(uint16_t bits)
+{
+    int sign = (bits >> 15) & 1;
+    int expo = (bits >> 7) & 0xFF;
+    int mant = bits & 0x7F;
+    double mag;
+    if (expo == 0xFF)
+        mag = mant ? NAN : INFINITY;
+    else if (expo == 0)
+        mag = ldexp((double)mant, -133);              /* subnormal: m/128 * 2^-126 */
+    else
+        mag = ldexp(1.0 + mant / 128.0, expo - 127);  /* normal: 1.m * 2^(e-127)   */
+    return sign ? -mag : mag;
+}
+
+/* One output row of the BF16 GEMM: D[m, 0:N] = bf16(sum_k A[m,k] * B[n,k]). */
+static void bf16_gemm_row(const double *tab, const uint16_t *a_row, const uint16_t *b,
+                          int64_t N, int64_t K, double *acc_row, uint16_t *d_row)
+{
+    for (int64_t n = 0; n < N; ++n) {
+        const uint16_t *b_row = b + n * K;
+        double s = 0.0;
+        for (int64_t k = 0; k < K; ++k)
+            s += tab[a_row[k]] * tab[b_row[k]];
+        if (acc_row)
+            acc_row[n] = s;
+        if (d_row)
+            d_row[n] = oracle_bf16_from_double(s);
+    }
+}
+
+static double *bf16_table(void)
+{
+    double *tab = (double *)malloc(65536 * sizeof(double));
+    if (tab)
+        for (int i = 0; i < 65536; ++i)
+            tab[i] = oracle_bf16_decode((uint16_t)i);
+    return tab;
+}
+
+/* Dense NT with BF16 operands: a [M,K], b [N,K] (BF16 bits); acc [M,N]
+ * (double, may be NULL), d [M,N] (BF16 bits, may be NULL).  Returns 0, -1 on
+ * bad sizes, -3 if out of memory. */
+int oracle_bf16_gemm_nt(const uint16_t *a, const uint16_t *b, int64_t M, int64_t N, int64_t K,
+                        double *acc, uint16_t *d)
+{
+    if (M < 0 || N < 0 || K < 0)
+        return -1;
+    double *tab = bf16_table();
+    if (!tab)
+        return -3;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t m = 0; m < M; ++m)
+        bf16_gemm_row(tab, a + m * K, b, N, K, acc ? acc + m * N : NULL, d ? d + m * N : NULL);
+    free(tab);
+    return 0;
+}
+
+/* Contiguous grouped, BF16 operands: a [M_sum,K], b [G,N,K], m_indices
+ * [M_sum]; a negative index marks a padding row, left unwritten.  Returns 0,
+ * -1 on bad sizes, -2 if some index is >= G, -3 if out of memory. */
+int oracle_bf16_grouped_contiguous(const uint16_t *a, const uint16_t *b, const int32_t *m_indices,
+                                   int64_t M_sum, int64_t N, int64_t K, int64_t G,
+                                   double *acc, uint16_t *d)
+{
+    if (M_sum < 0 || N < 0 || K < 0 || G < 0)
+        return -1;
+    for (int64_t r = 0; r < M_sum; ++r)
+        if (m_indices[r] >= G)
+            return -2;
+    double *tab = bf16_table();
+    if (!tab)
+        return -3;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < M_sum; ++r) {
+        int32_t e = m_indices[r];
+        if (e < 0)
+            continue;
+        bf16_gemm_row(tab, a + r * K, b + e * N * K, N, K,
+                      acc ? acc + r * N : NULL, d ? d + r * N : NULL);
+    }
+    free(tab);
+    return 0;
+}
+
+/* Masked grouped, BF16 operands: a [G,max_m,K], b [G,N,K], masked_m [G];
+ * rows m >= clamp(masked_m[g], 0, max_m) of group g are not written.
+ * Returns 0, -1 on bad sizes, -3 if out of memory. */
+int oracle_bf16_grouped_masked(const uint16_t *a, const uint16_t *b, const int32_t *masked_m,
+                               int64_t G, int64_t max_m, int64_t N, int64_t K,
+                               double *acc, uint16_t *d)
+{
+    if (G < 0 || max_m < 0 || N < 0 || K < 0)
+        return -1;
+    double *tab = bf16_table();
+    if (!tab)
+        return -3;
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (int64_t g = 0; g < G; ++g) {
+        for (int64_t m = 0; m < max_m; ++m) {
+            int64_t valid = masked_m[g] < 0 ? 0 : (masked_m[g] > max_m ? max_m : masked_m[g]);
+            if (m >= valid)
+                continue;
+            int64_t r = g * max_m + m;
+            bf16_gemm_row(tab, a + r * K, b + g * N * K, N, K,
+                          acc ? acc + r * N : NULL, d ? d + r * N : NULL);
+        }
+    }
+    free(tab);
     return 0;
 }
 

@@ -13,6 +13,9 @@ What each pin compares against:
 * the BF16 rounding: hand-worked cases (golden file), and torch's FP32->BF16
   conversion for values that are exactly FP32 (where one rounding from double
   equals one rounding from FP32);
+* the BF16 operand GEMM: every one of the 65536 operand patterns against the
+  FP32 widening and ml_dtypes; numpy float64 matmul; Python-float loops (bit
+  for bit); exact integer results; an empty K; the grouped forms row by row;
 * the GEMM: a hand-worked tiny example (golden file); brute force with numpy's
   float64 matmul on ml_dtypes-decoded operands; exact integer results; one-hot
   selection; power-of-two scale invariance; and for the grouped forms, the same
@@ -317,11 +320,138 @@ def pin_masked(o, seed=16):
                 assert np.all(d[g, m] == SENTINEL), (g, m)
 
 
+# ------------------------------------------------------ BF16 operand GEMM --
+
+def decode_bf16_np(bits) -> np.ndarray:
+    """BF16 bit patterns -> float64 by widening to FP32 bit patterns
+    (independent of the oracle's table)."""
+    return (np.asarray(bits, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def random_bf16(rng, shape, scale=1.0) -> np.ndarray:
+    x = torch.from_numpy((rng.standard_normal(shape) * scale).astype(np.float32))
+    return x.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def bf16_of_ints(ints: np.ndarray) -> np.ndarray:
+    """Exact BF16 patterns of small integers (|i| <= 256), through torch."""
+    x = torch.from_numpy(np.asarray(ints, np.float32))
+    return x.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def pin_bf16_operand_table(o):
+    """All 65536 patterns against the FP32 widening and ml_dtypes' bfloat16."""
+    bits = np.arange(65536, dtype=np.uint32)
+    ref = decode_bf16_np(bits.astype(np.uint16))
+    with np.errstate(invalid="ignore"):
+        ref2 = bits.astype(np.uint16).view(ml_dtypes.bfloat16).astype(np.float64)
+    got = np.array([o.bf16_decode(i) for i in range(65536)])
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan) and np.array_equal(np.isnan(ref2), nan)
+    assert np.array_equal(got[~nan], ref[~nan]) and np.array_equal(ref2[~nan], ref[~nan])
+    assert np.array_equal(np.signbit(got[~nan]), np.signbit(ref[~nan]))
+    # spot values from the format definition
+    assert o.bf16_decode(0x3F80) == 1.0 and o.bf16_decode(0xC040) == -3.0
+    assert o.bf16_decode(0x0001) == 2.0 ** -133 and o.bf16_decode(0x0080) == 2.0 ** -126
+    assert o.bf16_decode(0x7F7F) == (2 - 2.0 ** -7) * 2.0 ** 127
+    assert o.bf16_decode(0xFF80) == -np.inf
+
+
+BF16_BRUTE_SHAPES = [(1, 1, 1), (3, 5, 7), (8, 9, 64), (5, 130, 200), (2, 257, 64)]
+
+
+def pin_bf16_gemm_brute_force(o, seed=17):
+    rng = np.random.default_rng(seed)
+    for (M, N, K) in BF16_BRUTE_SHAPES:
+        a = random_bf16(rng, (M, K))
+        b = random_bf16(rng, (N, K), scale=4.0)
+        d, acc = o.bf16_gemm_nt(a, b)
+        ref = decode_bf16_np(a) @ decode_bf16_np(b).T
+        assert np.allclose(acc, ref, rtol=1e-12, atol=1e-300), (M, N, K)
+        assert np.array_equal(d, bf16_nearest_even(acc).reshape(M, N)), (M, N, K)
+
+
+def pin_bf16_gemm_python_loops(o, seed=18):
+    """Tiny case summed with Python floats in k order: the same IEEE double
+    operations, so the accumulator must match bit for bit."""
+    rng = np.random.default_rng(seed)
+    M, N, K = 2, 3, 11
+    a = random_bf16(rng, (M, K))
+    b = random_bf16(rng, (N, K))
+    d, acc = o.bf16_gemm_nt(a, b)
+    da, db = decode_bf16_np(a), decode_bf16_np(b)
+    for m in range(M):
+        for n in range(N):
+            s = 0.0
+            for k in range(K):
+                s += float(da[m, k]) * float(db[n, k])
+            assert acc[m, n] == s, (m, n)
+            assert d[m, n] == bf16_nearest_even(np.array([s]))[0], (m, n)
+
+
+def pin_bf16_gemm_integer_exact(o, seed=19):
+    rng = np.random.default_rng(seed)
+    for (M, N, K) in [(4, 6, 64), (9, 17, 256), (3, 140, 192)]:
+        ia = rng.integers(-8, 9, (M, K))
+        ib = rng.integers(-8, 9, (N, K))
+        d, acc = o.bf16_gemm_nt(bf16_of_ints(ia), bf16_of_ints(ib))
+        exact = ia @ ib.T                                   # |.| <= 64 K, exact in FP32
+        assert np.array_equal(acc, exact.astype(np.float64))
+        assert np.array_equal(d, bf16_of_ints(exact.astype(np.float32)))
+
+
+def pin_bf16_gemm_empty_k(o):
+    d, acc = o.bf16_gemm_nt(np.zeros((3, 0), np.uint16), np.zeros((5, 0), np.uint16))
+    assert np.array_equal(acc, np.zeros((3, 5))) and np.all(d == 0)
+
+
+def pin_bf16_grouped(o, seed=20):
+    rng = np.random.default_rng(seed)
+    # contiguous: padding rows keep the sentinel; expert rows equal the
+    # per-expert dense GEMM on the same rows
+    G, N, K = 3, 136, 128
+    counts = [2, 0, 129]
+    padded = [(-(-c // 128)) * 128 for c in counts]
+    m_idx = np.full(sum(padded), -1, np.int32)
+    off = 0
+    for g, c in enumerate(counts):
+        m_idx[off:off + c] = g
+        off += padded[g]
+    a = random_bf16(rng, (len(m_idx), K))
+    b = random_bf16(rng, (G, N, K))
+    d = np.full((len(m_idx), N), SENTINEL, np.uint16)
+    o.bf16_grouped_contiguous(a, b, m_idx, d=d)
+    for r in range(len(m_idx)):
+        e = m_idx[r]
+        if e < 0:
+            assert np.all(d[r] == SENTINEL), r
+        else:
+            ref = decode_bf16_np(a[r]) @ decode_bf16_np(b[e]).T
+            assert np.array_equal(d[r], bf16_nearest_even(ref)), r
+    # masked: rows m >= masked_m[g] (clamped to [0, max_m]) keep the sentinel
+    G, max_m, N, K = 4, 5, 72, 64
+    masked_m = np.array([5, 0, 2, 8], np.int32)
+    a = random_bf16(rng, (G, max_m, K))
+    b = random_bf16(rng, (G, N, K))
+    d = np.full((G, max_m, N), SENTINEL, np.uint16)
+    o.bf16_grouped_masked(a, b, masked_m, d=d)
+    for g in range(G):
+        valid = min(max(int(masked_m[g]), 0), max_m)
+        for m in range(max_m):
+            if m < valid:
+                ref = decode_bf16_np(a[g, m]) @ decode_bf16_np(b[g]).T
+                assert np.array_equal(d[g, m], bf16_nearest_even(ref)), (g, m)
+            else:
+                assert np.all(d[g, m] == SENTINEL), (g, m)
+
+
 ALL_PINS = [
     pin_e4m3_golden, pin_e4m3_structure, pin_e4m3_libraries,
     pin_bf16_golden, pin_bf16_vs_torch_on_fp32_values, pin_bf16_vs_candidates_on_wide_values,
     pin_tiny_worked_gemm, pin_dense_brute_force, pin_dense_integer_exact, pin_dense_one_hot,
     pin_dense_scale_invariance, pin_contiguous, pin_masked,
+    pin_bf16_operand_table, pin_bf16_gemm_brute_force, pin_bf16_gemm_python_loops,
+    pin_bf16_gemm_integer_exact, pin_bf16_gemm_empty_k, pin_bf16_grouped,
 ]
 
 

@@ -41,6 +41,17 @@ MUTANTS = [
     ("contiguous_pad_as_expert0", "if (e < 0)\n            continue;", "if (e < 0)\n            e = 0;"),
     ("contiguous_wrong_sfb_group", "sfb + e * NB * KB", "sfb"),
     ("masked_wrong_b_group", "b + g * N * K, sfb + g * NB * KB", "b, sfb + g * NB * KB"),
+    ("bf16_operand_bias_126", "ldexp(1.0 + mant / 128.0, expo - 127)", "ldexp(1.0 + mant / 128.0, expo - 126)"),
+    ("bf16_operand_mantissa_64", "ldexp(1.0 + mant / 128.0, expo - 127)", "ldexp(1.0 + mant / 64.0, expo - 127)"),
+    ("bf16_operand_subnormal", "ldexp((double)mant, -133)", "ldexp((double)mant, -134)"),
+    ("bf16_operand_sign_dropped", "int sign = (bits >> 15) & 1;", "int sign = 0;"),
+    ("bf16_operand_nan_as_inf", "mag = mant ? NAN : INFINITY;", "mag = INFINITY;"),
+    ("bf16_gemm_transposed_b", "const uint16_t *b_row = b + n * K;", "const uint16_t *b_row = b + (n % 2) * K;"),
+    ("bf16_gemm_skip_first_k", "s += tab[a_row[k]] * tab[b_row[k]];", "s += k ? tab[a_row[k]] * tab[b_row[k]] : 0.0;"),
+    ("bf16_gemm_float_acc", "double s = 0.0;\n        for", "float s = 0.0f;\n        for"),
+    ("bf16_gemm_a_row_for_b", "s += tab[a_row[k]] * tab[b_row[k]];", "s += tab[a_row[k]] * tab[a_row[k]];"),
+    ("bf16_contiguous_wrong_group", "bf16_gemm_row(tab, a + r * K, b + e * N * K,", "bf16_gemm_row(tab, a + r * K, b,"),
+    ("bf16_masked_wrong_group", "bf16_gemm_row(tab, a + r * K, b + g * N * K,", "bf16_gemm_row(tab, a + r * K, b,"),
 ]
 
 _CHILD = r"""
