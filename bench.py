@@ -7,7 +7,9 @@ DeepGEMM pages' DeepSeek-V3/R1 inference shapes, M in {64, 128} x (N, K) in
 power-of-two block scales, every step through the library's public call.
 The metric for M <= 128 is HBM bandwidth: algorithmic bytes (A, B, their
 scales, and D) per second.  The other workloads ("smoke", "prefill",
-"contiguous", "masked") report TFLOPS and are for profiling and study.
+"contiguous", "masked") report TFLOPS and are for profiling and study, as
+are "bf16-decode" and "bf16-prefill": the same dense shapes on BF16 operands
+(no scales), measured against the BF16 tensor peak.
 
 Timing: inputs sit in HBM, R copies of them at different addresses are rotated
 so that the bytes touched between two visits of one copy exceed the 126 MB L2;
@@ -67,13 +69,27 @@ def build_workload(name: str, seed: int = 0):
         return [("contiguous", workloads.contiguous_problem(**workloads.CONTIGUOUS_MOE, seed=seed))]
     if name == "masked":
         return [("masked", workloads.masked_problem(**workloads.MASKED_MOE, seed=seed))]
+    if name == "bf16-decode":
+        return [("bf16_dense", workloads.bf16_dense_problem(m, n, k, seed=seed + i))
+                for i, (m, n, k) in enumerate(workloads.DECODE_SHAPES)]
+    if name == "bf16-prefill":
+        return [("bf16_dense", workloads.bf16_dense_problem(m, n, k, seed=seed + i))
+                for i, (m, n, k) in enumerate(workloads.PREFILL_SHAPES)]
     raise ValueError(name)
+
+
+def is_bf16(name: str) -> bool:
+    return name.startswith("bf16-")
 
 
 def workload_meta(name: str):
     """(metric, unit, bound) for a workload."""
     if name in ("decode", "smoke"):
         return "FP8 GEMM HBM bandwidth (M<=128)", "GB/s", "hbm"
+    if name == "bf16-decode":
+        return "BF16 GEMM HBM bandwidth (M<=128)", "GB/s", "hbm"
+    if name == "bf16-prefill":
+        return "BF16 GEMM TFLOPS", "TFLOP/s", "tensor"
     return "FP8 GEMM TFLOPS", "TFLOP/s", "tensor"
 
 
@@ -90,12 +106,15 @@ def scale_units(x: float, unit: str, seconds: float) -> float:
 
 SPEC_HBM_GBS = 8000.0     # B200 HBM3e, vendor figure
 SPEC_FP8_TFLOPS = 4500.0  # B200 dense E4M3, vendor figure
+SPEC_BF16_TFLOPS = 2250.0  # B200 dense BF16, vendor figure
 
 
-def roofline_terms(items, ms: float, hbm_gbs: float, fp8_tflops: float) -> dict:
+def roofline_terms(items, ms: float, hbm_gbs: float, fp8_tflops: float,
+                   spec_tflops: float = SPEC_FP8_TFLOPS) -> dict:
     """Roofline of one step: every GEMM's time bound is the larger of its
-    FLOPs at the FP8 peak and its algorithmic bytes at the HBM bandwidth; the
-    step's bound is the sum.  ``bound`` names the term that dominates the sum."""
+    FLOPs at the tensor peak of its operand type (``fp8_tflops``; the BF16
+    peak for BF16 operands) and its algorithmic bytes at the HBM bandwidth;
+    the step's bound is the sum.  ``bound`` names the term that dominates."""
     def t_roof(hbm, fp8):
         return sum(max(p.flops() / (fp8 * 1e12), p.bytes() / (hbm * 1e9)) for _, p in items)
     t_flop = sum(p.flops() for _, p in items) / (fp8_tflops * 1e12)
@@ -103,7 +122,7 @@ def roofline_terms(items, ms: float, hbm_gbs: float, fp8_tflops: float) -> dict:
     t = t_roof(hbm_gbs, fp8_tflops)
     return {"bound": "tensor" if t_flop >= t_byte else "hbm", "t_roof_s": t,
             "frac_time": t / (ms / 1e3),
-            "frac_time_spec": t_roof(SPEC_HBM_GBS, SPEC_FP8_TFLOPS) / (ms / 1e3)}
+            "frac_time_spec": t_roof(SPEC_HBM_GBS, spec_tflops) / (ms / 1e3)}
 
 
 # --------------------------------------------------------------- helpers --
@@ -126,12 +145,19 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
+def profile_name(workload: str) -> str:
+    """Stem of a workload's ncu summaries under ``profiles/``."""
+    if is_bf16(workload):
+        return "bf16_gemm_" + workload[len("bf16-"):]
+    return "fp8_gemm_" + workload
+
+
 def profiled_traffic(workload: str):
     """DRAM bytes per launch of the dominant kernel, from the committed ncu
-    summary ``profiles/fp8_gemm_<workload>_traffic.md`` (its lines
+    summary ``profiles/<stem>_traffic.md`` (its lines
     ``traffic_bytes_per_launch:`` and ``kernel_source_hash:``), or None if the
     summary is absent or was taken on other kernel sources."""
-    path = os.path.join(ROOT, "profiles", f"fp8_gemm_{workload}_traffic.md")
+    path = os.path.join(ROOT, "profiles", f"{profile_name(workload)}_traffic.md")
     rec = {}
     try:
         with open(path) as f:
@@ -254,21 +280,32 @@ def run_gpu(args):
     items = build_workload(args.workload, seed=args.seed)
     metric, unit, _ = workload_meta(args.workload)
     units = step_units(items, unit)
-    set_bytes = sum(p.a.nbytes + p.b.nbytes + p.sfa.nbytes + p.sfb.nbytes for _, p in items)
+    set_bytes = sum(p.a.nbytes + p.b.nbytes + getattr(p, "sfa", p.a[:0]).nbytes
+                    + getattr(p, "sfb", p.a[:0]).nbytes for _, p in items)
     R = max(2, math.ceil(3 * L2_BYTES / max(set_bytes, 1)))
-    if args.workload in ("prefill", "contiguous", "masked"):
+    if args.workload in ("prefill", "contiguous", "masked", "bf16-prefill"):
         R = max(2, min(R, 4))
     flush_note = f"inputs rotated over {R} copies ({R * set_bytes / 2**20:.0f} MiB > 3x L2)"
 
     # device copies: R rotation sets of the inputs, one output per GEMM
+    def host_tensor(x):
+        # BF16 operands arrive as uint16 bit patterns
+        if x.dtype == np.uint16:
+            return torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16)
+        return torch.from_numpy(np.ascontiguousarray(x))
+
     def to_dev(x):
-        return torch.from_numpy(np.ascontiguousarray(x)).to(dev)
+        return host_tensor(x).to(dev)
+
+    def operands(p):
+        names = ("a", "sfa", "b", "sfb") if hasattr(p, "sfa") else ("a", "b")
+        return {k: getattr(p, k) for k in names}
 
     sets = []
     for r in range(R):
         one = []
         for kind, p in items:
-            t = {"a": to_dev(p.a), "sfa": to_dev(p.sfa), "b": to_dev(p.b), "sfb": to_dev(p.sfb)}
+            t = {k: to_dev(v) for k, v in operands(p).items()}
             if kind == "contiguous":
                 t["m_indices"] = to_dev(p.m_indices)
             if kind == "masked":
@@ -277,7 +314,7 @@ def run_gpu(args):
         sets.append(one)
     outs = []
     for kind, p in items:
-        if kind == "dense":
+        if kind in ("dense", "bf16_dense"):
             outs.append(torch.empty((p.M, p.N), dtype=torch.bfloat16, device=dev))
         elif kind == "contiguous":
             outs.append(torch.empty((p.M_sum, p.N), dtype=torch.bfloat16, device=dev))
@@ -288,6 +325,8 @@ def run_gpu(args):
         (kind, p), t, d = items[j], sets[r][j], outs[j]
         if kind == "dense":
             dg.fp8_gemm_nt(t["a"], t["sfa"], t["b"], t["sfb"], d)
+        elif kind == "bf16_dense":
+            dg.bf16_gemm_nt(t["a"], t["b"], d)
         elif kind == "contiguous":
             dg.m_grouped_fp8_gemm_nt_contiguous(t["a"], t["sfa"], t["b"], t["sfb"],
                                                 t["m_indices"], d)
@@ -375,8 +414,7 @@ def run_gpu(args):
     # ---- end to end: host buffers, copies inside the timed region ----
     pinned = []
     for kind, p in items:
-        t = {"a": torch.from_numpy(p.a).pin_memory(), "sfa": torch.from_numpy(p.sfa).pin_memory(),
-             "b": torch.from_numpy(p.b).pin_memory(), "sfb": torch.from_numpy(p.sfb).pin_memory()}
+        t = {k: host_tensor(v).pin_memory() for k, v in operands(p).items()}
         if kind == "contiguous":
             t["m_indices"] = torch.from_numpy(p.m_indices).pin_memory()
         if kind == "masked":
@@ -418,12 +456,16 @@ def run_gpu(args):
 
     peaks, peak_kind = load_peaks()
     hbm_peak = float(peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"]))
-    # E4M3 dense peak = 2x the measured BF16 figure (nominal FP8:BF16 ratio 4.5:2.25)
-    fp8_peak = 2.0 * float(peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"]))
-    roof = roofline_terms(items, ms, hbm_peak, fp8_peak)
+    # E4M3 dense peak = 2x the measured BF16 figure (nominal FP8:BF16 ratio
+    # 4.5:2.25); BF16 operands take the measured BF16 figure itself
+    bf16_peak = float(peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"]))
+    bf16 = is_bf16(args.workload)
+    tensor_peak = bf16_peak if bf16 else 2.0 * bf16_peak
+    roof = roofline_terms(items, ms, hbm_peak, tensor_peak,
+                          SPEC_BF16_TFLOPS if bf16 else SPEC_FP8_TFLOPS)
     bound = roof["bound"]
     r_unit = "GB/s" if bound == "hbm" else "TFLOP/s"
-    peak = hbm_peak if bound == "hbm" else fp8_peak
+    peak = hbm_peak if bound == "hbm" else tensor_peak
     achieved = scale_units(step_units(items, r_unit), r_unit, ms / 1e3)
     value = whole_job_value(units, world, ms, unit)
     launches_per_step = len(items)
@@ -438,7 +480,7 @@ def run_gpu(args):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "e4m3",
+        "dtype": "bf16" if bf16 else "e4m3",
         "data": "synthetic",
         "config": {
             "workload": args.workload,
@@ -457,7 +499,7 @@ def run_gpu(args):
             "unit": r_unit,
             "frac": round(achieved / peak, 4),
             "traffic": profiled_traffic(args.workload),
-            "peak_source": f"{peak_kind} ({'hbm_gbs copy' if bound == 'hbm' else '2 x bf16_tflops'})",
+            "peak_source": f"{peak_kind} ({'hbm_gbs copy' if bound == 'hbm' else 'bf16_tflops' if bf16 else '2 x bf16_tflops'})",
             "roofline_time_us": round(roof["t_roof_s"] * 1e6, 3),
             "frac_time": round(roof["frac_time"], 4),
             "frac_time_spec": round(roof["frac_time_spec"], 4),
@@ -476,7 +518,7 @@ def run_gpu(args):
 
 
 def _shape(p):
-    if isinstance(p, workloads.DenseProblem):
+    if isinstance(p, (workloads.DenseProblem, workloads.Bf16DenseProblem)):
         return {"M": p.M, "N": p.N, "K": p.K}
     if isinstance(p, workloads.ContiguousProblem):
         return {"M_sum": p.M_sum, "N": p.N, "K": p.K, "G": p.G, "valid_rows": p.valid_rows()}
@@ -490,7 +532,7 @@ def _row_units(items, unit):
     """Total rows per GEMM, for scaling a row sample up to the full step."""
     out = []
     for kind, p in items:
-        if kind == "dense":
+        if kind in ("dense", "bf16_dense"):
             out.append(p.M)
         else:
             out.append(p.valid_rows())
@@ -500,6 +542,8 @@ def _row_units(items, unit):
 def _oracle_rows(o, kind, p, rows: np.ndarray):
     if kind == "dense":
         o.gemm_nt(p.a[rows], p.sfa[rows], p.b, p.sfb, want_acc=False)
+    elif kind == "bf16_dense":
+        o.bf16_gemm_nt(p.a[rows], p.b, want_acc=False)
     elif kind == "contiguous":
         valid = np.nonzero(p.m_indices >= 0)[0][rows]
         o.grouped_contiguous(p.a[valid], p.sfa[valid], p.b, p.sfb, p.m_indices[valid])
@@ -614,7 +658,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="decode",
-                    choices=("decode", "smoke", "prefill", "contiguous", "masked"))
+                    choices=("decode", "smoke", "prefill", "contiguous", "masked", "bf16-decode",
+                             "bf16-prefill"))
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--per-gemm-reps", type=int, default=20,

@@ -9,6 +9,8 @@
  *   M-grouped contiguous  D[r,:]        = A[r,:] B[m_indices[r]]^T  for every row r
  *   M-grouped masked      D[g,m,:]      = A[g,m,:] B[g]^T           for m < masked_m[g]
  *
+ * and the same three forms on BF16 operands without scales (dg_bf16_*).
+ *
  * Sources: the operation and its fine-grained scaling and FP32 promotion are
  * described in the DeepGEMM release article (deepseek.csdn.net), part 1.2
  * "precision safeguards"; the call names fp8_gemm_nt and
@@ -36,7 +38,7 @@
  *    produced by scale = 2^ceil(log2(amax/448)); the kernel uses the exponent
  *    field only.
  *  - Requirements (checked on the host, DG_ERR_INVALID_ARG otherwise):
- *    K > 0 and K % 128 == 0; N > 0 and N % 16 == 0; a, b and d 16-byte
+ *    K > 0 and K % 128 == 0 (BF16 operands: K % 64 == 0); N > 0 and N % 16 == 0; a, b and d 16-byte
  *    aligned, sfa/sfb 4-byte aligned, m_indices/masked_m 4-byte aligned.
  *    A zero-row problem (M == 0, M_sum == 0, G == 0 or max_m == 0) is a
  *    no-op returning DG_OK.
@@ -132,6 +134,26 @@ dg_status dg_m_grouped_fp8_gemm_nt_masked(const void* a, const float* sfa, const
                                           const float* sfb, void* d, const int* masked_m, int G,
                                           int max_m, int N, int K, int expected_m,
                                           dg_stream_t stream);
+
+/* The three GEMM forms on BF16 operands (DeepGEMM project card,
+ * aiproducthub.cn, "core features": BF16 beside FP8 and FP4 in the unified
+ * dense GEMM family; grouped GEMMs in contiguous and masked layouts for MoE).
+ * No scale factors: D = bf16(A * B^T), FP32 accumulation, one rounding.
+ * a and b hold BF16 elements (2 bytes), both K-major; d is BF16; K % 64 == 0
+ * (one 128-byte K block is 64 elements).  Shapes, m_indices, masked_m,
+ * expected_m, untouched rows and every other rule are those of the FP8
+ * functions with the same form:
+ *   dense:      a [M,K], b [N,K], d [M,N]
+ *   contiguous: a [M_sum,K], b [G,N,K], d [M_sum,N], m_indices [M_sum]
+ *   masked:     a [G,max_m,K], b [G,N,K], d [G,max_m,N], masked_m [G] */
+dg_status dg_bf16_gemm_nt(const void* a, const void* b, void* d, int M, int N, int K,
+                          dg_stream_t stream);
+dg_status dg_m_grouped_bf16_gemm_nt_contiguous(const void* a, const void* b, void* d,
+                                               const int* m_indices, int M_sum, int N, int K,
+                                               int G, dg_stream_t stream);
+dg_status dg_m_grouped_bf16_gemm_nt_masked(const void* a, const void* b, void* d,
+                                           const int* masked_m, int G, int max_m, int N, int K,
+                                           int expected_m, dg_stream_t stream);
 
 /* Cap on the number of SMs the GEMMs use (release article, part 4.2:
  * set_num_sms).  n <= 0 restores the default (all SMs of the device).

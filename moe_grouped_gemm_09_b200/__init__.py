@@ -1,5 +1,5 @@
 """FP8 (E4M3) block-scaled GEMM for NVIDIA B200 (sm_100a): dense and MoE
-M-grouped (contiguous and masked layouts).
+M-grouped (contiguous and masked layouts), and the same forms on BF16 operands.
 
 This module is a thin binding over the C ABI of ``libdg.so`` (declared in
 ``include/dg.h``): it checks tensor types and devices, passes raw device
@@ -47,6 +47,9 @@ _gemm_tt = _decl("dg_fp8_gemm_tt", [_P, _P, _P, _P, _P, _I, _I, _I, _P])
 _gemm_nt_f32 = _decl("dg_fp8_gemm_nt_f32", [_P, _P, _P, _P, _P, _P, _I, _I, _I, _P])
 _gemm_contig = _decl("dg_m_grouped_fp8_gemm_nt_contiguous", [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P])
 _gemm_masked = _decl("dg_m_grouped_fp8_gemm_nt_masked", [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P])
+_bf16_gemm_nt = _decl("dg_bf16_gemm_nt", [_P, _P, _P, _I, _I, _I, _P])
+_bf16_gemm_contig = _decl("dg_m_grouped_bf16_gemm_nt_contiguous", [_P, _P, _P, _P, _I, _I, _I, _I, _P])
+_bf16_gemm_masked = _decl("dg_m_grouped_bf16_gemm_nt_masked", [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P])
 _set_num_sms = _decl("dg_set_num_sms", [_I])
 _get_num_sms = _decl("dg_get_num_sms", [])
 _get_last_err = _decl("dg_get_last_device_error", [ctypes.POINTER(ctypes.c_int)])
@@ -68,7 +71,8 @@ EXPORTED_SYMBOLS = ("dg_fp8_gemm_nt", "dg_m_grouped_fp8_gemm_nt_contiguous",
                     "dg_m_grouped_fp8_gemm_nt_masked", "dg_set_num_sms", "dg_get_num_sms",
                     "dg_get_last_device_error", "dg_set_wait_timeout_ms", "dg_status_string",
                     "dg_query_config", "dg_version", "dg_fp8_gemm_nt_noalloc", "dg_fp8_gemm_nn",
-                    "dg_fp8_gemm_tn", "dg_fp8_gemm_tt", "dg_fp8_gemm_nt_f32")
+                    "dg_fp8_gemm_tn", "dg_fp8_gemm_tt", "dg_fp8_gemm_nt_f32", "dg_bf16_gemm_nt",
+                    "dg_m_grouped_bf16_gemm_nt_contiguous", "dg_m_grouped_bf16_gemm_nt_masked")
 
 DEVICE_ERRORS = {
     0x101: "wait timeout in the TMA producer",
@@ -269,6 +273,72 @@ def m_grouped_fp8_gemm_nt_masked(a: torch.Tensor, sfa: torch.Tensor, b: torch.Te
         _check(_gemm_masked(a.data_ptr(), sfa.data_ptr(), b.data_ptr(), sfb.data_ptr(),
                             d.data_ptr(), masked_m.data_ptr(), G, max_m, N, K, int(expected_m),
                             _stream_ptr(dev)), "dg_m_grouped_fp8_gemm_nt_masked")
+    return d
+
+
+def _bf16(t: torch.Tensor, name: str) -> torch.Tensor:
+    if t.dtype != torch.bfloat16:
+        raise TypeError(f"{name}: expected bfloat16, got {t.dtype}")
+    return t
+
+
+def bf16_gemm_nt(a: torch.Tensor, b: torch.Tensor, d: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Dense ``D[M,N] = A[M,K] B[N,K]^T`` on BF16 operands (K-major, K % 64 == 0),
+    FP32 accumulation, BF16 output.  Runs on the current stream."""
+    _bf16(a, "a"); _bf16(b, "b")
+    M, K = a.shape
+    N = b.shape[0]
+    dev = a.device
+    _need(a, "a", torch.bfloat16, (M, K), dev)
+    _need(b, "b", torch.bfloat16, (N, K), dev)
+    if d is None:
+        d = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    _need(d, "d", torch.bfloat16, (M, N), dev)
+    with torch.cuda.device(dev):
+        _check(_bf16_gemm_nt(a.data_ptr(), b.data_ptr(), d.data_ptr(), M, N, K, _stream_ptr(dev)),
+               "dg_bf16_gemm_nt")
+    return d
+
+
+def m_grouped_bf16_gemm_nt_contiguous(a: torch.Tensor, b: torch.Tensor, m_indices: torch.Tensor,
+                                      d: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Contiguous grouped GEMM on BF16 operands: ``D[r] = A[r] B[m_indices[r]]^T``;
+    rows with index -1 are left untouched.  ``a [M_sum,K]``, ``b [G,N,K]``."""
+    _bf16(a, "a"); _bf16(b, "b")
+    M_sum, K = a.shape
+    G, N, _ = b.shape
+    dev = a.device
+    _need(a, "a", torch.bfloat16, (M_sum, K), dev)
+    _need(b, "b", torch.bfloat16, (G, N, K), dev)
+    _need(m_indices, "m_indices", torch.int32, (M_sum,), dev)
+    if d is None:
+        d = torch.empty((M_sum, N), dtype=torch.bfloat16, device=dev)
+    _need(d, "d", torch.bfloat16, (M_sum, N), dev)
+    with torch.cuda.device(dev):
+        _check(_bf16_gemm_contig(a.data_ptr(), b.data_ptr(), d.data_ptr(), m_indices.data_ptr(),
+                                 M_sum, N, K, G, _stream_ptr(dev)),
+               "dg_m_grouped_bf16_gemm_nt_contiguous")
+    return d
+
+
+def m_grouped_bf16_gemm_nt_masked(a: torch.Tensor, b: torch.Tensor, masked_m: torch.Tensor,
+                                  expected_m: int, d: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Masked grouped GEMM on BF16 operands: ``D[g, m] = A[g, m] B[g]^T`` for
+    ``m < masked_m[g]``; other rows are never written."""
+    _bf16(a, "a"); _bf16(b, "b")
+    G, max_m, K = a.shape
+    N = b.shape[1]
+    dev = a.device
+    _need(a, "a", torch.bfloat16, (G, max_m, K), dev)
+    _need(b, "b", torch.bfloat16, (G, N, K), dev)
+    _need(masked_m, "masked_m", torch.int32, (G,), dev)
+    if d is None:
+        d = torch.empty((G, max_m, N), dtype=torch.bfloat16, device=dev)
+    _need(d, "d", torch.bfloat16, (G, max_m, N), dev)
+    with torch.cuda.device(dev):
+        _check(_bf16_gemm_masked(a.data_ptr(), b.data_ptr(), d.data_ptr(), masked_m.data_ptr(),
+                                 G, max_m, N, K, int(expected_m), _stream_ptr(dev)),
+               "dg_m_grouped_bf16_gemm_nt_masked")
     return d
 
 

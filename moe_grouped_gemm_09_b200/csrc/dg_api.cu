@@ -26,7 +26,7 @@ struct DeviceState {
   bool ready = false;
   int num_sms = 0;
   int* error_word = nullptr;      // one int, device memory
-  bool smem_attr_set[7][kNumVariants] = {};  // per form (below) and variant
+  bool smem_attr_set[10][kNumVariants] = {};  // per form (below) and variant
   bool limits_known = false;
   ClusterLimits limits = {};      // co-resident split-K clusters per variant and size
 };
@@ -159,18 +159,23 @@ int effective_sms(const DeviceState& st) {
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-// 4-D tensor map over E4M3 bytes [groups][rows][K] viewed as
-// {128 bytes of K, rows, K/128 blocks, groups} with strides {K, 128, rows*K}:
-// a box of {128, box_rows, kps, 1} brings kps K blocks of box_rows rows, laid
+// 4-D tensor map over an operand [groups][rows][K] whose rows are kb = K *
+// elem_bytes bytes (E4M3: 1, BF16: 2), viewed as {one 128-byte K block,
+// rows, kb/128 blocks, groups} with byte strides {kb, 128, rows*kb}: a box of
+// {128 bytes, box_rows, kps, 1} brings kps K blocks of box_rows rows, laid
 // out in shared memory as kps consecutive [box_rows][128 B] tiles with the
 // 128-byte swizzle.
 dg_status make_map(CUtensorMap* map, const void* base, uint64_t K, uint64_t rows, uint64_t groups,
-                   uint32_t box_rows, uint32_t kps) {
-  cuuint64_t dims[4] = {128, rows, K / 128, groups};
-  cuuint64_t strides[3] = {K, 128, K * rows};  // bytes, for dims 1..3
-  cuuint32_t box[4] = {128, box_rows, kps, 1};
+                   uint32_t box_rows, uint32_t kps, uint32_t elem_bytes = 1) {
+  const uint64_t kb = K * elem_bytes;
+  const cuuint32_t block = 128 / elem_bytes;  // elements of one 128-byte K block
+  cuuint64_t dims[4] = {block, rows, kb / 128, groups};
+  cuuint64_t strides[3] = {kb, 128, kb * rows};  // bytes, for dims 1..3
+  cuuint32_t box[4] = {block, box_rows, kps, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims,
+  CUresult r = g_encode(map, elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                             : CU_TENSOR_MAP_DATA_TYPE_UINT8,
+                        4, const_cast<void*>(base), dims,
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -191,11 +196,16 @@ dg_status make_d_map(CUtensorMap* map, void* base, uint64_t N, uint64_t rows) {
 }
 
 // Launch forms: the three GEMM forms, then the dense form with M-major A
-// and/or N-major B, then the dense form with FP32 output (D = A B^T + C); the
-// forms differ in their kernel instantiation.
+// and/or N-major B, then the dense form with FP32 output (D = A B^T + C),
+// then the three GEMM forms on BF16 operands; the forms differ in their
+// kernel instantiation.
 enum Form : int { kFormDense = 0, kFormContiguous = 1, kFormMasked = 2, kFormNN = 3, kFormTN = 4,
-                  kFormTT = 5, kFormF32 = 6 };
-constexpr int kind_of_form(int f) { return f < 3 ? f : kDense; }
+                  kFormTT = 5, kFormF32 = 6, kFormBf16Dense = 7, kFormBf16Contiguous = 8,
+                  kFormBf16Masked = 9 };
+constexpr bool is_bf16_form(int f) { return f >= kFormBf16Dense; }
+constexpr int kind_of_form(int f) {
+  return f < 3 ? f : is_bf16_form(f) ? f - kFormBf16Dense : kDense;
+}
 constexpr int layout_of_form(int f) {
   return f == kFormNN ? kLayoutNN : f == kFormTN ? kLayoutTN : f == kFormTT ? kLayoutTT : kLayoutNT;
 }
@@ -219,11 +229,14 @@ dg_status make_map_mn(CUtensorMap* map, const void* base, uint64_t mn, uint64_t 
   return r == CUDA_SUCCESS ? DG_OK : DG_ERR_CUDA;
 }
 
-template <int V>
+template <int V, bool SCALED = true>
 using ShapeOf = std::conditional_t<
     kVariants[V].pair, PairShape<kVariants[V].block_n, kVariants[V].stages>,
     KernelShape<kVariants[V].block_n, kVariants[V].stages, kVariants[V].num_acc,
-                kVariants[V].kps, kVariants[V].a_rows, kVariants[V].small>>;
+                kVariants[V].kps, kVariants[V].a_rows, kVariants[V].small, SCALED>>;
+// The geometry a form's kernel is built with (BF16 operands: no scale factors).
+template <int FORM, int V>
+using FormShape = ShapeOf<V, !is_bf16_form(FORM)>;
 
 // Kernels are instantiated only for the (form, variant) pairs that exist:
 // the decode, 256-row and pair variants serve the dense form only.
@@ -236,9 +249,11 @@ constexpr std::array<int, sizeof...(V)> variant_table(std::integer_sequence<int,
 template <int FORM, int V>
 constexpr bool kBuilt =
     FORM == kFormDense ||
-    ((FORM == kFormContiguous || FORM == kFormMasked) && !kVariants[V].decode &&
-     kVariants[V].a_rows != 256 && !kVariants[V].pair) ||
-    (FORM >= kFormNN && mn_capable(kVariants[V]));
+    ((FORM == kFormContiguous || FORM == kFormMasked || FORM == kFormBf16Contiguous ||
+      FORM == kFormBf16Masked) &&
+     !kVariants[V].decode && kVariants[V].a_rows != 256 && !kVariants[V].pair) ||
+    (FORM == kFormBf16Dense && kVariants[V].a_rows != 256 && !kVariants[V].pair) ||
+    (FORM >= kFormNN && FORM <= kFormF32 && mn_capable(kVariants[V]));
 
 template <int FORM, int V>
 auto kernel_of() {
@@ -247,7 +262,8 @@ auto kernel_of() {
     return fp8_gemm_pair_kernel<var.block_n, var.stages>;
   } else {
     return fp8_gemm_kernel<kind_of_form(FORM), var.block_n, var.stages, var.num_acc, var.kps,
-                           var.a_rows, var.small, layout_of_form(FORM), FORM == kFormF32>;
+                           var.a_rows, var.small, layout_of_form(FORM), FORM == kFormF32,
+                           is_bf16_form(FORM)>;
   }
 }
 
@@ -258,7 +274,7 @@ dg_status set_smem_attr(DeviceState& st) {
   } else {
     if (!st.smem_attr_set[KIND][V]) {
       if (cudaFuncSetAttribute(kernel_of<KIND, V>(), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               ShapeOf<V>::kSmemBytes) != cudaSuccess)
+                               FormShape<KIND, V>::kSmemBytes) != cudaSuccess)
         return DG_ERR_CUDA;
       st.smem_attr_set[KIND][V] = true;
     }
@@ -324,7 +340,7 @@ dg_status launch_variant(DeviceState& st, const CUtensorMap& ta, const CUtensorM
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid, 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = ShapeOf<V>::kSmemBytes;
+    cfg.dynamicSmemBytes = FormShape<KIND, V>::kSmemBytes;
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -367,13 +383,16 @@ dg_status run(int form, const void* a, const float* sfa, const void* b, const fl
   const int kind = kind_of_form(form);
   const int layout = layout_of_form(form);
   const bool a_mn = (layout & 1) != 0, b_mn = (layout & 2) != 0;
+  const bool bf16 = is_bf16_form(form);
   // ---- argument checks (no device work) ----
+  // A K block is 128 bytes of a row: 128 E4M3 or 64 BF16 elements.
+  const int k_block = bf16 ? kBlockK / 2 : kBlockK;
   if (rows < 0 || G < 0) return DG_ERR_INVALID_ARG;
-  if (K <= 0 || K % 128 != 0 || N <= 0 || N % 16 != 0) return DG_ERR_INVALID_ARG;
+  if (K <= 0 || K % k_block != 0 || N <= 0 || N % 16 != 0) return DG_ERR_INVALID_ARG;
   if (rows == 0 || G == 0) return DG_OK;
-  if (!a || !sfa || !b || !sfb || !d) return DG_ERR_INVALID_ARG;
-  if (!aligned(a, 16) || !aligned(b, 16) || !aligned(d, 16) || !aligned(sfa, 4) ||
-      !aligned(sfb, 4))
+  if (!a || !b || !d || (!bf16 && (!sfa || !sfb))) return DG_ERR_INVALID_ARG;
+  if (!aligned(a, 16) || !aligned(b, 16) || !aligned(d, 16) ||
+      (!bf16 && (!aligned(sfa, 4) || !aligned(sfb, 4))))
     return DG_ERR_INVALID_ARG;
   if (kind == kContiguous && (!m_indices || !aligned(m_indices, 4) || rows % 128 != 0))
     return DG_ERR_INVALID_ARG;
@@ -385,6 +404,8 @@ dg_status run(int form, const void* a, const float* sfa, const void* b, const fl
   if (a_rows > 0x7fffffffLL || static_cast<long long>(G) * N > 0x7fffffffLL)
     return DG_ERR_UNSUPPORTED;
   if (K > (1 << 24)) return DG_ERR_UNSUPPORTED;
+  // the picker and the kernel count K in 128-byte blocks of a row
+  const int k_bytes = bf16 ? 2 * K : K;
 
   std::lock_guard<std::mutex> lock(g_mutex);
   DeviceState* st = nullptr;
@@ -395,13 +416,14 @@ dg_status run(int form, const void* a, const float* sfa, const void* b, const fl
     s = ensure_cluster_limits(*st);
     if (s != DG_OK) return s;
   }
-  PickedConfig pc = pick_config(kind, rows, N, K, G, expected_m, sms, &st->limits,
-                                /*allow_pair=*/true,
+  PickedConfig pc = pick_config(kind, rows, N, k_bytes, G, expected_m, sms, &st->limits,
+                                /*allow_pair=*/!bf16,
                                 /*mn_operands=*/layout != kLayoutNT || form == kFormF32);
-  forced_config(kind, rows, N, K, G, sms, &pc);
+  forced_config(kind, rows, N, k_bytes, G, sms, &pc);
   const Variant var = kVariants[pc.variant];
   if ((layout != kLayoutNT || form == kFormF32) && (!mn_capable(var) || pc.split_k > 1))
     return DG_ERR_UNSUPPORTED;
+  if (bf16 && (var.pair || var.a_rows == 256)) return DG_ERR_UNSUPPORTED;
 
   GemmArgs args = {};
   args.rows = rows;
@@ -410,7 +432,7 @@ dg_status run(int form, const void* a, const float* sfa, const void* b, const fl
   args.G = (kind == kDense) ? 1 : G;
   args.num_m_blocks = ceil_div(rows, tile_rows(var));
   args.num_n_blocks = ceil_div(N, var.block_n);
-  args.k_blocks = K / kBlockK;
+  args.k_blocks = k_bytes / kBlockK;
   args.split_k = pc.split_k;
   args.kb_per_split = ceil_div(args.k_blocks, pc.split_k);
   args.nb128 = ceil_div(N, 128);
@@ -446,11 +468,13 @@ dg_status run(int form, const void* a, const float* sfa, const void* b, const fl
 
   CUtensorMap ta, tb;
   const int b_groups = (kind == kDense) ? 1 : G;
+  const uint32_t elem = bf16 ? 2 : 1;
   s = a_mn ? make_map_mn(&ta, a, rows, K)
-           : make_map(&ta, a, K, rows, kind == kMasked ? G : 1, args.a_box_rows, var.kps);
+           : make_map(&ta, a, K, rows, kind == kMasked ? G : 1, args.a_box_rows, var.kps, elem);
   if (s != DG_OK) return s;
   s = b_mn ? make_map_mn(&tb, b, N, K)
-           : make_map(&tb, b, K, N, b_groups, var.pair ? var.block_n / 2 : var.block_n, var.kps);
+           : make_map(&tb, b, K, N, b_groups, var.pair ? var.block_n / 2 : var.block_n, var.kps,
+                      elem);
   if (s != DG_OK) return s;
   CUtensorMap td;
   s = make_d_map(&td, d, N, static_cast<uint64_t>(a_rows));
@@ -472,7 +496,13 @@ dg_status run(int form, const void* a, const float* sfa, const void* b, const fl
     case kFormNN: return launch<kFormNN>(*st, pc.variant, ta, tb, td, args, pc.grid, stream);
     case kFormTN: return launch<kFormTN>(*st, pc.variant, ta, tb, td, args, pc.grid, stream);
     case kFormTT: return launch<kFormTT>(*st, pc.variant, ta, tb, td, args, pc.grid, stream);
-    default: return launch<kFormF32>(*st, pc.variant, ta, tb, td, args, pc.grid, stream);
+    case kFormF32: return launch<kFormF32>(*st, pc.variant, ta, tb, td, args, pc.grid, stream);
+    case kFormBf16Dense:
+      return launch<kFormBf16Dense>(*st, pc.variant, ta, tb, td, args, pc.grid, stream);
+    case kFormBf16Contiguous:
+      return launch<kFormBf16Contiguous>(*st, pc.variant, ta, tb, td, args, pc.grid, stream);
+    default:
+      return launch<kFormBf16Masked>(*st, pc.variant, ta, tb, td, args, pc.grid, stream);
   }
 }
 
@@ -527,6 +557,26 @@ dg_status dg_m_grouped_fp8_gemm_nt_masked(const void* a, const float* sfa, const
                                           dg_stream_t stream) {
   return run(kFormMasked, a, sfa, b, sfb, d, nullptr, masked_m, max_m, N, K, G, expected_m,
              reinterpret_cast<cudaStream_t>(stream));
+}
+
+dg_status dg_bf16_gemm_nt(const void* a, const void* b, void* d, int M, int N, int K,
+                          dg_stream_t stream) {
+  return run(kFormBf16Dense, a, nullptr, b, nullptr, d, nullptr, nullptr, M, N, K, 1, 0,
+             reinterpret_cast<cudaStream_t>(stream));
+}
+
+dg_status dg_m_grouped_bf16_gemm_nt_contiguous(const void* a, const void* b, void* d,
+                                               const int* m_indices, int M_sum, int N, int K,
+                                               int G, dg_stream_t stream) {
+  return run(kFormBf16Contiguous, a, nullptr, b, nullptr, d, m_indices, nullptr, M_sum, N, K, G,
+             0, reinterpret_cast<cudaStream_t>(stream));
+}
+
+dg_status dg_m_grouped_bf16_gemm_nt_masked(const void* a, const void* b, void* d,
+                                           const int* masked_m, int G, int max_m, int N, int K,
+                                           int expected_m, dg_stream_t stream) {
+  return run(kFormBf16Masked, a, nullptr, b, nullptr, d, nullptr, masked_m, max_m, N, K, G,
+             expected_m, reinterpret_cast<cudaStream_t>(stream));
 }
 
 dg_status dg_set_num_sms(int n) {

@@ -116,19 +116,23 @@ __host__ __device__ constexpr int pow2_ceil(int x) {
 //            CTAs per SM, so that the next kernel's CTAs can start (and warm
 //            L2) while this kernel drains; it runs one tile per CTA and
 //            stages its epilogue in the then idle operand ring
-template <int BLOCK_N, int STAGES, int NUM_ACC, int KPS = 1, int A_ROWS = 128, bool SMALL = false>
+//   SCALED   block-scaled E4M3 operands (scale factors staged per stage in
+//            shared memory and TMEM); false for BF16 operands, whose K block
+//            is 64 elements, the same 128 bytes of a row
+template <int BLOCK_N, int STAGES, int NUM_ACC, int KPS = 1, int A_ROWS = 128, bool SMALL = false,
+          bool SCALED = true>
 struct KernelShape {
   static constexpr int kHalves = A_ROWS == 256 ? 2 : 1;  // 128-row MMA halves of a tile
   static constexpr int kTileM = kBlockM * kHalves;        // output rows of a tile
-  static constexpr int kABytes = KPS * A_ROWS * kBlockK;  // one E4M3 byte per element
+  static constexpr int kABytes = KPS * A_ROWS * kBlockK;  // kBlockK bytes of a row per K block
   static constexpr int kBBytes = KPS * BLOCK_N * kBlockK;
   static constexpr int kSfbChunks = (BLOCK_N + 127) / 128;
   // 128-row scale blocks of B one tile can touch (a tile that is not aligned
   // to 128 rows straddles one more)
   static constexpr int kSfbBlocks = kSfbChunks + (BLOCK_N % 128 != 0 && 128 % BLOCK_N != 0 ? 1 : 0);
   // SFA 512 B per 128 rows of A + SFB 512 B per 128 rows of B
-  static constexpr int kSfBytes = 512 * (kHalves + kSfbChunks);
-  static constexpr int kSfCols = 4 * (kHalves + kSfbChunks);  // TMEM columns per stage
+  static constexpr int kSfBytes = SCALED ? 512 * (kHalves + kSfbChunks) : 0;
+  static constexpr int kSfCols = SCALED ? 4 * (kHalves + kSfbChunks) : 0;  // TMEM columns per stage
   static constexpr int kAccCols = NUM_ACC * kHalves * BLOCK_N;
   static constexpr int kTmemCols = pow2_ceil(kAccCols + STAGES * kSfCols);
   static constexpr int kBarBytes = 8 * (2 * STAGES + 2 * NUM_ACC + 2);
@@ -298,13 +302,16 @@ struct StageWalker {
   }
 };
 
+// BF16: the same GEMM forms on BF16 operands (no scales): the ring, the tile
+// scheduler, split-K and the epilogue are shared; the scale-factor warp idles
+// and every 128-byte K block is four kind::f16 MMAs (K = 16 each).
 template <int KIND, int BLOCK_N, int STAGES, int NUM_ACC, int KPS, int A_ROWS, bool SMALL,
-          int LAYOUT = kLayoutNT, bool OUT_F32 = false>
+          int LAYOUT = kLayoutNT, bool OUT_F32 = false, bool BF16 = false>
 __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     const __grid_constant__ CUtensorMap tmap_b,
                     const __grid_constant__ CUtensorMap tmap_d, const GemmArgs p) {
-  using Shape = KernelShape<BLOCK_N, STAGES, NUM_ACC, KPS, A_ROWS, SMALL>;
+  using Shape = KernelShape<BLOCK_N, STAGES, NUM_ACC, KPS, A_ROWS, SMALL, !BF16>;
   constexpr int A_BYTES = Shape::kABytes;
   constexpr int B_BYTES = Shape::kBBytes;
   constexpr int SF_BYTES = Shape::kSfBytes;
@@ -328,6 +335,8 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
   // tiles made of whole 128-column boxes.
   constexpr bool A_MN = (LAYOUT & 1) != 0;
   constexpr bool B_MN = (LAYOUT & 2) != 0;
+  static_assert(!BF16 || (LAYOUT == kLayoutNT && !OUT_F32),
+                "BF16 operands: K-major A and B, BF16 output");
   // FP32 output (D = A B^T + C): the dense form, no split-K (host-checked)
   static_assert(!OUT_F32 || (KIND == kDense && A_ROWS == 128 && !SMALL), "FP32 output form");
   static_assert(LAYOUT == kLayoutNT ||
@@ -366,7 +375,8 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      ptx::mbar_init(&full[s], 2);   // producer arrive.expect_tx + scale warp arrive
+      // producer arrive.expect_tx (+ the scale warp's arrive for E4M3 operands)
+      ptx::mbar_init(&full[s], BF16 ? 1 : 2);
       ptx::mbar_init(&empty[s], 1);  // tcgen05.commit
     }
     for (int a = 0; a < NUM_ACC; ++a) {
@@ -621,7 +631,22 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer --
     if constexpr (kLateWait) ptx::grid_dependency_wait();
-    constexpr uint32_t idesc = ptx::idesc_mxf8_e4m3_ue8m0(kBlockM, BLOCK_N, A_MN, B_MN);
+    constexpr uint32_t idesc = BF16 ? ptx::idesc_bf16_f32(kBlockM, BLOCK_N)
+                                    : ptx::idesc_mxf8_e4m3_ue8m0(kBlockM, BLOCK_N, A_MN, B_MN);
+    // Scale factors of ring slot s into its TMEM columns: SFA words of each
+    // 128-row half, then SFB words of each 128-row chunk of the tile's B rows.
+    auto copy_sf = [&](int s) {
+      const uint32_t sfa_tmem = tmem_base + ACC_COLS + s * SF_COLS;
+      const uint32_t sfb_tmem = sfa_tmem + 4 * HALVES;
+      const uint32_t sf_smem = ptx::smem_addr(sSF + s * SF_BYTES);
+#pragma unroll
+      for (int h = 0; h < HALVES; ++h)
+        ptx::tc_cp_32x128b_warpx4(sfa_tmem + 4 * h, ptx::sdesc_sf_32x16(sf_smem + 512 * h));
+#pragma unroll
+      for (int h = 0; h < SFB_CHUNKS; ++h)
+        ptx::tc_cp_32x128b_warpx4(sfb_tmem + 4 * h,
+                                  ptx::sdesc_sf_32x16(sf_smem + 512 * (HALVES + h)));
+    };
     int it = 0, acc_it = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
@@ -641,19 +666,29 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
         ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
         if (!ok) break;
         ptx::tc_fence_after_sync();
-        if (lane == 0) {
-          // per stage: SFA words of each 128-row half, then SFB words of
-          // each 128-row chunk of the tile's B rows
+        if (BF16 && lane == 0) {
+          // BF16 operands: four K = 16 MMAs per 128-byte K block, no scales
+          const uint32_t a_base = ptx::smem_addr(sA + s * A_BYTES);
+          const uint32_t b_base = ptx::smem_addr(sB + s * B_BYTES);
+#pragma unroll
+          for (int j = 0; j < KPS; ++j) {
+            if (kb + j >= ti.kb_end) break;
+            const uint64_t db = ptx::sdesc_kmajor_sw128(b_base + j * BLOCK_N * kBlockK);
+#pragma unroll
+            for (int h = 0; h < HALVES; ++h) {
+              const uint64_t da = ptx::sdesc_kmajor_sw128(a_base + j * p.a_box_rows * kBlockK +
+                                                          h * kBlockM * kBlockK);
+#pragma unroll
+              for (int ks = 0; ks < kBlockK / 32; ++ks)
+                ptx::tc_mma_bf16(d_tmem + h * BLOCK_N, da + (32 >> 4) * ks, db + (32 >> 4) * ks,
+                                 idesc, kb + j > ti.kb_begin || ks > 0);
+            }
+          }
+          ptx::tc_commit(&empty[s]);
+        } else if (!BF16 && lane == 0) {
           const uint32_t sfa_tmem = tmem_base + ACC_COLS + s * SF_COLS;
           const uint32_t sfb_tmem = sfa_tmem + 4 * HALVES;
-          const uint32_t sf_smem = ptx::smem_addr(sSF + s * SF_BYTES);
-#pragma unroll
-          for (int h = 0; h < HALVES; ++h)
-            ptx::tc_cp_32x128b_warpx4(sfa_tmem + 4 * h, ptx::sdesc_sf_32x16(sf_smem + 512 * h));
-#pragma unroll
-          for (int h = 0; h < SFB_CHUNKS; ++h)
-            ptx::tc_cp_32x128b_warpx4(sfb_tmem + 4 * h,
-                                      ptx::sdesc_sf_32x16(sf_smem + 512 * (HALVES + h)));
+          copy_sf(s);
           const uint32_t a_base = ptx::smem_addr(sA + s * A_BYTES);
           const uint32_t b_base = ptx::smem_addr(sB + s * B_BYTES);
 #pragma unroll
@@ -700,7 +735,7 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
       ptx::mbar_wait_drain(drain, 0, 50000000ull);
     }
     __syncwarp();
-  } else if (warp == 2) {
+  } else if (warp == 2 && !BF16) {
     // --------------------------------------------- scale-factor producer --
     // The FP32 scales of a stage are loaded PF stages before they are
     // written, so the global-load latency overlaps several pipeline stages.

@@ -398,6 +398,18 @@ __device__ __forceinline__ void tc_mma_mxf8_block_scale(uint32_t d_tmem, uint64_
       : "memory");
 }
 
+// D (+)= A * B^T on BF16 operands (kind::f16, K = 16 per instruction, FP32
+// accumulator in TMEM), no scale factors.
+__device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, bool accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate ? 1u : 0u)
+      : "memory");
+}
+
 // Each thread of the warp reads 32 consecutive 32-bit columns of its own TMEM
 // lane (lane quarter = warp index % 4).
 __device__ __forceinline__ void tc_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[32]) {
@@ -474,6 +486,16 @@ __host__ __device__ constexpr uint32_t idesc_mxf8_e4m3_ue8m0(int m, int n, bool 
          | (1u << 23)                             // scale format: UE8M0
          | (static_cast<uint32_t>(m >> 4) << 24)  // M / 16
          | (0u << 29);                            // A scale-factor byte id
+}
+
+// Instruction descriptor of tcgen05.mma.kind::f16 for BF16 x BF16 operands,
+// both K-major, FP32 accumulation, M = m, N = n (multiple of 16 up to 256).
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int m, int n) {
+  return (1u << 4)                                // D format: F32
+         | (1u << 7)                              // A format: BF16
+         | (1u << 10)                             // B format: BF16
+         | (static_cast<uint32_t>(n >> 3) << 17)  // N / 8
+         | (static_cast<uint32_t>(m >> 4) << 24); // M / 16
 }
 
 }  // namespace ptx

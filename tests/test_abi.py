@@ -82,6 +82,20 @@ def test_f32_form_rejects_bad_arguments(dg):
     assert dg._gemm_nt_f32(None, None, None, None, None, None, 0, 16, 128, None) == 0
 
 
+def test_bf16_forms_reject_bad_arguments(dg):
+    # K must be a whole number of 64-element (128-byte) blocks; no scales needed
+    assert dg._bf16_gemm_nt(FAKE, FAKE, FAKE, 4, 16, 96, None) == 1
+    assert dg._bf16_gemm_nt(FAKE, FAKE, FAKE, 4, 15, 64, None) == 1
+    assert dg._bf16_gemm_nt(None, FAKE, FAKE, 4, 16, 64, None) == 1
+    assert dg._bf16_gemm_nt(FAKE, FAKE, FAKE + 8, 4, 16, 64, None) == 1
+    assert dg._bf16_gemm_nt(None, None, None, 0, 16, 64, None) == 0
+    assert dg._bf16_gemm_contig(FAKE, FAKE, FAKE, FAKE, 100, 16, 64, 2, None) == 1
+    assert dg._bf16_gemm_contig(FAKE, FAKE, FAKE, None, 128, 16, 64, 2, None) == 1
+    assert dg._bf16_gemm_masked(FAKE, FAKE, FAKE, None, 2, 64, 16, 64, 1, None) == 1
+    assert dg._bf16_gemm_masked(FAKE, FAKE, FAKE, FAKE, 5000, 64, 16, 64, 1, None) == 2
+    assert dg._bf16_gemm_masked(None, None, None, None, 0, 64, 16, 64, 1, None) == 0
+
+
 def test_zero_rows_is_a_noop(dg):
     # no device is touched for an empty problem, even with null pointers
     assert dg._gemm_nt(None, None, None, None, None, 0, 16, 128, None) == 0

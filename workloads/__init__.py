@@ -2,11 +2,12 @@
 oracle checks and the benchmark.
 
 This module only *produces inputs*: random FP32 matrices, their quantisation to
-FP8 E4M3 with power-of-two block scales, and the MoE group structure (per-expert
-token counts, ``m_indices``, ``masked_m``).  It holds none of the GEMM's own
-arithmetic: no decoding of E4M3 bytes, no scale application, no accumulation and
-no BF16 rounding.  Those live, independently, in ``oracle/`` (CPU) and in the
-CUDA library.
+FP8 E4M3 with power-of-two block scales (or, for the BF16-operand GEMM, their
+rounding to BF16 operands by ``ml_dtypes``), and the MoE group structure
+(per-expert token counts, ``m_indices``, ``masked_m``).  It holds none of the
+GEMM's own arithmetic: no decoding of operands, no scale application, no
+accumulation and no rounding of the result.  Those live, independently, in
+``oracle/`` (CPU) and in the CUDA library.
 
 Input recipe (the pages' workloads are DeepSeek-V3/R1 inference GEMMs, prefill
 and decode, dense and MoE-grouped; see the DeepGEMM release articles, sections on
@@ -24,7 +25,9 @@ performance and on the MoE grouped layouts):
   each expert's segment padded up to a multiple of 128 rows, padding rows marked
   ``-1`` in ``m_indices`` and filled with random FP8 bytes (so that a kernel that
   forgets to skip them is caught);
-* masked grouped layout: ``masked_m[g]`` uniform in ``[0, max_m]``.
+* masked grouped layout: ``masked_m[g]`` uniform in ``[0, max_m]``;
+* BF16 operands: the same N(0, 1) values (same streams) rounded to BF16 with
+  round-to-nearest-even, and the same group structure; no scales.
 """
 from __future__ import annotations
 
@@ -222,6 +225,105 @@ def masked_problem(G: int = 32, max_m: int = 256, N: int = 4096, K: int = 7168, 
         expected_m = max(1, int(round(float(np.clip(masked_m, 0, max_m).mean()))))
     return MaskedProblem(qa.reshape(G, max_m, K), sa.reshape(G, max_m, K // BLOCK_K), qb, sb,
                          masked_m, G, max_m, N, K, int(expected_m))
+
+
+def to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """FP32 values -> BF16 operand bit patterns (round to nearest even, ml_dtypes)."""
+    return np.asarray(x, np.float32).astype(ml_dtypes.bfloat16).view(np.uint16)
+
+
+@dataclasses.dataclass
+class Bf16DenseProblem:
+    a: np.ndarray     # uint16 [M, K]  BF16 bits, K-major
+    b: np.ndarray     # uint16 [N, K]  BF16 bits, K-major
+    M: int
+    N: int
+    K: int
+
+    def flops(self) -> float:
+        return 2.0 * self.M * self.N * self.K
+
+    def bytes(self) -> float:
+        return float(self.a.nbytes + self.b.nbytes + 2 * self.M * self.N)
+
+
+def bf16_dense_problem(M: int, N: int, K: int, seed: int = 0) -> Bf16DenseProblem:
+    a = to_bf16_bits(_normal(_rng(seed, _TAG_A), (M, K)))
+    b = to_bf16_bits(_normal(_rng(seed, _TAG_B, 0), (N, K)))
+    return Bf16DenseProblem(a, b, M, N, K)
+
+
+@dataclasses.dataclass
+class Bf16ContiguousProblem:
+    a: np.ndarray          # uint16 [M_sum, K]
+    b: np.ndarray          # uint16 [G, N, K]
+    m_indices: np.ndarray  # int32 [M_sum]; expert id or -1 for padding rows
+    counts: np.ndarray     # int64 [G]
+    M_sum: int
+    N: int
+    K: int
+    G: int
+
+    def valid_rows(self) -> int:
+        return int((self.m_indices >= 0).sum())
+
+    def flops(self) -> float:
+        return 2.0 * self.valid_rows() * self.N * self.K
+
+    def bytes(self) -> float:
+        used = int((self.counts > 0).sum())
+        v = self.valid_rows()
+        return float(2 * v * self.K + used * 2 * self.N * self.K + 2 * v * self.N + 4 * self.M_sum)
+
+
+def bf16_contiguous_problem(G: int, N: int, K: int, counts: np.ndarray, align: int = 128,
+                            seed: int = 0) -> Bf16ContiguousProblem:
+    counts = np.asarray(counts, dtype=np.int64)
+    assert counts.shape == (G,)
+    padded = -(-counts // align) * align
+    M_sum = int(padded.sum())
+    m_indices = np.full(M_sum, -1, np.int32)
+    off = 0
+    for g in range(G):
+        m_indices[off:off + counts[g]] = g
+        off += int(padded[g])
+    a = to_bf16_bits(_normal(_rng(seed, _TAG_A), (M_sum, K)))
+    b = np.stack([to_bf16_bits(_normal(_rng(seed, _TAG_B, g), (N, K))) for g in range(G)])
+    return Bf16ContiguousProblem(a, b, m_indices, counts, M_sum, N, K, G)
+
+
+@dataclasses.dataclass
+class Bf16MaskedProblem:
+    a: np.ndarray         # uint16 [G, max_m, K]
+    b: np.ndarray         # uint16 [G, N, K]
+    masked_m: np.ndarray  # int32 [G]
+    G: int
+    max_m: int
+    N: int
+    K: int
+    expected_m: int
+
+    def valid_rows(self) -> int:
+        return int(np.clip(self.masked_m, 0, self.max_m).sum())
+
+    def flops(self) -> float:
+        return 2.0 * self.valid_rows() * self.N * self.K
+
+    def bytes(self) -> float:
+        mm = np.clip(self.masked_m, 0, self.max_m)
+        v = int(mm.sum())
+        used = int((mm > 0).sum())
+        return float(2 * v * self.K + used * 2 * self.N * self.K + 2 * v * self.N + 4 * self.G)
+
+
+def bf16_masked_problem(G: int, max_m: int, N: int, K: int, masked_m: np.ndarray,
+                        seed: int = 0) -> Bf16MaskedProblem:
+    masked_m = np.asarray(masked_m, dtype=np.int32)
+    assert masked_m.shape == (G,)
+    a = to_bf16_bits(_normal(_rng(seed, _TAG_A), (G * max_m, K))).reshape(G, max_m, K)
+    b = np.stack([to_bf16_bits(_normal(_rng(seed, _TAG_B, g), (N, K))) for g in range(G)])
+    expected_m = max(1, int(round(float(np.clip(masked_m, 0, max_m).mean()))))
+    return Bf16MaskedProblem(a, b, masked_m, G, max_m, N, K, expected_m)
 
 
 def sentinel_d(*shape: int) -> np.ndarray:
