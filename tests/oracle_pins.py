@@ -325,7 +325,8 @@ def pin_masked(o, seed=16):
 def decode_bf16_np(bits) -> np.ndarray:
     """BF16 bit patterns -> float64 by widening to FP32 bit patterns
     (independent of the oracle's table)."""
-    return (np.asarray(bits, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    with np.errstate(invalid="ignore"):  # NaN patterns widen to NaN
+        return (np.asarray(bits, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
 def random_bf16(rng, shape, scale=1.0) -> np.ndarray:
