@@ -133,6 +133,10 @@ struct KernelShape {
   // SFA 512 B per 128 rows of A + SFB 512 B per 128 rows of B
   static constexpr int kSfBytes = SCALED ? 512 * (kHalves + kSfbChunks) : 0;
   static constexpr int kSfCols = SCALED ? 4 * (kHalves + kSfbChunks) : 0;  // TMEM columns per stage
+  // stages whose K blocks share one set of scale words: four one-block
+  // stages; a stage of several K blocks has words of its own (the decode
+  // variants, where the per-stage scale path measured faster)
+  static constexpr int kSfGroup = KPS == 1 ? 4 : 1;
   static constexpr int kAccCols = NUM_ACC * kHalves * BLOCK_N;
   static constexpr int kTmemCols = pow2_ceil(kAccCols + STAGES * kSfCols);
   static constexpr int kBarBytes = 8 * (2 * STAGES + 2 * NUM_ACC + 2);
@@ -157,7 +161,8 @@ struct KernelShape {
                 "a single-tile CTA stages its whole output tile in the ring");
   static_assert(kTmemCols <= 512, "TMEM budget exceeded");
   static_assert(BLOCK_N % 32 == 0 && BLOCK_N >= 32 && BLOCK_N <= 256, "BLOCK_N");
-  static_assert(KPS >= 1 && KPS <= 4, "up to four K blocks share one scale-factor word");
+  static_assert(KPS >= 1 && KPS <= 4 && 4 % KPS == 0,
+                "four K blocks (a whole number of stages) share one scale-factor word");
   static_assert(A_ROWS == 64 || A_ROWS == 128 || A_ROWS == 256, "A_ROWS");
   static_assert(A_ROWS != 256 || (!SMALL && KPS == 1), "two-half tiles are general variants");
   static_assert((BLOCK_N * kBlockK) % 1024 == 0, "B sub-tiles must keep 1024-byte alignment");
@@ -320,6 +325,7 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
   constexpr int SFB_BLOCKS = Shape::kSfbBlocks;
   constexpr int HALVES = Shape::kHalves;
   constexpr int TILE_M = Shape::kTileM;
+  constexpr int SF_GROUP = Shape::kSfGroup;
   constexpr int ACC_COLS = Shape::kAccCols;
   constexpr int TMEM_COLS = Shape::kTmemCols;
   constexpr int RED_PITCH = BLOCK_N + 4;  // floats per row of a parked split-K partial
@@ -633,12 +639,13 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
     if constexpr (kLateWait) ptx::grid_dependency_wait();
     constexpr uint32_t idesc = BF16 ? ptx::idesc_bf16_f32(kBlockM, BLOCK_N)
                                     : ptx::idesc_mxf8_e4m3_ue8m0(kBlockM, BLOCK_N, A_MN, B_MN);
-    // Scale factors of ring slot s into its TMEM columns: SFA words of each
-    // 128-row half, then SFB words of each 128-row chunk of the tile's B rows.
-    auto copy_sf = [&](int s) {
-      const uint32_t sfa_tmem = tmem_base + ACC_COLS + s * SF_COLS;
+    // Scale words of one group, from its shared-memory slot into the TMEM
+    // columns of the same slot: SFA words of each 128-row half, then SFB
+    // words of each 128-row chunk of the tile's B rows.
+    auto copy_sf = [&](int slot) {
+      const uint32_t sfa_tmem = tmem_base + ACC_COLS + slot * SF_COLS;
       const uint32_t sfb_tmem = sfa_tmem + 4 * HALVES;
-      const uint32_t sf_smem = ptx::smem_addr(sSF + s * SF_BYTES);
+      const uint32_t sf_smem = ptx::smem_addr(sSF + slot * SF_BYTES);
 #pragma unroll
       for (int h = 0; h < HALVES; ++h)
         ptx::tc_cp_32x128b_warpx4(sfa_tmem + 4 * h, ptx::sdesc_sf_32x16(sf_smem + 512 * h));
@@ -648,6 +655,12 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
                                   ptx::sdesc_sf_32x16(sf_smem + 512 * (HALVES + h)));
     };
     int it = 0, acc_it = 0;
+    // scale-word groups walked, and the slot of the current group's words:
+    // the slot of a group is its count modulo STAGES, in shared memory and
+    // TMEM alike.  A group has at least one stage, so the slot's previous
+    // group ended at least STAGES stages earlier, and its MMAs (and copy)
+    // are complete once this stage's full barrier has flipped.
+    int gc = 0, sf_slot = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
       const Tile ti = get_tile<KIND>(t, p, s_prefix, lane);
@@ -662,6 +675,12 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
       for (int kb = ti.kb_begin; kb < ti.kb_end; kb += KPS, ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
+        const int q = (kb - ti.kb_begin) / KPS;  // stage within the tile
+        const bool group_first = q % SF_GROUP == 0;
+        if (group_first) {
+          sf_slot = gc % STAGES;
+          ++gc;
+        }
         if (lane == 0) ok = ptx::mbar_wait(&full[s], ph, ctl, kDevTimeoutMma);
         ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
         if (!ok) break;
@@ -686,16 +705,18 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
           }
           ptx::tc_commit(&empty[s]);
         } else if (!BF16 && lane == 0) {
-          const uint32_t sfa_tmem = tmem_base + ACC_COLS + s * SF_COLS;
+          const uint32_t sfa_tmem = tmem_base + ACC_COLS + sf_slot * SF_COLS;
           const uint32_t sfb_tmem = sfa_tmem + 4 * HALVES;
-          copy_sf(s);
+          if (group_first) copy_sf(sf_slot);
           const uint32_t a_base = ptx::smem_addr(sA + s * A_BYTES);
           const uint32_t b_base = ptx::smem_addr(sB + s * B_BYTES);
 #pragma unroll
           for (int j = 0; j < KPS; ++j) {
             if (kb + j >= ti.kb_end) break;
-            // K block j of the stage: its scale factors are byte j of every
-            // TMEM scale word (selected by the scale-factor id)
+            // K block j of the stage is K block sb of its group: its scale
+            // factors are byte sb of every TMEM scale word (selected by the
+            // scale-factor id)
+            const uint32_t sb = static_cast<uint32_t>((q % SF_GROUP) * KPS + j);
             // a K step of 32 moves 32 bytes along a K-major row, or 4 swizzle
             // atoms (4096 bytes) down an M-/N-major tile
             constexpr uint32_t kStepA = A_MN ? 4096 >> 4 : 32 >> 4;
@@ -703,8 +724,8 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
             const uint64_t db =
                 B_MN ? ptx::sdesc_mnmajor_sw128(b_base, 128 * kBlockK)
                      : ptx::sdesc_kmajor_sw128(b_base + j * BLOCK_N * kBlockK);
-            const uint32_t id = idesc | (static_cast<uint32_t>(j) << 29) | (static_cast<uint32_t>(j) << 4);
-            const uint32_t byte_sel = static_cast<uint32_t>(j) << 30;
+            const uint32_t id = idesc | (sb << 29) | (sb << 4);
+            const uint32_t byte_sel = sb << 30;
 #pragma unroll
             for (int h = 0; h < HALVES; ++h) {
               // half h: A rows 128h.. of the stage's tile, its own accumulator
@@ -736,108 +757,253 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
     }
     __syncwarp();
   } else if (warp == 2 && !BF16) {
-    // --------------------------------------------- scale-factor producer --
-    // The FP32 scales of a stage are loaded PF stages before they are
-    // written, so the global-load latency overlaps several pipeline stages.
-    // Scale words pack the stage's K blocks: byte j belongs to K block j.
-    constexpr int PF = (8 + KPS - 1) / KPS;
-    const int KB = p.k_blocks;
-    float va[PF][HALVES][4][KPS];
-    float vb[PF][SFB_BLOCKS][KPS];
-    StageWalker<KIND, KPS> ld, wr;
-    ld.start(blockIdx.x, gridDim.x, total, p, s_prefix, lane);
-    wr.start(blockIdx.x, gridDim.x, total, p, s_prefix, lane);
-    if constexpr (kLateWait) ptx::grid_dependency_wait();
+    if constexpr (SF_GROUP == 1) {
+      // --------------------------------------------- scale-factor producer --
+      // The FP32 scales of a stage are loaded PF stages before they are
+      // written, so the global-load latency overlaps several pipeline stages.
+      // Scale words pack the stage's K blocks: byte j belongs to K block j.
+      constexpr int PF = (8 + KPS - 1) / KPS;
+      const int KB = p.k_blocks;
+      float va[PF][HALVES][4][KPS];
+      float vb[PF][SFB_BLOCKS][KPS];
+      StageWalker<KIND, KPS> ld, wr;
+      ld.start(blockIdx.x, gridDim.x, total, p, s_prefix, lane);
+      wr.start(blockIdx.x, gridDim.x, total, p, s_prefix, lane);
+      if constexpr (kLateWait) ptx::grid_dependency_wait();
 
-    auto issue = [&](float (&a)[HALVES][4][KPS], float (&b)[SFB_BLOCKS][KPS]) {
-      const Tile& ti = ld.w.ti;
-#pragma unroll
-      for (int h = 0; h < HALVES; ++h) {
-        const int m0 = ti.m_blk * TILE_M + kBlockM * h;  // first row of this half
-        const int row_base = (KIND == kMasked ? ti.group * p.rows : 0) + m0;
-        const int rows_left = p.rows - m0;  // rows of this half that exist
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int r = 32 * c + lane;
-#pragma unroll
+      auto issue = [&](float (&a)[HALVES][4][KPS], float (&b)[SFB_BLOCKS][KPS]) {
+        const Tile& ti = ld.w.ti;
+  #pragma unroll
+        for (int h = 0; h < HALVES; ++h) {
+          const int m0 = ti.m_blk * TILE_M + kBlockM * h;  // first row of this half
+          const int row_base = (KIND == kMasked ? ti.group * p.rows : 0) + m0;
+          const int rows_left = p.rows - m0;  // rows of this half that exist
+  #pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const int r = 32 * c + lane;
+  #pragma unroll
+            for (int j = 0; j < KPS; ++j)
+              a[h][c][j] = (r < rows_left && ld.kb + j < ti.kb_end)
+                               ? __ldg(p.sfa + (size_t)(row_base + r) * KB + ld.kb + j)
+                               : 1.0f;
+          }
+        }
+        // B scale blocks are 128 rows: the tile's rows touch blocks b0, b0 + 1, ...
+        const float* sfb_g = p.sfb + (size_t)ti.group * p.nb128 * KB;
+        const int b0 = ti.n_blk * BLOCK_N / 128;
+  #pragma unroll
+        for (int i = 0; i < SFB_BLOCKS; ++i) {
+          const int nb = min(b0 + i, p.nb128 - 1);
+  #pragma unroll
           for (int j = 0; j < KPS; ++j)
-            a[h][c][j] = (r < rows_left && ld.kb + j < ti.kb_end)
-                             ? __ldg(p.sfa + (size_t)(row_base + r) * KB + ld.kb + j)
-                             : 1.0f;
+            b[i][j] = (ld.kb + j < ti.kb_end) ? __ldg(sfb_g + (size_t)nb * KB + ld.kb + j) : 1.0f;
+        }
+        ld.next(p, s_prefix, lane);
+      };
+
+  #pragma unroll
+      for (int j = 0; j < PF; ++j)
+        if (!ld.done) issue(va[j], vb[j]);
+
+      int it = 0;
+      bool ok = true;
+      while (!wr.done && ok) {
+  #pragma unroll
+        for (int slot = 0; slot < PF; ++slot) {
+          if (wr.done || !ok) break;
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (lane == 0) ok = ptx::mbar_wait(&empty[s], ph ^ 1, ctl, kDevTimeoutScales);
+          ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+          if (!ok) break;
+          uint8_t* sf = sSF + s * SF_BYTES;
+          // A scales: TMEM lane l, column c holds row 32c + l of the half.
+  #pragma unroll
+          for (int h = 0; h < HALVES; ++h) {
+            uint32_t w[4];
+  #pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              uint32_t x = 0x7F7F7F7Fu;  // unused bytes: scale 1
+  #pragma unroll
+              for (int j = 0; j < KPS; ++j)
+                x = (x & ~(0xFFu << (8 * j))) | (ue8m0(va[slot][h][c][j]) << (8 * j));
+              w[c] = x;
+            }
+            *reinterpret_cast<uint4*>(sf + 512 * h + 16 * lane) = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+          // B scales, same layout per 128-row chunk of the tile's B rows: row
+          // r of the tile takes the scale of its own 128-row block of B
+          const int n_off = (wr.w.ti.n_blk * BLOCK_N) % 128;  // tile start within its block
+  #pragma unroll
+          for (int h = 0; h < SFB_CHUNKS; ++h) {
+            uint32_t w[4];
+  #pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const int idx = min((n_off + 128 * h + 32 * c + lane) / 128, SFB_BLOCKS - 1);
+              uint32_t x = 0x7F7F7F7Fu;
+  #pragma unroll
+              for (int j = 0; j < KPS; ++j) {
+                float v = vb[slot][0][j];
+  #pragma unroll
+                for (int i = 1; i < SFB_BLOCKS; ++i)
+                  if (idx == i) v = vb[slot][i][j];
+                x = (x & ~(0xFFu << (8 * j))) | (ue8m0(v) << (8 * j));
+              }
+              w[c] = x;
+            }
+            *reinterpret_cast<uint4*>(sf + 512 * (HALVES + h) + 16 * lane) =
+                make_uint4(w[0], w[1], w[2], w[3]);
+          }
+          ptx::fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(&full[s]);
+          if (!ld.done) issue(va[slot], vb[slot]);
+          wr.next(p, s_prefix, lane);
+          ++it;
         }
       }
-      // B scale blocks are 128 rows: the tile's rows touch blocks b0, b0 + 1, ...
-      const float* sfb_g = p.sfb + (size_t)ti.group * p.nb128 * KB;
-      const int b0 = ti.n_blk * BLOCK_N / 128;
-#pragma unroll
-      for (int i = 0; i < SFB_BLOCKS; ++i) {
-        const int nb = min(b0 + i, p.nb128 - 1);
-#pragma unroll
-        for (int j = 0; j < KPS; ++j)
-          b[i][j] = (ld.kb + j < ti.kb_end) ? __ldg(sfb_g + (size_t)nb * KB + ld.kb + j) : 1.0f;
-      }
-      ld.next(p, s_prefix, lane);
-    };
+    } else {
+      // --------------------------------------------- scale-factor producer --
+      // A tile's K blocks form groups of up to four (SF_GROUP stages of KPS
+      // blocks), and one set of scale words serves a whole group: byte b of a
+      // word is the group's K block b, selected by the MMA's scale-factor id,
+      // so a group costs one tcgen05.cp instead of one per stage.  A group's
+      // words go to the shared-memory slot of the group counter modulo STAGES
+      // at the group's first stage; every stage still takes its empty slot and
+      // arrives on its full barrier.  The FP32 scales of a group are loaded
+      // two groups ahead (a float4 per row when the rows allow it).
+      constexpr int GK = SF_GROUP * KPS;  // K blocks of a full group (4)
+      const int KB = p.k_blocks;
+      float va[2][HALVES][4][GK];
+      float vb[2][SFB_BLOCKS][GK];
+      StageWalker<KIND, GK> ld;    // walks the groups
+      StageWalker<KIND, KPS> wr;   // walks the stages
+      ld.start(blockIdx.x, gridDim.x, total, p, s_prefix, lane);
+      wr.start(blockIdx.x, gridDim.x, total, p, s_prefix, lane);
+      if constexpr (kLateWait) ptx::grid_dependency_wait();
+      // rows of sfa and sfb start on 16-byte boundaries: whole float4s per group
+      const bool vec = GK == 4 && KB % 4 == 0 &&
+                       (reinterpret_cast<uintptr_t>(p.sfa) & 15) == 0 &&
+                       (reinterpret_cast<uintptr_t>(p.sfb) & 15) == 0;
 
-#pragma unroll
-    for (int j = 0; j < PF; ++j)
-      if (!ld.done) issue(va[j], vb[j]);
+      auto issue = [&](float (&a)[HALVES][4][GK], float (&b)[SFB_BLOCKS][GK]) {
+        const Tile& ti = ld.w.ti;
+        const int kb0 = ld.kb;                       // first K block of the group
+        const bool v4 = vec && (kb0 & 3) == 0;       // then kb0 + 4 <= KB as well
+  #pragma unroll
+        for (int h = 0; h < HALVES; ++h) {
+          const int m0 = ti.m_blk * TILE_M + kBlockM * h;  // first row of this half
+          const int row_base = (KIND == kMasked ? ti.group * p.rows : 0) + m0;
+          const int rows_left = p.rows - m0;  // rows of this half that exist
+  #pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const int r = 32 * c + lane;
+            const float* src = p.sfa + (size_t)(row_base + r) * KB + kb0;
+            if (r < rows_left && v4) {
+              const float4 x = __ldg(reinterpret_cast<const float4*>(src));
+              a[h][c][0] = x.x; a[h][c][1] = x.y; a[h][c][2] = x.z; a[h][c][3] = x.w;
+            } else {
+  #pragma unroll
+              for (int j = 0; j < GK; ++j)
+                a[h][c][j] = (r < rows_left && kb0 + j < ti.kb_end) ? __ldg(src + j) : 1.0f;
+            }
+          }
+        }
+        // B scale blocks are 128 rows: the tile's rows touch blocks b0, b0 + 1, ...
+        const float* sfb_g = p.sfb + (size_t)ti.group * p.nb128 * KB;
+        const int b0 = ti.n_blk * BLOCK_N / 128;
+  #pragma unroll
+        for (int i = 0; i < SFB_BLOCKS; ++i) {
+          const int nb = min(b0 + i, p.nb128 - 1);
+          const float* src = sfb_g + (size_t)nb * KB + kb0;
+          if (v4) {
+            const float4 x = __ldg(reinterpret_cast<const float4*>(src));
+            b[i][0] = x.x; b[i][1] = x.y; b[i][2] = x.z; b[i][3] = x.w;
+          } else {
+  #pragma unroll
+            for (int j = 0; j < GK; ++j)
+              b[i][j] = (kb0 + j < ti.kb_end) ? __ldg(src + j) : 1.0f;
+          }
+        }
+        ld.next(p, s_prefix, lane);
+      };
 
-    int it = 0;
-    bool ok = true;
-    while (!wr.done && ok) {
-#pragma unroll
-      for (int slot = 0; slot < PF; ++slot) {
-        if (wr.done || !ok) break;
+      if (!ld.done) issue(va[0], vb[0]);
+      if (!ld.done) issue(va[1], vb[1]);
+
+      int it = 0, gc = 0;  // stages and groups walked
+      bool ok = true;
+      // one stage: take its empty slot, (at a group's first stage) write the
+      // group's words, arrive on its full barrier
+      auto stage = [&](bool first, const float (&a)[HALVES][4][GK],
+                       const float (&b)[SFB_BLOCKS][GK]) -> bool {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
-        if (lane == 0) ok = ptx::mbar_wait(&empty[s], ph ^ 1, ctl, kDevTimeoutScales);
-        ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-        if (!ok) break;
-        uint8_t* sf = sSF + s * SF_BYTES;
-        // A scales: TMEM lane l, column c holds row 32c + l of the half.
-#pragma unroll
-        for (int h = 0; h < HALVES; ++h) {
-          uint32_t w[4];
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t x = 0x7F7F7F7Fu;  // unused bytes: scale 1
-#pragma unroll
-            for (int j = 0; j < KPS; ++j)
-              x = (x & ~(0xFFu << (8 * j))) | (ue8m0(va[slot][h][c][j]) << (8 * j));
-            w[c] = x;
-          }
-          *reinterpret_cast<uint4*>(sf + 512 * h + 16 * lane) = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-        // B scales, same layout per 128-row chunk of the tile's B rows: row
-        // r of the tile takes the scale of its own 128-row block of B
-        const int n_off = (wr.w.ti.n_blk * BLOCK_N) % 128;  // tile start within its block
-#pragma unroll
-        for (int h = 0; h < SFB_CHUNKS; ++h) {
-          uint32_t w[4];
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const int idx = min((n_off + 128 * h + 32 * c + lane) / 128, SFB_BLOCKS - 1);
-            uint32_t x = 0x7F7F7F7Fu;
-#pragma unroll
-            for (int j = 0; j < KPS; ++j) {
-              float v = vb[slot][0][j];
-#pragma unroll
-              for (int i = 1; i < SFB_BLOCKS; ++i)
-                if (idx == i) v = vb[slot][i][j];
-              x = (x & ~(0xFFu << (8 * j))) | (ue8m0(v) << (8 * j));
+        bool good = true;
+        if (lane == 0) good = ptx::mbar_wait(&empty[s], ph ^ 1, ctl, kDevTimeoutScales);
+        good = __shfl_sync(0xFFFFFFFFu, good, 0);
+        if (!good) return false;
+        if (first) {
+          uint8_t* sf = sSF + (gc % STAGES) * SF_BYTES;
+          const int n_valid = min(GK, wr.w.ti.kb_end - wr.kb);  // K blocks of this group
+          // A scales: TMEM lane l, column c holds row 32c + l of the half.
+  #pragma unroll
+          for (int h = 0; h < HALVES; ++h) {
+            uint32_t w[4];
+  #pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              uint32_t x = 0x7F7F7F7Fu;  // unused bytes: scale 1
+  #pragma unroll
+              for (int j = 0; j < GK; ++j)
+                if (j < n_valid) x = (x & ~(0xFFu << (8 * j))) | (ue8m0(a[h][c][j]) << (8 * j));
+              w[c] = x;
             }
-            w[c] = x;
+            *reinterpret_cast<uint4*>(sf + 512 * h + 16 * lane) = make_uint4(w[0], w[1], w[2], w[3]);
           }
-          *reinterpret_cast<uint4*>(sf + 512 * (HALVES + h) + 16 * lane) =
-              make_uint4(w[0], w[1], w[2], w[3]);
+          // B scales, same layout per 128-row chunk of the tile's B rows: row
+          // r of the tile takes the scale of its own 128-row block of B
+          const int n_off = (wr.w.ti.n_blk * BLOCK_N) % 128;  // tile start within its block
+  #pragma unroll
+          for (int h = 0; h < SFB_CHUNKS; ++h) {
+            uint32_t w[4];
+  #pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const int idx = min((n_off + 128 * h + 32 * c + lane) / 128, SFB_BLOCKS - 1);
+              uint32_t x = 0x7F7F7F7Fu;
+  #pragma unroll
+              for (int j = 0; j < GK; ++j) {
+                float v = b[0][j];
+  #pragma unroll
+                for (int i = 1; i < SFB_BLOCKS; ++i)
+                  if (idx == i) v = b[i][j];
+                if (j < n_valid) x = (x & ~(0xFFu << (8 * j))) | (ue8m0(v) << (8 * j));
+              }
+              w[c] = x;
+            }
+            *reinterpret_cast<uint4*>(sf + 512 * (HALVES + h) + 16 * lane) =
+                make_uint4(w[0], w[1], w[2], w[3]);
+          }
+          ptx::fence_proxy_async_smem();
+          __syncwarp();
+          ++gc;
         }
-        ptx::fence_proxy_async_smem();
-        __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&full[s]);
-        if (!ld.done) issue(va[slot], vb[slot]);
         wr.next(p, s_prefix, lane);
         ++it;
+        return true;
+      };
+
+      while (!wr.done && ok) {
+  #pragma unroll
+        for (int buf = 0; buf < 2; ++buf) {
+          if (wr.done || !ok) break;
+          // the group's first stage (walking always stops at one), then the rest
+          ok = stage(true, va[buf], vb[buf]);
+          if (!ok) break;
+          if (!ld.done) issue(va[buf], vb[buf]);  // the group after next
+          while (ok && !wr.done && ((wr.kb - wr.w.ti.kb_begin) / KPS) % SF_GROUP != 0)
+            ok = stage(false, va[buf], vb[buf]);
+        }
       }
     }
   } else if (warp >= 4) {
