@@ -1,5 +1,6 @@
 // FP8 (E4M3) block-scaled GEMM D = A * B^T for sm_100a, dense and MoE
-// M-grouped (contiguous and masked layouts).
+// M-grouped (contiguous and masked layouts); the same kernel template also
+// serves BF16 operands without scales (BF16 = true).
 //
 // What it computes (DeepGEMM release article, deepseek.csdn.net, part 1.2;
 // DeepGEMM project card, aiproducthub.cn, "core features" and "technical
@@ -22,7 +23,11 @@
 //    (128-byte swizzle) into a multi-stage shared-memory ring; warp 1 owns the
 //    TMEM allocation and issues tcgen05.cp (scales) + tcgen05.mma; warp 2
 //    turns the FP32 scales into the UE8M0 layout that tcgen05.cp expects,
-//    loading them several stages ahead so that their latency stays hidden;
+//    loading them several stages ahead so that their latency stays hidden.
+//    One set of scale words serves up to four consecutive K blocks (one per
+//    byte, chosen by the MMA's scale-factor id): the two or four K blocks of
+//    a decode variant's stage, or four one-block stages in the others, so the
+//    copy into TMEM is not paid for every K block;
 //    warps 4..7 drain the TMEM accumulator (tcgen05.ld), convert to BF16 and
 //    store.
 //  * Split-K (decode shapes, too few output tiles for the SMs): the CTAs that
