@@ -81,6 +81,30 @@ def test_dense_scale_layout(dg):
     check_close(got, ref, "scale layout")
 
 
+def test_dense_scales_not_16_byte_aligned(dg):
+    """Scale tensors that start 4 bytes past a 16-byte boundary (the ABI asks
+    only for 4-byte alignment): the kernels must fall back from whole-float4
+    scale loads and still read every row's own scales."""
+    rng = np.random.default_rng(7)
+    M, N, K = 300, 400, 1024
+    p = workloads.dense_problem(M, N, K, seed=4)
+    p.sfa = np.ldexp(1.0, rng.integers(-8, 4, p.sfa.shape)).astype(np.float32)
+    p.sfb = np.ldexp(1.0, rng.integers(-8, 4, p.sfb.shape)).astype(np.float32)
+    sfa_buf = torch.empty(p.sfa.size + 4, dtype=torch.float32, device="cuda")
+    sfb_buf = torch.empty(p.sfb.size + 4, dtype=torch.float32, device="cuda")
+    sfa = sfa_buf[1:1 + p.sfa.size].view(p.sfa.shape)
+    sfb = sfb_buf[1:1 + p.sfb.size].view(p.sfb.shape)
+    sfa.copy_(dev(p.sfa))
+    sfb.copy_(dev(p.sfb))
+    assert sfa.data_ptr() % 16 == 4 and sfb.data_ptr() % 16 == 4
+    d = sentinel_like((M, N))
+    dg.fp8_gemm_nt(dev(p.a), sfa, dev(p.b), sfb, d)
+    torch.cuda.synchronize()
+    assert dg.get_last_device_error() == 0
+    ref, _ = oracle.default().gemm_nt(p.a, p.sfa, p.b, p.sfb, want_acc=False)
+    check_close(d_bits(d), ref, "unaligned scales")
+
+
 # Every general variant, forced, on one ragged shape with a random power-of-two
 # scale per A row and per B block (the picker would choose only some of them
 # for this shape).  "192:1:1:256:0" is the two-half 256-row tile; its 192-wide
