@@ -21,12 +21,13 @@ namespace dg {
 namespace {
 
 constexpr int kMaxDevices = 64;
+constexpr int kNumForms = 10;  // launch forms (enum Form below)
 
 struct DeviceState {
   bool ready = false;
   int num_sms = 0;
   int* error_word = nullptr;      // one int, device memory
-  bool smem_attr_set[10][kNumVariants] = {};  // per form (below) and variant
+  bool smem_attr_set[kNumForms][kNumVariants] = {};  // per form and variant
   bool limits_known = false;
   ClusterLimits limits = {};      // co-resident split-K clusters per variant and size
 };
@@ -202,6 +203,7 @@ dg_status make_d_map(CUtensorMap* map, void* base, uint64_t N, uint64_t rows) {
 enum Form : int { kFormDense = 0, kFormContiguous = 1, kFormMasked = 2, kFormNN = 3, kFormTN = 4,
                   kFormTT = 5, kFormF32 = 6, kFormBf16Dense = 7, kFormBf16Contiguous = 8,
                   kFormBf16Masked = 9 };
+static_assert(kFormBf16Masked + 1 == kNumForms, "one shared-memory attribute row per form");
 constexpr bool is_bf16_form(int f) { return f >= kFormBf16Dense; }
 constexpr int kind_of_form(int f) {
   return f < 3 ? f : is_bf16_form(f) ? f - kFormBf16Dense : kDense;
