@@ -179,6 +179,9 @@ const char* dg_status_string(dg_status s);
 /* Configuration the picker chooses for a problem, without launching anything
  * and without a GPU (num_sms is given explicitly).  kind: 0 dense, 1
  * contiguous, 2 masked; rows: M, M_sum or max_m; expected_m only for masked.
+ * The picker counts K in 128-byte blocks of a row: for the BF16-operand
+ * calls pass 2 * K (their tile geometry is that of the E4M3 call with twice
+ * the K, without the scale factors' shared memory and TMEM columns).
  * For the masked form the grid is an upper bound (the real tile count is
  * read from masked_m on the device). */
 typedef struct {
