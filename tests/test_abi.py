@@ -164,3 +164,27 @@ def test_query_rejects_bad_input(dg):
         dg.query_config(3, 64, 128, 128)
     with pytest.raises(dg.DgError):
         dg.query_config(0, 64, 100, 128)
+
+
+# ------------------------------------------------ the Python binding's checks --
+
+def test_binding_rejects_wrong_dtypes_and_host_tensors(dg):
+    """The binding validates tensors before any call into the library: wrong
+    element types raise TypeError, host (CPU) tensors ValueError."""
+    import torch
+    a8 = torch.zeros((4, 128), dtype=torch.uint8)
+    sfa = torch.ones((4, 1), dtype=torch.float32)
+    b8 = torch.zeros((16, 128), dtype=torch.uint8)
+    sfb = torch.ones((1, 1), dtype=torch.float32)
+    with pytest.raises(TypeError):
+        dg.fp8_gemm_nt(a8.float(), sfa, b8, sfb)
+    with pytest.raises(ValueError):
+        dg.fp8_gemm_nt(a8, sfa, b8, sfb)                  # not on a CUDA device
+    a16 = torch.zeros((4, 64), dtype=torch.bfloat16)
+    b16 = torch.zeros((16, 64), dtype=torch.bfloat16)
+    with pytest.raises(TypeError):
+        dg.bf16_gemm_nt(a16.float(), b16)
+    with pytest.raises(TypeError):
+        dg.m_grouped_bf16_gemm_nt_contiguous(a8, b16.unsqueeze(0), torch.zeros(4, dtype=torch.int32))
+    with pytest.raises(ValueError):
+        dg.bf16_gemm_nt(a16, b16)                         # not on a CUDA device
