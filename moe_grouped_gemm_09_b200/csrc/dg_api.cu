@@ -80,7 +80,11 @@ dg_status device_state(DeviceState** out, int* dev_out) {
       if (e && std::atoi(e) > 0) g_timeout_ns = 1000000ull * std::atoi(e);
     }
     st.num_sms = prop.multiProcessorCount;
-    if (cudaMalloc(&st.error_word, sizeof(int)) != cudaSuccess) return DG_ERR_CUDA;
+    if (!st.error_word && cudaMalloc(&st.error_word, sizeof(int)) != cudaSuccess) {
+      st.error_word = nullptr;
+      return DG_ERR_CUDA;
+    }
+    // (a failure below keeps the word for the next attempt instead of leaking it)
     if (cudaMemset(st.error_word, 0, sizeof(int)) != cudaSuccess) return DG_ERR_CUDA;
     if (cudaDeviceSynchronize() != cudaSuccess) return DG_ERR_CUDA;
     st.ready = true;
