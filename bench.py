@@ -6,10 +6,16 @@ DeepGEMM pages' DeepSeek-V3/R1 inference shapes, M in {64, 128} x (N, K) in
 {(2112, 7168), (32768, 512), (7168, 2048)}, each with its own E4M3 operands and
 power-of-two block scales, every step through the library's public call.
 The metric for M <= 128 is HBM bandwidth: algorithmic bytes (A, B, their
-scales, and D) per second.  The other workloads ("smoke", "prefill",
-"contiguous", "masked") report TFLOPS and are for profiling and study, as
-are "bf16-decode" and "bf16-prefill": the same dense shapes on BF16 operands
-(no scales), measured against the BF16 tensor peak.
+scales, and D) per second.  The same run then times the other configurations
+of the metric -- "smoke" (dense 64 x 512 x 1024), "prefill" (four dense
+M = 4096 GEMMs, TFLOPS), "contiguous" and "masked" (the two MoE grouped
+layouts, TFLOPS) -- the same way and reports each, with its own roofline and
+CPU-oracle baseline, under ``workloads`` in the same JSON line; the headline
+``value`` stays the decode step.  ``--workload`` makes any of them (or
+"bf16-decode" / "bf16-prefill": the same dense shapes on BF16 operands,
+against the BF16 tensor peak) the headline instead.  The tensor peak of the
+E4M3 roofline is the vendor library's measured dense E4M3 GEMM rate
+(``profiles/fp8_peak.md``, written from ``--measure-fp8-peak``).
 
 Timing: inputs sit in HBM, R copies of them at different addresses are rotated
 so that the bytes touched between two visits of one copy exceed the 126 MB L2;
@@ -24,9 +30,10 @@ Under torchrun every rank runs the same per-rank workload on its own GPU (no
 data-path collective: the GEMMs of a step are independent problems), so the
 scaling is weak and ``value`` counts the bytes of all ranks.
 
-``--impl reference`` times the CPU oracle instead, on the host cores, on a
-bounded sample of the same step (the oracle is test infrastructure; this leg
-and the ``cpu_baseline`` object are the only product uses of it).
+``--impl reference`` times the CPU oracle instead, on the host cores: whole
+steps when they fit the time budget (decode: about half a second a step),
+else a bounded row sample of each step (the oracle is test infrastructure;
+this leg and the ``cpu_baseline`` objects are the only product uses of it).
 """
 from __future__ import annotations
 
@@ -254,73 +261,63 @@ def whole_job_value(units_per_step: float, world: int, ms_per_step: float, unit:
 
 # ---------------------------------------------------------------- GPU arm --
 
-def run_gpu(args):
-    import torch
-    import torch.distributed as dist
+def fp8_peak(peaks: dict):
+    """Dense E4M3 tensor peak (TFLOP/s) and where it comes from: the measured
+    figure of ``profiles/fp8_peak.md`` (a large FP8 library GEMM timed on this
+    pool's B200s; ``--measure-fp8-peak`` writes it), else 2 x the measured
+    BF16 figure (the nominal 4.5 : 2.25 FP8 : BF16 ratio)."""
+    path = os.path.join(ROOT, "profiles", "fp8_peak.md")
+    try:
+        with open(path) as f:
+            for line in f:
+                if line.startswith("fp8_tflops:"):
+                    return float(line.split(":", 1)[1].strip()), "measured (fp8_peak.md, cuBLASLt E4M3)"
+    except (OSError, ValueError):
+        pass
+    bf16 = float(peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"]))
+    return 2.0 * bf16, "2 x bf16_tflops (nominal FP8:BF16 ratio)"
 
-    import moe_grouped_gemm_09_b200 as dg
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        torch.cuda.set_device(local_rank)
-        dist.init_process_group("nccl", device_id=torch.device("cuda", local_rank),
-                                timeout=__import__("datetime").timedelta(seconds=120))
-    dev = torch.device("cuda", local_rank if world > 1 else torch.cuda.current_device())
-    torch.cuda.set_device(dev)
+class GpuContext:
+    """Device, stream and rank plumbing shared by the timed workloads."""
 
-    def barrier():
-        if world > 1:
+    def __init__(self):
+        import torch
+        import torch.distributed as dist
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+        if self.world > 1:
+            torch.cuda.set_device(local_rank)
+            dist.init_process_group("nccl", device_id=torch.device("cuda", local_rank),
+                                    timeout=__import__("datetime").timedelta(seconds=120))
+        self.dev = torch.device("cuda", local_rank if self.world > 1 else torch.cuda.current_device())
+        torch.cuda.set_device(self.dev)
+        self.stream = torch.cuda.Stream(device=self.dev)
+
+    def barrier(self):
+        if self.world > 1:
+            import torch.distributed as dist
             dist.barrier()
 
-    def max_over_ranks(x: float) -> float:
-        return reduce_max(x, world, dev)
+    def max_over_ranks(self, x: float) -> float:
+        return reduce_max(x, self.world, self.dev)
 
-    items = build_workload(args.workload, seed=args.seed)
-    metric, unit, _ = workload_meta(args.workload)
-    units = step_units(items, unit)
-    set_bytes = sum(p.a.nbytes + p.b.nbytes + getattr(p, "sfa", p.a[:0]).nbytes
-                    + getattr(p, "sfb", p.a[:0]).nbytes for _, p in items)
-    R = max(2, math.ceil(3 * L2_BYTES / max(set_bytes, 1)))
-    if args.workload in ("prefill", "contiguous", "masked", "bf16-prefill"):
-        R = max(2, min(R, 4))
-    flush_note = f"inputs rotated over {R} copies ({R * set_bytes / 2**20:.0f} MiB > 3x L2)"
 
-    # device copies: R rotation sets of the inputs, one output per GEMM
-    def host_tensor(x):
-        # BF16 operands arrive as uint16 bit patterns
-        if x.dtype == np.uint16:
-            return torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16)
-        return torch.from_numpy(np.ascontiguousarray(x))
+def _host_tensor(x):
+    import torch
+    # BF16 operands arrive as uint16 bit patterns
+    if x.dtype == np.uint16:
+        return torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16)
+    return torch.from_numpy(np.ascontiguousarray(x))
 
-    def to_dev(x):
-        return host_tensor(x).to(dev)
 
-    def operands(p):
-        names = ("a", "sfa", "b", "sfb") if hasattr(p, "sfa") else ("a", "b")
-        return {k: getattr(p, k) for k in names}
+def _operands(p):
+    names = ("a", "sfa", "b", "sfb") if hasattr(p, "sfa") else ("a", "b")
+    return {k: getattr(p, k) for k in names}
 
-    sets = []
-    for r in range(R):
-        one = []
-        for kind, p in items:
-            t = {k: to_dev(v) for k, v in operands(p).items()}
-            if kind == "contiguous":
-                t["m_indices"] = to_dev(p.m_indices)
-            if kind == "masked":
-                t["masked_m"] = to_dev(p.masked_m)
-            one.append(t)
-        sets.append(one)
-    outs = []
-    for kind, p in items:
-        if kind in ("dense", "bf16_dense"):
-            outs.append(torch.empty((p.M, p.N), dtype=torch.bfloat16, device=dev))
-        elif kind == "contiguous":
-            outs.append(torch.empty((p.M_sum, p.N), dtype=torch.bfloat16, device=dev))
-        else:
-            outs.append(torch.empty((p.G, p.max_m, p.N), dtype=torch.bfloat16, device=dev))
 
+def _launcher(dg, items, sets, outs):
     def launch_one(j, r):
         (kind, p), t, d = items[j], sets[r][j], outs[j]
         if kind == "dense":
@@ -333,24 +330,67 @@ def run_gpu(args):
         else:
             dg.m_grouped_fp8_gemm_nt_masked(t["a"], t["sfa"], t["b"], t["sfb"],
                                             t["masked_m"], p.expected_m, d)
+    return launch_one
+
+
+def time_workload(ctx: GpuContext, name: str, args, steps: int, per_gemm: bool, e2e: bool,
+                  rotations: int = 0) -> dict:
+    """Times ``steps`` steps of one workload (inputs resident in HBM, rotated
+    over more than 3 x L2, one CUDA graph per rotation cycle, CUDA events on
+    the launching stream, max over ranks); optionally the per-GEMM graphs and
+    the end-to-end pass through the public call with host buffers."""
+    import torch
+    import moe_grouped_gemm_09_b200 as dg
+
+    dev, stream = ctx.dev, ctx.stream
+    items = build_workload(name, seed=args.seed)
+    metric, unit, _ = workload_meta(name)
+    set_bytes = sum(p.a.nbytes + p.b.nbytes + getattr(p, "sfa", p.a[:0]).nbytes
+                    + getattr(p, "sfb", p.a[:0]).nbytes for _, p in items)
+    R = max(2, math.ceil(3 * L2_BYTES / max(set_bytes, 1)))
+    if name in ("prefill", "contiguous", "masked", "bf16-prefill"):
+        R = max(2, min(R, 4))
+    if rotations > 0:
+        R = rotations
+    flush_note = f"inputs rotated over {R} copies ({R * set_bytes / 2**20:.0f} MiB"
+    flush_note += " > 3x L2)" if R * set_bytes > 3 * L2_BYTES else ", not above 3x L2)"
+
+    sets = []
+    for r in range(R):
+        one = []
+        for kind, p in items:
+            t = {k: _host_tensor(v).to(dev) for k, v in _operands(p).items()}
+            if kind == "contiguous":
+                t["m_indices"] = _host_tensor(p.m_indices).to(dev)
+            if kind == "masked":
+                t["masked_m"] = _host_tensor(p.masked_m).to(dev)
+            one.append(t)
+        sets.append(one)
+    outs = []
+    for kind, p in items:
+        if kind in ("dense", "bf16_dense"):
+            outs.append(torch.empty((p.M, p.N), dtype=torch.bfloat16, device=dev))
+        elif kind == "contiguous":
+            outs.append(torch.empty((p.M_sum, p.N), dtype=torch.bfloat16, device=dev))
+        else:
+            outs.append(torch.empty((p.G, p.max_m, p.N), dtype=torch.bfloat16, device=dev))
+    launch_one = _launcher(dg, items, sets, outs)
 
     def launch_step(r):
         for j in range(len(items)):
             launch_one(j, r)
 
-    stream = torch.cuda.Stream(device=dev)
     torch.cuda.synchronize(dev)
     with torch.cuda.stream(stream):
-        for i in range(args.warmup):          # eager warm-up (also sizes the workspace)
+        for i in range(args.warmup):          # eager warm-up (also the device set-up)
             launch_step(i % R)
     torch.cuda.synchronize(dev)
     if dg.get_last_device_error() != 0:
-        raise RuntimeError("device error during warm-up")
+        raise RuntimeError(f"{name}: device error during warm-up")
 
     # One graph holds a whole rotation cycle (steps on sets 0..R-1, so that
     # consecutive launches overlap through programmatic dependent launch
-    # across step boundaries too), one the first `K mod R` steps of a cycle;
-    # one graph per set adds events around each launch.
+    # across step boundaries too), one the first `steps mod R` steps of a cycle.
     def capture(n_steps):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
@@ -359,162 +399,255 @@ def run_gpu(args):
         return g
 
     cycle = capture(R)
-    rem = args.steps % R
+    rem = steps % R
     tail = capture(rem) if rem else None
-    # per GEMM of the step: one graph of its launches on every rotation set
-    per_gemm_graphs = []
-    for j in range(len(items)):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            for r in range(R):
-                launch_one(j, r)
-        per_gemm_graphs.append(g)
     with torch.cuda.stream(stream):
         cycle.replay()
         cycle.replay()
     torch.cuda.synchronize(dev)
 
-    # ---- timed region: exactly K steps ----
+    # ---- timed region: exactly `steps` steps ----
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier()
+    ctx.barrier()
     torch.cuda.synchronize(dev)
     with ClockSampler(dev.index) as clocks:
         with torch.cuda.stream(stream):
             start.record(stream)
-            for _ in range(args.steps // R):   # exactly args.steps steps in all
+            for _ in range(steps // R):
                 cycle.replay()
             if tail is not None:
                 tail.replay()
             end.record(stream)
         torch.cuda.synchronize(dev)
-    barrier()
-    ms = start.elapsed_time(end) / args.steps
-    ms = max_over_ranks(ms)
+    ctx.barrier()
+    ms = ctx.max_over_ranks(start.elapsed_time(end) / steps)
     if dg.get_last_device_error() != 0:
-        raise RuntimeError("device error during the timed steps")
-
-    # The one kernel of the step is the dominant kernel: its average launch
-    # duration over the timed region is ms / launches and its algorithmic
-    # bytes (or FLOPs) per launch are the step's / launches, so the achieved
-    # rate (below) is the step's units over the timed time.
+        raise RuntimeError(f"{name}: device error during the timed steps")
 
     # ---- per GEMM (second timed pass): R back-to-back launches of one shape ----
     kernel_ms = []
-    for j, g in enumerate(per_gemm_graphs):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            g.replay()
-            e0.record(stream)
-            for _ in range(args.per_gemm_reps):
+    if per_gemm:
+        for j in range(len(items)):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for r in range(R):
+                    launch_one(j, r)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
                 g.replay()
-            e1.record(stream)
-        torch.cuda.synchronize(dev)
-        kernel_ms.append(e0.elapsed_time(e1) / (args.per_gemm_reps * R))
+                e0.record(stream)
+                for _ in range(args.per_gemm_reps):
+                    g.replay()
+                e1.record(stream)
+            torch.cuda.synchronize(dev)
+            kernel_ms.append(e0.elapsed_time(e1) / (args.per_gemm_reps * R))
+            del g
 
     # ---- end to end: host buffers, copies inside the timed region ----
-    pinned = []
-    for kind, p in items:
-        t = {k: host_tensor(v).pin_memory() for k, v in operands(p).items()}
-        if kind == "contiguous":
-            t["m_indices"] = torch.from_numpy(p.m_indices).pin_memory()
-        if kind == "masked":
-            t["masked_m"] = torch.from_numpy(p.masked_m).pin_memory()
-        pinned.append(t)
-    host_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
-    h2d = sum(v.numel() * v.element_size() for t in pinned for v in t.values())
-    d2h = sum(o.numel() * o.element_size() for o in outs)
-    e2e_steps = max(3, min(args.steps, args.e2e_steps))
+    e2e_res = None
+    if e2e:
+        pinned = []
+        for kind, p in items:
+            t = {k: _host_tensor(v).pin_memory() for k, v in _operands(p).items()}
+            if kind == "contiguous":
+                t["m_indices"] = torch.from_numpy(p.m_indices).pin_memory()
+            if kind == "masked":
+                t["masked_m"] = torch.from_numpy(p.masked_m).pin_memory()
+            pinned.append(t)
+        host_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
+        h2d = sum(v.numel() * v.element_size() for t in pinned for v in t.values())
+        d2h = sum(o.numel() * o.element_size() for o in outs)
+        e2e_steps = max(3, min(steps, args.e2e_steps))
 
-    def e2e_step():
-        for t_h, t_d in zip(pinned, sets[0]):
-            for k in t_h:
-                t_d[k].copy_(t_h[k], non_blocking=True)
-        launch_step(0)
-        for o_h, o_d in zip(host_out, outs):
-            o_h.copy_(o_d, non_blocking=True)
+        def e2e_step():
+            for t_h, t_d in zip(pinned, sets[0]):
+                for k in t_h:
+                    t_d[k].copy_(t_h[k], non_blocking=True)
+            launch_step(0)
+            for o_h, o_d in zip(host_out, outs):
+                o_h.copy_(o_d, non_blocking=True)
 
-    with torch.cuda.stream(stream):
-        for _ in range(2):
-            e2e_step()
-    torch.cuda.synchronize(dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier()
-    torch.cuda.synchronize(dev)
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        for _ in range(e2e_steps):
-            e2e_step()
-        e1.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps)
+        with torch.cuda.stream(stream):
+            for _ in range(2):
+                e2e_step()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ctx.barrier()
+        torch.cuda.synchronize(dev)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(e2e_steps):
+                e2e_step()
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ctx.barrier()
+        e2e_ms = ctx.max_over_ranks(e0.elapsed_time(e1) / e2e_steps)
+        e2e_res = {"value": round(whole_job_value(step_units(items, unit), ctx.world, e2e_ms, unit), 3),
+                   "unit": unit, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
-    # ---- CPU baseline (rank 0, single-GPU run only) ----
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = run_oracle_sample(items, unit, budget_s=args.cpu_budget_s)
+    del cycle, tail
+    return {"items": items, "ms": ms, "R": R, "flush_note": flush_note, "kernel_ms": kernel_ms,
+            "clocks": clocks.summary(), "e2e": e2e_res, "metric": metric, "unit": unit}
 
+
+def workload_record(name: str, t: dict, world: int, steps: int, warmup: int) -> dict:
+    """The JSON record of one timed workload: metric, value, roofline."""
+    items, ms, unit = t["items"], t["ms"], t["unit"]
     peaks, peak_kind = load_peaks()
     hbm_peak = float(peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"]))
-    # E4M3 dense peak = 2x the measured BF16 figure (nominal FP8:BF16 ratio
-    # 4.5:2.25); BF16 operands take the measured BF16 figure itself
-    bf16_peak = float(peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"]))
-    bf16 = is_bf16(args.workload)
-    tensor_peak = bf16_peak if bf16 else 2.0 * bf16_peak
+    bf16 = is_bf16(name)
+    if bf16:
+        tensor_peak = float(peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"]))
+        tensor_src = f"{peak_kind} (bf16_tflops)"
+    else:
+        tensor_peak, tensor_src = fp8_peak(peaks)
     roof = roofline_terms(items, ms, hbm_peak, tensor_peak,
                           SPEC_BF16_TFLOPS if bf16 else SPEC_FP8_TFLOPS)
     bound = roof["bound"]
     r_unit = "GB/s" if bound == "hbm" else "TFLOP/s"
     peak = hbm_peak if bound == "hbm" else tensor_peak
     achieved = scale_units(step_units(items, r_unit), r_unit, ms / 1e3)
-    value = whole_job_value(units, world, ms, unit)
     launches_per_step = len(items)
-    res = {
-        "metric": metric,
-        "value": round(value, 3),
+    return {
+        "metric": t["metric"],
+        "value": round(whole_job_value(step_units(items, unit), world, ms, unit), 3),
         "unit": unit,
-        "n_gpus": world,
-        "steps": args.steps,
-        "warmup": args.warmup,
         "ms_per_step": round(ms, 6),
-        "higher_is_better": True,
-        "scaling": "weak",
-        "vs_baseline": None,
+        "steps": steps,
+        "warmup": warmup,
         "dtype": "bf16" if bf16 else "e4m3",
-        "data": "synthetic",
         "config": {
-            "workload": args.workload,
+            "workload": name,
             "gemms": [dict(kind=k, **_shape(p)) for k, p in items],
-            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-            "l2": flush_note,
-            "graph": f"one CUDA graph per rotation cycle of {R} steps",
+            "l2": t["flush_note"],
+            "graph": f"one CUDA graph per rotation cycle of {t['R']} steps",
         },
-        "e2e": {"value": round(whole_job_value(units, world, e2e_ms, unit), 3), "unit": unit,
-                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
-        "gpu_launches": int(args.steps * launches_per_step),
+        "gpu_launches": int(steps * launches_per_step),
         "roofline": {
             "bound": bound,
             "achieved": round(achieved, 3),
-            "peak": peak,
+            "peak": round(peak, 1),
             "unit": r_unit,
             "frac": round(achieved / peak, 4),
-            "traffic": profiled_traffic(args.workload),
-            "peak_source": f"{peak_kind} ({'hbm_gbs copy' if bound == 'hbm' else 'bf16_tflops' if bf16 else '2 x bf16_tflops'})",
+            "traffic": profiled_traffic(name),
+            "peak_source": f"{peak_kind} (hbm_gbs copy)" if bound == "hbm" else tensor_src,
+            "tensor_peak_tflops": round(tensor_peak, 1),
             "roofline_time_us": round(roof["t_roof_s"] * 1e6, 3),
             "frac_time": round(roof["frac_time"], 4),
             "frac_time_spec": round(roof["frac_time_spec"], 4),
             "launch_avg_us": round(ms * 1e3 / launches_per_step, 3),
-            "per_gemm_us": [round(x * 1e3, 3) for x in kernel_ms],
+            "per_gemm_us": [round(x * 1e3, 3) for x in t["kernel_ms"]],
         },
-        "clocks": clocks.summary(),
+        "clocks": t["clocks"],
     }
-    if cpu is not None:
-        res["cpu_baseline"] = cpu
-    if rank == 0:
+
+
+EXTRA_WORKLOADS = ("smoke", "prefill", "contiguous", "masked")
+
+
+def run_gpu(args):
+    import torch
+
+    ctx = GpuContext()
+    main = time_workload(ctx, args.workload, args, args.steps, per_gemm=True, e2e=True,
+                         rotations=args.rotations)
+    rec = workload_record(args.workload, main, ctx.world, args.steps, args.warmup)
+    res = {
+        "metric": rec["metric"],
+        "value": rec["value"],
+        "unit": rec["unit"],
+        "n_gpus": ctx.world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": rec["ms_per_step"],
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": rec["dtype"],
+        "data": "synthetic",
+        "config": dict(rec["config"], parallelism=(f"replicas x{ctx.world}" if ctx.world > 1
+                                                   else "single GPU")),
+        "e2e": main["e2e"],
+        "gpu_launches": rec["gpu_launches"],
+        "roofline": rec["roofline"],
+        "clocks": rec["clocks"],
+    }
+    cpu_ok = ctx.rank == 0 and ctx.world == 1 and not args.no_cpu_baseline
+    if cpu_ok:
+        res["cpu_baseline"] = run_oracle_sample(main["items"], main["unit"],
+                                                budget_s=args.cpu_budget_s)
+    del main
+    torch.cuda.empty_cache()
+
+    # The other configurations of the same metric, timed the same way in the
+    # same process (the headline `value` stays the workload above).
+    extras = [w for w in (args.extra_workloads.split(",") if args.extra_workloads else [])
+              if w and w != args.workload]
+    if extras:
+        res["workloads"] = {}
+        for w in extras:
+            t = time_workload(ctx, w, args, args.steps, per_gemm=(w == "prefill"), e2e=False,
+                              rotations=args.rotations)
+            r = workload_record(w, t, ctx.world, args.steps, args.warmup)
+            if cpu_ok:
+                r["cpu_baseline"] = run_oracle_sample(t["items"], t["unit"],
+                                                      budget_s=args.extra_cpu_budget_s)
+            res["workloads"][w] = r
+            del t
+            torch.cuda.empty_cache()
+    if ctx.rank == 0:
         print(json.dumps(res), flush=True)
-    if world > 1:
-        del cycle, tail, per_gemm_graphs
+    if ctx.world > 1:
+        import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def measure_fp8_peak(args):
+    """Dense E4M3 peak of this GPU from the vendor library: torch._scaled_mm
+    (cuBLASLt) on an 8192^3 E4M3 x E4M3 GEMM with FP32 per-tensor scales and
+    BF16 output, best of 20 CUDA-event-timed launches (burst) and the mean
+    over a 4 s back-to-back loop (sustained)."""
+    import torch
+    dev = torch.device("cuda", 0)
+    n = args.peak_size
+    a = torch.randn((n, n), device=dev).to(torch.float8_e4m3fn)
+    b = torch.randn((n, n), device=dev).to(torch.float8_e4m3fn)
+    one = torch.ones((), device=dev)
+
+    def mm():
+        return torch._scaled_mm(a, b.t(), scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+
+    for _ in range(5):
+        mm()
+    torch.cuda.synchronize()
+    best = 1e30
+    for _ in range(20):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        mm()
+        e1.record()
+        torch.cuda.synchronize()
+        best = min(best, e0.elapsed_time(e1))
+    flop = 2.0 * n ** 3
+    with ClockSampler(0) as clocks:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        iters = 0
+        t_end = time.perf_counter() + 4.0
+        while time.perf_counter() < t_end:
+            for _ in range(20):
+                mm()
+            iters += 20
+            torch.cuda.synchronize()
+        e1.record()
+        torch.cuda.synchronize()
+    sustained_ms = e0.elapsed_time(e1) / iters
+    print(json.dumps({"fp8_tflops": round(flop / best / 1e9, 1),
+                      "fp8_tflops_sustained": round(flop / sustained_ms / 1e9, 1),
+                      "shape": [n, n, n], "how": "torch._scaled_mm E4M3 x E4M3 -> BF16, "
+                      "per-tensor FP32 scales; best of 20 launches / mean of a 4 s loop",
+                      "clocks": clocks.summary(), "gpu": torch.cuda.get_device_name(0)}),
+          flush=True)
 
 
 def _shape(p):
@@ -602,7 +735,11 @@ def run_oracle_sample(items, unit, budget_s: float):
 
 
 def run_reference(args):
-    """The oracle as the reference arm: K timed steps, each a bounded sample."""
+    """The oracle as the reference arm: K timed steps on the host cores.  A
+    step is one whole step of the workload when the oracle finishes one in a
+    few seconds (decode: about half a second on 16 threads), else a bounded
+    row sample of it (one output row per host thread of one GEMM, round robin
+    over the GEMMs) scaled to the full step by rows."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
@@ -612,27 +749,47 @@ def run_reference(args):
     metric, unit, _ = workload_meta(args.workload)
     units = step_units(items, unit)
     rows_total = _row_units(items, unit)
-    # each step: one output row per host thread, of one GEMM (round robin over
-    # the GEMMs, walking down their rows); scaled to the full step by rows
-    per = max(1, o.num_threads())
-    cursor = [0] * len(items)
 
-    def one_step(i):
-        j = i % len(items)
-        n = min(per, rows_total[j])
-        rows = (cursor[j] + np.arange(n)) % rows_total[j]
-        cursor[j] = int((cursor[j] + n) % rows_total[j])
-        _oracle_rows(o, items[j][0], items[j][1], rows)
-        return n / rows_total[j] / len(items)
+    def whole_step():
+        for (kind, p), n in zip(items, rows_total):
+            _oracle_rows(o, kind, p, np.arange(n))
 
-    for i in range(args.warmup):
-        one_step(i)
-    full_equiv = 0.0
+    # one probe step decides whole steps or a row sample
     t0 = time.perf_counter()
-    for i in range(args.steps):
-        full_equiv += one_step(i)
-    dt = time.perf_counter() - t0
-    full_s = dt / full_equiv
+    whole_step()
+    probe_s = time.perf_counter() - t0
+    whole = probe_s * (args.steps + args.warmup) <= args.reference_budget_s
+    if whole:
+        for _ in range(max(0, args.warmup - 1)):
+            whole_step()
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            whole_step()
+        dt = time.perf_counter() - t0
+        full_s = dt / args.steps
+        sample = f"{args.steps} whole steps back to back ({dt:.1f} s)"
+    else:
+        per = max(1, o.num_threads())
+        cursor = [0] * len(items)
+
+        def one_step(i):
+            j = i % len(items)
+            n = min(per, rows_total[j])
+            rows = (cursor[j] + np.arange(n)) % rows_total[j]
+            cursor[j] = int((cursor[j] + n) % rows_total[j])
+            _oracle_rows(o, items[j][0], items[j][1], rows)
+            return n / rows_total[j] / len(items)
+
+        for i in range(args.warmup):
+            one_step(i)
+        full_equiv = 0.0
+        t0 = time.perf_counter()
+        for i in range(args.steps):
+            full_equiv += one_step(i)
+        dt = time.perf_counter() - t0
+        full_s = dt / full_equiv
+        sample = (f"{args.steps} timed steps of {per} output rows each (one GEMM per step, "
+                  f"round robin), {dt:.1f} s, scaled to full steps by rows")
     value = scale_units(units, unit, full_s)
     res = {
         "impl": "reference",
@@ -642,9 +799,7 @@ def run_reference(args):
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": args.workload, "gemms": [dict(kind=k, **_shape(p)) for k, p in items]},
         "cpu_baseline": {"value": round(value, 4), "unit": unit, "cores": o.num_threads(),
-                         "kind": "oracle",
-                         "sample": f"{args.steps} timed steps of {per} output rows each (one GEMM per "
-                                   f"step, round robin), {dt:.1f} s, scaled to full steps by rows"},
+                         "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 4), "unit": unit, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -654,7 +809,7 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="decode",
@@ -665,11 +820,25 @@ def main():
     ap.add_argument("--per-gemm-reps", type=int, default=20,
                     help="replays of each single-GEMM graph behind per_gemm_us")
     ap.add_argument("--cpu-budget-s", type=float, default=20.0)
+    ap.add_argument("--extra-cpu-budget-s", type=float, default=4.0,
+                    help="oracle time per extra workload's cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--extra-workloads", default=",".join(EXTRA_WORKLOADS),
+                    help="comma-separated workloads timed after the main one and reported "
+                         "under 'workloads' ('' for none)")
+    ap.add_argument("--rotations", type=int, default=0,
+                    help="input copies rotated between steps (0: enough to exceed 3x L2)")
+    ap.add_argument("--reference-budget-s", type=float, default=120.0,
+                    help="reference arm: whole oracle steps if they fit in this time")
+    ap.add_argument("--measure-fp8-peak", action="store_true",
+                    help="time the vendor library's dense E4M3 GEMM and print its TFLOP/s")
+    ap.add_argument("--peak-size", type=int, default=8192)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    if args.impl == "reference":
+    if args.measure_fp8_peak:
+        measure_fp8_peak(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_gpu(args)

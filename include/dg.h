@@ -36,7 +36,10 @@
  *      d    bfloat16 [rows of A, N], overwritten (no C / beta input).
  *    The scales must be positive normal powers of two (2^-126 .. 2^127), as
  *    produced by scale = 2^ceil(log2(amax/448)); the kernel uses the exponent
- *    field only.
+ *    field only.  With dg_set_check_scales(1) (or DG_CHECK_SCALES=1 in the
+ *    environment) the kernels check every scale they read and record device
+ *    error 0x301 for one that breaks this rule (the result is then
+ *    undefined); the check is off by default.
  *  - Requirements (checked on the host, DG_ERR_INVALID_ARG otherwise):
  *    K > 0 and K % 128 == 0 (BF16 operands: K % 64 == 0); N > 0 and N % 16 == 0; a, b and d 16-byte
  *    aligned, sfa/sfb 4-byte aligned, m_indices/masked_m 4-byte aligned.
@@ -47,9 +50,12 @@
  *    pointers live on must be the calling thread's current CUDA device.
  *  - Errors: argument errors return before anything is launched; launch
  *    errors return DG_ERR_CUDA.  A kernel that finds an inconsistency on the
- *    device (a wait that runs out of time, an m_indices block naming two
- *    experts, an expert index >= G) records a code that
- *    dg_get_last_device_error() reports after the stream is synchronised.
+ *    device records a code that dg_get_last_device_error() reports after the
+ *    stream is synchronised: 0x101..0x104 a wait that ran out of time (TMA
+ *    producer, scale producer, MMA issuer, epilogue; the kernel then stops
+ *    early and D is partly written), 0x201 an m_indices block naming two
+ *    experts, 0x202 an expert index >= G, 0x301 a scale that is not a
+ *    positive normal power of two (only when the check is on).
  *  - Results are deterministic: the same inputs give bit-identical outputs
  *    on every run (no floating-point atomics; split-K partial sums are added
  *    in a fixed order).
@@ -169,9 +175,23 @@ int dg_get_num_sms(void);
 dg_status dg_get_last_device_error(int* code);
 
 /* Per-launch time limit of every wait inside the kernels, in milliseconds
- * (default 1000).  A wait that runs out records a device error and the kernel
- * returns instead of hanging. */
+ * (default 1000, or DG_WAIT_TIMEOUT_MS from the environment).  A wait that
+ * runs out records a device error (0x101..0x104) and the kernel returns
+ * instead of hanging.  Applies to launches enqueued after the call, from
+ * every thread and entry point.  ms <= 0: DG_ERR_INVALID_ARG. */
 dg_status dg_set_wait_timeout_ms(int ms);
+/* The same limit in nanoseconds, for limits shorter than a millisecond (a
+ * wait needs at least one poll of the GPU's global timer, whose ticks are
+ * tens to hundreds of nanoseconds apart, before it can run out). */
+dg_status dg_set_wait_timeout_ns(long long ns);
+
+/* Turns the kernels' check of the scale contract on (enable != 0) or off:
+ * every scale a kernel reads must be a positive normal power of two, and one
+ * that is not records device error 0x301.  Off by default; the environment
+ * variable DG_CHECK_SCALES=1 turns it on at first use.  Applies to launches
+ * enqueued after the call, from every thread and entry point; the check
+ * costs a few instructions per scale and none when off. */
+dg_status dg_set_check_scales(int enable);
 
 /* Human-readable name of a status code.  Never NULL. */
 const char* dg_status_string(dg_status s);
@@ -218,12 +238,23 @@ dg_status dg_query_config(int kind, int rows, int N, int K, int G, int expected_
  * Every call shares the one array, which keeps the last call's contents;
  * calls whose kernels overlap on the GPU (different streams, or several
  * threads) share it too.  The SM cap of dg_set_num_sms does not apply here
- * (all SMs are used), and device-side error codes of this call stay in the
- * array: dg_get_last_device_error does not report them.  Waits inside the
- * kernel are bounded as in every call. */
+ * (all SMs are used).  Waits inside the kernel are bounded by the same limit
+ * as every call (dg_set_wait_timeout_ms / _ns), and DG_NO_PREFETCH and
+ * DG_CHECK_SCALES apply as they do elsewhere.  Device-side error codes of
+ * this call go to the array's error word, not to the one
+ * dg_get_last_device_error reads: read them with
+ * dg_fp8_gemm_nt_noalloc_get_last_device_error. */
 dg_status dg_fp8_gemm_nt_noalloc(const void* a, const float* sfa, const void* b,
                                  const float* sfb, void* d, int M, int N, int K,
                                  dg_stream_t stream);
+
+/* Reads and clears the error word of dg_fp8_gemm_nt_noalloc on the current
+ * device (codes as for dg_get_last_device_error; 0: none since the last
+ * read).  Synchronises the device, then copies the word through the CUDA
+ * symbol API, which allocates no device memory.  Since every no-alloc call
+ * shares the word, a code may come from any of the calls since the last
+ * read.  Returns DG_ERR_CUDA if the device cannot be queried. */
+dg_status dg_fp8_gemm_nt_noalloc_get_last_device_error(int* code);
 
 /* Library version, "major.minor.patch". */
 const char* dg_version(void);

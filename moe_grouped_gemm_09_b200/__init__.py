@@ -54,7 +54,10 @@ _set_num_sms = _decl("dg_set_num_sms", [_I])
 _get_num_sms = _decl("dg_get_num_sms", [])
 _get_last_err = _decl("dg_get_last_device_error", [ctypes.POINTER(ctypes.c_int)])
 _set_timeout = _decl("dg_set_wait_timeout_ms", [_I])
+_set_timeout_ns = _decl("dg_set_wait_timeout_ns", [ctypes.c_longlong])
+_set_check_scales = _decl("dg_set_check_scales", [_I])
 _gemm_nt_noalloc = _decl("dg_fp8_gemm_nt_noalloc", [_P, _P, _P, _P, _P, _I, _I, _I, _P])
+_noalloc_err = _decl("dg_fp8_gemm_nt_noalloc_get_last_device_error", [ctypes.POINTER(ctypes.c_int)])
 _status_string = _decl("dg_status_string", [_I], ctypes.c_char_p)
 _version = _decl("dg_version", [], ctypes.c_char_p)
 
@@ -72,7 +75,9 @@ EXPORTED_SYMBOLS = ("dg_fp8_gemm_nt", "dg_m_grouped_fp8_gemm_nt_contiguous",
                     "dg_get_last_device_error", "dg_set_wait_timeout_ms", "dg_status_string",
                     "dg_query_config", "dg_version", "dg_fp8_gemm_nt_noalloc", "dg_fp8_gemm_nn",
                     "dg_fp8_gemm_tn", "dg_fp8_gemm_tt", "dg_fp8_gemm_nt_f32", "dg_bf16_gemm_nt",
-                    "dg_m_grouped_bf16_gemm_nt_contiguous", "dg_m_grouped_bf16_gemm_nt_masked")
+                    "dg_m_grouped_bf16_gemm_nt_contiguous", "dg_m_grouped_bf16_gemm_nt_masked",
+                    "dg_set_wait_timeout_ns", "dg_fp8_gemm_nt_noalloc_get_last_device_error",
+                    "dg_set_check_scales")
 
 DEVICE_ERRORS = {
     0x101: "wait timeout in the TMA producer",
@@ -81,6 +86,7 @@ DEVICE_ERRORS = {
     0x104: "wait timeout in the epilogue",
     0x201: "a 128-row block of m_indices names two experts",
     0x202: "an m_indices entry is >= the number of groups",
+    0x301: "a scale that is not a positive normal power of two",
 }
 
 
@@ -212,7 +218,8 @@ def fp8_gemm_nt_noalloc(a: torch.Tensor, sfa: torch.Tensor, b: torch.Tensor, sfb
                         d: torch.Tensor) -> torch.Tensor:
     """Dense GEMM through the entry point that allocates no device memory (its
     scratch is a fixed array inside the library), for callers that cannot
-    allocate.  ``d`` must be given.  Calls must not overlap on the GPU."""
+    allocate.  ``d`` must be given.  Calls must not overlap on the GPU.  Its
+    device error codes are read with :func:`noalloc_get_last_device_error`."""
     _fp8_bytes(a, "a"); _fp8_bytes(b, "b")
     M, K = a.shape
     N = b.shape[0]
@@ -358,8 +365,27 @@ def get_last_device_error() -> int:
     return code.value
 
 
+def noalloc_get_last_device_error() -> int:
+    """Synchronise, then read and clear the error word of the no-alloc entry
+    point (0: none since the last read)."""
+    code = ctypes.c_int(0)
+    _check(_noalloc_err(ctypes.byref(code)), "dg_fp8_gemm_nt_noalloc_get_last_device_error")
+    return code.value
+
+
 def set_wait_timeout_ms(ms: int) -> None:
     _check(_set_timeout(int(ms)), "dg_set_wait_timeout_ms")
+
+
+def set_check_scales(enable: bool) -> None:
+    """Make later launches check every scale against the contract (a positive
+    normal power of two; device error 0x301 otherwise)."""
+    _check(_set_check_scales(1 if enable else 0), "dg_set_check_scales")
+
+
+def set_wait_timeout_ns(ns: int) -> None:
+    """Time limit of every wait inside later launches, in nanoseconds."""
+    _check(_set_timeout_ns(int(ns)), "dg_set_wait_timeout_ns")
 
 
 def query_config(kind: int, rows: int, N: int, K: int, G: int = 1, expected_m: int = 0,

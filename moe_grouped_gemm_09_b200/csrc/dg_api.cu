@@ -7,27 +7,21 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
-#include <array>
 #include <mutex>
-#include <type_traits>
-#include <utility>
 
 #include "../../include/dg.h"
-#include "dg_config.h"
-#include "sm100_fp8_gemm.cuh"
-#include "sm100_fp8_gemm_pair.cuh"
+#include "dg_internal.h"
 
 namespace dg {
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kNumForms = 10;  // launch forms (enum Form below)
 
 struct DeviceState {
   bool ready = false;
   int num_sms = 0;
   int* error_word = nullptr;      // one int, device memory
-  bool smem_attr_set[kNumForms][kNumVariants] = {};  // per form and variant
+  bool attr_set[kNumForms][kNumVariants] = {};  // shared-memory limit raised, per form and variant
   bool limits_known = false;
   ClusterLimits limits = {};      // co-resident split-K clusters per variant and size
 };
@@ -35,51 +29,58 @@ struct DeviceState {
 std::mutex g_mutex;
 DeviceState g_dev[kMaxDevices];
 int g_num_sms_cap = 0;            // 0: all SMs
+
+// Settings every entry point reads (guarded by their own mutex: the no-alloc
+// entry point reads them without holding g_mutex).
+std::mutex g_settings_mutex;
 unsigned long long g_timeout_ns = 1000ull * 1000 * 1000;
 bool g_timeout_from_env = false;
+int g_check_scales = -1;          // -1: not decided yet (read DG_CHECK_SCALES)
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+std::once_flag g_encode_once;
 EncodeTiledFn g_encode = nullptr;
 
-dg_status from_cuda(cudaError_t e) { return e == cudaSuccess ? DG_OK : DG_ERR_CUDA; }
+EncodeTiledFn encoder() {
+  std::call_once(g_encode_once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  });
+  return g_encode;
+}
+
+bool env_flag(const char* name) {
+  const char* e = std::getenv(name);
+  return e && e[0] && e[0] != '0';
+}
 
 bool print_configs() {
-  static int v = -1;
-  if (v < 0) {
-    const char* e = std::getenv("DG_PRINT_CONFIGS");
-    v = (e && e[0] && e[0] != '0') ? 1 : 0;
-  }
-  return v == 1;
+  static const bool v = env_flag("DG_PRINT_CONFIGS");
+  return v;
 }
 
 // Initialise (once) the state of the current device.  Caller holds g_mutex.
-dg_status device_state(DeviceState** out, int* dev_out) {
+dg_status device_state(DeviceState** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return DG_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return DG_ERR_UNSUPPORTED;
   DeviceState& st = g_dev[dev];
   if (!st.ready) {
-    cudaDeviceProp prop;
-    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return DG_ERR_CUDA;
-    if (prop.major != 10 || prop.minor != 0) return DG_ERR_ARCH;
-    if (!g_encode) {
-      cudaDriverEntryPointQueryResult q;
-      void* fn = nullptr;
-      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
-              cudaSuccess ||
-          q != cudaDriverEntryPointSuccess || fn == nullptr)
-        return DG_ERR_CUDA;
-      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
-    }
-    if (!g_timeout_from_env) {
-      g_timeout_from_env = true;
-      const char* e = std::getenv("DG_WAIT_TIMEOUT_MS");
-      if (e && std::atoi(e) > 0) g_timeout_ns = 1000000ull * std::atoi(e);
-    }
-    st.num_sms = prop.multiProcessorCount;
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return DG_ERR_CUDA;
+    if (major != 10 || minor != 0) return DG_ERR_ARCH;
+    if (!encoder()) return DG_ERR_CUDA;
+    st.num_sms = sms;
     if (!st.error_word && cudaMalloc(&st.error_word, sizeof(int)) != cudaSuccess) {
       st.error_word = nullptr;
       return DG_ERR_CUDA;
@@ -90,16 +91,13 @@ dg_status device_state(DeviceState** out, int* dev_out) {
     st.ready = true;
   }
   *out = &st;
-  if (dev_out) *dev_out = dev;
   return DG_OK;
 }
 
-// Rows per TMA box of A: a whole tile (128 rows, or 256 for a two-half
-// variant), except that a dense A shorter than one 128-row block is fetched
-// with a box of its own (16-row rounded) height, so the SM moves no padding.
-int a_box_rows(int kind, int rows, const Variant& var) {
-  if (var.a_rows == 256) return 256;
-  if (var.pair) return kBlockM;
+// Rows per TMA box of A: a whole 128-row tile, except that a dense A shorter
+// than one 128-row block is fetched with a box of its own (16-row rounded)
+// height, so the SM moves no padding.
+int a_box_rows(int kind, int rows) {
   if (kind != kDense || rows >= kBlockM) return kBlockM;
   return ((rows + 15) / 16) * 16;
 }
@@ -114,18 +112,16 @@ void forced_config(int kind, int rows, int N, int K, int G, int sms, PickedConfi
   if (!e || !e[0]) return;
   int bn = 0, sk = 1;
   if (std::sscanf(e, "%d:%d", &bn, &sk) < 1) return;
-  int kps = 0, ar = 0, sm = -1, pr = -1;
-  std::sscanf(e, "%*d:%*d:%d:%d:%d:%d", &kps, &ar, &sm, &pr);
+  int kps = 0, ar = 0, sm = -1;
+  std::sscanf(e, "%*d:%*d:%d:%d:%d", &kps, &ar, &sm);
   int v = -1;
   for (int i = 0; i < kNumVariants; ++i) {
     const Variant& x = kVariants[i];
     if (x.block_n != bn) continue;
     if (kps ? (x.kps != kps || (ar && x.a_rows != ar)) : x.decode) continue;
     if (sm >= 0 && x.small != (sm != 0)) continue;
-    if (x.pair != (pr > 0)) continue;
-    if ((x.decode || x.a_rows == 256 || x.pair) && kind != kDense) continue;
-    if ((x.a_rows == 256 || x.pair) && rows < 256) continue;
-    if (a_box_rows(kind, rows, x) > x.a_rows) continue;
+    if (x.decode && kind != kDense) continue;
+    if (a_box_rows(kind, rows) > x.a_rows) continue;
     v = i;
   }
   const int KB = K / kBlockK;
@@ -137,29 +133,7 @@ void forced_config(int kind, int rows, int N, int K, int G, int sms, PickedConfi
   pc->variant = v;
   pc->split_k = sk;
   pc->out_tiles = static_cast<int>(tiles);
-  if (kVariants[v].pair) {
-    const long long pairs = tiles < sms / 2 ? tiles : sms / 2;
-    pc->grid = static_cast<int>(2 * (pairs > 0 ? pairs : 1));
-    return;
-  }
   pc->grid = sk > 1 ? static_cast<int>(tiles) * sk : static_cast<int>(tiles < sms ? tiles : sms);
-}
-
-// L2 prefetch of the first tile before the dependency wait; DG_NO_PREFETCH=1
-// turns it off (for measurements).
-int prefetch_enabled() {
-  static int v = -1;
-  if (v < 0) {
-    const char* e = std::getenv("DG_NO_PREFETCH");
-    v = (e && e[0] && e[0] != '0') ? 0 : 1;
-  }
-  return v;
-}
-
-int effective_sms(const DeviceState& st) {
-  int n = st.num_sms;
-  if (g_num_sms_cap > 0 && g_num_sms_cap < n) n = g_num_sms_cap;
-  return n;
 }
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -178,12 +152,11 @@ dg_status make_map(CUtensorMap* map, const void* base, uint64_t K, uint64_t rows
   cuuint64_t strides[3] = {kb, 128, kb * rows};  // bytes, for dims 1..3
   cuuint32_t box[4] = {block, box_rows, kps, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = g_encode(map, elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
-                                             : CU_TENSOR_MAP_DATA_TYPE_UINT8,
-                        4, const_cast<void*>(base), dims,
-                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = encoder()(map, elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                              : CU_TENSOR_MAP_DATA_TYPE_UINT8,
+                         4, const_cast<void*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? DG_OK : DG_ERR_CUDA;
 }
 
@@ -194,31 +167,10 @@ dg_status make_d_map(CUtensorMap* map, void* base, uint64_t N, uint64_t rows) {
   cuuint64_t strides[1] = {N * 2};
   cuuint32_t box[2] = {64, 32};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                        CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = encoder()(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? DG_OK : DG_ERR_CUDA;
-}
-
-// Launch forms: the three GEMM forms, then the dense form with M-major A
-// and/or N-major B, then the dense form with FP32 output (D = A B^T + C),
-// then the three GEMM forms on BF16 operands; the forms differ in their
-// kernel instantiation.
-enum Form : int { kFormDense = 0, kFormContiguous = 1, kFormMasked = 2, kFormNN = 3, kFormTN = 4,
-                  kFormTT = 5, kFormF32 = 6, kFormBf16Dense = 7, kFormBf16Contiguous = 8,
-                  kFormBf16Masked = 9 };
-static_assert(kFormBf16Masked + 1 == kNumForms, "one shared-memory attribute row per form");
-constexpr bool is_bf16_form(int f) { return f >= kFormBf16Dense; }
-constexpr int kind_of_form(int f) {
-  return f < 3 ? f : is_bf16_form(f) ? f - kFormBf16Dense : kDense;
-}
-constexpr int layout_of_form(int f) {
-  return f == kFormNN ? kLayoutNN : f == kFormTN ? kLayoutTN : f == kFormTT ? kLayoutTT : kLayoutNT;
-}
-// Variants that serve M-/N-major operands and the FP32 output form: general
-// ones with 128-column B boxes.
-constexpr bool mn_capable(const Variant& v) {
-  return !v.decode && !v.small && !v.pair && v.kps == 1 && v.a_rows == 128 && v.block_n % 128 == 0;
 }
 
 // 2-D tensor map over an M-/N-major operand stored as [K, mn] bytes (mn
@@ -228,210 +180,143 @@ dg_status make_map_mn(CUtensorMap* map, const void* base, uint64_t mn, uint64_t 
   cuuint64_t strides[1] = {mn};
   cuuint32_t box[2] = {128, 128};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
-                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = encoder()(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? DG_OK : DG_ERR_CUDA;
 }
 
-template <int V, bool SCALED = true>
-using ShapeOf = std::conditional_t<
-    kVariants[V].pair, PairShape<kVariants[V].block_n, kVariants[V].stages>,
-    KernelShape<kVariants[V].block_n, kVariants[V].stages, kVariants[V].num_acc,
-                kVariants[V].kps, kVariants[V].a_rows, kVariants[V].small, SCALED>>;
-// The geometry a form's kernel is built with (BF16 operands: no scale factors).
-template <int FORM, int V>
-using FormShape = ShapeOf<V, !is_bf16_form(FORM)>;
-
-// Kernels are instantiated only for the (form, variant) pairs that exist:
-// the decode, 256-row and pair variants serve the dense form only.
-// Per-variant shared-memory bytes (what = 0) or TMEM columns (what = 1).
-template <int what, int... V>
-constexpr std::array<int, sizeof...(V)> variant_table(std::integer_sequence<int, V...>) {
-  return {(what == 0 ? ShapeOf<V>::kSmemBytes : ShapeOf<V>::kTmemCols)...};
+int effective_sms(const DeviceState& st) {
+  int n = st.num_sms;
+  if (g_num_sms_cap > 0 && g_num_sms_cap < n) n = g_num_sms_cap;
+  return n;
 }
 
-template <int FORM, int V>
-constexpr bool kBuilt =
-    FORM == kFormDense ||
-    ((FORM == kFormContiguous || FORM == kFormMasked || FORM == kFormBf16Contiguous ||
-      FORM == kFormBf16Masked) &&
-     !kVariants[V].decode && kVariants[V].a_rows != 256 && !kVariants[V].pair) ||
-    (FORM == kFormBf16Dense && kVariants[V].a_rows != 256 && !kVariants[V].pair) ||
-    (FORM >= kFormNN && FORM <= kFormF32 && mn_capable(kVariants[V]));
-
-template <int FORM, int V>
-auto kernel_of() {
-  constexpr Variant var = kVariants[V];
-  if constexpr (var.pair) {
-    return fp8_gemm_pair_kernel<var.block_n, var.stages>;
-  } else {
-    return fp8_gemm_kernel<kind_of_form(FORM), var.block_n, var.stages, var.num_acc, var.kps,
-                           var.a_rows, var.small, layout_of_form(FORM), FORM == kFormF32,
-                           is_bf16_form(FORM)>;
+dg_status launch_plan(DeviceState& st, const LaunchPlan& pl, cudaStream_t stream) {
+  bool* row = st.attr_set[pl.form];
+  switch (pl.form) {
+    case kFormDense: return launch_fp8_dense(row, pl, stream);
+    case kFormContiguous:
+    case kFormMasked: return launch_fp8_grouped(row, pl, stream);
+    case kFormNN:
+    case kFormTN:
+    case kFormTT:
+    case kFormF32: return launch_fp8_layouts(row, pl, stream);
+    case kFormBf16Dense: return launch_bf16_dense(row, pl, stream);
+    default: return launch_bf16_grouped(row, pl, stream);
   }
 }
 
-template <int KIND, int V>
-dg_status set_smem_attr(DeviceState& st) {
-  if constexpr (!kBuilt<KIND, V>) {
-    return DG_ERR_UNSUPPORTED;
-  } else {
-    if (!st.smem_attr_set[KIND][V]) {
-      if (cudaFuncSetAttribute(kernel_of<KIND, V>(), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               FormShape<KIND, V>::kSmemBytes) != cudaSuccess)
-        return DG_ERR_CUDA;
-      st.smem_attr_set[KIND][V] = true;
-    }
-    return DG_OK;
-  }
-}
-
-// How many clusters of each size the device co-schedules: split-K clusters of
-// every decode variant, and SM pairs of every pair variant (a cluster must fit
-// in one GPC, so fewer pairs than SMs / 2 may be resident at once).
-template <int V>
-dg_status query_cluster_limits(DeviceState& st) {
-  if constexpr (kVariants[V].decode || kVariants[V].pair) {
-    dg_status s = set_smem_attr<kDense, V>(st);
-    if (s != DG_OK) return s;
-    for (int c = kVariants[V].pair ? 2 : 1; c <= (kVariants[V].pair ? 2 : kMaxSplitK); ++c) {
-      cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3(c, 1, 1);
-      cfg.blockDim = dim3(kThreads, 1, 1);
-      cfg.dynamicSmemBytes = ShapeOf<V>::kSmemBytes;
-      cudaLaunchAttribute attr[1];
-      attr[0].id = cudaLaunchAttributeClusterDimension;
-      attr[0].val.clusterDim.x = c;
-      attr[0].val.clusterDim.y = 1;
-      attr[0].val.clusterDim.z = 1;
-      cfg.attrs = attr;
-      cfg.numAttrs = 1;
-      int n = 0;
-      if (cudaOccupancyMaxActiveClusters(&n, kernel_of<kDense, V>(), &cfg) != cudaSuccess) {
-        cudaGetLastError();  // clear; treat as "not known"
-        n = 0;
-      }
-      st.limits.max_clusters[V][c] = n;
-    }
-  }
-  return DG_OK;
-}
-
-template <int... V>
-dg_status query_all_cluster_limits(DeviceState& st, std::integer_sequence<int, V...>) {
-  dg_status s = DG_OK;
-  ((s = (s == DG_OK ? query_cluster_limits<V>(st) : s)), ...);
-  return s;
-}
-
-dg_status ensure_cluster_limits(DeviceState& st) {
-  if (st.limits_known) return DG_OK;
-  dg_status s = query_all_cluster_limits(st, std::make_integer_sequence<int, kNumVariants>{});
+// Shared path of every GEMM entry point.
+dg_status run(const GemmCall& call, cudaStream_t stream) {
+  bool empty = false;
+  dg_status s = check_gemm_call(call, &empty);  // before any device work
+  if (s != DG_OK || empty) return s;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceState* st = nullptr;
+  s = device_state(&st);
   if (s != DG_OK) return s;
-  st.limits_known = true;
-  return DG_OK;
-}
-
-template <int KIND, int V>
-dg_status launch_variant(DeviceState& st, const CUtensorMap& ta, const CUtensorMap& tb,
-                         const CUtensorMap& td, const GemmArgs& args, int grid,
-                         cudaStream_t stream) {
-  if constexpr (!kBuilt<KIND, V>) {
-    return DG_ERR_UNSUPPORTED;
-  } else {
-    dg_status s = set_smem_attr<KIND, V>(st);
+  if (kind_of_form(call.form) == kDense && !st->limits_known) {
+    s = query_decode_cluster_limits(st->attr_set[kFormDense], &st->limits);
     if (s != DG_OK) return s;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid, 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = FormShape<KIND, V>::kSmemBytes;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    int n_attr = 1;
-    if (args.split_k > 1 || kVariants[V].pair) {  // the CTAs of one output tile form a cluster
-      attr[1].id = cudaLaunchAttributeClusterDimension;
-      attr[1].val.clusterDim.x = kVariants[V].pair ? 2 : args.split_k;
-      attr[1].val.clusterDim.y = 1;
-      attr[1].val.clusterDim.z = 1;
-      n_attr = 2;
-    }
-    cfg.attrs = attr;
-    cfg.numAttrs = n_attr;
-    return from_cuda(cudaLaunchKernelEx(&cfg, kernel_of<KIND, V>(), ta, tb, td, args));
+    st->limits_known = true;
   }
+  LaunchPlan pl;
+  s = plan_gemm(call, DeviceFacts{effective_sms(*st), &st->limits}, st->error_word, &pl);
+  if (s != DG_OK || pl.grid == 0) return s;
+  return launch_plan(*st, pl, stream);
 }
 
-template <int KIND, int... V>
-dg_status launch_dispatch(DeviceState& st, int variant, const CUtensorMap& ta,
-                          const CUtensorMap& tb, const CUtensorMap& td, const GemmArgs& args,
-                          int grid, cudaStream_t stream, std::integer_sequence<int, V...>) {
-  dg_status s = DG_ERR_UNSUPPORTED;
-  ((variant == V ? (s = launch_variant<KIND, V>(st, ta, tb, td, args, grid, stream), 0) : 0),
-   ...);
-  return s;
+}  // namespace
+
+unsigned long long wait_timeout_ns() {
+  std::lock_guard<std::mutex> lock(g_settings_mutex);
+  if (!g_timeout_from_env) {
+    g_timeout_from_env = true;
+    const char* e = std::getenv("DG_WAIT_TIMEOUT_MS");
+    if (e && std::atoi(e) > 0) g_timeout_ns = 1000000ull * std::atoi(e);
+  }
+  return g_timeout_ns;
 }
 
-template <int KIND>
-dg_status launch(DeviceState& st, int variant, const CUtensorMap& ta, const CUtensorMap& tb,
-                 const CUtensorMap& td, const GemmArgs& args, int grid, cudaStream_t stream) {
-  return launch_dispatch<KIND>(st, variant, ta, tb, td, args, grid, stream,
-                               std::make_integer_sequence<int, kNumVariants>{});
+// L2 prefetch of the first tile before the dependency wait; DG_NO_PREFETCH=1
+// turns it off (for measurements).
+int prefetch_enabled() {
+  static const int v = env_flag("DG_NO_PREFETCH") ? 0 : 1;
+  return v;
 }
 
-// Shared path of the three GEMM forms.
-dg_status run(int form, const void* a, const float* sfa, const void* b, const float* sfb,
-              void* d, const int* m_indices, const int* masked_m, int rows, int N, int K, int G,
-              int expected_m, cudaStream_t stream, const float* c = nullptr) {
+// The kernels check every scale they read against the contract (a positive
+// normal power of two) and report device error 0x301: off unless
+// DG_CHECK_SCALES=1 or dg_set_check_scales(1).
+int check_scales_enabled() {
+  std::lock_guard<std::mutex> lock(g_settings_mutex);
+  if (g_check_scales < 0) g_check_scales = env_flag("DG_CHECK_SCALES") ? 1 : 0;
+  return g_check_scales;
+}
+
+dg_status check_gemm_call(const GemmCall& call, bool* empty) {
+  const int form = call.form;
   const int kind = kind_of_form(form);
   const int layout = layout_of_form(form);
-  const bool a_mn = (layout & 1) != 0, b_mn = (layout & 2) != 0;
+  const bool a_mn = (layout & 1) != 0;
   const bool bf16 = is_bf16_form(form);
-  // ---- argument checks (no device work) ----
+  const int rows = call.rows, N = call.N, K = call.K, G = call.G;
+  *empty = false;
   // A K block is 128 bytes of a row: 128 E4M3 or 64 BF16 elements.
   const int k_block = bf16 ? kBlockK / 2 : kBlockK;
   if (rows < 0 || G < 0) return DG_ERR_INVALID_ARG;
   if (K <= 0 || K % k_block != 0 || N <= 0 || N % 16 != 0) return DG_ERR_INVALID_ARG;
-  if (rows == 0 || G == 0) return DG_OK;
-  if (!a || !b || !d || (!bf16 && (!sfa || !sfb))) return DG_ERR_INVALID_ARG;
-  if (!aligned(a, 16) || !aligned(b, 16) || !aligned(d, 16) ||
-      (!bf16 && (!aligned(sfa, 4) || !aligned(sfb, 4))))
+  if (rows == 0 || G == 0) {
+    *empty = true;
+    return DG_OK;
+  }
+  if (!call.a || !call.b || !call.d || (!bf16 && (!call.sfa || !call.sfb)))
     return DG_ERR_INVALID_ARG;
-  if (kind == kContiguous && (!m_indices || !aligned(m_indices, 4) || rows % 128 != 0))
+  if (!aligned(call.a, 16) || !aligned(call.b, 16) || !aligned(call.d, 16) ||
+      (!bf16 && (!aligned(call.sfa, 4) || !aligned(call.sfb, 4))))
+    return DG_ERR_INVALID_ARG;
+  if (kind == kContiguous &&
+      (!call.m_indices || !aligned(call.m_indices, 4) || rows % 128 != 0))
     return DG_ERR_INVALID_ARG;
   if (a_mn && rows % 16 != 0) return DG_ERR_INVALID_ARG;  // [K, M] rows of whole 16-byte units
-  if (form == kFormF32 && c && !aligned(c, 16)) return DG_ERR_INVALID_ARG;
-  if (kind == kMasked && (!masked_m || !aligned(masked_m, 4))) return DG_ERR_INVALID_ARG;
+  if (form == kFormF32 && call.c && !aligned(call.c, 16)) return DG_ERR_INVALID_ARG;
+  if (kind == kMasked && (!call.masked_m || !aligned(call.masked_m, 4))) return DG_ERR_INVALID_ARG;
   if (kind == kMasked && G > kMaxMaskedGroups) return DG_ERR_UNSUPPORTED;
   const long long a_rows = (kind == kMasked) ? static_cast<long long>(G) * rows : rows;
   if (a_rows > 0x7fffffffLL || static_cast<long long>(G) * N > 0x7fffffffLL)
     return DG_ERR_UNSUPPORTED;
   if (K > (1 << 24)) return DG_ERR_UNSUPPORTED;
+  return DG_OK;
+}
+
+dg_status plan_gemm(const GemmCall& call, const DeviceFacts& facts, int* error_word,
+                    LaunchPlan* pl) {
+  pl->grid = 0;
+  bool empty = false;
+  dg_status s = check_gemm_call(call, &empty);
+  if (s != DG_OK || empty) return s;
+  const int form = call.form;
+  const int kind = kind_of_form(form);
+  const int layout = layout_of_form(form);
+  const bool a_mn = (layout & 1) != 0, b_mn = (layout & 2) != 0;
+  const bool bf16 = is_bf16_form(form);
+  const int rows = call.rows, N = call.N, K = call.K, G = call.G;
+  const long long a_rows = (kind == kMasked) ? static_cast<long long>(G) * rows : rows;
   // the picker and the kernel count K in 128-byte blocks of a row
   const int k_bytes = bf16 ? 2 * K : K;
+  const int sms = facts.num_sms;
 
-  std::lock_guard<std::mutex> lock(g_mutex);
-  DeviceState* st = nullptr;
-  dg_status s = device_state(&st, nullptr);
-  if (s != DG_OK) return s;
-  const int sms = effective_sms(*st);
-  if (kind == kDense) {
-    s = ensure_cluster_limits(*st);
-    if (s != DG_OK) return s;
-  }
-  PickedConfig pc = pick_config(kind, rows, N, k_bytes, G, expected_m, sms, &st->limits,
-                                /*allow_pair=*/!bf16,
+  PickedConfig pc = pick_config(kind, rows, N, k_bytes, G, call.expected_m, sms, facts.limits,
                                 /*mn_operands=*/layout != kLayoutNT || form == kFormF32);
   forced_config(kind, rows, N, k_bytes, G, sms, &pc);
   const Variant var = kVariants[pc.variant];
   if ((layout != kLayoutNT || form == kFormF32) && (!mn_capable(var) || pc.split_k > 1))
     return DG_ERR_UNSUPPORTED;
-  if (bf16 && (var.pair || var.a_rows == 256)) return DG_ERR_UNSUPPORTED;
 
-  GemmArgs args = {};
+  GemmArgs& args = pl->args;
+  args = GemmArgs{};
   args.rows = rows;
   args.N = N;
   args.K = K;
@@ -442,27 +327,19 @@ dg_status run(int form, const void* a, const float* sfa, const void* b, const fl
   args.split_k = pc.split_k;
   args.kb_per_split = ceil_div(args.k_blocks, pc.split_k);
   args.nb128 = ceil_div(N, 128);
-  args.sfa = sfa;
-  args.sfb = sfb;
-  args.d = static_cast<__nv_bfloat16*>(d);
-  args.d_f32 = form == kFormF32 ? static_cast<float*>(d) : nullptr;
-  args.c_f32 = form == kFormF32 ? c : nullptr;
-  args.m_indices = m_indices;
-  args.masked_m = masked_m;
-  args.error_word = st->error_word;
-  args.timeout_ns = g_timeout_ns;
-  args.a_box_rows = a_mn ? kBlockM : a_box_rows(kind, rows, var);
-  if (args.a_box_rows > var.a_rows) return DG_ERR_UNSUPPORTED;
-  if ((var.a_rows == 256 || var.pair) && (kind != kDense || pc.split_k > 1))
-    return DG_ERR_UNSUPPORTED;
-  if (var.pair) {
-    // no more pairs than the device co-schedules: a pair launched beyond that
-    // would only start once another has finished all its tiles
-    const int resident = cluster_limit(&st->limits, pc.variant, 2, sms);
-    if (pc.grid / 2 > resident) pc.grid = 2 * resident;
-    if (pc.grid % 2 != 0 || pc.grid < 2) return DG_ERR_UNSUPPORTED;
-  }
+  args.sfa = call.sfa;
+  args.sfb = call.sfb;
+  args.d = static_cast<__nv_bfloat16*>(call.d);
+  args.d_f32 = form == kFormF32 ? static_cast<float*>(call.d) : nullptr;
+  args.c_f32 = form == kFormF32 ? call.c : nullptr;
+  args.m_indices = call.m_indices;
+  args.masked_m = call.masked_m;
+  args.error_word = error_word;
+  args.timeout_ns = wait_timeout_ns();
+  args.a_box_rows = a_mn ? kBlockM : a_box_rows(kind, rows);
   args.prefetch = prefetch_enabled();
+  args.check_scales = bf16 ? 0 : check_scales_enabled();
+  if (args.a_box_rows > var.a_rows) return DG_ERR_UNSUPPORTED;
   // a small variant runs one tile per CTA (its epilogue reuses the ring)
   if (var.small && (kind != kDense || pc.grid != args.num_m_blocks * args.num_n_blocks * pc.split_k))
     return DG_ERR_UNSUPPORTED;
@@ -472,117 +349,109 @@ dg_status run(int form, const void* a, const float* sfa, const void* b, const fl
        rows > kBlockM || !split_fits(var, rows, pc.split_k)))
     return DG_ERR_UNSUPPORTED;
 
-  CUtensorMap ta, tb;
   const int b_groups = (kind == kDense) ? 1 : G;
   const uint32_t elem = bf16 ? 2 : 1;
-  s = a_mn ? make_map_mn(&ta, a, rows, K)
-           : make_map(&ta, a, K, rows, kind == kMasked ? G : 1, args.a_box_rows, var.kps, elem);
+  s = a_mn ? make_map_mn(&pl->ta, call.a, rows, K)
+                     : make_map(&pl->ta, call.a, K, rows, kind == kMasked ? G : 1,
+                                args.a_box_rows, var.kps, elem);
   if (s != DG_OK) return s;
-  s = b_mn ? make_map_mn(&tb, b, N, K)
-           : make_map(&tb, b, K, N, b_groups, var.pair ? var.block_n / 2 : var.block_n, var.kps,
-                      elem);
+  s = b_mn ? make_map_mn(&pl->tb, call.b, N, K)
+           : make_map(&pl->tb, call.b, K, N, b_groups, var.block_n, var.kps, elem);
   if (s != DG_OK) return s;
-  CUtensorMap td;
-  s = make_d_map(&td, d, N, static_cast<uint64_t>(a_rows));
+  s = make_d_map(&pl->td, call.d, N, static_cast<uint64_t>(a_rows));
   if (s != DG_OK) return s;
 
   if (print_configs())
     std::fprintf(stderr,
-                 "[dg] kind=%d rows=%d N=%d K=%d G=%d expected_m=%d -> BLOCK_N=%d stages=%d "
-                 "acc=%d split_k=%d grid=%d\n",
-                 kind, rows, N, K, G, expected_m, var.block_n, var.stages, var.num_acc,
-                 pc.split_k, pc.grid);
-
-  switch (form) {
-    case kFormDense: return launch<kFormDense>(*st, pc.variant, ta, tb, td, args, pc.grid, stream);
-    case kFormContiguous:
-      return launch<kFormContiguous>(*st, pc.variant, ta, tb, td, args, pc.grid, stream);
-    case kFormMasked:
-      return launch<kFormMasked>(*st, pc.variant, ta, tb, td, args, pc.grid, stream);
-    case kFormNN: return launch<kFormNN>(*st, pc.variant, ta, tb, td, args, pc.grid, stream);
-    case kFormTN: return launch<kFormTN>(*st, pc.variant, ta, tb, td, args, pc.grid, stream);
-    case kFormTT: return launch<kFormTT>(*st, pc.variant, ta, tb, td, args, pc.grid, stream);
-    case kFormF32: return launch<kFormF32>(*st, pc.variant, ta, tb, td, args, pc.grid, stream);
-    case kFormBf16Dense:
-      return launch<kFormBf16Dense>(*st, pc.variant, ta, tb, td, args, pc.grid, stream);
-    case kFormBf16Contiguous:
-      return launch<kFormBf16Contiguous>(*st, pc.variant, ta, tb, td, args, pc.grid, stream);
-    default:
-      return launch<kFormBf16Masked>(*st, pc.variant, ta, tb, td, args, pc.grid, stream);
-  }
+                 "[dg] form=%d rows=%d N=%d K=%d G=%d expected_m=%d -> BLOCK_N=%d stages=%d "
+                 "kps=%d acc=%d split_k=%d grid=%d\n",
+                 form, rows, N, K, G, call.expected_m, var.block_n, var.stages, var.kps,
+                 var.num_acc, pc.split_k, pc.grid);
+  pl->form = form;
+  pl->variant = pc.variant;
+  pl->grid = pc.grid;
+  return DG_OK;
 }
 
-}  // namespace
 }  // namespace dg
 
 using namespace dg;
+
+namespace {
+
+cudaStream_t as_stream(dg_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+dg_status dense_call(int form, const void* a, const float* sfa, const void* b, const float* sfb,
+                     void* d, int M, int N, int K, dg_stream_t stream, const float* c = nullptr) {
+  GemmCall call{form, a, sfa, b, sfb, d, c, nullptr, nullptr, M, N, K, 1, 0};
+  return run(call, as_stream(stream));
+}
+
+}  // namespace
 
 extern "C" {
 
 dg_status dg_fp8_gemm_nt(const void* a, const float* sfa, const void* b, const float* sfb,
                          void* d, int M, int N, int K, dg_stream_t stream) {
-  return run(kFormDense, a, sfa, b, sfb, d, nullptr, nullptr, M, N, K, 1, 0,
-             reinterpret_cast<cudaStream_t>(stream));
+  return dense_call(kFormDense, a, sfa, b, sfb, d, M, N, K, stream);
 }
 
 dg_status dg_fp8_gemm_nn(const void* a, const float* sfa, const void* b, const float* sfb,
                          void* d, int M, int N, int K, dg_stream_t stream) {
-  return run(kFormNN, a, sfa, b, sfb, d, nullptr, nullptr, M, N, K, 1, 0,
-             reinterpret_cast<cudaStream_t>(stream));
+  return dense_call(kFormNN, a, sfa, b, sfb, d, M, N, K, stream);
 }
 
 dg_status dg_fp8_gemm_tn(const void* a, const float* sfa, const void* b, const float* sfb,
                          void* d, int M, int N, int K, dg_stream_t stream) {
-  return run(kFormTN, a, sfa, b, sfb, d, nullptr, nullptr, M, N, K, 1, 0,
-             reinterpret_cast<cudaStream_t>(stream));
+  return dense_call(kFormTN, a, sfa, b, sfb, d, M, N, K, stream);
 }
 
 dg_status dg_fp8_gemm_tt(const void* a, const float* sfa, const void* b, const float* sfb,
                          void* d, int M, int N, int K, dg_stream_t stream) {
-  return run(kFormTT, a, sfa, b, sfb, d, nullptr, nullptr, M, N, K, 1, 0,
-             reinterpret_cast<cudaStream_t>(stream));
+  return dense_call(kFormTT, a, sfa, b, sfb, d, M, N, K, stream);
 }
 
 dg_status dg_fp8_gemm_nt_f32(const void* a, const float* sfa, const void* b, const float* sfb,
                              const float* c, float* d, int M, int N, int K, dg_stream_t stream) {
-  return run(kFormF32, a, sfa, b, sfb, d, nullptr, nullptr, M, N, K, 1, 0,
-             reinterpret_cast<cudaStream_t>(stream), c);
+  return dense_call(kFormF32, a, sfa, b, sfb, d, M, N, K, stream, c);
 }
 
 dg_status dg_m_grouped_fp8_gemm_nt_contiguous(const void* a, const float* sfa, const void* b,
                                               const float* sfb, void* d, const int* m_indices,
                                               int M_sum, int N, int K, int G,
                                               dg_stream_t stream) {
-  return run(kFormContiguous, a, sfa, b, sfb, d, m_indices, nullptr, M_sum, N, K, G, 0,
-             reinterpret_cast<cudaStream_t>(stream));
+  GemmCall call{kFormContiguous, a, sfa, b, sfb, d, nullptr, m_indices, nullptr, M_sum, N, K, G, 0};
+  return run(call, as_stream(stream));
 }
 
 dg_status dg_m_grouped_fp8_gemm_nt_masked(const void* a, const float* sfa, const void* b,
                                           const float* sfb, void* d, const int* masked_m, int G,
                                           int max_m, int N, int K, int expected_m,
                                           dg_stream_t stream) {
-  return run(kFormMasked, a, sfa, b, sfb, d, nullptr, masked_m, max_m, N, K, G, expected_m,
-             reinterpret_cast<cudaStream_t>(stream));
+  GemmCall call{kFormMasked, a, sfa, b, sfb, d, nullptr, nullptr, masked_m, max_m, N, K, G,
+                expected_m};
+  return run(call, as_stream(stream));
 }
 
 dg_status dg_bf16_gemm_nt(const void* a, const void* b, void* d, int M, int N, int K,
                           dg_stream_t stream) {
-  return run(kFormBf16Dense, a, nullptr, b, nullptr, d, nullptr, nullptr, M, N, K, 1, 0,
-             reinterpret_cast<cudaStream_t>(stream));
+  return dense_call(kFormBf16Dense, a, nullptr, b, nullptr, d, M, N, K, stream);
 }
 
 dg_status dg_m_grouped_bf16_gemm_nt_contiguous(const void* a, const void* b, void* d,
                                                const int* m_indices, int M_sum, int N, int K,
                                                int G, dg_stream_t stream) {
-  return run(kFormBf16Contiguous, a, nullptr, b, nullptr, d, m_indices, nullptr, M_sum, N, K, G,
-             0, reinterpret_cast<cudaStream_t>(stream));
+  GemmCall call{kFormBf16Contiguous, a, nullptr, b, nullptr, d, nullptr, m_indices, nullptr,
+                M_sum, N, K, G, 0};
+  return run(call, as_stream(stream));
 }
 
 dg_status dg_m_grouped_bf16_gemm_nt_masked(const void* a, const void* b, void* d,
                                            const int* masked_m, int G, int max_m, int N, int K,
                                            int expected_m, dg_stream_t stream) {
-  return run(kFormBf16Masked, a, nullptr, b, nullptr, d, nullptr, masked_m, max_m, N, K, G,
-             expected_m, reinterpret_cast<cudaStream_t>(stream));
+  GemmCall call{kFormBf16Masked, a, nullptr, b, nullptr, d, nullptr, nullptr, masked_m, max_m,
+                N, K, G, expected_m};
+  return run(call, as_stream(stream));
 }
 
 dg_status dg_set_num_sms(int n) {
@@ -594,7 +463,7 @@ dg_status dg_set_num_sms(int n) {
 int dg_get_num_sms(void) {
   std::lock_guard<std::mutex> lock(g_mutex);
   DeviceState* st = nullptr;
-  if (device_state(&st, nullptr) != DG_OK) return -1;
+  if (device_state(&st) != DG_OK) return -1;
   return effective_sms(*st);
 }
 
@@ -602,7 +471,7 @@ dg_status dg_get_last_device_error(int* code) {
   if (!code) return DG_ERR_INVALID_ARG;
   std::lock_guard<std::mutex> lock(g_mutex);
   DeviceState* st = nullptr;
-  dg_status s = device_state(&st, nullptr);
+  dg_status s = device_state(&st);
   if (s != DG_OK) return s;
   if (cudaDeviceSynchronize() != cudaSuccess) return DG_ERR_CUDA;
   int v = 0;
@@ -616,12 +485,23 @@ dg_status dg_get_last_device_error(int* code) {
   return DG_OK;
 }
 
+dg_status dg_set_wait_timeout_ns(long long ns) {
+  if (ns <= 0) return DG_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(g_settings_mutex);
+  g_timeout_from_env = true;
+  g_timeout_ns = static_cast<unsigned long long>(ns);
+  return DG_OK;
+}
+
+dg_status dg_set_check_scales(int enable) {
+  std::lock_guard<std::mutex> lock(g_settings_mutex);
+  g_check_scales = enable ? 1 : 0;
+  return DG_OK;
+}
+
 dg_status dg_set_wait_timeout_ms(int ms) {
   if (ms <= 0) return DG_ERR_INVALID_ARG;
-  std::lock_guard<std::mutex> lock(g_mutex);
-  g_timeout_from_env = true;
-  g_timeout_ns = 1000000ull * static_cast<unsigned long long>(ms);
-  return DG_OK;
+  return dg_set_wait_timeout_ns(1000000LL * ms);
 }
 
 const char* dg_status_string(dg_status s) {
@@ -649,14 +529,12 @@ dg_status dg_query_config(int kind, int rows, int N, int K, int G, int expected_
   out->num_acc = v.num_acc;
   out->split_k = pc.split_k;
   out->grid = pc.grid;
-  constexpr auto smem = variant_table<0>(std::make_integer_sequence<int, kNumVariants>{});
-  constexpr auto tmem = variant_table<1>(std::make_integer_sequence<int, kNumVariants>{});
-  out->smem_bytes = smem[pc.variant];
-  out->tmem_cols = tmem[pc.variant];
+  out->smem_bytes = variant_smem_bytes(pc.variant);
+  out->tmem_cols = variant_tmem_cols(pc.variant);
   out->kps = v.kps;
   return DG_OK;
 }
 
-const char* dg_version(void) { return "0.1.0"; }
+const char* dg_version(void) { return "0.2.0"; }
 
 }  // extern "C"

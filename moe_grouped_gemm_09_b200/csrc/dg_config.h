@@ -17,16 +17,12 @@ struct Variant {
   int stages;
   int num_acc;
   int kps;      // 128-wide K blocks per ring stage (one TMA box of each operand)
-  int a_rows;   // rows of A a stage holds (64: dense A of at most 64 rows;
-                // 256: a tile of two 128-row halves sharing each B tile)
+  int a_rows;   // rows of A a stage holds (64: dense A of at most 64 rows)
   bool decode;  // built for dense problems of at most one 128-row block
   bool small;   // two CTAs fit per SM; one tile per CTA
-  bool pair;    // one 256-row tile per pair of SMs (a 2-CTA cluster issuing
-                // tcgen05 cta_group::2 MMAs); dense form only
 };
 
-// The compiled variants: general ones first (every form; the 256-row one
-// serves the dense form only, and only when forced), then the
+// The compiled variants: general ones first (every form), then the
 // decode-shaped dense ones, whose stages are several K blocks deep so that
 // each TMA box moves 32-64 KB, then the small decode ones (at most ~100 KB of
 // shared memory and 256 TMEM columns, so that the next kernel's CTAs can be
@@ -36,7 +32,6 @@ constexpr Variant kVariants[] = {
     {128, 6, 2, 1, 128, false, false},
     {64, 8, 2, 1, 128, false, false},
     {32, 9, 2, 1, 128, false, false},
-    {192, 3, 1, 1, 256, false, false},
     {128, 2, 1, 4, 64, true, false},
     {64, 3, 2, 4, 64, true, false},
     {256, 2, 1, 2, 64, true, false},
@@ -47,7 +42,6 @@ constexpr Variant kVariants[] = {
     {64, 3, 1, 2, 64, true, true},
     {128, 3, 1, 1, 128, true, true},
     {64, 2, 1, 2, 128, true, true},
-    {256, 6, 1, 1, 128, false, false, true},
 };
 constexpr int kNumVariants = sizeof(kVariants) / sizeof(kVariants[0]);
 constexpr int kMaxSplitK = 8;  // portable cluster size
@@ -61,11 +55,11 @@ struct PickedConfig {
 
 inline int ceil_div(long long a, long long b) { return static_cast<int>((a + b - 1) / b); }
 
-// Output rows of one tile of a variant.
-inline int tile_rows(const Variant& v) { return (v.a_rows == 256 || v.pair) ? 256 : 128; }
+// Output rows of one tile (every variant: one 128-row MMA block).
+inline int tile_rows(const Variant&) { return 128; }
 
-// How many clusters of `cluster` CTAs of variant `variant` the device can run
-// at once.  max_clusters[v][s] for s in 1..kMaxSplitK; a value <= 0 means
+// How many split-K clusters of `cluster` CTAs of variant `variant` the device
+// can run at once.  max_clusters[v][s] for s in 1..kMaxSplitK; a value <= 0 means
 // "not known": then the SM count divided by the cluster size is assumed.
 struct ClusterLimits {
   int max_clusters[kNumVariants][kMaxSplitK + 1];
@@ -145,7 +139,7 @@ inline bool pick_decode(int rows, int N, int K, int num_sms, const ClusterLimits
 // kind: 0 dense, 1 contiguous, 2 masked.  rows: M, M_sum or max_m.
 inline PickedConfig pick_config(int kind, int rows, int N, int K, int G, int expected_m,
                                 int num_sms, const ClusterLimits* lim = nullptr,
-                                bool allow_pair = true, bool mn_operands = false) {
+                                bool mn_operands = false) {
   PickedConfig best{1, 1, 1, 1};
   if (kind == 0 && rows <= 128 && !mn_operands &&
       pick_decode(rows, N, K, num_sms, lim, &best))
@@ -170,14 +164,6 @@ inline PickedConfig pick_config(int kind, int rows, int N, int K, int G, int exp
     // M-/N-major operands: one K block per stage and whole 128-column B boxes
     if (mn_operands && (var.decode || var.kps != 1 || var.block_n % 128 != 0)) continue;
     if (var.decode && (kind != 0 || var.kps != 2 || var.block_n != 256)) continue;
-    // The 256-row variant (fewer operand bytes per FLOP) measured no faster
-    // than the 128 x 256 tiles on B200: the ring is bound by the latency of
-    // the bytes in flight, not by their count.  It is taken only when forced.
-    if (var.a_rows == 256) continue;
-    // The SM-pair variant is correct but measured slower than the single-SM
-    // 128 x 256 tiles on B200 (1.6-1.7 against 1.8-2.0 PFLOP/s on the prefill
-    // shapes); it is taken only when forced.
-    if (var.pair) continue;
     const int bn = var.block_n;
     if (bn > 128 && N <= 128) continue;
     const int tm = tile_rows(var);
@@ -205,7 +191,6 @@ inline PickedConfig pick_config(int kind, int rows, int N, int K, int G, int exp
   best.out_tiles = tiles > 0x7fffffff ? 0x7fffffff : static_cast<int>(tiles);
   best.grid = tiles < num_sms ? static_cast<int>(tiles) : num_sms;
   if (best.grid < 1) best.grid = 1;
-  (void)allow_pair;  // reserved for the pair variant once the picker takes it
   return best;
 }
 

@@ -70,6 +70,8 @@ enum DeviceError : int {
   kDevTimeoutEpilogue = 0x104,
   kDevMixedExperts = 0x201,   // a 128-row block of m_indices names two experts
   kDevExpertRange = 0x202,    // an m_indices entry is >= G
+  kDevBadScale = 0x301,       // a scale that is not a positive normal power of two (checked
+                              // only when GemmArgs::check_scales is set)
 };
 
 struct GemmArgs {
@@ -93,6 +95,7 @@ struct GemmArgs {
   unsigned long long timeout_ns;
   int a_box_rows;    // rows of A one TMA box brings (128, or fewer for a short dense A)
   int prefetch;      // 1: warm L2 with the first tile before waiting on the previous kernel
+  int check_scales;  // 1: report scales that are not positive normal powers of two
 };
 
 constexpr int kBlockM = 128;
@@ -115,8 +118,7 @@ __host__ __device__ constexpr int pow2_ceil(int x) {
 //   KPS      128-wide K blocks per ring stage: every stage is one TMA box of A
 //            and one of B, each KPS K blocks deep (bigger boxes stream faster)
 //   A_ROWS   rows of A a stage holds room for (64 for a dense A of at most 64
-//            rows, 128, or 256 for a tile of two 128-row MMA halves that
-//            share every B tile: fewer operand bytes per FLOP)
+//            rows, else 128)
 //   SMALL    a decode variant small enough (shared memory and TMEM) for two
 //            CTAs per SM, so that the next kernel's CTAs can start (and warm
 //            L2) while this kernel drains; it runs one tile per CTA and
@@ -127,8 +129,6 @@ __host__ __device__ constexpr int pow2_ceil(int x) {
 template <int BLOCK_N, int STAGES, int NUM_ACC, int KPS = 1, int A_ROWS = 128, bool SMALL = false,
           bool SCALED = true>
 struct KernelShape {
-  static constexpr int kHalves = A_ROWS == 256 ? 2 : 1;  // 128-row MMA halves of a tile
-  static constexpr int kTileM = kBlockM * kHalves;        // output rows of a tile
   static constexpr int kABytes = KPS * A_ROWS * kBlockK;  // kBlockK bytes of a row per K block
   static constexpr int kBBytes = KPS * BLOCK_N * kBlockK;
   static constexpr int kSfbChunks = (BLOCK_N + 127) / 128;
@@ -136,13 +136,13 @@ struct KernelShape {
   // to 128 rows straddles one more)
   static constexpr int kSfbBlocks = kSfbChunks + (BLOCK_N % 128 != 0 && 128 % BLOCK_N != 0 ? 1 : 0);
   // SFA 512 B per 128 rows of A + SFB 512 B per 128 rows of B
-  static constexpr int kSfBytes = SCALED ? 512 * (kHalves + kSfbChunks) : 0;
-  static constexpr int kSfCols = SCALED ? 4 * (kHalves + kSfbChunks) : 0;  // TMEM columns per stage
+  static constexpr int kSfBytes = SCALED ? 512 * (1 + kSfbChunks) : 0;
+  static constexpr int kSfCols = SCALED ? 4 * (1 + kSfbChunks) : 0;  // TMEM columns per stage
   // stages whose K blocks share one set of scale words: four one-block
   // stages; a stage of several K blocks has words of its own (the decode
   // variants, where the per-stage scale path measured faster)
   static constexpr int kSfGroup = KPS == 1 ? 4 : 1;
-  static constexpr int kAccCols = NUM_ACC * kHalves * BLOCK_N;
+  static constexpr int kAccCols = NUM_ACC * BLOCK_N;
   static constexpr int kTmemCols = pow2_ceil(kAccCols + STAGES * kSfCols);
   static constexpr int kBarBytes = 8 * (2 * STAGES + 2 * NUM_ACC + 2);
   // epilogue: each of the 4 epilogue warps stages 32 rows x kEpiCols BF16
@@ -168,8 +168,7 @@ struct KernelShape {
   static_assert(BLOCK_N % 32 == 0 && BLOCK_N >= 32 && BLOCK_N <= 256, "BLOCK_N");
   static_assert(KPS >= 1 && KPS <= 4 && 4 % KPS == 0,
                 "four K blocks (a whole number of stages) share one scale-factor word");
-  static_assert(A_ROWS == 64 || A_ROWS == 128 || A_ROWS == 256, "A_ROWS");
-  static_assert(A_ROWS != 256 || (!SMALL && KPS == 1), "two-half tiles are general variants");
+  static_assert(A_ROWS == 64 || A_ROWS == 128, "A_ROWS");
   static_assert((BLOCK_N * kBlockK) % 1024 == 0, "B sub-tiles must keep 1024-byte alignment");
 };
 
@@ -181,6 +180,15 @@ struct Tile {
 // A positive power-of-two FP32 value is 2^(e-127) with e its exponent field;
 // UE8M0 encodes 2^(e-127) as the byte e.
 __device__ __forceinline__ uint32_t ue8m0(float v) { return (__float_as_uint(v) >> 23) & 0xFFu; }
+
+// The scales' contract: a positive normal power of two (sign 0, mantissa 0,
+// exponent field neither 0 nor 255), the only values whose exponent byte is
+// the whole value.
+__device__ __forceinline__ bool scale_ok(float v) {
+  const uint32_t u = __float_as_uint(v);
+  const uint32_t e = (u >> 23) & 0xFFu;
+  return (u & 0x807FFFFFu) == 0 && e != 0 && e != 0xFFu;
+}
 
 // Expert of a 128-row block in the contiguous layout: the largest m_indices
 // entry of the block (padding rows are -1).  Warp-collective.
@@ -328,8 +336,6 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
   constexpr int SF_COLS = Shape::kSfCols;
   constexpr int SFB_CHUNKS = Shape::kSfbChunks;
   constexpr int SFB_BLOCKS = Shape::kSfbBlocks;
-  constexpr int HALVES = Shape::kHalves;
-  constexpr int TILE_M = Shape::kTileM;
   constexpr int SF_GROUP = Shape::kSfGroup;
   constexpr int ACC_COLS = Shape::kAccCols;
   constexpr int TMEM_COLS = Shape::kTmemCols;
@@ -340,7 +346,6 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
   static_assert(kBlockM * RED_PITCH * 4 <= STAGES * (A_BYTES + B_BYTES),
                 "split-K partial must fit in the operand ring");
   static_assert((KPS == 1 && !SMALL) || KIND == kDense, "decode variants serve the dense form");
-  static_assert(HALVES == 1 || KIND == kDense, "a 256-row tile could straddle two groups");
   // M-major A / N-major B: 2-D maps over [K, M] / [K, N] with boxes of 128
   // MN bytes x 128 K rows; one K block per stage, whole 128-row A boxes, and B
   // tiles made of whole 128-column boxes.
@@ -364,8 +369,8 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
   // when every CTA has a single tile (always for a small variant), the operand
   // ring, idle once that tile's MMAs are done, with one tile per warp and chunk
   const int n_tiles_total = (KIND == kMasked ? -1 : p.num_m_blocks * p.num_n_blocks * p.split_k);
-  const bool one_tile = HALVES == 1 && (SMALL || (n_tiles_total >= 0 &&
-                                                  n_tiles_total <= static_cast<int>(gridDim.x)));
+  const bool one_tile =
+      SMALL || (n_tiles_total >= 0 && n_tiles_total <= static_cast<int>(gridDim.x));
   uint8_t* sEpi = one_tile ? sA : sB + STAGES * B_BYTES;
   uint8_t* sSF = sB + STAGES * B_BYTES + Shape::kEpiBytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(sSF + STAGES * SF_BYTES);
@@ -423,9 +428,9 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
           ptx::tma_prefetch_l2_4d(&tmap_b, 0, ti.n_blk * BLOCK_N, kb, 0);
         }
         if constexpr (A_MN) {
-          ptx::tma_prefetch_l2_2d(&tmap_a, ti.m_blk * TILE_M, kb * kBlockK);
+          ptx::tma_prefetch_l2_2d(&tmap_a, ti.m_blk * kBlockM, kb * kBlockK);
         } else {
-          if (!SMALL) ptx::tma_prefetch_l2_4d(&tmap_a, 0, ti.m_blk * TILE_M, kb, 0);
+          if (!SMALL) ptx::tma_prefetch_l2_4d(&tmap_a, 0, ti.m_blk * kBlockM, kb, 0);
         }
       }
     }
@@ -470,11 +475,11 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
   // at stage0 to D, or (split-K) FP32 into the parked partial.
   constexpr int NCH_ALL = BLOCK_N / Shape::kEpiCols;
   const CUtensorMap* dmap = &tmap_d;
-  auto drain_acc = [&](const Tile& ti, int a, int h, int q, int c_begin, int c_end,
-                       uint8_t* stage0, bool report) {
+  auto drain_acc = [&](const Tile& ti, int a, int q, int c_begin, int c_end, uint8_t* stage0,
+                       bool report) {
     // which output row this thread owns, and whether it may be written
     const int row_local = 32 * q + lane;  // accumulator row = TMEM lane
-    const int m_in_group = ti.m_blk * TILE_M + kBlockM * h + row_local;
+    const int m_in_group = ti.m_blk * kBlockM + row_local;
     bool valid;
     size_t grow;
     if (KIND == kMasked) {
@@ -491,7 +496,7 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
       }
     }
     const uint32_t t_row =
-        tmem_base + (static_cast<uint32_t>(32 * q) << 16) + (a * HALVES + h) * BLOCK_N;
+        tmem_base + (static_cast<uint32_t>(32 * q) << 16) + a * BLOCK_N;
     const int n0 = ti.n_blk * BLOCK_N;
 
     // A warp whose 32 rows are all outside the output (a short dense A, a
@@ -598,7 +603,7 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
       const Tile ti = get_tile<KIND>(t, p, s_prefix, lane);
       if (ti.skip) continue;
-      const int a_row = ti.m_blk * TILE_M;
+      const int a_row = ti.m_blk * kBlockM;
       const int a_grp = (KIND == kMasked) ? ti.group : 0;
       for (int kb = ti.kb_begin; kb < ti.kb_end; kb += KPS, ++it) {
         const int s = it % STAGES;
@@ -645,19 +650,16 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
     constexpr uint32_t idesc = BF16 ? ptx::idesc_bf16_f32(kBlockM, BLOCK_N)
                                     : ptx::idesc_mxf8_e4m3_ue8m0(kBlockM, BLOCK_N, A_MN, B_MN);
     // Scale words of one group, from its shared-memory slot into the TMEM
-    // columns of the same slot: SFA words of each 128-row half, then SFB
-    // words of each 128-row chunk of the tile's B rows.
+    // columns of the same slot: the SFA words of the tile's 128 rows, then
+    // the SFB words of each 128-row chunk of the tile's B rows.
     auto copy_sf = [&](int slot) {
       const uint32_t sfa_tmem = tmem_base + ACC_COLS + slot * SF_COLS;
-      const uint32_t sfb_tmem = sfa_tmem + 4 * HALVES;
+      const uint32_t sfb_tmem = sfa_tmem + 4;
       const uint32_t sf_smem = ptx::smem_addr(sSF + slot * SF_BYTES);
-#pragma unroll
-      for (int h = 0; h < HALVES; ++h)
-        ptx::tc_cp_32x128b_warpx4(sfa_tmem + 4 * h, ptx::sdesc_sf_32x16(sf_smem + 512 * h));
+      ptx::tc_cp_32x128b_warpx4(sfa_tmem, ptx::sdesc_sf_32x16(sf_smem));
 #pragma unroll
       for (int h = 0; h < SFB_CHUNKS; ++h)
-        ptx::tc_cp_32x128b_warpx4(sfb_tmem + 4 * h,
-                                  ptx::sdesc_sf_32x16(sf_smem + 512 * (HALVES + h)));
+        ptx::tc_cp_32x128b_warpx4(sfb_tmem + 4 * h, ptx::sdesc_sf_32x16(sf_smem + 512 * (1 + h)));
     };
     int it = 0, acc_it = 0;
     // scale-word groups walked, and the slot of the current group's words:
@@ -676,7 +678,7 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
       if (!ok) break;
       ptx::tc_fence_after_sync();
-      const uint32_t d_tmem = tmem_base + a * HALVES * BLOCK_N;
+      const uint32_t d_tmem = tmem_base + a * BLOCK_N;
       for (int kb = ti.kb_begin; kb < ti.kb_end; kb += KPS, ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
@@ -698,20 +700,16 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
           for (int j = 0; j < KPS; ++j) {
             if (kb + j >= ti.kb_end) break;
             const uint64_t db = ptx::sdesc_kmajor_sw128(b_base + j * BLOCK_N * kBlockK);
+            const uint64_t da = ptx::sdesc_kmajor_sw128(a_base + j * p.a_box_rows * kBlockK);
 #pragma unroll
-            for (int h = 0; h < HALVES; ++h) {
-              const uint64_t da = ptx::sdesc_kmajor_sw128(a_base + j * p.a_box_rows * kBlockK +
-                                                          h * kBlockM * kBlockK);
-#pragma unroll
-              for (int ks = 0; ks < kBlockK / 32; ++ks)
-                ptx::tc_mma_bf16(d_tmem + h * BLOCK_N, da + (32 >> 4) * ks, db + (32 >> 4) * ks,
-                                 idesc, kb + j > ti.kb_begin || ks > 0);
-            }
+            for (int ks = 0; ks < kBlockK / 32; ++ks)
+              ptx::tc_mma_bf16(d_tmem, da + (32 >> 4) * ks, db + (32 >> 4) * ks, idesc,
+                               kb + j > ti.kb_begin || ks > 0);
           }
           ptx::tc_commit(&empty[s]);
         } else if (!BF16 && lane == 0) {
           const uint32_t sfa_tmem = tmem_base + ACC_COLS + sf_slot * SF_COLS;
-          const uint32_t sfb_tmem = sfa_tmem + 4 * HALVES;
+          const uint32_t sfb_tmem = sfa_tmem + 4;
           if (group_first) copy_sf(sf_slot);
           const uint32_t a_base = ptx::smem_addr(sA + s * A_BYTES);
           const uint32_t b_base = ptx::smem_addr(sB + s * B_BYTES);
@@ -731,20 +729,13 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
                      : ptx::sdesc_kmajor_sw128(b_base + j * BLOCK_N * kBlockK);
             const uint32_t id = idesc | (sb << 29) | (sb << 4);
             const uint32_t byte_sel = sb << 30;
+            const uint64_t da = A_MN ? ptx::sdesc_mnmajor_sw128(a_base, 128 * kBlockK)
+                                     : ptx::sdesc_kmajor_sw128(a_base + j * p.a_box_rows * kBlockK);
 #pragma unroll
-            for (int h = 0; h < HALVES; ++h) {
-              // half h: A rows 128h.. of the stage's tile, its own accumulator
-              const uint64_t da =
-                  A_MN ? ptx::sdesc_mnmajor_sw128(a_base, 128 * kBlockK)
-                       : ptx::sdesc_kmajor_sw128(a_base + j * p.a_box_rows * kBlockK +
-                                                 h * kBlockM * kBlockK);
-#pragma unroll
-              for (int ks = 0; ks < kBlockK / 32; ++ks)
-                ptx::tc_mma_mxf8_block_scale(d_tmem + h * BLOCK_N, da + kStepA * ks,
-                                             db + kStepB * ks, id,
-                                             (sfa_tmem + 4 * h) | byte_sel, sfb_tmem | byte_sel,
-                                             kb + j > ti.kb_begin || ks > 0);
-            }
+            for (int ks = 0; ks < kBlockK / 32; ++ks)
+              ptx::tc_mma_mxf8_block_scale(d_tmem, da + kStepA * ks, db + kStepB * ks, id,
+                                           sfa_tmem | byte_sel, sfb_tmem | byte_sel,
+                                           kb + j > ti.kb_begin || ks > 0);
           }
           ptx::tc_commit(&empty[s]);
         }
@@ -769,29 +760,26 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
       // Scale words pack the stage's K blocks: byte j belongs to K block j.
       constexpr int PF = (8 + KPS - 1) / KPS;
       const int KB = p.k_blocks;
-      float va[PF][HALVES][4][KPS];
+      float va[PF][4][KPS];
       float vb[PF][SFB_BLOCKS][KPS];
       StageWalker<KIND, KPS> ld, wr;
       ld.start(blockIdx.x, gridDim.x, total, p, s_prefix, lane);
       wr.start(blockIdx.x, gridDim.x, total, p, s_prefix, lane);
       if constexpr (kLateWait) ptx::grid_dependency_wait();
 
-      auto issue = [&](float (&a)[HALVES][4][KPS], float (&b)[SFB_BLOCKS][KPS]) {
+      auto issue = [&](float (&a)[4][KPS], float (&b)[SFB_BLOCKS][KPS]) {
         const Tile& ti = ld.w.ti;
+        const int m0 = ti.m_blk * kBlockM;  // first row of the tile
+        const int row_base = (KIND == kMasked ? ti.group * p.rows : 0) + m0;
+        const int rows_left = p.rows - m0;  // rows of the tile that exist
   #pragma unroll
-        for (int h = 0; h < HALVES; ++h) {
-          const int m0 = ti.m_blk * TILE_M + kBlockM * h;  // first row of this half
-          const int row_base = (KIND == kMasked ? ti.group * p.rows : 0) + m0;
-          const int rows_left = p.rows - m0;  // rows of this half that exist
+        for (int c = 0; c < 4; ++c) {
+          const int r = 32 * c + lane;
   #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const int r = 32 * c + lane;
-  #pragma unroll
-            for (int j = 0; j < KPS; ++j)
-              a[h][c][j] = (r < rows_left && ld.kb + j < ti.kb_end)
-                               ? __ldg(p.sfa + (size_t)(row_base + r) * KB + ld.kb + j)
-                               : 1.0f;
-          }
+          for (int j = 0; j < KPS; ++j)
+            a[c][j] = (r < rows_left && ld.kb + j < ti.kb_end)
+                          ? __ldg(p.sfa + (size_t)(row_base + r) * KB + ld.kb + j)
+                          : 1.0f;
         }
         // B scale blocks are 128 rows: the tile's rows touch blocks b0, b0 + 1, ...
         const float* sfb_g = p.sfb + (size_t)ti.group * p.nb128 * KB;
@@ -822,19 +810,21 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
           ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
           if (!ok) break;
           uint8_t* sf = sSF + s * SF_BYTES;
-          // A scales: TMEM lane l, column c holds row 32c + l of the half.
-  #pragma unroll
-          for (int h = 0; h < HALVES; ++h) {
+          bool bad = false;  // a scale breaks the contract (checked on request)
+          // A scales: TMEM lane l, column c holds row 32c + l of the tile.
+          {
             uint32_t w[4];
   #pragma unroll
             for (int c = 0; c < 4; ++c) {
               uint32_t x = 0x7F7F7F7Fu;  // unused bytes: scale 1
   #pragma unroll
-              for (int j = 0; j < KPS; ++j)
-                x = (x & ~(0xFFu << (8 * j))) | (ue8m0(va[slot][h][c][j]) << (8 * j));
+              for (int j = 0; j < KPS; ++j) {
+                x = (x & ~(0xFFu << (8 * j))) | (ue8m0(va[slot][c][j]) << (8 * j));
+                if (p.check_scales) bad |= !scale_ok(va[slot][c][j]);
+              }
               w[c] = x;
             }
-            *reinterpret_cast<uint4*>(sf + 512 * h + 16 * lane) = make_uint4(w[0], w[1], w[2], w[3]);
+            *reinterpret_cast<uint4*>(sf + 16 * lane) = make_uint4(w[0], w[1], w[2], w[3]);
           }
           // B scales, same layout per 128-row chunk of the tile's B rows: row
           // r of the tile takes the scale of its own 128-row block of B
@@ -853,12 +843,15 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
                 for (int i = 1; i < SFB_BLOCKS; ++i)
                   if (idx == i) v = vb[slot][i][j];
                 x = (x & ~(0xFFu << (8 * j))) | (ue8m0(v) << (8 * j));
+                if (p.check_scales) bad |= !scale_ok(v);
               }
               w[c] = x;
             }
-            *reinterpret_cast<uint4*>(sf + 512 * (HALVES + h) + 16 * lane) =
+            *reinterpret_cast<uint4*>(sf + 512 * (1 + h) + 16 * lane) =
                 make_uint4(w[0], w[1], w[2], w[3]);
           }
+          if (p.check_scales && __any_sync(0xFFFFFFFFu, bad) && lane == 0)
+            atomicCAS(p.error_word, 0, kDevBadScale);
           ptx::fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) ptx::mbar_arrive(&full[s]);
@@ -879,7 +872,7 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
       // two groups ahead (a float4 per row when the rows allow it).
       constexpr int GK = SF_GROUP * KPS;  // K blocks of a full group (4)
       const int KB = p.k_blocks;
-      float va[2][HALVES][4][GK];
+      float va[2][4][GK];
       float vb[2][SFB_BLOCKS][GK];
       StageWalker<KIND, GK> ld;    // walks the groups
       StageWalker<KIND, KPS> wr;   // walks the stages
@@ -891,27 +884,24 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
                        (reinterpret_cast<uintptr_t>(p.sfa) & 15) == 0 &&
                        (reinterpret_cast<uintptr_t>(p.sfb) & 15) == 0;
 
-      auto issue = [&](float (&a)[HALVES][4][GK], float (&b)[SFB_BLOCKS][GK]) {
+      auto issue = [&](float (&a)[4][GK], float (&b)[SFB_BLOCKS][GK]) {
         const Tile& ti = ld.w.ti;
         const int kb0 = ld.kb;                       // first K block of the group
         const bool v4 = vec && (kb0 & 3) == 0;       // then kb0 + 4 <= KB as well
+        const int m0 = ti.m_blk * kBlockM;           // first row of the tile
+        const int row_base = (KIND == kMasked ? ti.group * p.rows : 0) + m0;
+        const int rows_left = p.rows - m0;           // rows of the tile that exist
   #pragma unroll
-        for (int h = 0; h < HALVES; ++h) {
-          const int m0 = ti.m_blk * TILE_M + kBlockM * h;  // first row of this half
-          const int row_base = (KIND == kMasked ? ti.group * p.rows : 0) + m0;
-          const int rows_left = p.rows - m0;  // rows of this half that exist
+        for (int c = 0; c < 4; ++c) {
+          const int r = 32 * c + lane;
+          const float* src = p.sfa + (size_t)(row_base + r) * KB + kb0;
+          if (r < rows_left && v4) {
+            const float4 x = __ldg(reinterpret_cast<const float4*>(src));
+            a[c][0] = x.x; a[c][1] = x.y; a[c][2] = x.z; a[c][3] = x.w;
+          } else {
   #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const int r = 32 * c + lane;
-            const float* src = p.sfa + (size_t)(row_base + r) * KB + kb0;
-            if (r < rows_left && v4) {
-              const float4 x = __ldg(reinterpret_cast<const float4*>(src));
-              a[h][c][0] = x.x; a[h][c][1] = x.y; a[h][c][2] = x.z; a[h][c][3] = x.w;
-            } else {
-  #pragma unroll
-              for (int j = 0; j < GK; ++j)
-                a[h][c][j] = (r < rows_left && kb0 + j < ti.kb_end) ? __ldg(src + j) : 1.0f;
-            }
+            for (int j = 0; j < GK; ++j)
+              a[c][j] = (r < rows_left && kb0 + j < ti.kb_end) ? __ldg(src + j) : 1.0f;
           }
         }
         // B scale blocks are 128 rows: the tile's rows touch blocks b0, b0 + 1, ...
@@ -940,7 +930,7 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
       bool ok = true;
       // one stage: take its empty slot, (at a group's first stage) write the
       // group's words, arrive on its full barrier
-      auto stage = [&](bool first, const float (&a)[HALVES][4][GK],
+      auto stage = [&](bool first, const float (&a)[4][GK],
                        const float (&b)[SFB_BLOCKS][GK]) -> bool {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
@@ -951,19 +941,22 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
         if (first) {
           uint8_t* sf = sSF + (gc % STAGES) * SF_BYTES;
           const int n_valid = min(GK, wr.w.ti.kb_end - wr.kb);  // K blocks of this group
-          // A scales: TMEM lane l, column c holds row 32c + l of the half.
-  #pragma unroll
-          for (int h = 0; h < HALVES; ++h) {
+          bool bad = false;  // a scale breaks the contract (checked on request)
+          // A scales: TMEM lane l, column c holds row 32c + l of the tile.
+          {
             uint32_t w[4];
   #pragma unroll
             for (int c = 0; c < 4; ++c) {
               uint32_t x = 0x7F7F7F7Fu;  // unused bytes: scale 1
   #pragma unroll
-              for (int j = 0; j < GK; ++j)
-                if (j < n_valid) x = (x & ~(0xFFu << (8 * j))) | (ue8m0(a[h][c][j]) << (8 * j));
+              for (int j = 0; j < GK; ++j) {
+                if (j >= n_valid) continue;
+                x = (x & ~(0xFFu << (8 * j))) | (ue8m0(a[c][j]) << (8 * j));
+                if (p.check_scales) bad |= !scale_ok(a[c][j]);
+              }
               w[c] = x;
             }
-            *reinterpret_cast<uint4*>(sf + 512 * h + 16 * lane) = make_uint4(w[0], w[1], w[2], w[3]);
+            *reinterpret_cast<uint4*>(sf + 16 * lane) = make_uint4(w[0], w[1], w[2], w[3]);
           }
           // B scales, same layout per 128-row chunk of the tile's B rows: row
           // r of the tile takes the scale of its own 128-row block of B
@@ -981,13 +974,17 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
   #pragma unroll
                 for (int i = 1; i < SFB_BLOCKS; ++i)
                   if (idx == i) v = b[i][j];
-                if (j < n_valid) x = (x & ~(0xFFu << (8 * j))) | (ue8m0(v) << (8 * j));
+                if (j >= n_valid) continue;
+                x = (x & ~(0xFFu << (8 * j))) | (ue8m0(v) << (8 * j));
+                if (p.check_scales) bad |= !scale_ok(v);
               }
               w[c] = x;
             }
-            *reinterpret_cast<uint4*>(sf + 512 * (HALVES + h) + 16 * lane) =
+            *reinterpret_cast<uint4*>(sf + 512 * (1 + h) + 16 * lane) =
                 make_uint4(w[0], w[1], w[2], w[3]);
           }
+          if (p.check_scales && __any_sync(0xFFFFFFFFu, bad) && lane == 0)
+            atomicCAS(p.error_word, 0, kDevBadScale);
           ptx::fence_proxy_async_smem();
           __syncwarp();
           ++gc;
@@ -1045,10 +1042,8 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
 
       const int split_col = helpers ? BLOCK_N / 2 : BLOCK_N;
       // staging: in one_tile mode warp w owns tiles [w * NCH_ALL, (w + 1) * NCH_ALL)
-#pragma unroll
-      for (int h = 0; h < HALVES; ++h)
-        drain_acc(ti, a, h, q, 0, split_col,
-                  sEpi + (one_tile ? warp * NCH_ALL : q) * 32 * Shape::kEpiPitch, true);
+      drain_acc(ti, a, q, 0, split_col,
+                sEpi + (one_tile ? warp * NCH_ALL : q) * 32 * Shape::kEpiPitch, true);
       ptx::tc_fence_before_sync();
       ptx::mbar_arrive(&acc_empty[a]);
       ++acc_it;
@@ -1071,7 +1066,7 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
         ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
         if (ok) {
           ptx::tc_fence_after_sync();
-          drain_acc(ti, 0, 0, warp, BLOCK_N / 2, BLOCK_N,
+          drain_acc(ti, 0, warp, BLOCK_N / 2, BLOCK_N,
                     sEpi + (warp * NCH_ALL + NCH_ALL / 2) * 32 * Shape::kEpiPitch, false);
         }
       }

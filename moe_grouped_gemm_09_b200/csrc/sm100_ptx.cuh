@@ -120,7 +120,6 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
-// 3-D tiled load of one box into shared memory, completing on `bar`.
 // 2-D tiled load of one box into shared memory, completing on `bar`.
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
                                             int c0, int c1) {
@@ -147,21 +146,6 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, u
       "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(smem_addr(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
-      : "memory");
-}
-
-// The same load issued by each CTA of an MMA pair (tcgen05 cta_group::2): the
-// box lands in this CTA's shared memory and completes on `bar_cluster`, an
-// mbarrier of either CTA of the pair (map_shared_rank), so that the pair's
-// leader sees both halves of a stage on one barrier.  Each CTA loads only its
-// own box.
-__device__ __forceinline__ void tma_load_4d_pair(void* dst, const CUtensorMap* map,
-                                                 uint32_t bar_cluster, int c0, int c1, int c2,
-                                                 int c3) {
-  asm volatile(
-      "cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(smem_addr(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
       : "memory");
 }
 
@@ -306,25 +290,6 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
                : "memory");
 }
 
-// Pair forms (tcgen05 cta_group::2): one warp of each CTA of the pair, with the
-// same warp index, performs the allocation (same column count, same slot
-// offset) and, at the end, the release.
-__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                   smem_addr(dst_smem)),
-               "r"(ncols)
-               : "memory");
-}
-
-__device__ __forceinline__ void tmem_relinquish_pair() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
-               : "memory");
-}
-
 __device__ __forceinline__ void tc_fence_before_sync() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
@@ -339,39 +304,6 @@ __device__ __forceinline__ void tc_commit(uint64_t* bar) {
   asm volatile(
       "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
           smem_addr(bar))
-      : "memory");
-}
-
-// Pair form of tc_commit, issued by the pair's leader: arrive on the mbarrier
-// at cluster address `bar_cluster` (this CTA's or the peer's, from
-// map_shared_rank) once all tcgen05 operations issued so far have completed.
-__device__ __forceinline__ void tc_commit_pair(uint32_t bar_cluster) {
-  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   bar_cluster)
-               : "memory");
-}
-
-// Pair form of tc_cp_32x128b_warpx4, issued by the leader: each CTA of the
-// pair copies from its own shared memory (same offset) into its own TMEM.
-__device__ __forceinline__ void tc_cp_pair_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
-               : "memory");
-}
-
-// Pair form of the block-scaled MMA, issued by the leader: M = 256 rows (128 of
-// A in each CTA's shared memory, at the same offset), N columns (N/2 rows of B
-// in each CTA), each CTA accumulating its 128 rows x N in its own TMEM.
-__device__ __forceinline__ void tc_mma_pair_mxf8_block_scale(uint32_t d_tmem, uint64_t a_desc,
-                                                             uint64_t b_desc, uint32_t idesc,
-                                                             uint32_t sfa_tmem, uint32_t sfb_tmem,
-                                                             bool accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
-          d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate ? 1u : 0u), "r"(sfa_tmem),
-      "r"(sfb_tmem)
       : "memory");
 }
 

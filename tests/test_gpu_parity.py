@@ -17,7 +17,7 @@ import torch
 import oracle
 import workloads
 from parity import (check_close, d_bits, dev, oracle_contiguous_rows, oracle_dense_rows,
-                    oracle_masked_rows, sample_rows, sentinel_like)
+                    sample_rows, sentinel_like)
 
 pytestmark = pytest.mark.gpu
 
@@ -107,11 +107,8 @@ def test_dense_scales_not_16_byte_aligned(dg):
 
 # Every general variant, forced, on one ragged shape with a random power-of-two
 # scale per A row and per B block (the picker would choose only some of them
-# for this shape).  "192:1:1:256:0" is the two-half 256-row tile; its 192-wide
-# column tiles straddle the 128-row scale blocks of B.  "256:1:1:128:0:1" is
-# the SM-pair variant (256 x 256 tiles, 2-CTA clusters): the last row tile
-# leaves the second CTA of its pair without a single valid row.
-FORCED_GENERAL = ["256:1", "128:1", "64:1", "32:1", "192:1:1:256:0", "256:1:1:128:0:1"]
+# for this shape).
+FORCED_GENERAL = ["256:1", "128:1", "64:1", "32:1"]
 
 
 @pytest.mark.parametrize("cfg", FORCED_GENERAL)
@@ -125,6 +122,30 @@ def test_dense_forced_variant(dg, cfg, monkeypatch):
     got = run_dense(dg, p)
     ref, _ = oracle.default().gemm_nt(p.a, p.sfa, p.b, p.sfb, want_acc=False)
     check_close(got, ref, f"forced {cfg}")
+
+
+# Every decode variant ("block_n:split_k:kps:a_rows:small"), forced, with and
+# without split-K clusters, on a short A (one 128-row block) with a ragged N
+# and random power-of-two scales per A row and per B block.
+FORCED_DECODE = [
+    (100, "128:1:2:128:0"), (100, "128:4:2:128:0"), (100, "64:2:2:128:0"), (100, "64:8:2:128:0"),
+    (64, "256:2:2:128:0"), (100, "128:1:1:128:1"), (100, "64:4:2:128:1"),
+    (64, "128:1:4:64:0"), (64, "128:4:4:64:0"), (40, "64:8:4:64:0"), (64, "256:2:2:64:0"),
+    (64, "128:8:2:64:1"), (17, "64:2:2:64:1"),
+]
+
+
+@pytest.mark.parametrize("M,cfg", FORCED_DECODE)
+def test_dense_forced_decode_variant(dg, M, cfg, monkeypatch):
+    rng = np.random.default_rng(M + len(cfg))
+    N, K = 400, 1024
+    p = workloads.dense_problem(M, N, K, seed=13)
+    p.sfa = np.ldexp(1.0, rng.integers(-10, 4, p.sfa.shape)).astype(np.float32)
+    p.sfb = np.ldexp(1.0, rng.integers(-10, 4, p.sfb.shape)).astype(np.float32)
+    monkeypatch.setenv("DG_FORCE_CONFIG", cfg)
+    got = run_dense(dg, p)
+    ref, _ = oracle.default().gemm_nt(p.a, p.sfa, p.b, p.sfb, want_acc=False)
+    check_close(got, ref, f"forced decode {cfg}")
 
 
 # The other operand layouts: the same problem handed over with A M-major
@@ -239,23 +260,22 @@ def test_dense_decode_full(dg, M, N, K):
     check_close(got, ref, f"decode {M}x{N}x{K}")
 
 
-@pytest.mark.parametrize("M,N,K", [(4096, 7168, 2048), (4352, 2112, 1024)])
-def test_dense_pair_variant_sampled(dg, M, N, K, monkeypatch):
-    """The SM-pair variant over many tiles per pair (persistent loop, ring
-    phases wrapping), sampled rows covering every tile boundary."""
-    monkeypatch.setenv("DG_FORCE_CONFIG", "256:1:1:128:0:1")
-    p = workloads.dense_problem(M, N, K, seed=3)
-    got = run_dense(dg, p)
-    rows = sample_rows(M, 48, seed=M + K)
-    check_close(got[rows], oracle_dense_rows(p, rows), f"pair {M}x{N}x{K}")
-
-
 @pytest.mark.parametrize("M,N,K", workloads.PREFILL_SHAPES)
 def test_dense_prefill_sampled(dg, M, N, K):
     p = workloads.dense_problem(M, N, K, seed=0)
     got = run_dense(dg, p)
     rows = sample_rows(M, 48, seed=M + N)
     check_close(got[rows], oracle_dense_rows(p, rows), f"prefill {M}x{N}x{K}")
+
+
+def test_dense_prefill_full(dg):
+    """One prefill-shaped GEMM (4096 x 2112 x 7168: 288 output tiles, two
+    waves, a ragged last column tile) compared on every output element."""
+    M, N, K = workloads.PREFILL_SHAPES[0]
+    p = workloads.dense_problem(M, N, K, seed=0)
+    got = run_dense(dg, p)
+    ref, _ = oracle.default().gemm_nt(p.a, p.sfa, p.b, p.sfb, want_acc=False)
+    check_close(got, ref, f"prefill full {M}x{N}x{K}")
 
 
 def test_dense_deterministic(dg):
@@ -305,15 +325,17 @@ def test_contiguous_small(dg):
     check_close(got[~pad], ref[~pad], "contiguous small")
 
 
-def test_contiguous_full_sampled(dg):
+def test_contiguous_full(dg):
+    """The contiguous MoE workload (32 experts, Zipf-skewed token counts),
+    every valid row against the oracle and every padding row untouched."""
     p = workloads.contiguous_problem(**workloads.CONTIGUOUS_MOE, seed=0)
     got = run_contiguous(dg, p)
     assert dg.get_last_device_error() == 0
     pad = p.m_indices < 0
     assert np.all(got[pad] == workloads.SENTINEL_BF16), "padding rows were written"
-    valid = np.nonzero(~pad)[0]
-    rows = valid[sample_rows(len(valid), 64, seed=9)]
-    check_close(got[rows], oracle_contiguous_rows(p, rows), "contiguous full")
+    ref = np.full((p.M_sum, p.N), workloads.SENTINEL_BF16, np.uint16)
+    oracle.default().grouped_contiguous(p.a, p.sfa, p.b, p.sfb, p.m_indices, d=ref)
+    check_close(got[~pad], ref[~pad], "contiguous full")
 
 
 def test_contiguous_mixed_block_reports(dg):
@@ -354,21 +376,17 @@ def test_masked_small(dg):
             check_close(got[g, :v], ref[g, :v], f"masked group {g}")
 
 
-def test_masked_full_sampled(dg):
+def test_masked_full(dg):
+    """The masked MoE workload (32 groups, masked_m uniform in [0, 256]),
+    every valid row against the oracle and every masked row untouched."""
     p = workloads.masked_problem(**workloads.MASKED_MOE, seed=0)
     got = run_masked(dg, p)
     assert dg.get_last_device_error() == 0
-    rng = np.random.default_rng(4)
-    pairs = []
-    for g in range(p.G):
-        v = int(p.masked_m[g])
-        assert np.all(got[g, v:] == workloads.SENTINEL_BF16), f"group {g}: masked rows written"
-        for m in sorted(set([0, v - 1] + rng.integers(0, max(v, 1), 2).tolist())):
-            if 0 <= m < v:
-                pairs.append((g, m))
-    ref = oracle_masked_rows(p, pairs)
-    got_rows = np.stack([got[g, m] for g, m in pairs])
-    check_close(got_rows, ref, "masked full")
+    ref = np.full((p.G, p.max_m, p.N), workloads.SENTINEL_BF16, np.uint16)
+    oracle.default().grouped_masked(p.a, p.sfa, p.b, p.sfb, p.masked_m, d=ref)
+    valid = np.arange(p.max_m)[None, :] < p.masked_m[:, None]
+    assert np.all(got[~valid] == workloads.SENTINEL_BF16), "masked rows were written"
+    check_close(got[valid], ref[valid], "masked full")
 
 
 def test_masked_expected_m_does_not_change_results(dg):
@@ -379,3 +397,35 @@ def test_masked_expected_m_does_not_change_results(dg):
     p.expected_m = 256
     c = run_masked(dg, p)
     assert np.array_equal(a, b) and np.array_equal(a, c)
+
+
+@pytest.mark.parametrize("M,N,K", [(64, 2112, 1024), (300, 400, 1024)])
+def test_scale_contract_check(dg, M, N, K):
+    """With the scale check on, valid scales run clean and match the oracle;
+    one A scale and one B scale with mantissa bits (1.5, 0.75: not powers of
+    two) record device error 0x301.  With the check off the same call records
+    nothing (the contract is the caller's)."""
+    p = workloads.dense_problem(M, N, K, seed=14)
+    a, b = dev(p.a), dev(p.b)
+    ref, _ = oracle.default().gemm_nt(p.a, p.sfa, p.b, p.sfb, want_acc=False)
+    bad_sfa, bad_sfb = p.sfa.copy(), p.sfb.copy()
+    bad_sfa[M // 2, K // 256] = 1.5
+    bad_sfb[-1, 0] = 0.75
+    try:
+        dg.set_check_scales(True)
+        d = sentinel_like((M, N))
+        dg.fp8_gemm_nt(a, dev(p.sfa), b, dev(p.sfb), d)
+        torch.cuda.synchronize()
+        assert dg.get_last_device_error() == 0
+        check_close(d_bits(d), ref, "valid scales, check on")
+        dg.fp8_gemm_nt(a, dev(bad_sfa), b, dev(p.sfb), sentinel_like((M, N)))
+        torch.cuda.synchronize()
+        assert dg.get_last_device_error() == 0x301
+        dg.fp8_gemm_nt(a, dev(p.sfa), b, dev(bad_sfb), sentinel_like((M, N)))
+        torch.cuda.synchronize()
+        assert dg.get_last_device_error() == 0x301
+    finally:
+        dg.set_check_scales(False)
+    dg.fp8_gemm_nt(a, dev(bad_sfa), b, dev(bad_sfb), sentinel_like((M, N)))
+    torch.cuda.synchronize()
+    assert dg.get_last_device_error() == 0
