@@ -60,6 +60,8 @@ def load(lib_path: str = _LIB_PATH):
     lib.oracle_grouped_contiguous.argtypes = [P, P, P, P, P, I64, I64, I64, I64, P, P]
     lib.oracle_grouped_masked.restype = ctypes.c_int
     lib.oracle_grouped_masked.argtypes = [P, P, P, P, P, I64, I64, I64, I64, P, P]
+    lib.oracle_k_grouped_tn.restype = ctypes.c_int
+    lib.oracle_k_grouped_tn.argtypes = [P, P, P, P, P, P, I64, I64, I64, I64, P]
     lib.oracle_bf16_decode.restype = ctypes.c_double
     lib.oracle_bf16_decode.argtypes = [ctypes.c_uint16]
     lib.oracle_bf16_gemm_nt.restype = ctypes.c_int
@@ -168,6 +170,30 @@ class Oracle:
         return d, acc
 
     # -- BF16 operands (no scales) --
+    def k_grouped_tn(self, a, sfa, b, sfb, ks, c=None):
+        """K-grouped GEMM (weight gradient): ``acc[g] = C[g] + A_g^T B_g`` over
+        the K rows of group g.  ``a [K_sum, M]`` and ``b [K_sum, N]`` E4M3 bytes
+        (M-/N-major), ``sfa [M, K_sum/128]``, ``sfb [ceil(N/128), K_sum/128]``,
+        ``ks`` int32 [G] (multiples of 128 summing to K_sum), ``c`` float32
+        [G, M, N] or None.  Returns ``acc`` float64 [G, M, N]."""
+        a = _c(a, np.uint8); b = _c(b, np.uint8)
+        sfa = _c(sfa, np.float32); sfb = _c(sfb, np.float32)
+        ks = _c(ks, np.int32)
+        K_sum, M = a.shape
+        N = b.shape[1]
+        G = ks.shape[0]
+        assert b.shape[0] == K_sum and sfa.shape == (M, K_sum // 128)
+        assert sfb.shape == (-(-N // 128), K_sum // 128)
+        if c is not None:
+            c = _c(c, np.float32)
+            assert c.shape == (G, M, N)
+        acc = np.empty((G, M, N), np.float64)
+        rc = self.lib.oracle_k_grouped_tn(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(ks),
+                                          _ptr(c), G, M, N, K_sum, _ptr(acc))
+        if rc != 0:
+            raise ValueError(f"oracle_k_grouped_tn: bad arguments (rc={rc})")
+        return acc
+
     def bf16_decode(self, bits: int) -> float:
         return float(self.lib.oracle_bf16_decode(int(bits)))
 

@@ -37,6 +37,8 @@
  *    part 4.2, names m_grouped_gemm_fp8_masked; project card, "core
  *    features": grouped GEMM, contiguous and masked layouts).  masked_m is
  *    clamped to [0, max_m].
+ *  - K-grouped layout (the weight gradient of the grouped forms in
+ *    training): see oracle_k_grouped_tn below.
  *
  * BF16 GEMM (same three forms, BF16 operands, no scales): the project card,
  * section "core features", lists BF16 beside FP8 and FP4 in its unified
@@ -224,6 +226,70 @@ int oracle_grouped_masked(const uint8_t *a, const float *sfa, const uint8_t *b,
                      acc ? acc + r * N : NULL, d ? d + r * N : NULL);
         }
     }
+    return 0;
+}
+
+/* ---- K-grouped form (MoE weight gradient) -------------------------------- */
+
+/* The training backward pass of an M-grouped GEMM (project card, section
+ * "core features": the unified GEMM family serves training forward and
+ * backward, with NT / TN / NN / TT layouts on SM100) needs, per expert g,
+ * the gradient of its weights: a GEMM whose reduction runs over that
+ * expert's tokens only.  The tokens of all experts are concatenated along
+ * the reduction axis ("K grouped"):
+ *
+ *   acc[g, m, n] = C[g, m, n] + sum_{k in K_g} A_hat[k, m] * B_hat[k, n],
+ *   K_g = [k_off[g], k_off[g] + ks[g]),  k_off[g] = ks[0] + ... + ks[g-1],
+ *
+ * with A stored [K_sum, M] (M-major: one row per token) and B [K_sum, N]
+ * (N-major), A_hat[k, m] = dec(a[k, m]) * sfa[m, k/128] (one scale per output
+ * row per 128 tokens) and B_hat[k, n] = dec(b[k, n]) * sfb[n/128, k/128]
+ * (128 x 128 blocks): the scale conventions of the dense call, with k the
+ * global token index.  Every ks[g] is a multiple of 128 (each expert's
+ * segment is padded as in the contiguous forward), so no scale block spans
+ * two experts.  The sum runs k ascending in double; C may be NULL (zero).
+ * Returns 0, -1 on bad sizes, -2 if the ks do not tile [0, K_sum) in
+ * multiples of 128. */
+int oracle_k_grouped_tn(const uint8_t *a, const float *sfa, const uint8_t *b, const float *sfb,
+                        const int32_t *ks, const float *c, int64_t G, int64_t M, int64_t N,
+                        int64_t K_sum, double *acc)
+{
+    if (K_sum % ORACLE_BLOCK_K != 0 || G < 0 || M < 0 || N < 0)
+        return -1;
+    int64_t total = 0;
+    for (int64_t g = 0; g < G; ++g) {
+        if (ks[g] < 0 || ks[g] % ORACLE_BLOCK_K != 0)
+            return -2;
+        total += ks[g];
+    }
+    if (total != K_sum)
+        return -2;
+    double tab[256];
+    oracle_e4m3_table(tab);
+    int64_t KB = K_sum / ORACLE_BLOCK_K;
+    int64_t *k_off = (int64_t *)malloc(sizeof(int64_t) * (size_t)(G + 1));
+    if (!k_off)
+        return -1;
+    k_off[0] = 0;
+    for (int64_t g = 0; g < G; ++g)
+        k_off[g + 1] = k_off[g] + ks[g];
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (int64_t g = 0; g < G; ++g) {
+        for (int64_t m = 0; m < M; ++m) {
+            for (int64_t n = 0; n < N; ++n) {
+                double s = 0.0;
+                for (int64_t k = k_off[g]; k < k_off[g + 1]; ++k) {
+                    double ah = tab[a[k * M + m]] * (double)sfa[m * KB + k / ORACLE_BLOCK_K];
+                    double bh = tab[b[k * N + n]] *
+                                (double)sfb[(n / ORACLE_BLOCK_N) * KB + k / ORACLE_BLOCK_K];
+                    s += ah * bh;
+                }
+                int64_t o = (g * M + m) * N + n;
+                acc[o] = (c ? (double)c[o] : 0.0) + s;
+            }
+        }
+    }
+    free(k_off);
     return 0;
 }
 

@@ -16,6 +16,9 @@ What each pin compares against:
 * the BF16 operand GEMM: every one of the 65536 operand patterns against the
   FP32 widening and ml_dtypes; numpy float64 matmul; Python-float loops (bit
   for bit); exact integer results; an empty K; the grouped forms row by row;
+* the K-grouped (weight-gradient) form: numpy float64 per group plus C, the
+  dense oracle on each group's slice (bit for bit) and over all of K (the sum
+  over groups), exact integer results, an empty group leaving C;
 * the GEMM: a hand-worked tiny example (golden file); brute force with numpy's
   float64 matmul on ml_dtypes-decoded operands; exact integer results; one-hot
   selection; power-of-two scale invariance; and for the grouped forms, the same
@@ -446,6 +449,81 @@ def pin_bf16_grouped(o, seed=20):
                 assert np.all(d[g, m] == SENTINEL), (g, m)
 
 
+# ------------------------------------------------- K-grouped (weight grad) --
+
+def _k_grouped_case(rng, ks, M, N, with_c=True):
+    K_sum = int(np.sum(ks))
+    a = random_e4m3(rng, (K_sum, M))           # [K_sum, M], M-major
+    b = random_e4m3(rng, (K_sum, N))           # [K_sum, N], N-major
+    sfa = random_pow2_scales(rng, (M, K_sum // 128))
+    sfb = random_pow2_scales(rng, (-(-N // 128), K_sum // 128))
+    c = rng.standard_normal((len(ks), M, N)).astype(np.float32) * 64 if with_c else None
+    return a, sfa, b, sfb, np.asarray(ks, np.int32), c
+
+
+def pin_k_grouped_brute_force(o, seed=21):
+    """Per group, numpy float64 on ml_dtypes-decoded operands over the group's
+    rows of K only, plus C; an empty group leaves exactly C."""
+    rng = np.random.default_rng(seed)
+    ks = [256, 0, 128, 384]
+    M, N = 24, 136
+    a, sfa, b, sfb, ks, c = _k_grouped_case(rng, ks, M, N)
+    acc = o.k_grouped_tn(a, sfa, b, sfb, ks, c)
+    k0 = 0
+    for g, kg in enumerate(ks):
+        kb = slice(k0 // 128, (k0 + kg) // 128)
+        ah = decode_ml(a[k0:k0 + kg]).T * np.repeat(sfa[:, kb].astype(np.float64), 128, axis=1)
+        sfb_rows = np.repeat(sfb[:, kb].astype(np.float64), 128, axis=0)[:N]
+        bh = decode_ml(b[k0:k0 + kg]).T * np.repeat(sfb_rows, 128, axis=1)
+        ref = c[g].astype(np.float64) + ah @ bh.T
+        tol = 1e-12 * (np.abs(c[g]).astype(np.float64) + np.abs(ah) @ np.abs(bh).T) + 1e-300
+        assert np.all(np.abs(acc[g] - ref) <= tol), g
+        if kg == 0:
+            assert np.array_equal(acc[g], c[g].astype(np.float64)), g
+        k0 += kg
+
+
+def pin_k_grouped_is_per_group_dense(o, seed=22):
+    """Without C, group g's result is bit for bit the dense NT oracle run on
+    that group's rows of K (transposed to K-major) with that group's scale
+    columns; and the sum over groups equals the dense GEMM over all of K."""
+    rng = np.random.default_rng(seed)
+    ks = [128, 512, 0, 256]
+    M, N = 40, 264
+    a, sfa, b, sfb, ks, _ = _k_grouped_case(rng, ks, M, N, with_c=False)
+    acc = o.k_grouped_tn(a, sfa, b, sfb, ks, None)
+    k0 = 0
+    for g, kg in enumerate(ks):
+        if kg == 0:
+            assert np.all(acc[g] == 0.0), g
+            continue
+        kb = slice(k0 // 128, (k0 + kg) // 128)
+        _, dense = o.gemm_nt(np.ascontiguousarray(a[k0:k0 + kg].T), sfa[:, kb],
+                             np.ascontiguousarray(b[k0:k0 + kg].T), sfb[:, kb])
+        assert np.array_equal(acc[g], dense), g
+        k0 += kg
+    _, full = o.gemm_nt(np.ascontiguousarray(a.T), sfa, np.ascontiguousarray(b.T), sfb)
+    total = acc.sum(axis=0)
+    assert np.allclose(total, full, rtol=1e-12, atol=1e-9 * np.abs(full).max())
+
+
+def pin_k_grouped_integer_exact(o, seed=23):
+    """Values in {-1, 0, 1}, unit scales: every group's result is the integer
+    product of its slices exactly."""
+    rng = np.random.default_rng(seed)
+    ks = np.array([128, 256, 0, 128], np.int32)
+    M, N = 16, 48
+    K_sum = int(ks.sum())
+    enc = np.array([0xB8, 0x00, 0x38], np.uint8)
+    ia, ib = rng.integers(-1, 2, (K_sum, M)), rng.integers(-1, 2, (K_sum, N))
+    acc = o.k_grouped_tn(enc[ia + 1], np.ones((M, K_sum // 128), np.float32), enc[ib + 1],
+                         np.ones((1, K_sum // 128), np.float32), ks, None)
+    k0 = 0
+    for g, kg in enumerate(ks):
+        assert np.array_equal(acc[g], (ia[k0:k0 + kg].T @ ib[k0:k0 + kg]).astype(np.float64)), g
+        k0 += kg
+
+
 ALL_PINS = [
     pin_e4m3_golden, pin_e4m3_structure, pin_e4m3_libraries,
     pin_bf16_golden, pin_bf16_vs_torch_on_fp32_values, pin_bf16_vs_candidates_on_wide_values,
@@ -453,6 +531,7 @@ ALL_PINS = [
     pin_dense_scale_invariance, pin_contiguous, pin_masked,
     pin_bf16_operand_table, pin_bf16_gemm_brute_force, pin_bf16_gemm_python_loops,
     pin_bf16_gemm_integer_exact, pin_bf16_gemm_empty_k, pin_bf16_grouped,
+    pin_k_grouped_brute_force, pin_k_grouped_is_per_group_dense, pin_k_grouped_integer_exact,
 ]
 
 

@@ -52,6 +52,13 @@ MUTANTS = [
     ("bf16_gemm_a_row_for_b", "s += tab[a_row[k]] * tab[b_row[k]];", "s += tab[a_row[k]] * tab[a_row[k]];"),
     ("bf16_contiguous_wrong_group", "bf16_gemm_row(tab, a + r * K, b + e * N * K,", "bf16_gemm_row(tab, a + r * K, b,"),
     ("bf16_masked_wrong_group", "bf16_gemm_row(tab, a + r * K, b + g * N * K,", "bf16_gemm_row(tab, a + r * K, b,"),
+    ("kgrouped_local_scale_block", "sfa[m * KB + k / ORACLE_BLOCK_K]", "sfa[m * KB + (k - k_off[g]) / ORACLE_BLOCK_K]"),
+    ("kgrouped_group_shifted", "for (int64_t k = k_off[g]; k < k_off[g + 1]; ++k)",
+     "for (int64_t k = k_off[g] / 2; k < k_off[g + 1]; ++k)"),
+    ("kgrouped_addend_dropped", "acc[o] = (c ? (double)c[o] : 0.0) + s;", "acc[o] = s;"),
+    ("kgrouped_sfb_one_n_block", "(double)sfb[(n / ORACLE_BLOCK_N) * KB + k / ORACLE_BLOCK_K]",
+     "(double)sfb[k / ORACLE_BLOCK_K]"),
+    ("kgrouped_b_row_of_a", "tab[b[k * N + n]]", "tab[b[k * N + (n % M)]]"),
 ]
 
 _CHILD = r"""
