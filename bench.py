@@ -76,6 +76,8 @@ def build_workload(name: str, seed: int = 0):
         return [("contiguous", workloads.contiguous_problem(**workloads.CONTIGUOUS_MOE, seed=seed))]
     if name == "masked":
         return [("masked", workloads.masked_problem(**workloads.MASKED_MOE, seed=seed))]
+    if name == "k-grouped":
+        return [("k_grouped", workloads.k_grouped_problem(**workloads.K_GROUPED_MOE, seed=seed))]
     if name == "bf16-decode":
         return [("bf16_dense", workloads.bf16_dense_problem(m, n, k, seed=seed + i))
                 for i, (m, n, k) in enumerate(workloads.DECODE_SHAPES)]
@@ -327,6 +329,8 @@ def _launcher(dg, items, sets, outs):
         elif kind == "contiguous":
             dg.m_grouped_fp8_gemm_nt_contiguous(t["a"], t["sfa"], t["b"], t["sfb"],
                                                 t["m_indices"], d)
+        elif kind == "k_grouped":
+            dg.k_grouped_fp8_gemm_tn_contiguous(t["a"], t["sfa"], t["b"], t["sfb"], t["ks"], d=d)
         else:
             dg.m_grouped_fp8_gemm_nt_masked(t["a"], t["sfa"], t["b"], t["sfb"],
                                             t["masked_m"], p.expected_m, d)
@@ -348,7 +352,7 @@ def time_workload(ctx: GpuContext, name: str, args, steps: int, per_gemm: bool, 
     set_bytes = sum(p.a.nbytes + p.b.nbytes + getattr(p, "sfa", p.a[:0]).nbytes
                     + getattr(p, "sfb", p.a[:0]).nbytes for _, p in items)
     R = max(2, math.ceil(3 * L2_BYTES / max(set_bytes, 1)))
-    if name in ("prefill", "contiguous", "masked", "bf16-prefill"):
+    if name in ("prefill", "contiguous", "masked", "k-grouped", "bf16-prefill"):
         R = max(2, min(R, 4))
     if rotations > 0:
         R = rotations
@@ -364,6 +368,8 @@ def time_workload(ctx: GpuContext, name: str, args, steps: int, per_gemm: bool, 
                 t["m_indices"] = _host_tensor(p.m_indices).to(dev)
             if kind == "masked":
                 t["masked_m"] = _host_tensor(p.masked_m).to(dev)
+            if kind == "k_grouped":
+                t["ks"] = _host_tensor(p.ks).to(dev)
             one.append(t)
         sets.append(one)
     outs = []
@@ -372,6 +378,8 @@ def time_workload(ctx: GpuContext, name: str, args, steps: int, per_gemm: bool, 
             outs.append(torch.empty((p.M, p.N), dtype=torch.bfloat16, device=dev))
         elif kind == "contiguous":
             outs.append(torch.empty((p.M_sum, p.N), dtype=torch.bfloat16, device=dev))
+        elif kind == "k_grouped":
+            outs.append(torch.empty((p.G, p.M, p.N), dtype=torch.float32, device=dev))
         else:
             outs.append(torch.empty((p.G, p.max_m, p.N), dtype=torch.bfloat16, device=dev))
     launch_one = _launcher(dg, items, sets, outs)
@@ -453,6 +461,8 @@ def time_workload(ctx: GpuContext, name: str, args, steps: int, per_gemm: bool, 
                 t["m_indices"] = torch.from_numpy(p.m_indices).pin_memory()
             if kind == "masked":
                 t["masked_m"] = torch.from_numpy(p.masked_m).pin_memory()
+            if kind == "k_grouped":
+                t["ks"] = torch.from_numpy(p.ks).pin_memory()
             pinned.append(t)
         host_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
         h2d = sum(v.numel() * v.element_size() for t in pinned for v in t.values())
@@ -542,7 +552,7 @@ def workload_record(name: str, t: dict, world: int, steps: int, warmup: int) -> 
     }
 
 
-EXTRA_WORKLOADS = ("smoke", "prefill", "contiguous", "masked")
+EXTRA_WORKLOADS = ("smoke", "prefill", "contiguous", "masked", "k-grouped")
 
 
 def run_gpu(args):
@@ -655,6 +665,9 @@ def _shape(p):
         return {"M": p.M, "N": p.N, "K": p.K}
     if isinstance(p, workloads.ContiguousProblem):
         return {"M_sum": p.M_sum, "N": p.N, "K": p.K, "G": p.G, "valid_rows": p.valid_rows()}
+    if isinstance(p, workloads.KGroupedProblem):
+        return {"G": p.G, "M": p.M, "N": p.N, "K_sum": p.K_sum, "valid_tokens": p.valid_rows(),
+                "out": "fp32"}
     return {"G": p.G, "max_m": p.max_m, "N": p.N, "K": p.K, "valid_rows": p.valid_rows(),
             "expected_m": p.expected_m}
 
@@ -665,7 +678,7 @@ def _row_units(items, unit):
     """Total rows per GEMM, for scaling a row sample up to the full step."""
     out = []
     for kind, p in items:
-        if kind in ("dense", "bf16_dense"):
+        if kind in ("dense", "bf16_dense", "k_grouped"):
             out.append(p.M)
         else:
             out.append(p.valid_rows())
@@ -680,6 +693,9 @@ def _oracle_rows(o, kind, p, rows: np.ndarray):
     elif kind == "contiguous":
         valid = np.nonzero(p.m_indices >= 0)[0][rows]
         o.grouped_contiguous(p.a[valid], p.sfa[valid], p.b, p.sfb, p.m_indices[valid])
+    elif kind == "k_grouped":
+        # output rows m of every group: the columns m of A and their scales
+        o.k_grouped_tn(p.a[:, rows], p.sfa[rows], p.b, p.sfb, p.ks)
     else:
         pairs = [(g, m) for g in range(p.G) for m in range(min(max(int(p.masked_m[g]), 0), p.max_m))]
         sel = sorted(pairs[i] for i in rows)
@@ -813,8 +829,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="decode",
-                    choices=("decode", "smoke", "prefill", "contiguous", "masked", "bf16-decode",
-                             "bf16-prefill"))
+                    choices=("decode", "smoke", "prefill", "contiguous", "masked", "k-grouped",
+                             "bf16-decode", "bf16-prefill"))
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--per-gemm-reps", type=int, default=20,

@@ -54,7 +54,8 @@
  *    stream is synchronised: 0x101..0x104 a wait that ran out of time (TMA
  *    producer, scale producer, MMA issuer, epilogue; the kernel then stops
  *    early and D is partly written), 0x201 an m_indices block naming two
- *    experts, 0x202 an expert index >= G, 0x301 a scale that is not a
+ *    experts, 0x202 an expert index >= G, 0x203 K-grouped group sizes that
+ *    do not tile K in multiples of 128, 0x301 a scale that is not a
  *    positive normal power of two (only when the check is on).
  *  - Results are deterministic: the same inputs give bit-identical outputs
  *    on every run (no floating-point atomics; split-K partial sums are added
@@ -141,6 +142,35 @@ dg_status dg_m_grouped_fp8_gemm_nt_masked(const void* a, const float* sfa, const
                                           int max_m, int N, int K, int expected_m,
                                           dg_stream_t stream);
 
+/* K-grouped GEMM, contiguous layout: the weight gradient of the M-grouped
+ * forms in training (DeepGEMM project card, aiproducthub.cn, "core
+ * features": the unified GEMM family serves training forward and backward,
+ * with NT / TN / NN / TT layouts on SM100).  The tokens of all G groups
+ * (experts) are concatenated along the reduction axis K; group g owns the K
+ * rows [k_off[g], k_off[g] + ks[g]) with k_off[g] = ks[0] + ... + ks[g-1]:
+ *   D[g][M,N] = C[g] + sum over the K rows k of group g of A_hat[k,:]^T B_hat[k,:]
+ * a    E4M3 bytes [K_sum, M], M contiguous (M-major: one row per token);
+ * b    E4M3 bytes [K_sum, N], N contiguous (N-major);
+ * sfa  float32 [M, K_sum/128]: scale of output row m for the K block kb
+ *      (the global block index: k / 128);
+ * sfb  float32 [ceil(N/128), K_sum/128]: scale of the 128 x 128 block
+ *      (n/128, kb) of B;
+ * c, d float32 [G, M, N]; c may be NULL (D = the products) or equal d
+ *      (accumulate in place, as a training step does);
+ * ks   int32 [G] on the device: every ks[g] >= 0, a multiple of 128 (each
+ *      group's token segment padded to 128 rows, so no scale block spans two
+ *      groups), summing to K_sum.  A group with ks[g] == 0 gets D[g] = C[g]
+ *      (zeros without C).  Sizes that break these rules are found on the
+ *      device: nothing is written and device error 0x203 is recorded.
+ * M % 16 == 0 (M-major rows of whole 16-byte units), N % 16 == 0,
+ * K_sum > 0 and K_sum % 128 == 0, G <= 1024, a, b, c, d 16-byte aligned;
+ * otherwise DG_ERR_INVALID_ARG (DG_ERR_UNSUPPORTED for G > 1024).  The scale
+ * contract and everything else are those of the dense calls. */
+dg_status dg_k_grouped_fp8_gemm_tn_contiguous(const void* a, const float* sfa, const void* b,
+                                              const float* sfb, const float* c, float* d,
+                                              const int* ks, int G, int M, int N, int K_sum,
+                                              dg_stream_t stream);
+
 /* The three GEMM forms on BF16 operands (DeepGEMM project card,
  * aiproducthub.cn, "core features": BF16 beside FP8 and FP4 in the unified
  * dense GEMM family; grouped GEMMs in contiguous and masked layouts for MoE).
@@ -189,8 +219,10 @@ dg_status dg_set_wait_timeout_ns(long long ns);
  * every scale a kernel reads must be a positive normal power of two, and one
  * that is not records device error 0x301.  Off by default; the environment
  * variable DG_CHECK_SCALES=1 turns it on at first use.  Applies to launches
- * enqueued after the call, from every thread and entry point; the check
- * costs a few instructions per scale and none when off. */
+ * enqueued after the call, from every thread and entry point.  When on, each
+ * FP8 call first launches a small kernel on the same stream that reads every
+ * scale of sfa and sfb (one extra launch per call); when off, nothing is
+ * added. */
 dg_status dg_set_check_scales(int enable);
 
 /* Human-readable name of a status code.  Never NULL. */
@@ -198,7 +230,8 @@ const char* dg_status_string(dg_status s);
 
 /* Configuration the picker chooses for a problem, without launching anything
  * and without a GPU (num_sms is given explicitly).  kind: 0 dense, 1
- * contiguous, 2 masked; rows: M, M_sum or max_m; expected_m only for masked.
+ * contiguous, 2 masked, 3 K-grouped; rows: M, M_sum or max_m (K-grouped: M,
+ * the output rows of each group; K: K_sum); expected_m only for masked.
  * The picker counts K in 128-byte blocks of a row: for the BF16-operand
  * calls pass 2 * K (their tile geometry is that of the E4M3 call with twice
  * the K, without the scale factors' shared memory and TMEM columns).

@@ -47,6 +47,8 @@ _gemm_tt = _decl("dg_fp8_gemm_tt", [_P, _P, _P, _P, _P, _I, _I, _I, _P])
 _gemm_nt_f32 = _decl("dg_fp8_gemm_nt_f32", [_P, _P, _P, _P, _P, _P, _I, _I, _I, _P])
 _gemm_contig = _decl("dg_m_grouped_fp8_gemm_nt_contiguous", [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P])
 _gemm_masked = _decl("dg_m_grouped_fp8_gemm_nt_masked", [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P])
+_k_grouped = _decl("dg_k_grouped_fp8_gemm_tn_contiguous",
+                   [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P])
 _bf16_gemm_nt = _decl("dg_bf16_gemm_nt", [_P, _P, _P, _I, _I, _I, _P])
 _bf16_gemm_contig = _decl("dg_m_grouped_bf16_gemm_nt_contiguous", [_P, _P, _P, _P, _I, _I, _I, _I, _P])
 _bf16_gemm_masked = _decl("dg_m_grouped_bf16_gemm_nt_masked", [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P])
@@ -77,7 +79,7 @@ EXPORTED_SYMBOLS = ("dg_fp8_gemm_nt", "dg_m_grouped_fp8_gemm_nt_contiguous",
                     "dg_fp8_gemm_tn", "dg_fp8_gemm_tt", "dg_fp8_gemm_nt_f32", "dg_bf16_gemm_nt",
                     "dg_m_grouped_bf16_gemm_nt_contiguous", "dg_m_grouped_bf16_gemm_nt_masked",
                     "dg_set_wait_timeout_ns", "dg_fp8_gemm_nt_noalloc_get_last_device_error",
-                    "dg_set_check_scales")
+                    "dg_set_check_scales", "dg_k_grouped_fp8_gemm_tn_contiguous")
 
 DEVICE_ERRORS = {
     0x101: "wait timeout in the TMA producer",
@@ -86,6 +88,7 @@ DEVICE_ERRORS = {
     0x104: "wait timeout in the epilogue",
     0x201: "a 128-row block of m_indices names two experts",
     0x202: "an m_indices entry is >= the number of groups",
+    0x203: "K-grouped group sizes that do not tile K in multiples of 128",
     0x301: "a scale that is not a positive normal power of two",
 }
 
@@ -283,6 +286,37 @@ def m_grouped_fp8_gemm_nt_masked(a: torch.Tensor, sfa: torch.Tensor, b: torch.Te
     return d
 
 
+def k_grouped_fp8_gemm_tn_contiguous(a: torch.Tensor, sfa: torch.Tensor, b: torch.Tensor,
+                                     sfb: torch.Tensor, ks: torch.Tensor,
+                                     c: Optional[torch.Tensor] = None,
+                                     d: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """K-grouped GEMM (MoE weight gradient): ``D[g] = C[g] + A_g^T B_g`` over the
+    K rows of group g.  ``a [K_sum, M]`` and ``b [K_sum, N]`` E4M3 (M-/N-major,
+    one row per token), ``sfa [M, K_sum/128]``, ``sfb [ceil(N/128), K_sum/128]``,
+    ``ks`` int32 [G] on the device (multiples of 128 summing to K_sum), ``c`` and
+    ``d`` float32 [G, M, N] (``c`` optional, may be ``d``)."""
+    _fp8_bytes(a, "a"); _fp8_bytes(b, "b")
+    K_sum, M = a.shape
+    N = b.shape[1]
+    G = ks.shape[0]
+    dev = a.device
+    _need(a, "a", None, (K_sum, M), dev)
+    _need(b, "b", None, (K_sum, N), dev)
+    _need(sfa, "sfa", torch.float32, (M, K_sum // 128), dev)
+    _need(sfb, "sfb", torch.float32, ((N + 127) // 128, K_sum // 128), dev)
+    _need(ks, "ks", torch.int32, (G,), dev)
+    if c is not None:
+        _need(c, "c", torch.float32, (G, M, N), dev)
+    if d is None:
+        d = torch.empty((G, M, N), dtype=torch.float32, device=dev)
+    _need(d, "d", torch.float32, (G, M, N), dev)
+    with torch.cuda.device(dev):
+        _check(_k_grouped(a.data_ptr(), sfa.data_ptr(), b.data_ptr(), sfb.data_ptr(),
+                          None if c is None else c.data_ptr(), d.data_ptr(), ks.data_ptr(), G, M,
+                          N, K_sum, _stream_ptr(dev)), "dg_k_grouped_fp8_gemm_tn_contiguous")
+    return d
+
+
 def _bf16(t: torch.Tensor, name: str) -> torch.Tensor:
     if t.dtype != torch.bfloat16:
         raise TypeError(f"{name}: expected bfloat16, got {t.dtype}")
@@ -397,4 +431,4 @@ def query_config(kind: int, rows: int, N: int, K: int, G: int = 1, expected_m: i
     return {n: getattr(c, n) for n, _ in DgConfig._fields_}
 
 
-KIND_DENSE, KIND_CONTIGUOUS, KIND_MASKED = 0, 1, 2
+KIND_DENSE, KIND_CONTIGUOUS, KIND_MASKED, KIND_K_GROUPED = 0, 1, 2, 3

@@ -7,7 +7,9 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <algorithm>
 #include <mutex>
+#include <utility>
 
 #include "../../include/dg.h"
 #include "dg_internal.h"
@@ -128,7 +130,7 @@ void forced_config(int kind, int rows, int N, int K, int G, int sms, PickedConfi
   if (v < 0 || sk < 1 || sk > kMaxSplitK || sk > KB) return;
   if (sk > 1 && (kind != kDense || rows > kBlockM)) return;
   if ((sk - 1) * ceil_div(KB, sk) >= KB) return;
-  const long long groups = (kind == kMasked) ? G : 1;
+  const long long groups = (kind == kMasked || kind == kKGrouped) ? G : 1;
   const long long tiles = groups * ceil_div(rows, tile_rows(kVariants[v])) * ceil_div(N, bn);
   pc->variant = v;
   pc->split_k = sk;
@@ -202,7 +204,8 @@ dg_status launch_plan(DeviceState& st, const LaunchPlan& pl, cudaStream_t stream
     case kFormNN:
     case kFormTN:
     case kFormTT:
-    case kFormF32: return launch_fp8_layouts(row, pl, stream);
+    case kFormF32:
+    case kFormKGrouped: return launch_fp8_layouts(row, pl, stream);
     case kFormBf16Dense: return launch_bf16_dense(row, pl, stream);
     default: return launch_bf16_grouped(row, pl, stream);
   }
@@ -225,10 +228,41 @@ dg_status run(const GemmCall& call, cudaStream_t stream) {
   LaunchPlan pl;
   s = plan_gemm(call, DeviceFacts{effective_sms(*st), &st->limits}, st->error_word, &pl);
   if (s != DG_OK || pl.grid == 0) return s;
+  if (!is_bf16_form(call.form) && check_scales_enabled()) {
+    s = launch_scale_check(call, st->error_word, stream);
+    if (s != DG_OK) return s;
+  }
   return launch_plan(*st, pl, stream);
 }
 
+// Checks n scales against the contract and records kDevBadScale if one breaks
+// it.  Launched before a GEMM only when the check is turned on; the GEMM
+// kernels themselves use the exponent byte without looking at the rest.
+__global__ void check_scales_kernel(const float* __restrict__ s, long long n, int* error_word) {
+  bool bad = false;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x)
+    bad |= !scale_ok(__ldg(s + i));
+  if (__any_sync(0xFFFFFFFFu, bad) && (threadIdx.x & 31) == 0) atomicCAS(error_word, 0, kDevBadScale);
+}
+
 }  // namespace
+
+dg_status launch_scale_check(const GemmCall& call, int* error_word, cudaStream_t stream) {
+  const int kind = kind_of_form(call.form);
+  const long long kb = call.K / kBlockK;
+  const long long a_rows = kind == kMasked ? static_cast<long long>(call.G) * call.rows : call.rows;
+  // (K-grouped: one sfa [M, K/128] and one sfb for all groups)
+  const long long b_groups = (kind == kDense || kind == kKGrouped) ? 1 : call.G;
+  const long long n_sfa = a_rows * kb;
+  const long long n_sfb = b_groups * ceil_div(call.N, 128) * kb;
+  for (const auto& t : {std::make_pair(call.sfa, n_sfa), std::make_pair(call.sfb, n_sfb)}) {
+    const int blocks = static_cast<int>(std::min<long long>((t.second + 255) / 256, 1024));
+    check_scales_kernel<<<blocks, 256, 0, stream>>>(t.first, t.second, error_word);
+    if (cudaGetLastError() != cudaSuccess) return DG_ERR_CUDA;
+  }
+  return DG_OK;
+}
 
 unsigned long long wait_timeout_ns() {
   std::lock_guard<std::mutex> lock(g_settings_mutex);
@@ -281,10 +315,13 @@ dg_status check_gemm_call(const GemmCall& call, bool* empty) {
       (!call.m_indices || !aligned(call.m_indices, 4) || rows % 128 != 0))
     return DG_ERR_INVALID_ARG;
   if (a_mn && rows % 16 != 0) return DG_ERR_INVALID_ARG;  // [K, M] rows of whole 16-byte units
-  if (form == kFormF32 && call.c && !aligned(call.c, 16)) return DG_ERR_INVALID_ARG;
+  if (is_f32_form(form) && call.c && !aligned(call.c, 16)) return DG_ERR_INVALID_ARG;
   if (kind == kMasked && (!call.masked_m || !aligned(call.masked_m, 4))) return DG_ERR_INVALID_ARG;
-  if (kind == kMasked && G > kMaxMaskedGroups) return DG_ERR_UNSUPPORTED;
-  const long long a_rows = (kind == kMasked) ? static_cast<long long>(G) * rows : rows;
+  if (kind == kKGrouped && (!call.ks || !aligned(call.ks, 4))) return DG_ERR_INVALID_ARG;
+  if ((kind == kMasked || kind == kKGrouped) && G > kMaxMaskedGroups) return DG_ERR_UNSUPPORTED;
+  // rows of D (and of A for the masked form)
+  const long long a_rows =
+      (kind == kMasked || kind == kKGrouped) ? static_cast<long long>(G) * rows : rows;
   if (a_rows > 0x7fffffffLL || static_cast<long long>(G) * N > 0x7fffffffLL)
     return DG_ERR_UNSUPPORTED;
   if (K > (1 << 24)) return DG_ERR_UNSUPPORTED;
@@ -303,16 +340,17 @@ dg_status plan_gemm(const GemmCall& call, const DeviceFacts& facts, int* error_w
   const bool a_mn = (layout & 1) != 0, b_mn = (layout & 2) != 0;
   const bool bf16 = is_bf16_form(form);
   const int rows = call.rows, N = call.N, K = call.K, G = call.G;
-  const long long a_rows = (kind == kMasked) ? static_cast<long long>(G) * rows : rows;
+  const long long a_rows =
+      (kind == kMasked || kind == kKGrouped) ? static_cast<long long>(G) * rows : rows;
   // the picker and the kernel count K in 128-byte blocks of a row
   const int k_bytes = bf16 ? 2 * K : K;
   const int sms = facts.num_sms;
 
   PickedConfig pc = pick_config(kind, rows, N, k_bytes, G, call.expected_m, sms, facts.limits,
-                                /*mn_operands=*/layout != kLayoutNT || form == kFormF32);
+                                /*mn_operands=*/layout != kLayoutNT || is_f32_form(form));
   forced_config(kind, rows, N, k_bytes, G, sms, &pc);
   const Variant var = kVariants[pc.variant];
-  if ((layout != kLayoutNT || form == kFormF32) && (!mn_capable(var) || pc.split_k > 1))
+  if ((layout != kLayoutNT || is_f32_form(form)) && (!mn_capable(var) || pc.split_k > 1))
     return DG_ERR_UNSUPPORTED;
 
   GemmArgs& args = pl->args;
@@ -320,7 +358,7 @@ dg_status plan_gemm(const GemmCall& call, const DeviceFacts& facts, int* error_w
   args.rows = rows;
   args.N = N;
   args.K = K;
-  args.G = (kind == kDense) ? 1 : G;
+  args.G = (kind == kDense) ? 1 : G;  // K-grouped: groups of K, one D each
   args.num_m_blocks = ceil_div(rows, tile_rows(var));
   args.num_n_blocks = ceil_div(N, var.block_n);
   args.k_blocks = k_bytes / kBlockK;
@@ -330,15 +368,15 @@ dg_status plan_gemm(const GemmCall& call, const DeviceFacts& facts, int* error_w
   args.sfa = call.sfa;
   args.sfb = call.sfb;
   args.d = static_cast<__nv_bfloat16*>(call.d);
-  args.d_f32 = form == kFormF32 ? static_cast<float*>(call.d) : nullptr;
-  args.c_f32 = form == kFormF32 ? call.c : nullptr;
+  args.d_f32 = is_f32_form(form) ? static_cast<float*>(call.d) : nullptr;
+  args.c_f32 = is_f32_form(form) ? call.c : nullptr;
+  args.ks = call.ks;
   args.m_indices = call.m_indices;
   args.masked_m = call.masked_m;
   args.error_word = error_word;
   args.timeout_ns = wait_timeout_ns();
   args.a_box_rows = a_mn ? kBlockM : a_box_rows(kind, rows);
   args.prefetch = prefetch_enabled();
-  args.check_scales = bf16 ? 0 : check_scales_enabled();
   if (args.a_box_rows > var.a_rows) return DG_ERR_UNSUPPORTED;
   // a small variant runs one tile per CTA (its epilogue reuses the ring)
   if (var.small && (kind != kDense || pc.grid != args.num_m_blocks * args.num_n_blocks * pc.split_k))
@@ -433,6 +471,14 @@ dg_status dg_m_grouped_fp8_gemm_nt_masked(const void* a, const float* sfa, const
   return run(call, as_stream(stream));
 }
 
+dg_status dg_k_grouped_fp8_gemm_tn_contiguous(const void* a, const float* sfa, const void* b,
+                                              const float* sfb, const float* c, float* d,
+                                              const int* ks, int G, int M, int N, int K_sum,
+                                              dg_stream_t stream) {
+  GemmCall call{kFormKGrouped, a, sfa, b, sfb, d, c, nullptr, nullptr, M, N, K_sum, G, 0, ks};
+  return run(call, as_stream(stream));
+}
+
 dg_status dg_bf16_gemm_nt(const void* a, const void* b, void* d, int M, int N, int K,
                           dg_stream_t stream) {
   return dense_call(kFormBf16Dense, a, nullptr, b, nullptr, d, M, N, K, stream);
@@ -518,10 +564,11 @@ const char* dg_status_string(dg_status s) {
 
 dg_status dg_query_config(int kind, int rows, int N, int K, int G, int expected_m, int num_sms,
                           dg_config* out) {
-  if (!out || kind < 0 || kind > 2 || rows < 0 || N <= 0 || N % 16 != 0 || K <= 0 ||
+  if (!out || kind < 0 || kind > 3 || rows < 0 || N <= 0 || N % 16 != 0 || K <= 0 ||
       K % 128 != 0 || G < 1 || num_sms < 1)
     return DG_ERR_INVALID_ARG;
-  const PickedConfig pc = pick_config(kind, rows, N, K, G, expected_m, num_sms);
+  const PickedConfig pc = pick_config(kind, rows, N, K, G, expected_m, num_sms, nullptr,
+                                      /*mn_operands=*/kind == kKGrouped);
   const Variant v = kVariants[pc.variant];
   out->block_m = tile_rows(v);
   out->block_n = v.block_n;

@@ -136,7 +136,8 @@ inline bool pick_decode(int rows, int N, int K, int num_sms, const ClusterLimits
   return found;
 }
 
-// kind: 0 dense, 1 contiguous, 2 masked.  rows: M, M_sum or max_m.
+// kind: 0 dense, 1 contiguous, 2 masked, 3 K-grouped.  rows: M, M_sum, max_m,
+// or M (the output rows of each group of the K-grouped form).
 inline PickedConfig pick_config(int kind, int rows, int N, int K, int G, int expected_m,
                                 int num_sms, const ClusterLimits* lim = nullptr,
                                 bool mn_operands = false) {
@@ -156,6 +157,8 @@ inline PickedConfig pick_config(int kind, int rows, int N, int K, int G, int exp
   if (kind == 2) {
     eff_rows = expected_m > 0 ? (expected_m < rows ? expected_m : rows) : rows;
     groups = G;
+  } else if (kind == 3) {
+    groups = G;  // every group has all of its output tiles
   }
   double best_cost = 1e30;
   for (int v = 0; v < kNumVariants; ++v) {
@@ -182,8 +185,8 @@ inline PickedConfig pick_config(int kind, int rows, int N, int K, int G, int exp
   const int tm = tile_rows(kVariants[best.variant]);
   const int n_tiles = ceil_div(N, bn);
   long long tiles;
-  if (kind == 2) {
-    tiles = static_cast<long long>(G) * ceil_div(rows, tm) * n_tiles;  // upper bound
+  if (kind == 2 || kind == 3) {
+    tiles = static_cast<long long>(G) * ceil_div(rows, tm) * n_tiles;  // masked: upper bound
   } else {
     tiles = static_cast<long long>(ceil_div(rows, tm)) * n_tiles;
   }

@@ -16,21 +16,27 @@ namespace dg {
 
 // Launch forms: the three GEMM forms, then the dense form with M-major A
 // and/or N-major B, then the dense form with FP32 output (D = A B^T + C),
-// then the three GEMM forms on BF16 operands; the forms differ in their
-// kernel instantiation.
+// then the three GEMM forms on BF16 operands, then the K-grouped form (the
+// weight gradient: M-major A, N-major B, FP32 output per group); the forms
+// differ in their kernel instantiation.
 enum Form : int { kFormDense = 0, kFormContiguous = 1, kFormMasked = 2, kFormNN = 3, kFormTN = 4,
                   kFormTT = 5, kFormF32 = 6, kFormBf16Dense = 7, kFormBf16Contiguous = 8,
-                  kFormBf16Masked = 9 };
-constexpr int kNumForms = 10;
-static_assert(kFormBf16Masked + 1 == kNumForms, "one shared-memory attribute row per form");
+                  kFormBf16Masked = 9, kFormKGrouped = 10 };
+constexpr int kNumForms = 11;
+static_assert(kFormKGrouped + 1 == kNumForms, "one shared-memory attribute row per form");
 
-constexpr bool is_bf16_form(int f) { return f >= kFormBf16Dense; }
+constexpr bool is_bf16_form(int f) { return f >= kFormBf16Dense && f <= kFormBf16Masked; }
 constexpr int kind_of_form(int f) {
-  return f < 3 ? f : is_bf16_form(f) ? f - kFormBf16Dense : kDense;
+  return f < 3 ? f : is_bf16_form(f) ? f - kFormBf16Dense : f == kFormKGrouped ? kKGrouped : kDense;
 }
 constexpr int layout_of_form(int f) {
-  return f == kFormNN ? kLayoutNN : f == kFormTN ? kLayoutTN : f == kFormTT ? kLayoutTT : kLayoutNT;
+  return f == kFormNN ? kLayoutNN
+         : (f == kFormTN || f == kFormKGrouped) ? kLayoutTN
+         : f == kFormTT ? kLayoutTT
+                        : kLayoutNT;
 }
+// Forms whose kernel writes the FP32 accumulator (plus an optional addend).
+constexpr bool is_f32_form(int f) { return f == kFormF32 || f == kFormKGrouped; }
 // Variants that serve M-/N-major operands and the FP32 output form: general
 // ones with 128-column B boxes.
 constexpr bool mn_capable(const Variant& v) {
@@ -58,6 +64,7 @@ struct GemmCall {
   const int* m_indices;  // contiguous form
   const int* masked_m;   // masked form
   int rows, N, K, G, expected_m;
+  const int* ks = nullptr;  // K-grouped form: rows of K per group (device)
 };
 
 // Device facts the plan depends on (none of them needs device memory).
@@ -76,6 +83,10 @@ dg_status check_gemm_call(const GemmCall& call, bool* empty);
 // device word the kernel reports into.
 dg_status plan_gemm(const GemmCall& call, const DeviceFacts& facts, int* error_word,
                     LaunchPlan* plan);
+
+// Launches the scale-contract check of a call's sfa and sfb (FP8 forms) on
+// `stream`, reporting into `error_word`.
+dg_status launch_scale_check(const GemmCall& call, int* error_word, cudaStream_t stream);
 
 // Library-wide settings that every entry point applies.
 unsigned long long wait_timeout_ns();

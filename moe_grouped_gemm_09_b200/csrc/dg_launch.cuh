@@ -26,13 +26,13 @@ constexpr bool kBuilt =
     ((FORM == kFormContiguous || FORM == kFormMasked || FORM == kFormBf16Contiguous ||
       FORM == kFormBf16Masked) &&
      !kVariants[V].decode) ||
-    (FORM >= kFormNN && FORM <= kFormF32 && mn_capable(kVariants[V]));
+    ((FORM >= kFormNN && FORM <= kFormF32) || FORM == kFormKGrouped) && mn_capable(kVariants[V]);
 
 template <int FORM, int V>
 auto kernel_of() {
   constexpr Variant var = kVariants[V];
   return fp8_gemm_kernel<kind_of_form(FORM), var.block_n, var.stages, var.num_acc, var.kps,
-                         var.a_rows, var.small, layout_of_form(FORM), FORM == kFormF32,
+                         var.a_rows, var.small, layout_of_form(FORM), is_f32_form(FORM),
                          is_bf16_form(FORM)>;
 }
 

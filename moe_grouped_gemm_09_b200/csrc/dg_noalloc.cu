@@ -88,7 +88,12 @@ extern "C" dg_status dg_fp8_gemm_nt_noalloc(const void* a, const float* sfa, con
   LaunchPlan pl;
   s = plan_gemm(call, DeviceFacts{st->num_sms, &st->limits}, st->error_word, &pl);
   if (s != DG_OK || pl.grid == 0) return s;
-  return launch_fp8_dense(st->attr_set, pl, reinterpret_cast<cudaStream_t>(stream));
+  const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if (check_scales_enabled()) {
+    s = launch_scale_check(call, st->error_word, cs);
+    if (s != DG_OK) return s;
+  }
+  return launch_fp8_dense(st->attr_set, pl, cs);
 }
 
 extern "C" dg_status dg_fp8_gemm_nt_noalloc_get_last_device_error(int* code) {

@@ -54,7 +54,10 @@
 
 namespace dg {
 
-enum GemmKind : int { kDense = 0, kContiguous = 1, kMasked = 2 };
+// kKGrouped: the reduction axis is grouped (the weight gradient of the MoE
+// grouped forms in training): group g sums the K rows [k_off[g], k_off[g] +
+// ks[g]) of A [K_sum, M] and B [K_sum, N] into its own FP32 output D[g].
+enum GemmKind : int { kDense = 0, kContiguous = 1, kMasked = 2, kKGrouped = 3 };
 
 // Operand layouts of the dense form (DeepGEMM project card, core features:
 // NT / NN / TN / TT on SM100).  Bit 0: A is M-major ([K, M] in memory);
@@ -70,8 +73,10 @@ enum DeviceError : int {
   kDevTimeoutEpilogue = 0x104,
   kDevMixedExperts = 0x201,   // a 128-row block of m_indices names two experts
   kDevExpertRange = 0x202,    // an m_indices entry is >= G
-  kDevBadScale = 0x301,       // a scale that is not a positive normal power of two (checked
-                              // only when GemmArgs::check_scales is set)
+  kDevKGroups = 0x203,        // K-grouped: group sizes negative, not multiples of 128, or not
+                              // summing to K (nothing is computed)
+  kDevBadScale = 0x301,       // a scale that is not a positive normal power of two (reported
+                              // by check_scales_kernel, launched only on request)
 };
 
 struct GemmArgs {
@@ -91,11 +96,11 @@ struct GemmArgs {
   const float* c_f32;  // FP32 output form: C [rows, N] added to the product, or null
   const int* m_indices;  // contiguous: [rows]
   const int* masked_m;   // masked: [G]
+  const int* ks;         // K-grouped: rows of K of each group [G]
   int* error_word;
   unsigned long long timeout_ns;
   int a_box_rows;    // rows of A one TMA box brings (128, or fewer for a short dense A)
   int prefetch;      // 1: warm L2 with the first tile before waiting on the previous kernel
-  int check_scales;  // 1: report scales that are not positive normal powers of two
 };
 
 constexpr int kBlockM = 128;
@@ -230,6 +235,19 @@ __device__ __forceinline__ Tile get_tile(int t, const GemmArgs& p, const int* s_
     ti.m_blk = u % p.num_m_blocks;
     ti.n_blk = u / p.num_m_blocks;
     ti.group = 0;
+  } else if (KIND == kKGrouped) {
+    // every group has the same output tiles; its K range comes from the
+    // prefix of the group sizes (in K blocks); a group without K rows still
+    // has its output written (C, or zeros) by the epilogue
+    const int tpg = p.num_m_blocks * p.num_n_blocks;
+    ti.group = u / tpg;
+    const int local = u - ti.group * tpg;
+    ti.m_blk = local % p.num_m_blocks;
+    ti.n_blk = local / p.num_m_blocks;
+    ti.kb_begin = s_prefix[ti.group];
+    ti.kb_end = s_prefix[ti.group + 1];
+    ti.skip = ti.kb_begin >= ti.kb_end;
+    return ti;
   } else {
     // row-major over tiles: the CTAs of one wave cover a few consecutive
     // 128-row blocks (one or a few experts) and all their column tiles, so
@@ -354,9 +372,13 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
   static_assert(!BF16 || (LAYOUT == kLayoutNT && !OUT_F32),
                 "BF16 operands: K-major A and B, BF16 output");
   // FP32 output (D = A B^T + C): the dense form, no split-K (host-checked)
-  static_assert(!OUT_F32 || (KIND == kDense && A_ROWS == 128 && !SMALL), "FP32 output form");
+  static_assert(!OUT_F32 || ((KIND == kDense || KIND == kKGrouped) && A_ROWS == 128 && !SMALL),
+                "FP32 output form");
+  static_assert(KIND != kKGrouped || (OUT_F32 && LAYOUT == kLayoutTN),
+                "K-grouped: M-major A, N-major B, FP32 output");
   static_assert(LAYOUT == kLayoutNT ||
-                    (KIND == kDense && KPS == 1 && A_ROWS == 128 && !SMALL && BLOCK_N % 128 == 0),
+                    ((KIND == kDense || KIND == kKGrouped) && KPS == 1 && A_ROWS == 128 &&
+                     !SMALL && BLOCK_N % 128 == 0),
                 "M-/N-major operands: dense form, general variants with 128-column B boxes");
 
   extern __shared__ uint8_t smem_raw[];
@@ -368,7 +390,8 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
   // epilogue staging tiles (1024-aligned, swizzled): their own region, or,
   // when every CTA has a single tile (always for a small variant), the operand
   // ring, idle once that tile's MMAs are done, with one tile per warp and chunk
-  const int n_tiles_total = (KIND == kMasked ? -1 : p.num_m_blocks * p.num_n_blocks * p.split_k);
+  const int n_tiles_total =
+      (KIND == kMasked || KIND == kKGrouped) ? -1 : p.num_m_blocks * p.num_n_blocks * p.split_k;
   const bool one_tile =
       SMALL || (n_tiles_total >= 0 && n_tiles_total <= static_cast<int>(gridDim.x));
   uint8_t* sEpi = one_tile ? sA : sB + STAGES * B_BYTES;
@@ -381,7 +404,8 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
   uint64_t* recv_bar = drain + 1;  // split-K: partial slices pushed by the other CTAs
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(recv_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int* s_prefix = const_cast<int*>(abort_flag + 3);  // masked form only
+  int* s_kvalid = const_cast<int*>(abort_flag + 1);  // K-grouped form: group sizes consistent
+  int* s_prefix = const_cast<int*>(abort_flag + 3);  // masked and K-grouped forms
   // split-K: this CTA's FP32 partial, parked over the (by then idle) operand ring
   float* red = reinterpret_cast<float*>(sA);
 
@@ -434,6 +458,20 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
         }
       }
     }
+    if constexpr (!BF16) {
+      // ... and the scales that tile reads (one line holds 32 K blocks of a
+      // row): the scale warp's first loads then come from L2 instead of
+      // queueing behind the operand stream in DRAM
+      const int m0 = ti.m_blk * kBlockM;
+      const int rows_here = min(kBlockM, p.rows - m0);
+      for (int r = lane; r < rows_here; r += 32)
+        for (int kb = ti.kb_begin; kb < ti.kb_end; kb += 32)
+          ptx::prefetch_l2(p.sfa + (size_t)(m0 + r) * p.k_blocks + kb);
+      const int b0 = ti.n_blk * BLOCK_N / 128;
+      if (lane < SFB_BLOCKS && b0 + lane < p.nb128)
+        for (int kb = ti.kb_begin; kb < ti.kb_end; kb += 32)
+          ptx::prefetch_l2(p.sfb + (size_t)(b0 + lane) * p.k_blocks + kb);
+    }
   }
   // Barriers, the abort flag and the TMEM base are published before waiting
   // on the previous kernel, so that every role starts right after the wait.
@@ -465,10 +503,32 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
     }
     __syncthreads();
   }
+  if (KIND == kKGrouped) {
+    // K-block offsets of the groups, from the group sizes (device data); an
+    // inconsistent set of sizes computes nothing and says why
+    if (threadIdx.x == 96) {
+      int acc = 0;
+      bool bad = false;
+      for (int g = 0; g < p.G; ++g) {
+        s_prefix[g] = acc;
+        const int k = p.ks[g];
+        bad |= k < 0 || k % kBlockK != 0;
+        acc += max(k, 0) / kBlockK;
+      }
+      s_prefix[p.G] = acc;
+      bad |= acc != p.k_blocks;
+      if (bad) atomicCAS(p.error_word, 0, kDevKGroups);
+      *s_kvalid = bad ? 0 : 1;
+    }
+    __syncthreads();
+  }
 
   ptx::WaitCtl ctl{abort_flag, p.error_word, p.timeout_ns};
-  const int total = (KIND == kMasked ? s_prefix[p.G]
-                                     : p.num_m_blocks * p.num_n_blocks) * p.split_k;
+  const int total = (KIND == kMasked     ? s_prefix[p.G]
+                     : KIND == kKGrouped ? (*s_kvalid ? p.G : 0) * p.num_m_blocks *
+                                               p.num_n_blocks
+                                         : p.num_m_blocks * p.num_n_blocks) *
+                    p.split_k;
 
   // Drains TMEM accumulator buffer `a` of tile `ti`, lane quarter q (rows
   // 32q..32q+31), columns [c_begin, c_end): BF16 through the staging tiles
@@ -485,6 +545,9 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
     if (KIND == kMasked) {
       const int mm = min(max(__ldg(p.masked_m + ti.group), 0), p.rows);
       valid = m_in_group < mm;
+      grow = (size_t)ti.group * p.rows + m_in_group;
+    } else if (KIND == kKGrouped) {
+      valid = m_in_group < p.rows;
       grow = (size_t)ti.group * p.rows + m_in_group;
     } else {
       valid = m_in_group < p.rows;
@@ -782,7 +845,8 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
                           : 1.0f;
         }
         // B scale blocks are 128 rows: the tile's rows touch blocks b0, b0 + 1, ...
-        const float* sfb_g = p.sfb + (size_t)ti.group * p.nb128 * KB;
+        // (K-grouped: one sfb for all groups, indexed by the global K block)
+        const float* sfb_g = p.sfb + (KIND == kKGrouped ? 0 : (size_t)ti.group * p.nb128 * KB);
         const int b0 = ti.n_blk * BLOCK_N / 128;
   #pragma unroll
         for (int i = 0; i < SFB_BLOCKS; ++i) {
@@ -810,7 +874,6 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
           ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
           if (!ok) break;
           uint8_t* sf = sSF + s * SF_BYTES;
-          bool bad = false;  // a scale breaks the contract (checked on request)
           // A scales: TMEM lane l, column c holds row 32c + l of the tile.
           {
             uint32_t w[4];
@@ -818,10 +881,8 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
             for (int c = 0; c < 4; ++c) {
               uint32_t x = 0x7F7F7F7Fu;  // unused bytes: scale 1
   #pragma unroll
-              for (int j = 0; j < KPS; ++j) {
+              for (int j = 0; j < KPS; ++j)
                 x = (x & ~(0xFFu << (8 * j))) | (ue8m0(va[slot][c][j]) << (8 * j));
-                if (p.check_scales) bad |= !scale_ok(va[slot][c][j]);
-              }
               w[c] = x;
             }
             *reinterpret_cast<uint4*>(sf + 16 * lane) = make_uint4(w[0], w[1], w[2], w[3]);
@@ -843,15 +904,12 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
                 for (int i = 1; i < SFB_BLOCKS; ++i)
                   if (idx == i) v = vb[slot][i][j];
                 x = (x & ~(0xFFu << (8 * j))) | (ue8m0(v) << (8 * j));
-                if (p.check_scales) bad |= !scale_ok(v);
               }
               w[c] = x;
             }
             *reinterpret_cast<uint4*>(sf + 512 * (1 + h) + 16 * lane) =
                 make_uint4(w[0], w[1], w[2], w[3]);
           }
-          if (p.check_scales && __any_sync(0xFFFFFFFFu, bad) && lane == 0)
-            atomicCAS(p.error_word, 0, kDevBadScale);
           ptx::fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) ptx::mbar_arrive(&full[s]);
@@ -905,7 +963,8 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
           }
         }
         // B scale blocks are 128 rows: the tile's rows touch blocks b0, b0 + 1, ...
-        const float* sfb_g = p.sfb + (size_t)ti.group * p.nb128 * KB;
+        // (K-grouped: one sfb for all groups, indexed by the global K block)
+        const float* sfb_g = p.sfb + (KIND == kKGrouped ? 0 : (size_t)ti.group * p.nb128 * KB);
         const int b0 = ti.n_blk * BLOCK_N / 128;
   #pragma unroll
         for (int i = 0; i < SFB_BLOCKS; ++i) {
@@ -941,7 +1000,6 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
         if (first) {
           uint8_t* sf = sSF + (gc % STAGES) * SF_BYTES;
           const int n_valid = min(GK, wr.w.ti.kb_end - wr.kb);  // K blocks of this group
-          bool bad = false;  // a scale breaks the contract (checked on request)
           // A scales: TMEM lane l, column c holds row 32c + l of the tile.
           {
             uint32_t w[4];
@@ -949,11 +1007,8 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
             for (int c = 0; c < 4; ++c) {
               uint32_t x = 0x7F7F7F7Fu;  // unused bytes: scale 1
   #pragma unroll
-              for (int j = 0; j < GK; ++j) {
-                if (j >= n_valid) continue;
-                x = (x & ~(0xFFu << (8 * j))) | (ue8m0(a[c][j]) << (8 * j));
-                if (p.check_scales) bad |= !scale_ok(a[c][j]);
-              }
+              for (int j = 0; j < GK; ++j)
+                if (j < n_valid) x = (x & ~(0xFFu << (8 * j))) | (ue8m0(a[c][j]) << (8 * j));
               w[c] = x;
             }
             *reinterpret_cast<uint4*>(sf + 16 * lane) = make_uint4(w[0], w[1], w[2], w[3]);
@@ -974,17 +1029,13 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
   #pragma unroll
                 for (int i = 1; i < SFB_BLOCKS; ++i)
                   if (idx == i) v = b[i][j];
-                if (j >= n_valid) continue;
-                x = (x & ~(0xFFu << (8 * j))) | (ue8m0(v) << (8 * j));
-                if (p.check_scales) bad |= !scale_ok(v);
+                if (j < n_valid) x = (x & ~(0xFFu << (8 * j))) | (ue8m0(v) << (8 * j));
               }
               w[c] = x;
             }
             *reinterpret_cast<uint4*>(sf + 512 * (1 + h) + 16 * lane) =
                 make_uint4(w[0], w[1], w[2], w[3]);
           }
-          if (p.check_scales && __any_sync(0xFFFFFFFFu, bad) && lane == 0)
-            atomicCAS(p.error_word, 0, kDevBadScale);
           ptx::fence_proxy_async_smem();
           __syncwarp();
           ++gc;
@@ -1021,6 +1072,18 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
       if (ti.skip) {
         if (KIND == kContiguous && ti.group >= p.G && ep_tid == 0)
           atomicCAS(p.error_word, 0, kDevExpertRange);
+        if constexpr (KIND == kKGrouped && OUT_F32) {
+          // a group without K rows: its output is C (or zeros), no product
+          const int m = ti.m_blk * kBlockM + row_local;
+          if (m < p.rows) {
+            const size_t off = ((size_t)ti.group * p.rows + m) * p.N;
+            for (int n = ti.n_blk * BLOCK_N; n < min(p.N, (ti.n_blk + 1) * BLOCK_N); n += 4) {
+              const float4 v = p.c_f32 ? *reinterpret_cast<const float4*>(p.c_f32 + off + n)
+                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+              *reinterpret_cast<float4*>(p.d_f32 + off + n) = v;
+            }
+          }
+        }
         if (split) {
           // an empty K slice still contributes (zeros) to the cluster's sum
           const int valid_rows = min(p.rows - ti.m_blk * kBlockM, kBlockM);

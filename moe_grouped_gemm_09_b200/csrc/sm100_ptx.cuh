@@ -177,6 +177,18 @@ __device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* map, int c
       : "memory");
 }
 
+// Bring `bytes` contiguous bytes at `p` (16-byte aligned, a multiple of 16)
+// into L2 with one bulk request (no completion to wait for).
+__device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// Bring the 128-byte line holding `p` into L2 (no completion to wait for).
+// Safe before a dependency wait for the same reason as the TMA prefetches.
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p) : "memory");
+}
+
 // ------------------------------------------------------------------ cluster --
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {

@@ -159,9 +159,29 @@ def test_small_problem_grid_is_its_tile_count(dg):
     assert c["grid"] == (-(-300 // 128)) * (-(-96 // c["block_n"]))
 
 
+def test_k_grouped_plan_covers_every_group(dg):
+    """The K-grouped form (kind 3) takes persistent general tiles with whole
+    128-column B boxes, and its tiles are every group's output tiles."""
+    c = dg.query_config(3, 256, 384, 4096, G=8, num_sms=148)
+    assert c["block_n"] % 128 == 0 and c["split_k"] == 1 and c["kps"] == 1
+    assert c["grid"] == min(148, 8 * 2 * (-(-384 // c["block_n"])))
+
+
+def test_k_grouped_bad_arguments_rejected(dg):
+    fn = dg._k_grouped
+    # a, sfa, b, sfb, c, d, ks, G, M, N, K_sum, stream
+    assert fn(FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, 2, 24, 128, 256, None) == 1   # M % 16
+    assert fn(FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, 2, 32, 120, 256, None) == 1   # N % 16
+    assert fn(FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, 2, 32, 128, 200, None) == 1   # K % 128
+    assert fn(FAKE, FAKE, FAKE, FAKE, None, FAKE, None, 2, 32, 128, 256, None) == 1   # no ks
+    assert fn(FAKE, FAKE, FAKE, FAKE, FAKE + 4, FAKE, FAKE, 2, 32, 128, 256, None) == 1  # c align
+    assert fn(FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, 2000, 32, 128, 256, None) == 2  # G > 1024
+    assert fn(FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, 0, 32, 128, 256, None) == 0     # no groups
+
+
 def test_query_rejects_bad_input(dg):
     with pytest.raises(dg.DgError):
-        dg.query_config(3, 64, 128, 128)
+        dg.query_config(4, 64, 128, 128)
     with pytest.raises(dg.DgError):
         dg.query_config(0, 64, 100, 128)
 

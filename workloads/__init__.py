@@ -26,6 +26,9 @@ performance and on the MoE grouped layouts):
   ``-1`` in ``m_indices`` and filled with random FP8 bytes (so that a kernel that
   forgets to skip them is caught);
 * masked grouped layout: ``masked_m[g]`` uniform in ``[0, max_m]``;
+* K-grouped layout (weight gradient): the contiguous layout's token counts,
+  each expert's rows padded with zero rows to a multiple of 128; A (output
+  gradients) and B (layer inputs) stored one row per token;
 * BF16 operands: the same N(0, 1) values (same streams) rounded to BF16 with
   round-to-nearest-even, and the same group structure; no scales.
 """
@@ -227,6 +230,63 @@ def masked_problem(G: int = 32, max_m: int = 256, N: int = 4096, K: int = 7168, 
                          masked_m, G, max_m, N, K, int(expected_m))
 
 
+@dataclasses.dataclass
+class KGroupedProblem:
+    """The weight gradient of an M-grouped layer: per expert g,
+    dW[g] = dY_g^T X_g, the reduction running over the expert's tokens.  In the
+    K-grouped call's terms: A = dY as [K_sum, M] (one row per token), B = X as
+    [K_sum, N], group g owning ks[g] consecutive rows (its tokens, then zero
+    rows up to a multiple of 128)."""
+    a: np.ndarray        # uint8 [K_sum, M]  E4M3 bytes, M-major
+    sfa: np.ndarray      # float32 [M, K_sum/128]
+    b: np.ndarray        # uint8 [K_sum, N]  E4M3 bytes, N-major
+    sfb: np.ndarray      # float32 [ceil(N/128), K_sum/128]
+    ks: np.ndarray       # int32 [G]: rows of K of each group (multiples of 128)
+    counts: np.ndarray   # tokens of each group (the rest of its rows are zero)
+    G: int
+    M: int
+    N: int
+    K_sum: int
+
+    def valid_rows(self) -> int:
+        return int(self.counts.sum())
+
+    def flops(self) -> float:
+        return 2.0 * self.M * self.N * self.valid_rows()
+
+    def bytes(self) -> float:
+        v = self.valid_rows()
+        KB = self.K_sum // BLOCK_K
+        NB = -(-self.N // BLOCK_N_SCALE)
+        return float(v * (self.M + self.N) + 4 * (self.M + NB) * KB + 4 * self.G
+                     + 4 * self.G * self.M * self.N)
+
+
+def k_grouped_problem(G: int = 32, M: int = 4096, N: int = 7168, total_tokens: int = 8192,
+                      zipf_s: float = 1.1, align: int = 128, seed: int = 0,
+                      counts: Optional[np.ndarray] = None) -> KGroupedProblem:
+    """Token counts as in the contiguous layout (Zipf over the experts), each
+    expert's segment padded with zero rows to a multiple of ``align``; N(0, 1)
+    values for the real rows, quantised in 1 x 128 blocks along the tokens for
+    A (one scale per column of dY per 128 tokens) and 128 x 128 blocks for B."""
+    if counts is None:
+        counts = zipf_counts(total_tokens, G, zipf_s, seed)
+    counts = np.asarray(counts, dtype=np.int64)
+    ks = (-(-counts // align) * align).astype(np.int32)
+    K_sum = int(ks.sum())
+    real = np.zeros(K_sum, bool)
+    off = 0
+    for g in range(G):
+        real[off:off + counts[g]] = True
+        off += int(ks[g])
+    xa = _normal(_rng(seed, _TAG_A), (M, K_sum)) * real[None, :]
+    xb = _normal(_rng(seed, _TAG_B), (N, K_sum)) * real[None, :]
+    qa, sa = quantize_rows(xa, 1)
+    qb, sb = quantize_rows(xb, BLOCK_N_SCALE)
+    return KGroupedProblem(np.ascontiguousarray(qa.T), sa, np.ascontiguousarray(qb.T), sb, ks,
+                           counts, G, M, N, K_sum)
+
+
 def to_bf16_bits(x: np.ndarray) -> np.ndarray:
     """FP32 values -> BF16 operand bit patterns (round to nearest even, ml_dtypes)."""
     return np.asarray(x, np.float32).astype(ml_dtypes.bfloat16).view(np.uint16)
@@ -339,3 +399,5 @@ PREFILL_SHAPES = [(4096, n, k) for (n, k) in ((2112, 7168), (24576, 1536), (7168
                                               (4096, 7168))]
 CONTIGUOUS_MOE = dict(G=32, N=4096, K=7168, total_tokens=8192, zipf_s=1.1, align=128)
 MASKED_MOE = dict(G=32, max_m=256, N=4096, K=7168)
+# the weight gradient of the contiguous MoE layer: dW[g] [4096, 7168] per expert
+K_GROUPED_MOE = dict(G=32, M=4096, N=7168, total_tokens=8192, zipf_s=1.1, align=128)
