@@ -348,6 +348,9 @@ def time_workload(ctx: GpuContext, name: str, args, steps: int, per_gemm: bool, 
 
     dev, stream = ctx.dev, ctx.stream
     items = build_workload(name, seed=args.seed)
+    # dense workloads: B is the weights, so the weight preload applies
+    preload = args.weight_preload == "on" and all(k in ("dense", "bf16_dense") for k, _ in items)
+    dg.set_weight_preload(preload)
     metric, unit, _ = workload_meta(name)
     set_bytes = sum(p.a.nbytes + p.b.nbytes + getattr(p, "sfa", p.a[:0]).nbytes
                     + getattr(p, "sfb", p.a[:0]).nbytes for _, p in items)
@@ -432,6 +435,32 @@ def time_workload(ctx: GpuContext, name: str, args, steps: int, per_gemm: bool, 
     if dg.get_last_device_error() != 0:
         raise RuntimeError(f"{name}: device error during the timed steps")
 
+    # the same steps with the weight preload off, for comparison (the dense
+    # workloads are timed with it on: B is the weights, written by no kernel)
+    ms_no_preload = None
+    if preload:
+        dg.set_weight_preload(False)
+        plain = capture(R)
+        plain_tail = capture(rem) if rem else None
+        with torch.cuda.stream(stream):
+            plain.replay()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ctx.barrier()
+        torch.cuda.synchronize(dev)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(steps // R):
+                plain.replay()
+            if plain_tail is not None:
+                plain_tail.replay()
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ctx.barrier()
+        ms_no_preload = ctx.max_over_ranks(e0.elapsed_time(e1) / steps)
+        dg.set_weight_preload(True)
+        del plain, plain_tail
+
     # ---- per GEMM (second timed pass): R back-to-back launches of one shape ----
     kernel_ms = []
     if per_gemm:
@@ -496,8 +525,10 @@ def time_workload(ctx: GpuContext, name: str, args, steps: int, per_gemm: bool, 
                    "unit": unit, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
     del cycle, tail
+    dg.set_weight_preload(False)
     return {"items": items, "ms": ms, "R": R, "flush_note": flush_note, "kernel_ms": kernel_ms,
-            "clocks": clocks.summary(), "e2e": e2e_res, "metric": metric, "unit": unit}
+            "clocks": clocks.summary(), "e2e": e2e_res, "metric": metric, "unit": unit,
+            "preload": preload, "ms_no_preload": ms_no_preload}
 
 
 def workload_record(name: str, t: dict, world: int, steps: int, warmup: int) -> dict:
@@ -531,6 +562,7 @@ def workload_record(name: str, t: dict, world: int, steps: int, warmup: int) -> 
             "gemms": [dict(kind=k, **_shape(p)) for k, p in items],
             "l2": t["flush_note"],
             "graph": f"one CUDA graph per rotation cycle of {t['R']} steps",
+            "weight_preload": t["preload"],
         },
         "gpu_launches": int(steps * launches_per_step),
         "roofline": {
@@ -549,6 +581,9 @@ def workload_record(name: str, t: dict, world: int, steps: int, warmup: int) -> 
             "per_gemm_us": [round(x * 1e3, 3) for x in t["kernel_ms"]],
         },
         "clocks": t["clocks"],
+        **({"value_without_weight_preload": round(
+            whole_job_value(step_units(items, unit), world, t["ms_no_preload"], unit), 3)}
+           if t["ms_no_preload"] else {}),
     }
 
 
@@ -582,6 +617,8 @@ def run_gpu(args):
         "roofline": rec["roofline"],
         "clocks": rec["clocks"],
     }
+    if "value_without_weight_preload" in rec:
+        res["value_without_weight_preload"] = rec["value_without_weight_preload"]
     cpu_ok = ctx.rank == 0 and ctx.world == 1 and not args.no_cpu_baseline
     if cpu_ok:
         res["cpu_baseline"] = run_oracle_sample(main["items"], main["unit"],
@@ -846,6 +883,9 @@ def main():
                     help="input copies rotated between steps (0: enough to exceed 3x L2)")
     ap.add_argument("--reference-budget-s", type=float, default=120.0,
                     help="reference arm: whole oracle steps if they fit in this time")
+    ap.add_argument("--weight-preload", choices=("on", "off"), default="on",
+                    help="dense workloads: let each GEMM load B (the weights) before waiting "
+                         "on the previous kernel; the line also reports the value with it off")
     ap.add_argument("--measure-fp8-peak", action="store_true",
                     help="time the vendor library's dense E4M3 GEMM and print its TFLOP/s")
     ap.add_argument("--peak-size", type=int, default=8192)

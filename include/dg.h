@@ -225,6 +225,20 @@ dg_status dg_set_wait_timeout_ns(long long ns);
  * added. */
 dg_status dg_set_check_scales(int enable);
 
+/* Weight preload for the dense calls (enable != 0), off by default; the
+ * environment variable DG_WEIGHT_PRELOAD=1 turns it on at first use.  Every
+ * GEMM launch may start before the previous kernel on its stream has
+ * finished (programmatic dependent launch) and waits for it before reading
+ * its inputs.  With the preload on, a dense call's kernel loads the first
+ * ring stages of B before that wait, overlapping them with the previous
+ * kernel's tail; only A (and the scales) are read after it.  The caller
+ * declares by turning it on that B -- model weights in inference -- is
+ * never written by a kernel that may still run when a dense GEMM reading it
+ * is launched on the same stream.  Applies to launches enqueued after the
+ * call, from every thread and entry point; results are the same either way
+ * when that holds. */
+dg_status dg_set_weight_preload(int enable);
+
 /* Human-readable name of a status code.  Never NULL. */
 const char* dg_status_string(dg_status s);
 

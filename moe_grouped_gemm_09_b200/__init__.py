@@ -58,6 +58,7 @@ _get_last_err = _decl("dg_get_last_device_error", [ctypes.POINTER(ctypes.c_int)]
 _set_timeout = _decl("dg_set_wait_timeout_ms", [_I])
 _set_timeout_ns = _decl("dg_set_wait_timeout_ns", [ctypes.c_longlong])
 _set_check_scales = _decl("dg_set_check_scales", [_I])
+_set_weight_preload = _decl("dg_set_weight_preload", [_I])
 _gemm_nt_noalloc = _decl("dg_fp8_gemm_nt_noalloc", [_P, _P, _P, _P, _P, _I, _I, _I, _P])
 _noalloc_err = _decl("dg_fp8_gemm_nt_noalloc_get_last_device_error", [ctypes.POINTER(ctypes.c_int)])
 _status_string = _decl("dg_status_string", [_I], ctypes.c_char_p)
@@ -79,7 +80,8 @@ EXPORTED_SYMBOLS = ("dg_fp8_gemm_nt", "dg_m_grouped_fp8_gemm_nt_contiguous",
                     "dg_fp8_gemm_tn", "dg_fp8_gemm_tt", "dg_fp8_gemm_nt_f32", "dg_bf16_gemm_nt",
                     "dg_m_grouped_bf16_gemm_nt_contiguous", "dg_m_grouped_bf16_gemm_nt_masked",
                     "dg_set_wait_timeout_ns", "dg_fp8_gemm_nt_noalloc_get_last_device_error",
-                    "dg_set_check_scales", "dg_k_grouped_fp8_gemm_tn_contiguous")
+                    "dg_set_check_scales", "dg_k_grouped_fp8_gemm_tn_contiguous",
+                    "dg_set_weight_preload")
 
 DEVICE_ERRORS = {
     0x101: "wait timeout in the TMA producer",
@@ -415,6 +417,13 @@ def set_check_scales(enable: bool) -> None:
     """Make later launches check every scale against the contract (a positive
     normal power of two; device error 0x301 otherwise)."""
     _check(_set_check_scales(1 if enable else 0), "dg_set_check_scales")
+
+
+def set_weight_preload(enable: bool) -> None:
+    """Let later dense launches load B (weights) before waiting on the previous
+    kernel of their stream; the caller declares that no kernel that may still
+    run writes B."""
+    _check(_set_weight_preload(1 if enable else 0), "dg_set_weight_preload")
 
 
 def set_wait_timeout_ns(ns: int) -> None:

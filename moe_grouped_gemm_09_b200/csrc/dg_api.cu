@@ -38,6 +38,7 @@ std::mutex g_settings_mutex;
 unsigned long long g_timeout_ns = 1000ull * 1000 * 1000;
 bool g_timeout_from_env = false;
 int g_check_scales = -1;          // -1: not decided yet (read DG_CHECK_SCALES)
+int g_weight_preload = -1;        // -1: not decided yet (read DG_WEIGHT_PRELOAD)
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -104,9 +105,9 @@ int a_box_rows(int kind, int rows) {
   return ((rows + 15) / 16) * 16;
 }
 
-// DG_FORCE_CONFIG="<block_n>:<split_k>[:<kps>:<a_rows>[:<small>]]" overrides
+// DG_FORCE_CONFIG="<block_n>:<split_k>[:<kps>:<a_rows>[:<mode>]]" overrides
 // the picker (tuning sweeps); without kps/a_rows a general (one K block per
-// stage) variant.
+// stage) variant; mode 0 general, 1 decode, 2 small decode.
 // Ignored unless the variant exists and, for split_k > 1, the problem is a
 // dense one with a single 128-row block.
 void forced_config(int kind, int rows, int N, int K, int G, int sms, PickedConfig* pc) {
@@ -114,14 +115,14 @@ void forced_config(int kind, int rows, int N, int K, int G, int sms, PickedConfi
   if (!e || !e[0]) return;
   int bn = 0, sk = 1;
   if (std::sscanf(e, "%d:%d", &bn, &sk) < 1) return;
-  int kps = 0, ar = 0, sm = -1;
-  std::sscanf(e, "%*d:%*d:%d:%d:%d", &kps, &ar, &sm);
+  int kps = 0, ar = 0, mode = -1;
+  std::sscanf(e, "%*d:%*d:%d:%d:%d", &kps, &ar, &mode);
   int v = -1;
   for (int i = 0; i < kNumVariants; ++i) {
     const Variant& x = kVariants[i];
     if (x.block_n != bn) continue;
     if (kps ? (x.kps != kps || (ar && x.a_rows != ar)) : x.decode) continue;
-    if (sm >= 0 && x.small != (sm != 0)) continue;
+    if (mode >= 0 && (x.small ? 2 : x.decode ? 1 : 0) != mode) continue;
     if (x.decode && kind != kDense) continue;
     if (a_box_rows(kind, rows) > x.a_rows) continue;
     v = i;
@@ -170,6 +171,21 @@ dg_status make_d_map(CUtensorMap* map, void* base, uint64_t N, uint64_t rows) {
   cuuint32_t box[2] = {64, 32};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = encoder()(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? DG_OK : DG_ERR_CUDA;
+}
+
+// 3-D tensor map over an FP32 output D [groups][rows][N] (the FP32-output
+// forms: groups = 1 for the dense one) with a box of 32 rows x 32 columns
+// (128 bytes) and the 128-byte swizzle; rows past a group's end and columns
+// past N are clipped by the TMA unit.
+dg_status make_d_map_f32(CUtensorMap* map, void* base, uint64_t N, uint64_t rows, uint64_t groups) {
+  cuuint64_t dims[3] = {N, rows, groups};
+  cuuint64_t strides[2] = {N * 4, rows * N * 4};
+  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = encoder()(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                          CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? DG_OK : DG_ERR_CUDA;
@@ -247,6 +263,12 @@ __global__ void check_scales_kernel(const float* __restrict__ s, long long n, in
 }
 
 }  // namespace
+
+int weight_preload_enabled() {
+  std::lock_guard<std::mutex> lock(g_settings_mutex);
+  if (g_weight_preload < 0) g_weight_preload = env_flag("DG_WEIGHT_PRELOAD") ? 1 : 0;
+  return g_weight_preload;
+}
 
 dg_status launch_scale_check(const GemmCall& call, int* error_word, cudaStream_t stream) {
   const int kind = kind_of_form(call.form);
@@ -377,9 +399,11 @@ dg_status plan_gemm(const GemmCall& call, const DeviceFacts& facts, int* error_w
   args.timeout_ns = wait_timeout_ns();
   args.a_box_rows = a_mn ? kBlockM : a_box_rows(kind, rows);
   args.prefetch = prefetch_enabled();
+  args.preload_b = kind == kDense ? weight_preload_enabled() : 0;
   if (args.a_box_rows > var.a_rows) return DG_ERR_UNSUPPORTED;
-  // a small variant runs one tile per CTA (its epilogue reuses the ring)
-  if (var.small && (kind != kDense || pc.grid != args.num_m_blocks * args.num_n_blocks * pc.split_k))
+  // a decode variant runs one tile per CTA (its epilogue reuses the ring)
+  if (var.decode &&
+      (kind != kDense || pc.grid != args.num_m_blocks * args.num_n_blocks * pc.split_k))
     return DG_ERR_UNSUPPORTED;
   // split-K runs one tile per CTA, one cluster per output tile
   if (pc.split_k > 1 &&
@@ -396,7 +420,9 @@ dg_status plan_gemm(const GemmCall& call, const DeviceFacts& facts, int* error_w
   s = b_mn ? make_map_mn(&pl->tb, call.b, N, K)
            : make_map(&pl->tb, call.b, K, N, b_groups, var.block_n, var.kps, elem);
   if (s != DG_OK) return s;
-  s = make_d_map(&pl->td, call.d, N, static_cast<uint64_t>(a_rows));
+  s = is_f32_form(form)
+          ? make_d_map_f32(&pl->td, call.d, N, rows, kind == kKGrouped ? G : 1)
+          : make_d_map(&pl->td, call.d, N, static_cast<uint64_t>(a_rows));
   if (s != DG_OK) return s;
 
   if (print_configs())
@@ -536,6 +562,12 @@ dg_status dg_set_wait_timeout_ns(long long ns) {
   std::lock_guard<std::mutex> lock(g_settings_mutex);
   g_timeout_from_env = true;
   g_timeout_ns = static_cast<unsigned long long>(ns);
+  return DG_OK;
+}
+
+dg_status dg_set_weight_preload(int enable) {
+  std::lock_guard<std::mutex> lock(g_settings_mutex);
+  g_weight_preload = enable ? 1 : 0;
   return DG_OK;
 }
 

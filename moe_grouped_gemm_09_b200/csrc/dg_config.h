@@ -22,16 +22,19 @@ struct Variant {
   bool small;   // two CTAs fit per SM; one tile per CTA
 };
 
-// The compiled variants: general ones first (every form), then the
-// decode-shaped dense ones, whose stages are several K blocks deep so that
-// each TMA box moves 32-64 KB, then the small decode ones (at most ~100 KB of
-// shared memory and 256 TMEM columns, so that the next kernel's CTAs can be
-// resident and warm L2 with their weights while this kernel drains).
+// The compiled variants: general ones first (every form; the one with two K
+// blocks per stage serves the dense form, where it wins for short K), then
+// the decode-shaped dense ones, whose stages are several K blocks deep so
+// that each TMA box moves 32-64 KB, then the small decode ones (at most
+// ~100 KB of shared memory and 256 TMEM columns, so that the next kernel's
+// CTAs can be resident and warm L2 with their weights while this kernel
+// drains).
 constexpr Variant kVariants[] = {
     {256, 4, 1, 1, 128, false, false},
     {128, 6, 2, 1, 128, false, false},
     {64, 8, 2, 1, 128, false, false},
     {32, 9, 2, 1, 128, false, false},
+    {256, 2, 1, 2, 128, false, false},
     {128, 2, 1, 4, 64, true, false},
     {64, 3, 2, 4, 64, true, false},
     {256, 2, 1, 2, 64, true, false},
@@ -70,13 +73,32 @@ inline int cluster_limit(const ClusterLimits* lim, int v, int s, int num_sms) {
   return n > 0 ? n : num_sms / s;
 }
 
-// Split-K parks each CTA's FP32 partial and the slices the other CTAs push to
-// it in the (then idle) operand ring: (2 * rows + split) rows of BLOCK_N + 4
-// floats must fit.
+// Bytes of a decode variant's split-K receive region (E4M3 operands): the
+// shared-memory budget (227 KB, or 113 KB for a small variant) less the ring,
+// the scale-factor slots, the barriers and 16 bytes of flags (plus 1 KB of
+// alignment slack), capped at a whole A_ROWS x BLOCK_N FP32 partial.  The
+// kernel's own geometry (KernelShape::kRecvBytes) is checked against this at
+// compile time.
+constexpr int decode_recv_bytes(const Variant& v) {
+  if (!v.decode) return 0;
+  const int sf = 512 * (1 + (v.block_n + 127) / 128);
+  const int fixed = 1024 + v.stages * (v.kps * (v.a_rows + v.block_n) * 128 + sf) +
+                    8 * (2 * v.stages + 2 * v.num_acc + 2) + 16;
+  const int budget = (v.small ? 115712 : 232448) - fixed;
+  const int whole = v.a_rows * v.block_n * 4;
+  return ((budget < whole ? budget : whole) / 16) * 16;
+}
+
+// Split-K: column slice c of the tile belongs to CTA c of the cluster; every
+// CTA pushes each other CTA's slice of its valid rows into that CTA's receive
+// region, which must hold split - 1 slices of rows x BLOCK_N / split FP32;
+// slices are whole 16-byte BF16 groups (BLOCK_N / split a multiple of 8).
 inline bool split_fits(const Variant& var, int rows, int split) {
-  const long long ring = static_cast<long long>(var.stages) * var.kps * (var.a_rows + var.block_n) * 128;
-  const long long need = static_cast<long long>(2 * rows + split) * (var.block_n + 4) * 4;
-  return need <= ring;
+  if (split < 2) return true;
+  if (var.block_n % (8 * split) != 0) return false;
+  const long long need =
+      static_cast<long long>(split - 1) * rows * (var.block_n / split) * 4;
+  return need <= decode_recv_bytes(var);
 }
 
 // Decode-shaped dense problems (at most one 128-row block): HBM-bound.  Pick
@@ -166,7 +188,8 @@ inline PickedConfig pick_config(int kind, int rows, int N, int K, int G, int exp
     if (var.small || var.a_rows < 128) continue;
     // M-/N-major operands: one K block per stage and whole 128-column B boxes
     if (mn_operands && (var.decode || var.kps != 1 || var.block_n % 128 != 0)) continue;
-    if (var.decode && (kind != 0 || var.kps != 2 || var.block_n != 256)) continue;
+    // decode variants run one tile per CTA; several K blocks per stage: dense only
+    if (var.decode || (var.kps != 1 && kind != 0)) continue;
     const int bn = var.block_n;
     if (bn > 128 && N <= 128) continue;
     const int tm = tile_rows(var);

@@ -92,6 +92,7 @@ dg_status launch_scale_check(const GemmCall& call, int* error_word, cudaStream_t
 unsigned long long wait_timeout_ns();
 int prefetch_enabled();
 int check_scales_enabled();
+int weight_preload_enabled();
 
 // Per-form launches (one translation unit each).  `attr_set` is the caller's
 // per-device row of flags: whether the form's kernel of each variant has had

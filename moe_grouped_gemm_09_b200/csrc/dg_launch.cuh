@@ -13,26 +13,42 @@
 
 namespace dg {
 
+// Kernel mode of a variant: 0 general, 1 decode, 2 small decode.
+constexpr int mode_of(const Variant& v) { return v.small ? 2 : v.decode ? 1 : 0; }
+
 template <int V, bool SCALED = true>
 using ShapeOf = KernelShape<kVariants[V].block_n, kVariants[V].stages, kVariants[V].num_acc,
-                            kVariants[V].kps, kVariants[V].a_rows, kVariants[V].small, SCALED>;
+                            kVariants[V].kps, kVariants[V].a_rows, mode_of(kVariants[V]), SCALED>;
 
 // Kernels exist only for the (form, variant) pairs that are used: the decode
-// variants serve the dense forms, the M-/N-major and FP32-output forms take
-// the general variants with 128-column B boxes.
+// variants and the general ones with several K blocks per stage serve the
+// dense forms, the M-/N-major and FP32-output forms take the general
+// variants with 128-column B boxes.
 template <int FORM, int V>
 constexpr bool kBuilt =
     FORM == kFormDense || FORM == kFormBf16Dense ||
     ((FORM == kFormContiguous || FORM == kFormMasked || FORM == kFormBf16Contiguous ||
       FORM == kFormBf16Masked) &&
-     !kVariants[V].decode) ||
+     !kVariants[V].decode && kVariants[V].kps == 1) ||
     ((FORM >= kFormNN && FORM <= kFormF32) || FORM == kFormKGrouped) && mn_capable(kVariants[V]);
+
+// The host's view of the split-K receive region is the kernel's.
+template <int V>
+constexpr bool recv_matches() {
+  return ShapeOf<V>::kRecvBytes == decode_recv_bytes(kVariants[V]);
+}
+template <int... V>
+constexpr bool all_recv_match(std::integer_sequence<int, V...>) {
+  return (recv_matches<V>() && ...);
+}
+static_assert(all_recv_match(std::make_integer_sequence<int, kNumVariants>{}),
+              "decode_recv_bytes must mirror KernelShape::kRecvBytes");
 
 template <int FORM, int V>
 auto kernel_of() {
   constexpr Variant var = kVariants[V];
   return fp8_gemm_kernel<kind_of_form(FORM), var.block_n, var.stages, var.num_acc, var.kps,
-                         var.a_rows, var.small, layout_of_form(FORM), is_f32_form(FORM),
+                         var.a_rows, mode_of(var), layout_of_form(FORM), is_f32_form(FORM),
                          is_bf16_form(FORM)>;
 }
 

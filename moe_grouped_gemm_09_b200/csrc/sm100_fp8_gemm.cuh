@@ -32,11 +32,13 @@
 //    store.
 //  * Split-K (decode shapes, too few output tiles for the SMs): the CTAs that
 //    share an output tile form one thread-block cluster, each computes the
-//    partial sum of its K slice and parks it in its own shared memory; after
-//    a cluster barrier every CTA pushes the rows each other CTA owns to that
-//    CTA with one bulk copy (distributed shared memory), and every CTA sums
-//    the partials of its own rows in a fixed order (deterministic), then
-//    stores BF16.  No global scratch is used.
+//    partial sum of its K slice; column slice r of the tile belongs to CTA r.
+//    As soon as its accumulator is ready, every CTA pushes each other CTA's
+//    slice straight from registers into that CTA's receive region with
+//    asynchronous distributed-shared-memory stores that complete on the
+//    owner's barrier, keeps its own slice, and, once its incoming slices
+//    have landed, sums them in rank order (deterministic) and stores BF16.
+//    No global scratch is used.
 //  * Before waiting on the previous kernel (programmatic dependent launch),
 //    the producer asks TMA to prefetch its first tile's operands into L2.
 //  * A single-tile CTA (decode) drains its accumulator with all eight warps.
@@ -101,6 +103,8 @@ struct GemmArgs {
   unsigned long long timeout_ns;
   int a_box_rows;    // rows of A one TMA box brings (128, or fewer for a short dense A)
   int prefetch;      // 1: warm L2 with the first tile before waiting on the previous kernel
+  int preload_b;     // 1 (dense form): B is constant while kernels run (weights), so the
+                     // first ring stages of B may be loaded before that wait
 };
 
 constexpr int kBlockM = 128;
@@ -124,16 +128,19 @@ __host__ __device__ constexpr int pow2_ceil(int x) {
 //            and one of B, each KPS K blocks deep (bigger boxes stream faster)
 //   A_ROWS   rows of A a stage holds room for (64 for a dense A of at most 64
 //            rows, else 128)
-//   SMALL    a decode variant small enough (shared memory and TMEM) for two
-//            CTAs per SM, so that the next kernel's CTAs can start (and warm
-//            L2) while this kernel drains; it runs one tile per CTA and
-//            stages its epilogue in the then idle operand ring
+//   MODE     0: general (persistent CTAs, any number of tiles each);
+//            1: decode (dense form, one tile per CTA, split-K capable, the
+//            epilogue staged in the then idle operand ring);
+//            2: small decode, as 1 but small enough (shared memory and TMEM)
+//            for two CTAs per SM, so that the next kernel's CTAs can start
+//            (and warm L2) while this kernel drains
 //   SCALED   block-scaled E4M3 operands (scale factors staged per stage in
 //            shared memory and TMEM); false for BF16 operands, whose K block
 //            is 64 elements, the same 128 bytes of a row
-template <int BLOCK_N, int STAGES, int NUM_ACC, int KPS = 1, int A_ROWS = 128, bool SMALL = false,
+template <int BLOCK_N, int STAGES, int NUM_ACC, int KPS = 1, int A_ROWS = 128, int MODE = 0,
           bool SCALED = true>
 struct KernelShape {
+  static constexpr bool kSmall = MODE == 2;
   static constexpr int kABytes = KPS * A_ROWS * kBlockK;  // kBlockK bytes of a row per K block
   static constexpr int kBBytes = KPS * BLOCK_N * kBlockK;
   static constexpr int kSfbChunks = (BLOCK_N + 127) / 128;
@@ -156,16 +163,31 @@ struct KernelShape {
   // whole row segments
   static constexpr int kEpiCols = BLOCK_N % 64 == 0 ? 64 : 32;
   static constexpr int kEpiPitch = kEpiCols * 2;        // bytes per staged row
-  static constexpr int kEpiBytes = SMALL ? 0 : 4 * 32 * kEpiPitch;
-  // tmem slot, flags, and (grouped forms) the masked prefix
-  static constexpr int kMiscBytes = 16 + (SMALL ? 0 : 4 * (kMaxMaskedGroups + 1));
+  // Decode variants serve the dense form only and run one tile per CTA:
+  // their epilogue stages in the idle operand ring (no staging region of its
+  // own), they need no masked-group prefix, and they own a region that
+  // receives the partial sums pushed by the other CTAs of a split-K cluster.
+  static constexpr bool kDecode = MODE != 0;
+  static constexpr int kEpiBytes = kDecode ? 0 : 4 * 32 * kEpiPitch;
+  // tmem slot, flags, and (grouped forms) the masked or K-group prefix
+  static constexpr int kMiscBytes = 16 + (kDecode ? 0 : 4 * (kMaxMaskedGroups + 1));
   // A short A tile is read by the 128-row MMA past its end (rows that only
   // feed never-stored accumulator rows); the B ring follows the A ring, so
   // that read stays inside this CTA's shared memory.
-  static constexpr int kSmemBytes = 1024 /* alignment slack */ + STAGES * (kABytes + kBBytes) +
-                                    STAGES * kSfBytes + kEpiBytes + kBarBytes + kMiscBytes;
+  static constexpr int kFixedBytes = 1024 /* alignment slack */ + STAGES * (kABytes + kBBytes) +
+                                     STAGES * kSfBytes + kEpiBytes + kBarBytes + kMiscBytes;
+  // split-K receive region: what the budget leaves, at most a whole partial
+  // (A_ROWS x BLOCK_N FP32), in 16-byte units
+  static constexpr int kBudget = kSmall ? 115712 : 232448;
+  static constexpr int kRecvBytes =
+      !kDecode ? 0
+               : ((kBudget - kFixedBytes < A_ROWS * BLOCK_N * 4 ? kBudget - kFixedBytes
+                                                                : A_ROWS * BLOCK_N * 4) /
+                  16) * 16;
+  static constexpr int kSmemBytes = kFixedBytes + kRecvBytes;
+  static_assert(kRecvBytes >= 0, "receive region");
   static_assert(kSmemBytes <= 232448, "shared memory budget (227 KB) exceeded");
-  static_assert(!SMALL || (kSmemBytes <= 115712 && kTmemCols <= 256),
+  static_assert(!kSmall || (kSmemBytes <= 115712 && kTmemCols <= 256),
                 "a small variant must leave room for a second CTA on its SM");
   static_assert(STAGES * (kABytes + kBBytes) >= 8 * BLOCK_N * 64,
                 "a single-tile CTA stages its whole output tile in the ring");
@@ -341,13 +363,14 @@ struct StageWalker {
 // BF16: the same GEMM forms on BF16 operands (no scales): the ring, the tile
 // scheduler, split-K and the epilogue are shared; the scale-factor warp idles
 // and every 128-byte K block is four kind::f16 MMAs (K = 16 each).
-template <int KIND, int BLOCK_N, int STAGES, int NUM_ACC, int KPS, int A_ROWS, bool SMALL,
+template <int KIND, int BLOCK_N, int STAGES, int NUM_ACC, int KPS, int A_ROWS, int MODE,
           int LAYOUT = kLayoutNT, bool OUT_F32 = false, bool BF16 = false>
-__global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
+__global__ void __launch_bounds__(kThreads, MODE == 2 ? 2 : 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     const __grid_constant__ CUtensorMap tmap_b,
                     const __grid_constant__ CUtensorMap tmap_d, const GemmArgs p) {
-  using Shape = KernelShape<BLOCK_N, STAGES, NUM_ACC, KPS, A_ROWS, SMALL, !BF16>;
+  using Shape = KernelShape<BLOCK_N, STAGES, NUM_ACC, KPS, A_ROWS, MODE, !BF16>;
+  constexpr bool SMALL = Shape::kSmall;
   constexpr int A_BYTES = Shape::kABytes;
   constexpr int B_BYTES = Shape::kBBytes;
   constexpr int SF_BYTES = Shape::kSfBytes;
@@ -357,13 +380,8 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
   constexpr int SF_GROUP = Shape::kSfGroup;
   constexpr int ACC_COLS = Shape::kAccCols;
   constexpr int TMEM_COLS = Shape::kTmemCols;
-  constexpr int RED_PITCH = BLOCK_N + 4;  // floats per row of a parked split-K partial
-  // split-K: parked partial (valid rows) plus incoming slices (at most
-  // valid rows + split more) live in the idle operand ring; the host only
-  // picks a split for which (2 * valid rows + split) rows fit.
-  static_assert(kBlockM * RED_PITCH * 4 <= STAGES * (A_BYTES + B_BYTES),
-                "split-K partial must fit in the operand ring");
-  static_assert((KPS == 1 && !SMALL) || KIND == kDense, "decode variants serve the dense form");
+  static_assert((KPS == 1 && MODE == 0) || KIND == kDense,
+                "decode variants and several K blocks per stage: the dense form");
   // M-major A / N-major B: 2-D maps over [K, M] / [K, N] with boxes of 128
   // MN bytes x 128 K rows; one K block per stage, whole 128-row A boxes, and B
   // tiles made of whole 128-column boxes.
@@ -372,13 +390,13 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
   static_assert(!BF16 || (LAYOUT == kLayoutNT && !OUT_F32),
                 "BF16 operands: K-major A and B, BF16 output");
   // FP32 output (D = A B^T + C): the dense form, no split-K (host-checked)
-  static_assert(!OUT_F32 || ((KIND == kDense || KIND == kKGrouped) && A_ROWS == 128 && !SMALL),
+  static_assert(!OUT_F32 || ((KIND == kDense || KIND == kKGrouped) && A_ROWS == 128 && MODE == 0),
                 "FP32 output form");
   static_assert(KIND != kKGrouped || (OUT_F32 && LAYOUT == kLayoutTN),
                 "K-grouped: M-major A, N-major B, FP32 output");
   static_assert(LAYOUT == kLayoutNT ||
                     ((KIND == kDense || KIND == kKGrouped) && KPS == 1 && A_ROWS == 128 &&
-                     !SMALL && BLOCK_N % 128 == 0),
+                     MODE == 0 && BLOCK_N % 128 == 0),
                 "M-/N-major operands: dense form, general variants with 128-column B boxes");
 
   extern __shared__ uint8_t smem_raw[];
@@ -392,26 +410,39 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
   // ring, idle once that tile's MMAs are done, with one tile per warp and chunk
   const int n_tiles_total =
       (KIND == kMasked || KIND == kKGrouped) ? -1 : p.num_m_blocks * p.num_n_blocks * p.split_k;
+  // (a decode variant always runs one tile per CTA: the host launches it so)
   const bool one_tile =
-      SMALL || (n_tiles_total >= 0 && n_tiles_total <= static_cast<int>(gridDim.x));
+      Shape::kDecode || (n_tiles_total >= 0 && n_tiles_total <= static_cast<int>(gridDim.x));
   uint8_t* sEpi = one_tile ? sA : sB + STAGES * B_BYTES;
   uint8_t* sSF = sB + STAGES * B_BYTES + Shape::kEpiBytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sSF + STAGES * SF_BYTES);
+  // split-K: the slices of the partial sums the other CTAs of the cluster push
+  // to this one, [source slot][valid row][column of this CTA's slice] FP32
+  float* sRecv = reinterpret_cast<float*>(sSF + STAGES * SF_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sSF + STAGES * SF_BYTES + Shape::kRecvBytes);
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;
   uint64_t* acc_empty = acc_full + NUM_ACC;
   uint64_t* drain = acc_empty + NUM_ACC;
-  uint64_t* recv_bar = drain + 1;  // split-K: partial slices pushed by the other CTAs
+  uint64_t* recv_bar = drain + 1;  // split-K: all slices pushed to this CTA have landed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(recv_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* s_kvalid = const_cast<int*>(abort_flag + 1);  // K-grouped form: group sizes consistent
   int* s_prefix = const_cast<int*>(abort_flag + 3);  // masked and K-grouped forms
-  // split-K: this CTA's FP32 partial, parked over the (by then idle) operand ring
-  float* red = reinterpret_cast<float*>(sA);
+  // split-K: this CTA's own slice of its partial sums, kept over the (by then
+  // idle) operand ring
+  float* own = reinterpret_cast<float*>(sA);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
   const bool split = p.split_k > 1;
+  // Split-K (decode variants, one 128-row block, one output tile per cluster
+  // of split_k CTAs, CTA rank = K slice): column slice r of the tile
+  // (BLOCK_N / split_k columns) belongs to CTA r, which sums it over the
+  // cluster in rank order and stores it.
+  const int sk_rank = split ? static_cast<int>(ptx::cluster_ctarank()) : 0;
+  const int sk_cols = BLOCK_N / p.split_k;                 // columns of a slice
+  const int sk_rows = min(p.rows, kBlockM);                // valid rows (dense, one block)
+  const int sk_slot_floats = sk_rows * sk_cols;            // one source's slice
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -435,7 +466,7 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
     ptx::tmem_alloc(tmem_slot, TMEM_COLS);
     ptx::tmem_relinquish();
   }
-  if (KIND == kDense && p.prefetch && warp == 0 &&
+  if (KIND == kDense && p.prefetch && !p.preload_b && warp == 0 &&
       blockIdx.x < p.num_m_blocks * p.num_n_blocks * p.split_k) {
     // Warm L2 with this CTA's first tile while the previous kernel finishes
     // (the tile order of the dense form does not depend on device data).
@@ -458,20 +489,6 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
         }
       }
     }
-    if constexpr (!BF16) {
-      // ... and the scales that tile reads (one line holds 32 K blocks of a
-      // row): the scale warp's first loads then come from L2 instead of
-      // queueing behind the operand stream in DRAM
-      const int m0 = ti.m_blk * kBlockM;
-      const int rows_here = min(kBlockM, p.rows - m0);
-      for (int r = lane; r < rows_here; r += 32)
-        for (int kb = ti.kb_begin; kb < ti.kb_end; kb += 32)
-          ptx::prefetch_l2(p.sfa + (size_t)(m0 + r) * p.k_blocks + kb);
-      const int b0 = ti.n_blk * BLOCK_N / 128;
-      if (lane < SFB_BLOCKS && b0 + lane < p.nb128)
-        for (int kb = ti.kb_begin; kb < ti.kb_end; kb += 32)
-          ptx::prefetch_l2(p.sfb + (size_t)(b0 + lane) * p.k_blocks + kb);
-    }
   }
   // Barriers, the abort flag and the TMEM base are published before waiting
   // on the previous kernel, so that every role starts right after the wait.
@@ -479,6 +496,15 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
   __syncthreads();
   ptx::tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
+  if (split) {
+    // this CTA expects split_k - 1 slices; the first phase of the cluster
+    // barrier publishes its initialised barriers to the other CTAs, which
+    // wait on it before their first push
+    if (threadIdx.x == 0)
+      ptx::mbar_arrive_expect_tx(recv_bar,
+                                 static_cast<uint32_t>((p.split_k - 1) * sk_slot_floats * 4));
+    ptx::cluster_arrive_release();
+  }
   // Let the next kernel start its own prologue (once every CTA of this grid
   // got here).  Everything above reads no input; the inputs may be the
   // previous kernel's outputs, so every thread waits for that kernel (a no-op
@@ -535,6 +561,24 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
   // at stage0 to D, or (split-K) FP32 into the parked partial.
   constexpr int NCH_ALL = BLOCK_N / Shape::kEpiCols;
   const CUtensorMap* dmap = &tmap_d;
+  // Split-K: four consecutive partial sums of accumulator row `row`, columns
+  // c..c+3 of the tile, go to the CTA owning their column slice: into this
+  // CTA's own slice kept in the ring, or pushed into the owner's receive
+  // region (source slot: this CTA's rank, skipping the owner's own), landing
+  // on the owner's receive barrier.
+  auto split_put = [&](int row, int c, float4 v) {
+    const int owner = c / sk_cols;
+    const int col = c - owner * sk_cols;
+    if (owner == sk_rank) {
+      *reinterpret_cast<float4*>(own + row * sk_cols + col) = v;
+    } else {
+      const int slot = sk_rank < owner ? sk_rank : sk_rank - 1;
+      const uint32_t dst =
+          ptx::smem_addr(sRecv + (size_t)slot * sk_slot_floats + row * sk_cols + col);
+      ptx::st_async_v4(ptx::map_shared_rank(dst, owner), v,
+                       ptx::map_shared_rank(ptx::smem_addr(recv_bar), owner));
+    }
+  };
   auto drain_acc = [&](const Tile& ti, int a, int q, int c_begin, int c_end, uint8_t* stage0,
                        bool report) {
     // which output row this thread owns, and whether it may be written
@@ -578,34 +622,52 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
           ptx::tc_ld_32x32b_x32(t_row + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[CH - 32]));
         ptx::tc_wait_ld();
         if constexpr (OUT_F32) {
-          // FP32 output: each lane writes its own row's CH floats (whole
-          // 128-byte lines), adding C's if given (C may be D itself: every
-          // element is read and written by the same thread)
-          if (valid) {
-            const size_t off = grow * p.N + n0 + c0;
+          // FP32 output, in boxes of 32 rows x 32 columns: each lane adds its
+          // row's C values if given (C may be D itself: every element is read
+          // by the thread that stages it, before its box is stored), stages
+          // the row's 128 bytes in the warp's swizzled tile, and one TMA
+          // store writes the box (the tensor map is [groups][rows][N], so
+          // rows past a group's end and columns past N are clipped).
+          const size_t off = grow * p.N + n0 + c0;
+          const int grp = (KIND == kKGrouped) ? ti.group : 0;
 #pragma unroll
-            for (int j = 0; j < CH / 4; ++j) {
-              if (n0 + c0 + 4 * j >= p.N) break;
-              float4 v = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
-                                     __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
-              if (p.c_f32) {
-                const float4 cv = *reinterpret_cast<const float4*>(p.c_f32 + off + 4 * j);
-                v.x += cv.x; v.y += cv.y; v.z += cv.z; v.w += cv.w;
+          for (int hh = 0; hh < CH / 32; ++hh) {
+            float* v = reinterpret_cast<float*>(&r[32 * hh]);
+            if (p.c_f32 && valid) {
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                if (n0 + c0 + 32 * hh + 4 * j >= p.N) break;
+                const float4 cv =
+                    *reinterpret_cast<const float4*>(p.c_f32 + off + 32 * hh + 4 * j);
+                v[4 * j] += cv.x; v[4 * j + 1] += cv.y; v[4 * j + 2] += cv.z; v[4 * j + 3] += cv.w;
               }
-              *reinterpret_cast<float4*>(p.d_f32 + off + 4 * j) = v;
             }
+            uint8_t* stage = stage0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              *reinterpret_cast<float4*>(stage + lane * 128 + 16 * (j ^ (lane % 8))) =
+                  make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+            ptx::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              ptx::tma_store_3d(dmap, stage, n0 + c0 + 32 * hh,
+                                ti.m_blk * kBlockM + 32 * q, grp);
+              ptx::bulk_commit_group();
+              ptx::bulk_wait_group_read0();  // staging tile free again
+            }
+            __syncwarp();
           }
           continue;
         }
         uint8_t* stage = one_tile ? stage0 + ((c0 - c_begin) / CH) * 32 * Shape::kEpiPitch : stage0;
         if (split) {
-          // park the FP32 partial; the cluster reduces it below
+          // each column slice of the FP32 partial to the CTA that owns it
           if (valid) {
 #pragma unroll
             for (int j = 0; j < CH / 4; ++j)
-              *reinterpret_cast<float4*>(red + row_local * RED_PITCH + c0 + 4 * j) =
-                  make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
-                              __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+              split_put(row_local, c0 + 4 * j,
+                        make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                    __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3])));
           }
           continue;
         }
@@ -652,7 +714,6 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
         }
         __syncwarp();
       }
-      if (split) ptx::fence_proxy_async_smem();  // parked rows are read by bulk copies
     }
   };
   // A single-tile CTA's warps 0-3 are idle once their roles end: they drain
@@ -661,40 +722,66 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer --
+    // One box of A and one of B per stage, each KPS K blocks deep (blocks
+    // past K are zero-filled and still counted).  A short dense A (fewer than
+    // 128 rows) is fetched with a box of only its rows; the 128-row MMA then
+    // reads stale shared memory for the other rows, which only feeds
+    // accumulator rows that are never stored.
+    auto load_a = [&](int s, const Tile& ti, int kb) {
+      if constexpr (A_MN) {
+        ptx::tma_load_2d(sA + s * A_BYTES, &tmap_a, &full[s], ti.m_blk * kBlockM, kb * kBlockK);
+      } else {
+        ptx::tma_load_4d(sA + s * A_BYTES, &tmap_a, &full[s], 0, ti.m_blk * kBlockM, kb,
+                         (KIND == kMasked) ? ti.group : 0);
+      }
+    };
+    auto load_b = [&](int s, const Tile& ti, int kb) {
+      if constexpr (B_MN) {
+        // 128-column blocks of the tile, 128 x 128 bytes each
+#pragma unroll
+        for (int h = 0; h < BLOCK_N / 128; ++h)
+          ptx::tma_load_2d(sB + s * B_BYTES + h * 128 * kBlockK, &tmap_b, &full[s],
+                           ti.n_blk * BLOCK_N + 128 * h, kb * kBlockK);
+      } else {
+        ptx::tma_load_4d(sB + s * B_BYTES, &tmap_b, &full[s], 0, ti.n_blk * BLOCK_N, kb,
+                         ti.group);
+      }
+    };
+    const uint32_t stage_bytes = KPS * (p.a_box_rows + BLOCK_N) * kBlockK;
     int it = 0;
     bool ok = true;
+    // Weight preload (dense form, on request): B does not change while
+    // kernels run, so the first ring stages' B boxes go out before the wait on
+    // the previous kernel (whose outputs A may be); their A boxes follow the
+    // wait.  The ring is fresh, so those stages' slots are free.
+    int preloaded = 0;
+    if (kLateWait && p.preload_b && static_cast<int>(blockIdx.x) < total) {
+      const Tile ti = get_tile<KIND>(blockIdx.x, p, s_prefix, lane);
+      if (!ti.skip && lane == 0) {
+        for (int kb = ti.kb_begin; kb < ti.kb_end && preloaded < STAGES; kb += KPS, ++preloaded) {
+          ptx::mbar_arrive_expect_tx(&full[preloaded], stage_bytes);
+          load_b(preloaded, ti, kb);
+        }
+      }
+      preloaded = __shfl_sync(0xFFFFFFFFu, preloaded, 0);
+    }
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
       const Tile ti = get_tile<KIND>(t, p, s_prefix, lane);
       if (ti.skip) continue;
-      const int a_row = ti.m_blk * kBlockM;
-      const int a_grp = (KIND == kMasked) ? ti.group : 0;
       for (int kb = ti.kb_begin; kb < ti.kb_end; kb += KPS, ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
         if (lane == 0) {
-          ok = ptx::mbar_wait(&empty[s], ph ^ 1, ctl, kDevTimeoutProducer);
-          if (ok) {
-            // One box of A and one of B, each KPS K blocks deep (blocks past K
-            // are zero-filled and still counted).  A short dense A (fewer
-            // than 128 rows) is fetched with a box of only its rows; the
-            // 128-row MMA then reads stale shared memory for the other rows,
-            // which only feeds accumulator rows that are never stored.
-            ptx::mbar_arrive_expect_tx(&full[s], KPS * (p.a_box_rows + BLOCK_N) * kBlockK);
-            if (kLateWait && it == 0) ptx::grid_dependency_wait();
-            if constexpr (A_MN) {
-              ptx::tma_load_2d(sA + s * A_BYTES, &tmap_a, &full[s], a_row, kb * kBlockK);
-            } else {
-              ptx::tma_load_4d(sA + s * A_BYTES, &tmap_a, &full[s], 0, a_row, kb, a_grp);
-            }
-            if constexpr (B_MN) {
-              // 128-column blocks of the tile, 128 x 128 bytes each
-#pragma unroll
-              for (int h = 0; h < BLOCK_N / 128; ++h)
-                ptx::tma_load_2d(sB + s * B_BYTES + h * 128 * kBlockK, &tmap_b, &full[s],
-                                 ti.n_blk * BLOCK_N + 128 * h, kb * kBlockK);
-            } else {
-              ptx::tma_load_4d(sB + s * B_BYTES, &tmap_b, &full[s], 0, ti.n_blk * BLOCK_N, kb,
-                               ti.group);
+          if (it < preloaded) {
+            if (it == 0) ptx::grid_dependency_wait();
+            load_a(s, ti, kb);  // its B box and barrier bytes went out before the wait
+          } else {
+            ok = ptx::mbar_wait(&empty[s], ph ^ 1, ctl, kDevTimeoutProducer);
+            if (ok) {
+              ptx::mbar_arrive_expect_tx(&full[s], stage_bytes);
+              if (kLateWait && it == 0) ptx::grid_dependency_wait();
+              load_a(s, ti, kb);
+              load_b(s, ti, kb);
             }
           }
         }
@@ -1062,6 +1149,9 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
   } else if (warp >= 4) {
     // --------------------------------------------------------- epilogue --
     if constexpr (kLateWait) ptx::grid_dependency_wait();
+    // split-K: every CTA of the cluster has initialised its barriers (first
+    // phase of the cluster barrier) before this warp pushes to any of them
+    if (split) ptx::cluster_wait();
     const int q = warp & 3;                // TMEM lane quarter of this warp
     const int row_local = 32 * q + lane;   // accumulator row = TMEM lane
     const int ep_tid = threadIdx.x - 128;  // 0..127
@@ -1084,13 +1174,9 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
             }
           }
         }
-        if (split) {
+        if (split && row_local < sk_rows) {
           // an empty K slice still contributes (zeros) to the cluster's sum
-          const int valid_rows = min(p.rows - ti.m_blk * kBlockM, kBlockM);
-          if (row_local < valid_rows)
-            for (int c = 0; c < BLOCK_N; c += 4)
-              *reinterpret_cast<float4*>(red + row_local * RED_PITCH + c) = make_float4(0, 0, 0, 0);
-          ptx::fence_proxy_async_smem();  // parked rows are read by bulk copies
+          for (int c = 0; c < BLOCK_N; c += 4) split_put(row_local, c, make_float4(0, 0, 0, 0));
         }
         continue;
       }
@@ -1142,76 +1228,56 @@ __global__ void __launch_bounds__(kThreads, SMALL ? 2 : 1)
   if (split) {
     // ---------------------------------------- split-K cluster reduction --
     // One output tile per cluster, one K slice per CTA (rank = slice).  The
-    // tile's valid rows are cut into one slice per CTA; every CTA pushes the
-    // rows of each other CTA's slice of its parked partial to that CTA with
-    // one bulk copy (distributed shared memory), then sums the partials of
-    // its own slice in rank order and stores BF16.
-    const int S = p.split_k;
-    const uint32_t rank = ptx::cluster_ctarank();
-    const Tile ti = get_tile<KIND>(blockIdx.x, p, s_prefix, lane);
-    const int valid_rows = min(p.rows - ti.m_blk * kBlockM, kBlockM);
-    const int rows_per = (valid_rows + S - 1) / S;
-    auto slice_rows = [&](int r) { return max(0, min(valid_rows, (r + 1) * rows_per) - r * rows_per); };
-    // incoming slices land after the parked rows: slot `src` holds CTA src's rows
-    float* recv = red + valid_rows * RED_PITCH;
-    static_assert(RED_PITCH % 4 == 0, "16-byte rows");
-    __syncwarp();
-    ptx::cluster_sync();  // every CTA has parked its partial and is done with its ring
-    if (threadIdx.x == 0) {
-      const uint32_t mine = static_cast<uint32_t>(slice_rows(rank) * RED_PITCH * 4);
-      ptx::mbar_arrive_expect_tx(recv_bar, (S - 1) * mine);
-      const uint32_t bar_local = ptx::smem_addr(recv_bar);
-      const uint32_t slot_local = ptx::smem_addr(recv + rank * rows_per * RED_PITCH);
-      for (int dst = 0; dst < S; ++dst) {
-        const int n_rows = slice_rows(dst);
-        if (dst == static_cast<int>(rank) || n_rows == 0) continue;
-        ptx::bulk_copy_to_peer(ptx::map_shared_rank(slot_local, dst),
-                               red + dst * rows_per * RED_PITCH,
-                               static_cast<uint32_t>(n_rows * RED_PITCH * 4),
-                               ptx::map_shared_rank(bar_local, dst));
+    // epilogue has kept this CTA's column slice of its partial sums and
+    // pushed every other slice to the CTA that owns it; once the slices the
+    // other CTAs pushed here have landed, each epilogue thread sums its row
+    // of this CTA's slice over the cluster in rank order (deterministic) and
+    // stores it as BF16.
+    if (warp >= 4) {
+      const int row = threadIdx.x - 128;  // accumulator row of this thread
+      bool ok = !*abort_flag;
+      if (ok) {
+        ok = ptx::mbar_wait<true>(recv_bar, 0, ctl, kDevTimeoutEpilogue);
+      } else {
+        // after an abort, still let the slices the other CTAs pushed land
+        // (briefly) before this CTA can leave
+        ptx::mbar_wait_drain(recv_bar, 0, 20000000ull);
       }
-      ptx::bulk_commit_group();
-    }
-    {
-      __syncwarp();
-      bool ok = true;
-      if (lane == 0) ok = ptx::mbar_wait(recv_bar, 0, ctl, kDevTimeoutEpilogue);
-      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-      // every copy into this CTA has landed: the cluster barrier that keeps
-      // CTAs alive for incoming copies can complete while this CTA reduces
-      ptx::cluster_arrive_relaxed();
-      const int r0 = rank * rows_per;
-      constexpr int C8 = BLOCK_N / 8;
-      const int items = ok ? slice_rows(rank) * C8 : 0;
-      const int n0 = ti.n_blk * BLOCK_N;
-      for (int item = threadIdx.x; item < items; item += kThreads) {
-        const int lr = item / C8;  // row within the slice
-        const int c = 8 * (item % C8);
-        if (n0 + c >= p.N) continue;
-        float4 lo = make_float4(0, 0, 0, 0), hi = make_float4(0, 0, 0, 0);
+      const Tile ti = get_tile<KIND>(blockIdx.x, p, s_prefix, lane);
+      const int n0 = ti.n_blk * BLOCK_N + sk_rank * sk_cols;
+      if (ok && row < sk_rows) {
+        for (int c = 0; c < sk_cols; c += 8) {
+          if (n0 + c >= p.N) break;
+          float4 lo = make_float4(0, 0, 0, 0), hi = make_float4(0, 0, 0, 0);
 #pragma unroll
-        for (int src = 0; src < kMaxSplit; ++src) {  // fixed order: deterministic
-          if (src >= S) break;
-          const float* part = (src == static_cast<int>(rank))
-                                  ? red + (r0 + lr) * RED_PITCH + c
-                                  : recv + (src * rows_per + lr) * RED_PITCH + c;
-          const float4 x = *reinterpret_cast<const float4*>(part);
-          const float4 y = *reinterpret_cast<const float4*>(part + 4);
-          lo.x += x.x; lo.y += x.y; lo.z += x.z; lo.w += x.w;
-          hi.x += y.x; hi.y += y.y; hi.z += y.z; hi.w += y.w;
+          for (int src = 0; src < kMaxSplit; ++src) {  // fixed order: deterministic
+            if (src >= p.split_k) break;
+            const int slot = src < sk_rank ? src : src - 1;
+            const float* part = (src == sk_rank)
+                                    ? own + row * sk_cols + c
+                                    : sRecv + (size_t)slot * sk_slot_floats + row * sk_cols + c;
+            const float4 x = *reinterpret_cast<const float4*>(part);
+            const float4 y = *reinterpret_cast<const float4*>(part + 4);
+            lo.x += x.x; lo.y += x.y; lo.z += x.z; lo.w += x.w;
+            hi.x += y.x; hi.y += y.y; hi.z += y.z; hi.w += y.w;
+          }
+          uint4 v;
+          v.x = pack_bf16x2(lo.x, lo.y);
+          v.y = pack_bf16x2(lo.z, lo.w);
+          v.z = pack_bf16x2(hi.x, hi.y);
+          v.w = pack_bf16x2(hi.z, hi.w);
+          *reinterpret_cast<uint4*>(p.d + (size_t)row * p.N + n0 + c) = v;
         }
-        uint4 v;
-        v.x = pack_bf16x2(lo.x, lo.y);
-        v.y = pack_bf16x2(lo.z, lo.w);
-        v.z = pack_bf16x2(hi.x, hi.y);
-        v.w = pack_bf16x2(hi.z, hi.w);
-        const size_t grow = (size_t)ti.m_blk * kBlockM + r0 + lr;
-        *reinterpret_cast<uint4*>(p.d + grow * p.N + n0 + c) = v;
       }
+    } else {
+      // the first phase of the cluster barrier, for the threads that push nothing
+      ptx::cluster_wait();
     }
-    if (threadIdx.x == 0) ptx::bulk_wait_group_read0();  // outgoing copies done reading
-    __syncwarp();
-    ptx::cluster_wait();  // no CTA leaves while a copy into it may still land
+    // Second phase: this CTA needs nothing more from the others (its incoming
+    // slices have landed, or it gave up); no CTA leaves while a slice may
+    // still be on its way into it.
+    ptx::cluster_arrive_relaxed();
+    ptx::cluster_wait();
   }
 
   ptx::tc_fence_before_sync();

@@ -177,18 +177,6 @@ __device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* map, int c
       : "memory");
 }
 
-// Bring `bytes` contiguous bytes at `p` (16-byte aligned, a multiple of 16)
-// into L2 with one bulk request (no completion to wait for).
-__device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
-
-// Bring the 128-byte line holding `p` into L2 (no completion to wait for).
-// Safe before a dependency wait for the same reason as the TMA prefetches.
-__device__ __forceinline__ void prefetch_l2(const void* p) {
-  asm volatile("prefetch.global.L2 [%0];" ::"l"(p) : "memory");
-}
-
 // ------------------------------------------------------------------ cluster --
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
@@ -217,6 +205,9 @@ __device__ __forceinline__ void grid_dependency_wait() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
+__device__ __forceinline__ void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
 __device__ __forceinline__ void cluster_arrive_relaxed() {
   asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 }
@@ -240,6 +231,17 @@ __device__ __forceinline__ float4 ld_shared_cluster_f4(uint32_t addr) {
   return v;
 }
 
+// Asynchronous 16-byte store into the shared memory of a CTA of the cluster
+// (`dst_cluster` and `bar_cluster` from map_shared_rank): completes 16
+// transaction bytes on that CTA's mbarrier once the data has landed.
+__device__ __forceinline__ void st_async_v4(uint32_t dst_cluster, float4 v, uint32_t bar_cluster) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+          dst_cluster),
+      "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(bar_cluster)
+      : "memory");
+}
+
 // Bulk copy of `bytes` (multiple of 16, 16-byte aligned) from this CTA's
 // shared memory into the shared memory of another CTA of the cluster
 // (`dst_cluster`, an address from map_shared_rank), completing on that CTA's
@@ -260,6 +262,16 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void*
       "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
           reinterpret_cast<uint64_t>(map)),
       "r"(smem_addr(src)), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+// 3-D tiled store of one box from shared memory to global memory (bulk group).
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int c0,
+                                             int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(smem_addr(src)), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
 }
 

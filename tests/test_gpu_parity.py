@@ -108,7 +108,7 @@ def test_dense_scales_not_16_byte_aligned(dg):
 # Every general variant, forced, on one ragged shape with a random power-of-two
 # scale per A row and per B block (the picker would choose only some of them
 # for this shape).
-FORCED_GENERAL = ["256:1", "128:1", "64:1", "32:1"]
+FORCED_GENERAL = ["256:1", "128:1", "64:1", "32:1", "256:1:2:128:0"]
 
 
 @pytest.mark.parametrize("cfg", FORCED_GENERAL)
@@ -124,14 +124,15 @@ def test_dense_forced_variant(dg, cfg, monkeypatch):
     check_close(got, ref, f"forced {cfg}")
 
 
-# Every decode variant ("block_n:split_k:kps:a_rows:small"), forced, with and
+# Every decode variant ("block_n:split_k:kps:a_rows:mode", mode 1 decode, 2
+# small decode), forced, with and
 # without split-K clusters, on a short A (one 128-row block) with a ragged N
 # and random power-of-two scales per A row and per B block.
 FORCED_DECODE = [
-    (100, "128:1:2:128:0"), (100, "128:4:2:128:0"), (100, "64:2:2:128:0"), (100, "64:8:2:128:0"),
-    (64, "256:2:2:128:0"), (100, "128:1:1:128:1"), (100, "64:4:2:128:1"),
-    (64, "128:1:4:64:0"), (64, "128:4:4:64:0"), (40, "64:8:4:64:0"), (64, "256:2:2:64:0"),
-    (64, "128:8:2:64:1"), (17, "64:2:2:64:1"),
+    (100, "128:1:2:128:1"), (64, "128:4:2:128:1"), (100, "64:2:2:128:1"), (100, "64:8:2:128:1"),
+    (128, "64:4:2:128:1"), (64, "256:2:2:64:1"), (64, "256:8:2:64:1"), (100, "128:1:1:128:2"),
+    (40, "64:4:2:128:2"), (64, "128:1:4:64:1"), (64, "128:8:4:64:1"), (40, "64:8:4:64:1"),
+    (48, "128:2:2:64:2"), (17, "64:2:2:64:2"),
 ]
 
 
@@ -429,3 +430,33 @@ def test_scale_contract_check(dg, M, N, K):
     dg.fp8_gemm_nt(a, dev(bad_sfa), b, dev(bad_sfb), sentinel_like((M, N)))
     torch.cuda.synchronize()
     assert dg.get_last_device_error() == 0
+
+
+@pytest.mark.parametrize("M,N,K", workloads.DECODE_SHAPES + [(300, 400, 1024), (4096, 2112, 1024)])
+def test_weight_preload_gives_the_same_results(dg, M, N, K):
+    """With the weight preload on (B loaded before the wait on the previous
+    kernel), every decode shape (split-K clusters included) and persistent
+    tiles give bit-identical results to the preload off, and match the
+    oracle."""
+    p = workloads.dense_problem(M, N, K, seed=15)
+    try:
+        dg.set_weight_preload(True)
+        on = run_dense(dg, p)
+    finally:
+        dg.set_weight_preload(False)
+    off = run_dense(dg, p)
+    assert np.array_equal(on, off)
+    ref, _ = oracle.default().gemm_nt(p.a, p.sfa, p.b, p.sfb, want_acc=False)
+    check_close(on, ref, f"preload {M}x{N}x{K}")
+
+
+@pytest.mark.parametrize("M,N,K", [(64, 2112, 1024), (512, 384, 512)])
+def test_dependent_launches_with_weight_preload(dg, M, N, K):
+    """The graph of four dependent in-place FP32 accumulations with the
+    weight preload on: B is loaded early, but each launch still reads the D
+    the previous one wrote only after that launch has finished."""
+    try:
+        dg.set_weight_preload(True)
+        test_dependent_launches_in_a_graph(dg, M, N, K)
+    finally:
+        dg.set_weight_preload(False)

@@ -35,9 +35,10 @@ def dg():
     lib.set_wait_timeout_ns(DEFAULT_LIMIT_NS)
 
 
-# (force config "block_n:split_k:kps:a_rows:small", M, N, K): one output tile,
-# so one CTA without split and a cluster of two CTAs with split 2
-CASES = [("64:1:2:128:0", 64, 64, 16384), ("64:2:2:128:0", 64, 64, 16384)]
+# (force config "block_n:split_k:kps:a_rows:mode", M, N, K): one output tile of
+# a decode variant, so one CTA without split and a cluster of two CTAs with
+# split 2
+CASES = [("64:1:2:128:1", 64, 64, 16384), ("64:2:2:128:1", 64, 64, 16384)]
 
 
 @pytest.mark.parametrize("cfg,M,N,K", CASES)
