@@ -73,32 +73,13 @@ inline int cluster_limit(const ClusterLimits* lim, int v, int s, int num_sms) {
   return n > 0 ? n : num_sms / s;
 }
 
-// Bytes of a decode variant's split-K receive region (E4M3 operands): the
-// shared-memory budget (227 KB, or 113 KB for a small variant) less the ring,
-// the scale-factor slots, the barriers and 16 bytes of flags (plus 1 KB of
-// alignment slack), capped at a whole A_ROWS x BLOCK_N FP32 partial.  The
-// kernel's own geometry (KernelShape::kRecvBytes) is checked against this at
-// compile time.
-constexpr int decode_recv_bytes(const Variant& v) {
-  if (!v.decode) return 0;
-  const int sf = 512 * (1 + (v.block_n + 127) / 128);
-  const int fixed = 1024 + v.stages * (v.kps * (v.a_rows + v.block_n) * 128 + sf) +
-                    8 * (2 * v.stages + 2 * v.num_acc + 2) + 16;
-  const int budget = (v.small ? 115712 : 232448) - fixed;
-  const int whole = v.a_rows * v.block_n * 4;
-  return ((budget < whole ? budget : whole) / 16) * 16;
-}
-
-// Split-K: column slice c of the tile belongs to CTA c of the cluster; every
-// CTA pushes each other CTA's slice of its valid rows into that CTA's receive
-// region, which must hold split - 1 slices of rows x BLOCK_N / split FP32;
-// slices are whole 16-byte BF16 groups (BLOCK_N / split a multiple of 8).
+// Split-K parks each CTA's FP32 partial and the slices the other CTAs push to
+// it in the (then idle) operand ring: (2 * rows + split) rows of BLOCK_N + 4
+// floats must fit.
 inline bool split_fits(const Variant& var, int rows, int split) {
-  if (split < 2) return true;
-  if (var.block_n % (8 * split) != 0) return false;
-  const long long need =
-      static_cast<long long>(split - 1) * rows * (var.block_n / split) * 4;
-  return need <= decode_recv_bytes(var);
+  const long long ring = static_cast<long long>(var.stages) * var.kps * (var.a_rows + var.block_n) * 128;
+  const long long need = static_cast<long long>(2 * rows + split) * (var.block_n + 4) * 4;
+  return need <= ring;
 }
 
 // Decode-shaped dense problems (at most one 128-row block): HBM-bound.  Pick

@@ -32,18 +32,6 @@ constexpr bool kBuilt =
      !kVariants[V].decode && kVariants[V].kps == 1) ||
     ((FORM >= kFormNN && FORM <= kFormF32) || FORM == kFormKGrouped) && mn_capable(kVariants[V]);
 
-// The host's view of the split-K receive region is the kernel's.
-template <int V>
-constexpr bool recv_matches() {
-  return ShapeOf<V>::kRecvBytes == decode_recv_bytes(kVariants[V]);
-}
-template <int... V>
-constexpr bool all_recv_match(std::integer_sequence<int, V...>) {
-  return (recv_matches<V>() && ...);
-}
-static_assert(all_recv_match(std::make_integer_sequence<int, kNumVariants>{}),
-              "decode_recv_bytes must mirror KernelShape::kRecvBytes");
-
 template <int FORM, int V>
 auto kernel_of() {
   constexpr Variant var = kVariants[V];

@@ -32,13 +32,11 @@
 //    store.
 //  * Split-K (decode shapes, too few output tiles for the SMs): the CTAs that
 //    share an output tile form one thread-block cluster, each computes the
-//    partial sum of its K slice; column slice r of the tile belongs to CTA r.
-//    As soon as its accumulator is ready, every CTA pushes each other CTA's
-//    slice straight from registers into that CTA's receive region with
-//    asynchronous distributed-shared-memory stores that complete on the
-//    owner's barrier, keeps its own slice, and, once its incoming slices
-//    have landed, sums them in rank order (deterministic) and stores BF16.
-//    No global scratch is used.
+//    partial sum of its K slice and parks it in its own shared memory; after
+//    a cluster barrier every CTA pushes the rows each other CTA owns to that
+//    CTA with one bulk copy (distributed shared memory), and every CTA sums
+//    the partials of its own rows in a fixed order (deterministic), then
+//    stores BF16.  No global scratch is used.
 //  * Before waiting on the previous kernel (programmatic dependent launch),
 //    the producer asks TMA to prefetch its first tile's operands into L2.
 //  * A single-tile CTA (decode) drains its accumulator with all eight warps.
@@ -165,8 +163,7 @@ struct KernelShape {
   static constexpr int kEpiPitch = kEpiCols * 2;        // bytes per staged row
   // Decode variants serve the dense form only and run one tile per CTA:
   // their epilogue stages in the idle operand ring (no staging region of its
-  // own), they need no masked-group prefix, and they own a region that
-  // receives the partial sums pushed by the other CTAs of a split-K cluster.
+  // own) and they need no masked-group prefix.
   static constexpr bool kDecode = MODE != 0;
   static constexpr int kEpiBytes = kDecode ? 0 : 4 * 32 * kEpiPitch;
   // tmem slot, flags, and (grouped forms) the masked or K-group prefix
@@ -174,18 +171,8 @@ struct KernelShape {
   // A short A tile is read by the 128-row MMA past its end (rows that only
   // feed never-stored accumulator rows); the B ring follows the A ring, so
   // that read stays inside this CTA's shared memory.
-  static constexpr int kFixedBytes = 1024 /* alignment slack */ + STAGES * (kABytes + kBBytes) +
-                                     STAGES * kSfBytes + kEpiBytes + kBarBytes + kMiscBytes;
-  // split-K receive region: what the budget leaves, at most a whole partial
-  // (A_ROWS x BLOCK_N FP32), in 16-byte units
-  static constexpr int kBudget = kSmall ? 115712 : 232448;
-  static constexpr int kRecvBytes =
-      !kDecode ? 0
-               : ((kBudget - kFixedBytes < A_ROWS * BLOCK_N * 4 ? kBudget - kFixedBytes
-                                                                : A_ROWS * BLOCK_N * 4) /
-                  16) * 16;
-  static constexpr int kSmemBytes = kFixedBytes + kRecvBytes;
-  static_assert(kRecvBytes >= 0, "receive region");
+  static constexpr int kSmemBytes = 1024 /* alignment slack */ + STAGES * (kABytes + kBBytes) +
+                                    STAGES * kSfBytes + kEpiBytes + kBarBytes + kMiscBytes;
   static_assert(kSmemBytes <= 232448, "shared memory budget (227 KB) exceeded");
   static_assert(!kSmall || (kSmemBytes <= 115712 && kTmemCols <= 256),
                 "a small variant must leave room for a second CTA on its SM");
@@ -415,34 +402,28 @@ __global__ void __launch_bounds__(kThreads, MODE == 2 ? 2 : 1)
       Shape::kDecode || (n_tiles_total >= 0 && n_tiles_total <= static_cast<int>(gridDim.x));
   uint8_t* sEpi = one_tile ? sA : sB + STAGES * B_BYTES;
   uint8_t* sSF = sB + STAGES * B_BYTES + Shape::kEpiBytes;
-  // split-K: the slices of the partial sums the other CTAs of the cluster push
-  // to this one, [source slot][valid row][column of this CTA's slice] FP32
-  float* sRecv = reinterpret_cast<float*>(sSF + STAGES * SF_BYTES);
-  uint64_t* full = reinterpret_cast<uint64_t*>(sSF + STAGES * SF_BYTES + Shape::kRecvBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sSF + STAGES * SF_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;
   uint64_t* acc_empty = acc_full + NUM_ACC;
   uint64_t* drain = acc_empty + NUM_ACC;
-  uint64_t* recv_bar = drain + 1;  // split-K: all slices pushed to this CTA have landed
+  uint64_t* recv_bar = drain + 1;  // split-K: partial slices pushed by the other CTAs
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(recv_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* s_kvalid = const_cast<int*>(abort_flag + 1);  // K-grouped form: group sizes consistent
   int* s_prefix = const_cast<int*>(abort_flag + 3);  // masked and K-grouped forms
-  // split-K: this CTA's own slice of its partial sums, kept over the (by then
-  // idle) operand ring
-  float* own = reinterpret_cast<float*>(sA);
+  // split-K: this CTA's FP32 partial, parked over the (by then idle) operand ring
+  constexpr int RED_PITCH = BLOCK_N + 4;  // floats per row of a parked split-K partial
+  // split-K: parked partial (valid rows) plus incoming slices (at most
+  // valid rows + split more) live in the idle operand ring; the host only
+  // picks a split for which (2 * valid rows + split) rows fit.
+  static_assert(kBlockM * RED_PITCH * 4 <= STAGES * (A_BYTES + B_BYTES),
+                "split-K partial must fit in the operand ring");
+  float* red = reinterpret_cast<float*>(sA);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
   const bool split = p.split_k > 1;
-  // Split-K (decode variants, one 128-row block, one output tile per cluster
-  // of split_k CTAs, CTA rank = K slice): column slice r of the tile
-  // (BLOCK_N / split_k columns) belongs to CTA r, which sums it over the
-  // cluster in rank order and stores it.
-  const int sk_rank = split ? static_cast<int>(ptx::cluster_ctarank()) : 0;
-  const int sk_cols = BLOCK_N / p.split_k;                 // columns of a slice
-  const int sk_rows = min(p.rows, kBlockM);                // valid rows (dense, one block)
-  const int sk_slot_floats = sk_rows * sk_cols;            // one source's slice
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -496,15 +477,6 @@ __global__ void __launch_bounds__(kThreads, MODE == 2 ? 2 : 1)
   __syncthreads();
   ptx::tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
-  if (split) {
-    // this CTA expects split_k - 1 slices; the first phase of the cluster
-    // barrier publishes its initialised barriers to the other CTAs, which
-    // wait on it before their first push
-    if (threadIdx.x == 0)
-      ptx::mbar_arrive_expect_tx(recv_bar,
-                                 static_cast<uint32_t>((p.split_k - 1) * sk_slot_floats * 4));
-    ptx::cluster_arrive_release();
-  }
   // Let the next kernel start its own prologue (once every CTA of this grid
   // got here).  Everything above reads no input; the inputs may be the
   // previous kernel's outputs, so every thread waits for that kernel (a no-op
@@ -561,24 +533,6 @@ __global__ void __launch_bounds__(kThreads, MODE == 2 ? 2 : 1)
   // at stage0 to D, or (split-K) FP32 into the parked partial.
   constexpr int NCH_ALL = BLOCK_N / Shape::kEpiCols;
   const CUtensorMap* dmap = &tmap_d;
-  // Split-K: four consecutive partial sums of accumulator row `row`, columns
-  // c..c+3 of the tile, go to the CTA owning their column slice: into this
-  // CTA's own slice kept in the ring, or pushed into the owner's receive
-  // region (source slot: this CTA's rank, skipping the owner's own), landing
-  // on the owner's receive barrier.
-  auto split_put = [&](int row, int c, float4 v) {
-    const int owner = c / sk_cols;
-    const int col = c - owner * sk_cols;
-    if (owner == sk_rank) {
-      *reinterpret_cast<float4*>(own + row * sk_cols + col) = v;
-    } else {
-      const int slot = sk_rank < owner ? sk_rank : sk_rank - 1;
-      const uint32_t dst =
-          ptx::smem_addr(sRecv + (size_t)slot * sk_slot_floats + row * sk_cols + col);
-      ptx::st_async_v4(ptx::map_shared_rank(dst, owner), v,
-                       ptx::map_shared_rank(ptx::smem_addr(recv_bar), owner));
-    }
-  };
   auto drain_acc = [&](const Tile& ti, int a, int q, int c_begin, int c_end, uint8_t* stage0,
                        bool report) {
     // which output row this thread owns, and whether it may be written
@@ -661,13 +615,13 @@ __global__ void __launch_bounds__(kThreads, MODE == 2 ? 2 : 1)
         }
         uint8_t* stage = one_tile ? stage0 + ((c0 - c_begin) / CH) * 32 * Shape::kEpiPitch : stage0;
         if (split) {
-          // each column slice of the FP32 partial to the CTA that owns it
+          // park the FP32 partial; the cluster reduces it below
           if (valid) {
 #pragma unroll
             for (int j = 0; j < CH / 4; ++j)
-              split_put(row_local, c0 + 4 * j,
-                        make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
-                                    __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3])));
+              *reinterpret_cast<float4*>(red + row_local * RED_PITCH + c0 + 4 * j) =
+                  make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                              __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
           }
           continue;
         }
@@ -714,6 +668,7 @@ __global__ void __launch_bounds__(kThreads, MODE == 2 ? 2 : 1)
         }
         __syncwarp();
       }
+      if (split) ptx::fence_proxy_async_smem();  // parked rows are read by bulk copies
     }
   };
   // A single-tile CTA's warps 0-3 are idle once their roles end: they drain
@@ -1149,9 +1104,6 @@ __global__ void __launch_bounds__(kThreads, MODE == 2 ? 2 : 1)
   } else if (warp >= 4) {
     // --------------------------------------------------------- epilogue --
     if constexpr (kLateWait) ptx::grid_dependency_wait();
-    // split-K: every CTA of the cluster has initialised its barriers (first
-    // phase of the cluster barrier) before this warp pushes to any of them
-    if (split) ptx::cluster_wait();
     const int q = warp & 3;                // TMEM lane quarter of this warp
     const int row_local = 32 * q + lane;   // accumulator row = TMEM lane
     const int ep_tid = threadIdx.x - 128;  // 0..127
@@ -1174,9 +1126,13 @@ __global__ void __launch_bounds__(kThreads, MODE == 2 ? 2 : 1)
             }
           }
         }
-        if (split && row_local < sk_rows) {
+        if (split) {
           // an empty K slice still contributes (zeros) to the cluster's sum
-          for (int c = 0; c < BLOCK_N; c += 4) split_put(row_local, c, make_float4(0, 0, 0, 0));
+          const int valid_rows = min(p.rows - ti.m_blk * kBlockM, kBlockM);
+          if (row_local < valid_rows)
+            for (int c = 0; c < BLOCK_N; c += 4)
+              *reinterpret_cast<float4*>(red + row_local * RED_PITCH + c) = make_float4(0, 0, 0, 0);
+          ptx::fence_proxy_async_smem();  // parked rows are read by bulk copies
         }
         continue;
       }
@@ -1228,56 +1184,76 @@ __global__ void __launch_bounds__(kThreads, MODE == 2 ? 2 : 1)
   if (split) {
     // ---------------------------------------- split-K cluster reduction --
     // One output tile per cluster, one K slice per CTA (rank = slice).  The
-    // epilogue has kept this CTA's column slice of its partial sums and
-    // pushed every other slice to the CTA that owns it; once the slices the
-    // other CTAs pushed here have landed, each epilogue thread sums its row
-    // of this CTA's slice over the cluster in rank order (deterministic) and
-    // stores it as BF16.
-    if (warp >= 4) {
-      const int row = threadIdx.x - 128;  // accumulator row of this thread
-      bool ok = !*abort_flag;
-      if (ok) {
-        ok = ptx::mbar_wait<true>(recv_bar, 0, ctl, kDevTimeoutEpilogue);
-      } else {
-        // after an abort, still let the slices the other CTAs pushed land
-        // (briefly) before this CTA can leave
-        ptx::mbar_wait_drain(recv_bar, 0, 20000000ull);
+    // tile's valid rows are cut into one slice per CTA; every CTA pushes the
+    // rows of each other CTA's slice of its parked partial to that CTA with
+    // one bulk copy (distributed shared memory), then sums the partials of
+    // its own slice in rank order and stores BF16.
+    const int S = p.split_k;
+    const uint32_t rank = ptx::cluster_ctarank();
+    const Tile ti = get_tile<KIND>(blockIdx.x, p, s_prefix, lane);
+    const int valid_rows = min(p.rows - ti.m_blk * kBlockM, kBlockM);
+    const int rows_per = (valid_rows + S - 1) / S;
+    auto slice_rows = [&](int r) { return max(0, min(valid_rows, (r + 1) * rows_per) - r * rows_per); };
+    // incoming slices land after the parked rows: slot `src` holds CTA src's rows
+    float* recv = red + valid_rows * RED_PITCH;
+    static_assert(RED_PITCH % 4 == 0, "16-byte rows");
+    __syncwarp();
+    ptx::cluster_sync();  // every CTA has parked its partial and is done with its ring
+    if (threadIdx.x == 0) {
+      const uint32_t mine = static_cast<uint32_t>(slice_rows(rank) * RED_PITCH * 4);
+      ptx::mbar_arrive_expect_tx(recv_bar, (S - 1) * mine);
+      const uint32_t bar_local = ptx::smem_addr(recv_bar);
+      const uint32_t slot_local = ptx::smem_addr(recv + rank * rows_per * RED_PITCH);
+      for (int dst = 0; dst < S; ++dst) {
+        const int n_rows = slice_rows(dst);
+        if (dst == static_cast<int>(rank) || n_rows == 0) continue;
+        ptx::bulk_copy_to_peer(ptx::map_shared_rank(slot_local, dst),
+                               red + dst * rows_per * RED_PITCH,
+                               static_cast<uint32_t>(n_rows * RED_PITCH * 4),
+                               ptx::map_shared_rank(bar_local, dst));
       }
-      const Tile ti = get_tile<KIND>(blockIdx.x, p, s_prefix, lane);
-      const int n0 = ti.n_blk * BLOCK_N + sk_rank * sk_cols;
-      if (ok && row < sk_rows) {
-        for (int c = 0; c < sk_cols; c += 8) {
-          if (n0 + c >= p.N) break;
-          float4 lo = make_float4(0, 0, 0, 0), hi = make_float4(0, 0, 0, 0);
-#pragma unroll
-          for (int src = 0; src < kMaxSplit; ++src) {  // fixed order: deterministic
-            if (src >= p.split_k) break;
-            const int slot = src < sk_rank ? src : src - 1;
-            const float* part = (src == sk_rank)
-                                    ? own + row * sk_cols + c
-                                    : sRecv + (size_t)slot * sk_slot_floats + row * sk_cols + c;
-            const float4 x = *reinterpret_cast<const float4*>(part);
-            const float4 y = *reinterpret_cast<const float4*>(part + 4);
-            lo.x += x.x; lo.y += x.y; lo.z += x.z; lo.w += x.w;
-            hi.x += y.x; hi.y += y.y; hi.z += y.z; hi.w += y.w;
-          }
-          uint4 v;
-          v.x = pack_bf16x2(lo.x, lo.y);
-          v.y = pack_bf16x2(lo.z, lo.w);
-          v.z = pack_bf16x2(hi.x, hi.y);
-          v.w = pack_bf16x2(hi.z, hi.w);
-          *reinterpret_cast<uint4*>(p.d + (size_t)row * p.N + n0 + c) = v;
-        }
-      }
-    } else {
-      // the first phase of the cluster barrier, for the threads that push nothing
-      ptx::cluster_wait();
+      ptx::bulk_commit_group();
     }
-    // Second phase: this CTA needs nothing more from the others (its incoming
-    // slices have landed, or it gave up); no CTA leaves while a slice may
-    // still be on its way into it.
-    ptx::cluster_arrive_relaxed();
-    ptx::cluster_wait();
+    {
+      __syncwarp();
+      bool ok = true;
+      if (lane == 0) ok = ptx::mbar_wait(recv_bar, 0, ctl, kDevTimeoutEpilogue);
+      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+      // every copy into this CTA has landed: the cluster barrier that keeps
+      // CTAs alive for incoming copies can complete while this CTA reduces
+      ptx::cluster_arrive_relaxed();
+      const int r0 = rank * rows_per;
+      constexpr int C8 = BLOCK_N / 8;
+      const int items = ok ? slice_rows(rank) * C8 : 0;
+      const int n0 = ti.n_blk * BLOCK_N;
+      for (int item = threadIdx.x; item < items; item += kThreads) {
+        const int lr = item / C8;  // row within the slice
+        const int c = 8 * (item % C8);
+        if (n0 + c >= p.N) continue;
+        float4 lo = make_float4(0, 0, 0, 0), hi = make_float4(0, 0, 0, 0);
+#pragma unroll
+        for (int src = 0; src < kMaxSplit; ++src) {  // fixed order: deterministic
+          if (src >= S) break;
+          const float* part = (src == static_cast<int>(rank))
+                                  ? red + (r0 + lr) * RED_PITCH + c
+                                  : recv + (src * rows_per + lr) * RED_PITCH + c;
+          const float4 x = *reinterpret_cast<const float4*>(part);
+          const float4 y = *reinterpret_cast<const float4*>(part + 4);
+          lo.x += x.x; lo.y += x.y; lo.z += x.z; lo.w += x.w;
+          hi.x += y.x; hi.y += y.y; hi.z += y.z; hi.w += y.w;
+        }
+        uint4 v;
+        v.x = pack_bf16x2(lo.x, lo.y);
+        v.y = pack_bf16x2(lo.z, lo.w);
+        v.z = pack_bf16x2(hi.x, hi.y);
+        v.w = pack_bf16x2(hi.z, hi.w);
+        const size_t grow = (size_t)ti.m_blk * kBlockM + r0 + lr;
+        *reinterpret_cast<uint4*>(p.d + grow * p.N + n0 + c) = v;
+      }
+    }
+    if (threadIdx.x == 0) ptx::bulk_wait_group_read0();  // outgoing copies done reading
+    __syncwarp();
+    ptx::cluster_wait();  // no CTA leaves while a copy into it may still land
   }
 
   ptx::tc_fence_before_sync();

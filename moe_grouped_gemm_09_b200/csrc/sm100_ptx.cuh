@@ -205,9 +205,6 @@ __device__ __forceinline__ void grid_dependency_wait() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
-__device__ __forceinline__ void cluster_arrive_release() {
-  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-}
 __device__ __forceinline__ void cluster_arrive_relaxed() {
   asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 }
@@ -229,17 +226,6 @@ __device__ __forceinline__ float4 ld_shared_cluster_f4(uint32_t addr) {
                : "r"(addr)
                : "memory");
   return v;
-}
-
-// Asynchronous 16-byte store into the shared memory of a CTA of the cluster
-// (`dst_cluster` and `bar_cluster` from map_shared_rank): completes 16
-// transaction bytes on that CTA's mbarrier once the data has landed.
-__device__ __forceinline__ void st_async_v4(uint32_t dst_cluster, float4 v, uint32_t bar_cluster) {
-  asm volatile(
-      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
-          dst_cluster),
-      "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(bar_cluster)
-      : "memory");
 }
 
 // Bulk copy of `bytes` (multiple of 16, 16-byte aligned) from this CTA's
