@@ -319,6 +319,21 @@ def _operands(p):
     return {k: getattr(p, k) for k in names}
 
 
+def gemm_launches(kind: str, p) -> int:
+    """Kernel launches one GEMM call makes: 1, plus the tail launches of a
+    dense call whose last wave of tiles is split off (the library's own plan,
+    read through dg_query_config)."""
+    if kind not in ("dense", "bf16_dense"):
+        return 1
+    import moe_grouped_gemm_09_b200 as dg
+    k_bytes = p.K * (2 if kind == "bf16_dense" else 1)
+    return 1 + dg.query_config(dg.KIND_DENSE, p.M, p.N, k_bytes)["tail_launches"]
+
+
+def step_launches(items) -> int:
+    return sum(gemm_launches(k, p) for k, p in items)
+
+
 def _launcher(dg, items, sets, outs):
     def launch_one(j, r):
         (kind, p), t, d = items[j], sets[r][j], outs[j]
@@ -548,7 +563,7 @@ def workload_record(name: str, t: dict, world: int, steps: int, warmup: int) -> 
     r_unit = "GB/s" if bound == "hbm" else "TFLOP/s"
     peak = hbm_peak if bound == "hbm" else tensor_peak
     achieved = scale_units(step_units(items, r_unit), r_unit, ms / 1e3)
-    launches_per_step = len(items)
+    launches_per_step = step_launches(items)
     return {
         "metric": t["metric"],
         "value": round(whole_job_value(step_units(items, unit), world, ms, unit), 3),

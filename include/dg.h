@@ -86,7 +86,13 @@ typedef enum {
 
 /* Dense NT GEMM: D[M,N] = A[M,K] * B[N,K]^T.
  * a [M,K] E4M3, sfa [M, K/128], b [N,K] E4M3, sfb [ceil(N/128), K/128],
- * d [M,N] BF16.  M >= 0. */
+ * d [M,N] BF16.  M >= 0.
+ * Usually one kernel launch on `stream`.  When the last wave of output tiles
+ * would occupy at most half of the SMs (and K >= 4096), the call enqueues the
+ * whole waves as one launch and the remaining tiles, one or two rectangles of
+ * D, as up to two more launches of split-K tiles; dg_query_config reports the
+ * split, and DG_NO_TAIL_SPLIT=1 in the environment turns it off.  The same
+ * holds for dg_bf16_gemm_nt (K >= 2048 there) and dg_fp8_gemm_nt_noalloc. */
 dg_status dg_fp8_gemm_nt(const void* a, const float* sfa, const void* b, const float* sfb,
                          void* d, int M, int N, int K, dg_stream_t stream);
 
@@ -261,6 +267,11 @@ typedef struct {
   int smem_bytes;  /* dynamic shared memory per CTA */
   int tmem_cols;   /* TMEM columns allocated per CTA */
   int kps;         /* 128-wide K blocks per ring stage */
+  int main_tiles;  /* dense form: tiles of the first launch when the last wave
+                      is split off (0: one launch) */
+  int tail_launches; /* launches of 128 x 128 decode tiles after the first (0..2):
+                        the tiles past main_tiles, one rectangle of D each */
+  int tail_split;  /* K slices (CTAs per cluster) of the tail launches' tiles */
 } dg_config;
 
 dg_status dg_query_config(int kind, int rows, int N, int K, int G, int expected_m, int num_sms,

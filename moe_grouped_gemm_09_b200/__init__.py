@@ -68,7 +68,7 @@ _version = _decl("dg_version", [], ctypes.c_char_p)
 class DgConfig(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in
                 ("block_m", "block_n", "stages", "num_acc", "split_k", "grid", "smem_bytes", "tmem_cols",
-                 "kps")]
+                 "kps", "main_tiles", "tail_launches", "tail_split")]
 
 
 _query = _decl("dg_query_config", [_I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(DgConfig)])

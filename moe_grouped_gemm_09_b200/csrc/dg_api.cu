@@ -110,7 +110,8 @@ int a_box_rows(int kind, int rows) {
 // stage) variant; mode 0 general, 1 decode, 2 small decode.
 // Ignored unless the variant exists and, for split_k > 1, the problem is a
 // dense one with a single 128-row block.
-void forced_config(int kind, int rows, int N, int K, int G, int sms, PickedConfig* pc) {
+void forced_config(int kind, int rows, int N, int K, int G, int sms, bool f32_out,
+                   PickedConfig* pc) {
   const char* e = std::getenv("DG_FORCE_CONFIG");
   if (!e || !e[0]) return;
   int bn = 0, sk = 1;
@@ -120,7 +121,7 @@ void forced_config(int kind, int rows, int N, int K, int G, int sms, PickedConfi
   int v = -1;
   for (int i = 0; i < kNumVariants; ++i) {
     const Variant& x = kVariants[i];
-    if (x.block_n != bn) continue;
+    if (x.block_n != bn || x.f32 != f32_out) continue;
     if (kps ? (x.kps != kps || (ar && x.a_rows != ar)) : x.decode) continue;
     if (mode >= 0 && (x.small ? 2 : x.decode ? 1 : 0) != mode) continue;
     if (x.decode && kind != kDense) continue;
@@ -163,11 +164,12 @@ dg_status make_map(CUtensorMap* map, const void* base, uint64_t K, uint64_t rows
   return r == CUDA_SUCCESS ? DG_OK : DG_ERR_CUDA;
 }
 
-// 2-D tensor map over the BF16 output D [rows][N] with a box of 32 rows x
-// 64 columns and the 128-byte swizzle (the epilogue's staging layout).
-dg_status make_d_map(CUtensorMap* map, void* base, uint64_t N, uint64_t rows) {
+// 2-D tensor map over the BF16 output D [rows][N], rows ldd elements apart,
+// with a box of 32 rows x 64 columns and the 128-byte swizzle (the
+// epilogue's staging layout).
+dg_status make_d_map(CUtensorMap* map, void* base, uint64_t N, uint64_t rows, uint64_t ldd) {
   cuuint64_t dims[2] = {N, rows};
-  cuuint64_t strides[1] = {N * 2};
+  cuuint64_t strides[1] = {ldd * 2};
   cuuint32_t box[2] = {64, 32};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = encoder()(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
@@ -177,16 +179,16 @@ dg_status make_d_map(CUtensorMap* map, void* base, uint64_t N, uint64_t rows) {
 }
 
 // 3-D tensor map over an FP32 output D [groups][rows][N] (the FP32-output
-// forms: groups = 1 for the dense one) with a box of 32 rows x 32 columns
-// (128 bytes) and the 128-byte swizzle; rows past a group's end and columns
+// forms: groups = 1 for the dense one) with a box of 32 rows x 16 columns
+// (64 bytes) and the 64-byte swizzle; rows past a group's end and columns
 // past N are clipped by the TMA unit.
 dg_status make_d_map_f32(CUtensorMap* map, void* base, uint64_t N, uint64_t rows, uint64_t groups) {
   cuuint64_t dims[3] = {N, rows, groups};
   cuuint64_t strides[2] = {N * 4, rows * N * 4};
-  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t box[3] = {16, 32, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = encoder()(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
-                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
                          CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? DG_OK : DG_ERR_CUDA;
 }
@@ -241,14 +243,15 @@ dg_status run(const GemmCall& call, cudaStream_t stream) {
     if (s != DG_OK) return s;
     st->limits_known = true;
   }
-  LaunchPlan pl;
-  s = plan_gemm(call, DeviceFacts{effective_sms(*st), &st->limits}, st->error_word, &pl);
-  if (s != DG_OK || pl.grid == 0) return s;
+  LaunchPlans plans;
+  s = plan_gemm(call, DeviceFacts{effective_sms(*st), &st->limits}, st->error_word, &plans);
+  if (s != DG_OK || plans.n == 0) return s;
   if (!is_bf16_form(call.form) && check_scales_enabled()) {
     s = launch_scale_check(call, st->error_word, stream);
     if (s != DG_OK) return s;
   }
-  return launch_plan(*st, pl, stream);
+  for (int i = 0; i < plans.n && s == DG_OK; ++i) s = launch_plan(*st, plans.plan[i], stream);
+  return s;
 }
 
 // Checks n scales against the contract and records kDevBadScale if one breaks
@@ -350,12 +353,18 @@ dg_status check_gemm_call(const GemmCall& call, bool* empty) {
   return DG_OK;
 }
 
-dg_status plan_gemm(const GemmCall& call, const DeviceFacts& facts, int* error_word,
-                    LaunchPlan* pl) {
-  pl->grid = 0;
-  bool empty = false;
-  dg_status s = check_gemm_call(call, &empty);
-  if (s != DG_OK || empty) return s;
+namespace {
+
+// The last-wave split (see plan_tail) is on unless DG_NO_TAIL_SPLIT=1 (read
+// at every call, like DG_FORCE_CONFIG, for measurements).
+bool tail_split_enabled() { return !env_flag("DG_NO_TAIL_SPLIT"); }
+
+// Fills one launch of `call` (the whole problem, or a rectangle of D with A,
+// B and their scales offset to it): kernel arguments and tensor maps for the
+// given variant, split and grid; `ldd` is the row stride of D in elements and
+// `tile_limit` (> 0) stops the dense form after that many tiles.
+dg_status fill_plan(const GemmCall& call, int variant, int split, int grid, int ldd,
+                    int tile_limit, int* error_word, LaunchPlan* pl) {
   const int form = call.form;
   const int kind = kind_of_form(form);
   const int layout = layout_of_form(form);
@@ -364,15 +373,9 @@ dg_status plan_gemm(const GemmCall& call, const DeviceFacts& facts, int* error_w
   const int rows = call.rows, N = call.N, K = call.K, G = call.G;
   const long long a_rows =
       (kind == kMasked || kind == kKGrouped) ? static_cast<long long>(G) * rows : rows;
-  // the picker and the kernel count K in 128-byte blocks of a row
   const int k_bytes = bf16 ? 2 * K : K;
-  const int sms = facts.num_sms;
-
-  PickedConfig pc = pick_config(kind, rows, N, k_bytes, G, call.expected_m, sms, facts.limits,
-                                /*mn_operands=*/layout != kLayoutNT || is_f32_form(form));
-  forced_config(kind, rows, N, k_bytes, G, sms, &pc);
-  const Variant var = kVariants[pc.variant];
-  if ((layout != kLayoutNT || is_f32_form(form)) && (!mn_capable(var) || pc.split_k > 1))
+  const Variant var = kVariants[variant];
+  if ((layout != kLayoutNT || is_f32_form(form)) && (!mn_capable(var) || split > 1))
     return DG_ERR_UNSUPPORTED;
 
   GemmArgs& args = pl->args;
@@ -384,12 +387,13 @@ dg_status plan_gemm(const GemmCall& call, const DeviceFacts& facts, int* error_w
   args.num_m_blocks = ceil_div(rows, tile_rows(var));
   args.num_n_blocks = ceil_div(N, var.block_n);
   args.k_blocks = k_bytes / kBlockK;
-  args.split_k = pc.split_k;
-  args.kb_per_split = ceil_div(args.k_blocks, pc.split_k);
+  args.split_k = split;
+  args.kb_per_split = ceil_div(args.k_blocks, split);
   args.nb128 = ceil_div(N, 128);
   args.sfa = call.sfa;
   args.sfb = call.sfb;
   args.d = static_cast<__nv_bfloat16*>(call.d);
+  args.ldd = ldd;
   args.d_f32 = is_f32_form(form) ? static_cast<float*>(call.d) : nullptr;
   args.c_f32 = is_f32_form(form) ? call.c : nullptr;
   args.ks = call.ks;
@@ -400,20 +404,20 @@ dg_status plan_gemm(const GemmCall& call, const DeviceFacts& facts, int* error_w
   args.a_box_rows = a_mn ? kBlockM : a_box_rows(kind, rows);
   args.prefetch = prefetch_enabled();
   args.preload_b = kind == kDense ? weight_preload_enabled() : 0;
+  args.tile_limit = tile_limit;
   if (args.a_box_rows > var.a_rows) return DG_ERR_UNSUPPORTED;
   // a decode variant runs one tile per CTA (its epilogue reuses the ring)
-  if (var.decode &&
-      (kind != kDense || pc.grid != args.num_m_blocks * args.num_n_blocks * pc.split_k))
+  const long long tiles = static_cast<long long>(args.num_m_blocks) * args.num_n_blocks;
+  if (var.decode && (kind != kDense || tile_limit != 0 || grid != tiles * split))
     return DG_ERR_UNSUPPORTED;
   // split-K runs one tile per CTA, one cluster per output tile
-  if (pc.split_k > 1 &&
-      (kind != kDense || pc.grid != args.num_m_blocks * args.num_n_blocks * pc.split_k ||
-       rows > kBlockM || !split_fits(var, rows, pc.split_k)))
+  if (split > 1 && (kind != kDense || tile_limit != 0 || grid != tiles * split ||
+                    !split_fits(var, rows < kBlockM ? rows : kBlockM, split)))
     return DG_ERR_UNSUPPORTED;
 
   const int b_groups = (kind == kDense) ? 1 : G;
   const uint32_t elem = bf16 ? 2 : 1;
-  s = a_mn ? make_map_mn(&pl->ta, call.a, rows, K)
+  dg_status s = a_mn ? make_map_mn(&pl->ta, call.a, rows, K)
                      : make_map(&pl->ta, call.a, K, rows, kind == kMasked ? G : 1,
                                 args.a_box_rows, var.kps, elem);
   if (s != DG_OK) return s;
@@ -422,18 +426,77 @@ dg_status plan_gemm(const GemmCall& call, const DeviceFacts& facts, int* error_w
   if (s != DG_OK) return s;
   s = is_f32_form(form)
           ? make_d_map_f32(&pl->td, call.d, N, rows, kind == kKGrouped ? G : 1)
-          : make_d_map(&pl->td, call.d, N, static_cast<uint64_t>(a_rows));
+          : make_d_map(&pl->td, call.d, N, static_cast<uint64_t>(a_rows), ldd);
   if (s != DG_OK) return s;
 
   if (print_configs())
     std::fprintf(stderr,
                  "[dg] form=%d rows=%d N=%d K=%d G=%d expected_m=%d -> BLOCK_N=%d stages=%d "
-                 "kps=%d acc=%d split_k=%d grid=%d\n",
+                 "kps=%d acc=%d split_k=%d grid=%d tile_limit=%d\n",
                  form, rows, N, K, G, call.expected_m, var.block_n, var.stages, var.kps,
-                 var.num_acc, pc.split_k, pc.grid);
+                 var.num_acc, split, grid, tile_limit);
   pl->form = form;
-  pl->variant = pc.variant;
-  pl->grid = pc.grid;
+  pl->variant = variant;
+  pl->grid = grid;
+  return DG_OK;
+}
+
+}  // namespace
+
+dg_status plan_gemm(const GemmCall& call, const DeviceFacts& facts, int* error_word,
+                    LaunchPlans* plans) {
+  plans->n = 0;
+  bool empty = false;
+  dg_status s = check_gemm_call(call, &empty);
+  if (s != DG_OK || empty) return s;
+  const int form = call.form;
+  const int kind = kind_of_form(form);
+  const int layout = layout_of_form(form);
+  const bool bf16 = is_bf16_form(form);
+  const int rows = call.rows, N = call.N, K = call.K, G = call.G;
+  // the picker and the kernel count K in 128-byte blocks of a row
+  const int k_bytes = bf16 ? 2 * K : K;
+  const int sms = facts.num_sms;
+
+  PickedConfig pc = pick_config(kind, rows, N, k_bytes, G, call.expected_m, sms, facts.limits,
+                                /*mn_operands=*/layout != kLayoutNT || is_f32_form(form),
+                                /*f32_out=*/is_f32_form(form));
+  const PickedConfig picked = pc;
+  forced_config(kind, rows, N, k_bytes, G, sms, is_f32_form(form), &pc);
+  const bool forced = pc.variant != picked.variant || pc.split_k != picked.split_k;
+
+  TailPlan tp;
+  if (kind == kDense && layout == kLayoutNT && !is_f32_form(form) && !forced &&
+      tail_split_enabled())
+    tp = plan_tail(rows, N, k_bytes, sms, pc.variant, facts.limits);
+  const int main_grid = tp.main_tiles > 0 && tp.main_tiles < pc.grid ? tp.main_tiles : pc.grid;
+  s = fill_plan(call, pc.variant, pc.split_k, main_grid, N, tp.main_tiles, error_word,
+                &plans->plan[0]);
+  if (s != DG_OK) return s;
+  plans->n = 1;
+  // tail launches: a rectangle of D each, A and B (and their scales) offset
+  // to its first row and column
+  const size_t elem = bf16 ? 2 : 1;
+  const int KB = k_bytes / kBlockK;
+  for (int i = 0; i < tp.n_rects; ++i) {
+    const TailRect& r = tp.rect[i];
+    GemmCall sub = call;
+    sub.a = static_cast<const uint8_t*>(call.a) + static_cast<size_t>(r.row0) * K * elem;
+    sub.b = static_cast<const uint8_t*>(call.b) + static_cast<size_t>(r.col0) * K * elem;
+    if (!bf16) {
+      sub.sfa = call.sfa + static_cast<size_t>(r.row0) * KB;
+      sub.sfb = call.sfb + static_cast<size_t>(r.col0 / 128) * KB;
+    }
+    sub.d = static_cast<uint8_t*>(call.d) +
+            (static_cast<size_t>(r.row0) * N + r.col0) * sizeof(__nv_bfloat16);
+    sub.rows = r.rows;
+    sub.N = r.cols;
+    const int tiles = ceil_div(r.rows, 128) * ceil_div(r.cols, kVariants[tp.variant].block_n);
+    s = fill_plan(sub, tp.variant, tp.split, tiles * tp.split, N, 0, error_word,
+                  &plans->plan[plans->n]);
+    if (s != DG_OK) return s;
+    ++plans->n;
+  }
   return DG_OK;
 }
 
@@ -600,7 +663,8 @@ dg_status dg_query_config(int kind, int rows, int N, int K, int G, int expected_
       K % 128 != 0 || G < 1 || num_sms < 1)
     return DG_ERR_INVALID_ARG;
   const PickedConfig pc = pick_config(kind, rows, N, K, G, expected_m, num_sms, nullptr,
-                                      /*mn_operands=*/kind == kKGrouped);
+                                      /*mn_operands=*/kind == kKGrouped,
+                                      /*f32_out=*/kind == kKGrouped);
   const Variant v = kVariants[pc.variant];
   out->block_m = tile_rows(v);
   out->block_n = v.block_n;
@@ -611,6 +675,12 @@ dg_status dg_query_config(int kind, int rows, int N, int K, int G, int expected_
   out->smem_bytes = variant_smem_bytes(pc.variant);
   out->tmem_cols = variant_tmem_cols(pc.variant);
   out->kps = v.kps;
+  TailPlan tp;
+  if (kind == kDense) tp = plan_tail(rows, N, K, num_sms, pc.variant, nullptr);
+  out->main_tiles = tp.main_tiles;
+  out->tail_launches = tp.n_rects;
+  out->tail_split = tp.n_rects ? tp.split : 0;
+  if (tp.main_tiles > 0 && tp.main_tiles < out->grid) out->grid = tp.main_tiles;
   return DG_OK;
 }
 

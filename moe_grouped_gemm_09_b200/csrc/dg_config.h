@@ -20,21 +20,23 @@ struct Variant {
   int a_rows;   // rows of A a stage holds (64: dense A of at most 64 rows)
   bool decode;  // built for dense problems of at most one 128-row block
   bool small;   // two CTAs fit per SM; one tile per CTA
+  bool f32 = false;  // for the FP32-output forms only: 8 KB of epilogue staging per
+                     // epilogue warp, four output boxes in flight
 };
 
-// The compiled variants: general ones first (every form; the one with two K
-// blocks per stage serves the dense form, where it wins for short K), then
+// The compiled variants: general ones first (every form), then
 // the decode-shaped dense ones, whose stages are several K blocks deep so
 // that each TMA box moves 32-64 KB, then the small decode ones (at most
 // ~100 KB of shared memory and 256 TMEM columns, so that the next kernel's
 // CTAs can be resident and warm L2 with their weights while this kernel
-// drains).
+// drains), then the FP32-output ones (a shallower ring, room for four
+// output boxes in flight per epilogue warp: those forms are bound by writing
+// their FP32 output).
 constexpr Variant kVariants[] = {
     {256, 4, 1, 1, 128, false, false},
     {128, 6, 2, 1, 128, false, false},
     {64, 8, 2, 1, 128, false, false},
     {32, 9, 2, 1, 128, false, false},
-    {256, 2, 1, 2, 128, false, false},
     {128, 2, 1, 4, 64, true, false},
     {64, 3, 2, 4, 64, true, false},
     {256, 2, 1, 2, 64, true, false},
@@ -45,6 +47,8 @@ constexpr Variant kVariants[] = {
     {64, 3, 1, 2, 64, true, true},
     {128, 3, 1, 1, 128, true, true},
     {64, 2, 1, 2, 128, true, true},
+    {256, 3, 1, 1, 128, false, false, true},
+    {128, 4, 2, 1, 128, false, false, true},
 };
 constexpr int kNumVariants = sizeof(kVariants) / sizeof(kVariants[0]);
 constexpr int kMaxSplitK = 8;  // portable cluster size
@@ -143,18 +147,20 @@ inline bool pick_decode(int rows, int N, int K, int num_sms, const ClusterLimits
 // or M (the output rows of each group of the K-grouped form).
 inline PickedConfig pick_config(int kind, int rows, int N, int K, int G, int expected_m,
                                 int num_sms, const ClusterLimits* lim = nullptr,
-                                bool mn_operands = false) {
+                                bool mn_operands = false, bool f32_out = false) {
   PickedConfig best{1, 1, 1, 1};
-  if (kind == 0 && rows <= 128 && !mn_operands &&
+  if (kind == 0 && rows <= 128 && !mn_operands && !f32_out &&
       pick_decode(rows, N, K, num_sms, lim, &best))
     return best;
 
   // Everything else: persistent CTAs, no split.  Tile time is set by the
   // bytes the SM must pull through TMA per K block (A 16 KB + B BLOCK_N x
   // 128 B; measured on B200 to bound these compute-bound tiles), so choose
-  // the variant minimising waves x bytes per K block.  For the dense form a
-  // variant with two K blocks per stage (bigger boxes) also competes; it pays
-  // off for short K.
+  // the variant minimising waves x bytes per K block.  The FP32-output forms
+  // are bound by writing their output instead: waves x output columns per
+  // tile, the variant with two accumulators (its epilogue overlaps the next
+  // tile) ahead by 5 % (measured on the K-grouped workload: 0.96 against
+  // 0.99 ms).
   int eff_rows = rows;
   int groups = 1;
   if (kind == 2) {
@@ -166,7 +172,7 @@ inline PickedConfig pick_config(int kind, int rows, int N, int K, int G, int exp
   double best_cost = 1e30;
   for (int v = 0; v < kNumVariants; ++v) {
     const Variant& var = kVariants[v];
-    if (var.small || var.a_rows < 128) continue;
+    if (var.small || var.a_rows < 128 || var.f32 != f32_out) continue;
     // M-/N-major operands: one K block per stage and whole 128-column B boxes
     if (mn_operands && (var.decode || var.kps != 1 || var.block_n % 128 != 0)) continue;
     // decode variants run one tile per CTA; several K blocks per stage: dense only
@@ -178,8 +184,8 @@ inline PickedConfig pick_config(int kind, int rows, int N, int K, int G, int exp
     const int n_tiles = ceil_div(N, bn);
     const long long tiles = static_cast<long long>(m_blocks) * n_tiles;
     const int waves = ceil_div(tiles, num_sms);
-    double cost = waves * (tm / 8.0 + bn / 8.0);
-    if (var.kps == 2) cost *= (K <= 2048 ? 0.85 : 1.02);
+    double cost = f32_out ? waves * bn * (var.num_acc > 1 ? 0.95 : 1.0)
+                          : waves * (tm / 8.0 + bn / 8.0);
     if (cost < best_cost - 1e-9) {
       best_cost = cost;
       best.variant = v;
@@ -199,6 +205,84 @@ inline PickedConfig pick_config(int kind, int rows, int N, int K, int G, int exp
   best.grid = tiles < num_sms ? static_cast<int>(tiles) : num_sms;
   if (best.grid < 1) best.grid = 1;
   return best;
+}
+
+}  // namespace dg
+
+namespace dg {
+
+// Last-wave split of a dense GEMM.  The persistent kernel walks the output
+// tiles column by column (m fastest), one tile per SM per wave.  When the
+// last wave would hold at most a quarter as many tiles as there are SMs, each
+// of them a whole K loop while the other SMs idle, the first launch stops
+// after the whole waves (`main_tiles`) and the remaining tiles, one or two
+// rectangles of D (the last m-blocks of one column, then whole columns), run
+// as further launches of 128 x 128 tiles of a decode variant, split along K
+// across thread-block clusters so that they fill the SMs.
+struct TailRect {
+  int row0, rows;  // rows of D (and of A)
+  int col0, cols;  // columns of D (rows of B); col0 is a multiple of 128
+};
+struct TailPlan {
+  int main_tiles = 0;  // tiles of the first launch (0: no split)
+  int n_rects = 0;
+  TailRect rect[2] = {};
+  int variant = -1;    // decode variant of the tail launches
+  int split = 1;       // K slices per tail tile (CTAs per cluster)
+};
+
+inline TailPlan plan_tail(int rows, int N, int K, int num_sms, int main_variant,
+                          const ClusterLimits* lim) {
+  TailPlan tp;
+  const Variant& mv = kVariants[main_variant];
+  const int KB = K / 128;
+  // only the general variants with whole 128-column B scale blocks per tile
+  // (a rectangle then starts on a scale block), and long enough K loops that
+  // a wave is worth saving
+  if (mv.decode || mv.small || mv.block_n % 128 != 0 || KB < 32 || num_sms < 2) return tp;
+  const int mb = ceil_div(rows, 128), nb = ceil_div(N, mv.block_n);
+  const long long tiles = static_cast<long long>(mb) * nb;
+  if (tiles <= num_sms) return tp;
+  const int rem = static_cast<int>(tiles % num_sms);
+  if (rem == 0 || 2 * rem > num_sms) return tp;
+  int tail_v = -1;
+  for (int v = 0; v < kNumVariants; ++v) {
+    const Variant& x = kVariants[v];
+    if (x.decode && !x.small && x.block_n == 128 && x.a_rows == 128) tail_v = v;
+  }
+  if (tail_v < 0) return tp;
+  const int main_tiles = static_cast<int>(tiles) - rem;
+  const int c0 = main_tiles / mb, m0 = main_tiles % mb;
+  TailPlan out;
+  out.main_tiles = main_tiles;
+  out.variant = tail_v;
+  int c_next = c0;
+  if (m0 > 0) {
+    out.rect[out.n_rects++] = TailRect{m0 * 128, rows - m0 * 128, c0 * mv.block_n,
+                                       (N < (c0 + 1) * mv.block_n ? N : (c0 + 1) * mv.block_n) -
+                                           c0 * mv.block_n};
+    c_next = c0 + 1;
+  }
+  if (c_next < nb)
+    out.rect[out.n_rects++] = TailRect{0, rows, c_next * mv.block_n, N - c_next * mv.block_n};
+  int tail_tiles = 0;
+  for (int i = 0; i < out.n_rects; ++i)
+    tail_tiles += ceil_div(out.rect[i].rows, 128) * ceil_div(out.rect[i].cols, 128);
+  // the largest split whose clusters all fit in one wave, each CTA keeping at
+  // least four K blocks.  Unsplit, the tail's 128-column tiles would stream
+  // their whole K loop with every SM busy, while the partial wave they
+  // replace runs with few SMs contending for L2 (measured: 4096 x 4096 x 7168,
+  // 68 tiles past three waves, took 12 us longer as 136 unsplit tail tiles),
+  // so a split of at least 2 is required.
+  const Variant& tv = kVariants[tail_v];
+  for (int s = kMaxSplitK; s >= 2; s >>= 1) {
+    if (static_cast<long long>(tail_tiles) * s > num_sms || KB < 4 * s) continue;
+    if (s > 1 && (!split_fits(tv, 128, s) || cluster_limit(lim, tail_v, s, num_sms) < tail_tiles))
+      continue;
+    out.split = s;
+    return out;
+  }
+  return tp;  // the tail does not fit one wave even unsplit: keep one launch
 }
 
 }  // namespace dg

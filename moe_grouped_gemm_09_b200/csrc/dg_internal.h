@@ -77,12 +77,20 @@ struct DeviceFacts {
 // set when there is nothing to compute.
 dg_status check_gemm_call(const GemmCall& call, bool* empty);
 
+// The launches of one call, in stream order: one, or for a dense problem
+// whose last wave of tiles would leave most SMs idle, a first launch over the
+// whole waves and one or two tail launches (plan_tail).
+struct LaunchPlans {
+  int n = 0;
+  LaunchPlan plan[3];
+};
+
 // Checks the call's arguments, picks the kernel variant and grid, fills the
-// kernel arguments and encodes the tensor maps.  DG_OK with plan->grid == 0
+// kernel arguments and encodes the tensor maps.  DG_OK with plans->n == 0
 // means there is nothing to launch (an empty problem).  `error_word` is the
-// device word the kernel reports into.
+// device word the kernels report into.
 dg_status plan_gemm(const GemmCall& call, const DeviceFacts& facts, int* error_word,
-                    LaunchPlan* plan);
+                    LaunchPlans* plans);
 
 // Launches the scale-contract check of a call's sfa and sfb (FP8 forms) on
 // `stream`, reporting into `error_word`.

@@ -16,21 +16,24 @@ namespace dg {
 // Kernel mode of a variant: 0 general, 1 decode, 2 small decode.
 constexpr int mode_of(const Variant& v) { return v.small ? 2 : v.decode ? 1 : 0; }
 
-template <int V, bool SCALED = true>
+template <int V, bool SCALED = true, bool F32EPI = kVariants[V].f32>
 using ShapeOf = KernelShape<kVariants[V].block_n, kVariants[V].stages, kVariants[V].num_acc,
-                            kVariants[V].kps, kVariants[V].a_rows, mode_of(kVariants[V]), SCALED>;
+                            kVariants[V].kps, kVariants[V].a_rows, mode_of(kVariants[V]), SCALED,
+                            F32EPI>;
 
 // Kernels exist only for the (form, variant) pairs that are used: the decode
 // variants and the general ones with several K blocks per stage serve the
-// dense forms, the M-/N-major and FP32-output forms take the general
-// variants with 128-column B boxes.
+// dense forms, the M-/N-major forms take the general variants with
+// 128-column B boxes, and the FP32-output forms their own variants.
 template <int FORM, int V>
 constexpr bool kBuilt =
-    FORM == kFormDense || FORM == kFormBf16Dense ||
-    ((FORM == kFormContiguous || FORM == kFormMasked || FORM == kFormBf16Contiguous ||
-      FORM == kFormBf16Masked) &&
-     !kVariants[V].decode && kVariants[V].kps == 1) ||
-    ((FORM >= kFormNN && FORM <= kFormF32) || FORM == kFormKGrouped) && mn_capable(kVariants[V]);
+    kVariants[V].f32
+        ? is_f32_form(FORM) && mn_capable(kVariants[V])
+        : FORM == kFormDense || FORM == kFormBf16Dense ||
+              ((FORM == kFormContiguous || FORM == kFormMasked || FORM == kFormBf16Contiguous ||
+                FORM == kFormBf16Masked) &&
+               !kVariants[V].decode && kVariants[V].kps == 1) ||
+              (FORM >= kFormNN && FORM <= kFormTT && mn_capable(kVariants[V]));
 
 template <int FORM, int V>
 auto kernel_of() {
@@ -47,7 +50,8 @@ dg_status set_smem_attr(bool* attr_set) {
   } else {
     if (!attr_set[V]) {
       if (cudaFuncSetAttribute(kernel_of<FORM, V>(), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               ShapeOf<V, !is_bf16_form(FORM)>::kSmemBytes) != cudaSuccess)
+                               ShapeOf<V, !is_bf16_form(FORM), is_f32_form(FORM)>::kSmemBytes) !=
+          cudaSuccess)
         return DG_ERR_CUDA;
       attr_set[V] = true;
     }
@@ -65,7 +69,7 @@ dg_status launch_variant(bool* attr_set, const LaunchPlan& pl, cudaStream_t stre
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(pl.grid, 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = ShapeOf<V, !is_bf16_form(FORM)>::kSmemBytes;
+    cfg.dynamicSmemBytes = ShapeOf<V, !is_bf16_form(FORM), is_f32_form(FORM)>::kSmemBytes;
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -85,15 +85,16 @@ extern "C" dg_status dg_fp8_gemm_nt_noalloc(const void* a, const float* sfa, con
   NaDevice* st = nullptr;
   s = na_setup(&st);
   if (s != DG_OK) return s;
-  LaunchPlan pl;
-  s = plan_gemm(call, DeviceFacts{st->num_sms, &st->limits}, st->error_word, &pl);
-  if (s != DG_OK || pl.grid == 0) return s;
+  LaunchPlans plans;
+  s = plan_gemm(call, DeviceFacts{st->num_sms, &st->limits}, st->error_word, &plans);
+  if (s != DG_OK || plans.n == 0) return s;
   const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   if (check_scales_enabled()) {
     s = launch_scale_check(call, st->error_word, cs);
     if (s != DG_OK) return s;
   }
-  return launch_fp8_dense(st->attr_set, pl, cs);
+  for (int i = 0; i < plans.n && s == DG_OK; ++i) s = launch_fp8_dense(st->attr_set, plans.plan[i], cs);
+  return s;
 }
 
 extern "C" dg_status dg_fp8_gemm_nt_noalloc_get_last_device_error(int* code) {

@@ -91,7 +91,8 @@ struct GemmArgs {
   int nb128;         // ceil(N / 128): B scale blocks along N
   const float* sfa;  // [G * rows, k_blocks]   (dense/contiguous: G = 1 row space)
   const float* sfb;  // [G, nb128, k_blocks]
-  __nv_bfloat16* d;  // [G * rows, N]
+  __nv_bfloat16* d;  // [G * rows, N], rows ldd elements apart
+  int ldd;           // BF16 D: row stride in elements (N; larger for a sub-block of D)
   float* d_f32;      // FP32 output form: D [rows, N] (d unused)
   const float* c_f32;  // FP32 output form: C [rows, N] added to the product, or null
   const int* m_indices;  // contiguous: [rows]
@@ -103,6 +104,8 @@ struct GemmArgs {
   int prefetch;      // 1: warm L2 with the first tile before waiting on the previous kernel
   int preload_b;     // 1 (dense form): B is constant while kernels run (weights), so the
                      // first ring stages of B may be loaded before that wait
+  int tile_limit;    // dense form: > 0: compute only the first tile_limit output tiles of
+                     // the tile order (the rest go to a launch of their own)
 };
 
 constexpr int kBlockM = 128;
@@ -136,7 +139,7 @@ __host__ __device__ constexpr int pow2_ceil(int x) {
 //            shared memory and TMEM); false for BF16 operands, whose K block
 //            is 64 elements, the same 128 bytes of a row
 template <int BLOCK_N, int STAGES, int NUM_ACC, int KPS = 1, int A_ROWS = 128, int MODE = 0,
-          bool SCALED = true>
+          bool SCALED = true, bool F32EPI = false>
 struct KernelShape {
   static constexpr bool kSmall = MODE == 2;
   static constexpr int kABytes = KPS * A_ROWS * kBlockK;  // kBlockK bytes of a row per K block
@@ -165,7 +168,9 @@ struct KernelShape {
   // their epilogue stages in the idle operand ring (no staging region of its
   // own) and they need no masked-group prefix.
   static constexpr bool kDecode = MODE != 0;
-  static constexpr int kEpiBytes = kDecode ? 0 : 4 * 32 * kEpiPitch;
+  // (FP32-output forms: 8 KB per warp, four 2 KB output boxes in flight)
+  static constexpr int kF32Boxes = 4;
+  static constexpr int kEpiBytes = kDecode ? 0 : F32EPI ? 4 * kF32Boxes * 2048 : 4 * 32 * kEpiPitch;
   // tmem slot, flags, and (grouped forms) the masked or K-group prefix
   static constexpr int kMiscBytes = 16 + (kDecode ? 0 : 4 * (kMaxMaskedGroups + 1));
   // A short A tile is read by the 128-row MMA past its end (rows that only
@@ -356,7 +361,7 @@ __global__ void __launch_bounds__(kThreads, MODE == 2 ? 2 : 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     const __grid_constant__ CUtensorMap tmap_b,
                     const __grid_constant__ CUtensorMap tmap_d, const GemmArgs p) {
-  using Shape = KernelShape<BLOCK_N, STAGES, NUM_ACC, KPS, A_ROWS, MODE, !BF16>;
+  using Shape = KernelShape<BLOCK_N, STAGES, NUM_ACC, KPS, A_ROWS, MODE, !BF16, OUT_F32>;
   constexpr bool SMALL = Shape::kSmall;
   constexpr int A_BYTES = Shape::kABytes;
   constexpr int B_BYTES = Shape::kBBytes;
@@ -395,8 +400,11 @@ __global__ void __launch_bounds__(kThreads, MODE == 2 ? 2 : 1)
   // epilogue staging tiles (1024-aligned, swizzled): their own region, or,
   // when every CTA has a single tile (always for a small variant), the operand
   // ring, idle once that tile's MMAs are done, with one tile per warp and chunk
-  const int n_tiles_total =
-      (KIND == kMasked || KIND == kKGrouped) ? -1 : p.num_m_blocks * p.num_n_blocks * p.split_k;
+  // output tiles of the dense and contiguous forms (x split) this launch computes
+  const int flat_tiles =
+      (KIND == kDense && p.tile_limit > 0 ? p.tile_limit : p.num_m_blocks * p.num_n_blocks) *
+      p.split_k;
+  const int n_tiles_total = (KIND == kMasked || KIND == kKGrouped) ? -1 : flat_tiles;
   // (a decode variant always runs one tile per CTA: the host launches it so)
   const bool one_tile =
       Shape::kDecode || (n_tiles_total >= 0 && n_tiles_total <= static_cast<int>(gridDim.x));
@@ -448,7 +456,7 @@ __global__ void __launch_bounds__(kThreads, MODE == 2 ? 2 : 1)
     ptx::tmem_relinquish();
   }
   if (KIND == kDense && p.prefetch && !p.preload_b && warp == 0 &&
-      blockIdx.x < p.num_m_blocks * p.num_n_blocks * p.split_k) {
+      static_cast<int>(blockIdx.x) < flat_tiles) {
     // Warm L2 with this CTA's first tile while the previous kernel finishes
     // (the tile order of the dense form does not depend on device data).
     // A small variant prefetches the whole K range of B, the weights it
@@ -522,24 +530,27 @@ __global__ void __launch_bounds__(kThreads, MODE == 2 ? 2 : 1)
   }
 
   ptx::WaitCtl ctl{abort_flag, p.error_word, p.timeout_ns};
-  const int total = (KIND == kMasked     ? s_prefix[p.G]
-                     : KIND == kKGrouped ? (*s_kvalid ? p.G : 0) * p.num_m_blocks *
-                                               p.num_n_blocks
-                                         : p.num_m_blocks * p.num_n_blocks) *
-                    p.split_k;
+  const int total = KIND == kMasked     ? s_prefix[p.G] * p.split_k
+                    : KIND == kKGrouped ? (*s_kvalid ? p.G : 0) * p.num_m_blocks *
+                                              p.num_n_blocks * p.split_k
+                                        : flat_tiles;
 
   // Drains TMEM accumulator buffer `a` of tile `ti`, lane quarter q (rows
   // 32q..32q+31), columns [c_begin, c_end): BF16 through the staging tiles
   // at stage0 to D, or (split-K) FP32 into the parked partial.
   constexpr int NCH_ALL = BLOCK_N / Shape::kEpiCols;
   const CUtensorMap* dmap = &tmap_d;
-  auto drain_acc = [&](const Tile& ti, int a, int q, int c_begin, int c_end, uint8_t* stage0,
-                       bool report) {
-    // which output row this thread owns, and whether it may be written
+  int f32_boxes = 0;  // FP32-output boxes this thread's warp has stored (its box buffer)
+  // staging bytes of one epilogue warp in the staging region (persistent CTAs)
+  constexpr int kWarpEpiBytes = Shape::kEpiBytes / 4;
+  static_assert(!OUT_F32 || Shape::kEpiBytes == 4 * Shape::kF32Boxes * 2048,
+                "FP32 output: four 2 KB box buffers per epilogue warp");
+  // The output row of accumulator row 32q + lane of tile `ti` (`grow`, the
+  // row of D) and whether it is written; `report` flags a contiguous row of
+  // another expert.
+  auto out_row = [&](const Tile& ti, int q, bool report, bool& valid, size_t& grow) {
     const int row_local = 32 * q + lane;  // accumulator row = TMEM lane
     const int m_in_group = ti.m_blk * kBlockM + row_local;
-    bool valid;
-    size_t grow;
     if (KIND == kMasked) {
       const int mm = min(max(__ldg(p.masked_m + ti.group), 0), p.rows);
       valid = m_in_group < mm;
@@ -556,6 +567,57 @@ __global__ void __launch_bounds__(kThreads, MODE == 2 ? 2 : 1)
         valid = (e == ti.group);
       }
     }
+  };
+
+  // Stores BF16 columns [c0, c0 + 64) of this lane's output row, held as
+  // packed pairs in v[0..31], through the warp's staging tile: one TMA box of
+  // 32 rows x 64 columns (rows past the tensor's end and columns past N are
+  // clipped by the TMA unit), or whole row segments when some of the warp's
+  // rows are not written (grouped forms).  The staging tile is free again on
+  // return.
+  auto store_bf16_64 = [&](const uint32_t* v, uint8_t* stage, int n0, int c0, bool valid,
+                           size_t grow, bool tma_store) {
+    constexpr int CPR = 8;  // 16-byte chunks per staged row
+    // chunk j of row `lane` at chunk position j ^ (lane % 8): the 128-byte swizzle
+#pragma unroll
+    for (int j = 0; j < CPR; ++j)
+      *reinterpret_cast<uint4*>(stage + lane * 128 + 16 * (j ^ (lane % CPR))) =
+          make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+    if (tma_store) {
+      ptx::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        ptx::tma_store_2d(dmap, stage, n0 + c0, static_cast<int>(grow - lane));
+        ptx::bulk_commit_group();
+        ptx::bulk_wait_group_read0();
+      }
+      __syncwarp();
+      return;
+    }
+    __syncwarp();
+    constexpr int RPI = 32 / CPR;  // rows per store instruction
+    const int sub = lane % CPR;
+#pragma unroll
+    for (int i = 0; i < 32 / RPI; ++i) {
+      const int rr = RPI * i + lane / CPR;  // row within the warp's 32
+      const bool row_ok = __shfl_sync(0xFFFFFFFFu, valid, rr);
+      const int n = n0 + c0 + 8 * sub;
+      if (row_ok && n < p.N) {
+        const size_t g_row = grow - lane + rr;  // the rows of a warp are consecutive
+        *reinterpret_cast<uint4*>(p.d + g_row * p.ldd + n) =
+            *reinterpret_cast<const uint4*>(stage + rr * 128 + 16 * (sub ^ (rr % CPR)));
+      }
+    }
+    __syncwarp();
+  };
+
+  auto drain_acc = [&](const Tile& ti, int a, int q, int c_begin, int c_end, uint8_t* stage0,
+                       bool report) {
+    // which output row this thread owns, and whether it may be written
+    const int row_local = 32 * q + lane;  // accumulator row = TMEM lane
+    bool valid;
+    size_t grow;
+    out_row(ti, q, report, valid, grow);
     const uint32_t t_row =
         tmem_base + (static_cast<uint32_t>(32 * q) << 16) + a * BLOCK_N;
     const int n0 = ti.n_blk * BLOCK_N;
@@ -576,40 +638,44 @@ __global__ void __launch_bounds__(kThreads, MODE == 2 ? 2 : 1)
           ptx::tc_ld_32x32b_x32(t_row + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[CH - 32]));
         ptx::tc_wait_ld();
         if constexpr (OUT_F32) {
-          // FP32 output, in boxes of 32 rows x 32 columns: each lane adds its
-          // row's C values if given (C may be D itself: every element is read
-          // by the thread that stages it, before its box is stored), stages
-          // the row's 128 bytes in the warp's swizzled tile, and one TMA
-          // store writes the box (the tensor map is [groups][rows][N], so
-          // rows past a group's end and columns past N are clipped).
-          const size_t off = grow * p.N + n0 + c0;
+          // FP32 output in boxes of 32 rows x 16 columns (64 bytes a row):
+          // each lane adds its row's C values if given (C may be D: every
+          // element is read by the thread that stages it, before its box is
+          // stored), stages the row's 64 bytes in one of the warp's four
+          // 2 KB box buffers (16-byte chunk j of row l at position
+          // j ^ ((l / 2) % 4): the 64-byte swizzle), and one TMA store writes
+          // the box; the tensor map is [groups][rows][N], so rows past a
+          // group's end and columns past N are clipped.  A buffer is reused
+          // once the store issued from it four boxes earlier has read it:
+          // the form is bound by writing its output, and three stores stay
+          // in flight while the next box is staged.
           const int grp = (KIND == kKGrouped) ? ti.group : 0;
+          const size_t off = grow * p.N + n0 + c0;
 #pragma unroll
-          for (int hh = 0; hh < CH / 32; ++hh) {
-            float* v = reinterpret_cast<float*>(&r[32 * hh]);
+          for (int h = 0; h < CH / 16; ++h) {
+            float* v = reinterpret_cast<float*>(&r[16 * h]);
             if (p.c_f32 && valid) {
 #pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                if (n0 + c0 + 32 * hh + 4 * j >= p.N) break;
-                const float4 cv =
-                    *reinterpret_cast<const float4*>(p.c_f32 + off + 32 * hh + 4 * j);
+              for (int j = 0; j < 4; ++j) {
+                if (n0 + c0 + 16 * h + 4 * j >= p.N) break;
+                const float4 cv = *reinterpret_cast<const float4*>(p.c_f32 + off + 16 * h + 4 * j);
                 v[4 * j] += cv.x; v[4 * j + 1] += cv.y; v[4 * j + 2] += cv.z; v[4 * j + 3] += cv.w;
               }
             }
-            uint8_t* stage = stage0;
+            uint8_t* stage = stage0 + (f32_boxes % Shape::kF32Boxes) * 2048;
+            if (lane == 0) ptx::bulk_wait_group_read<Shape::kF32Boxes - 1>();
+            __syncwarp();
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-              *reinterpret_cast<float4*>(stage + lane * 128 + 16 * (j ^ (lane % 8))) =
+            for (int j = 0; j < 4; ++j)
+              *reinterpret_cast<float4*>(stage + lane * 64 + 16 * (j ^ ((lane >> 1) & 3))) =
                   make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
             ptx::fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-              ptx::tma_store_3d(dmap, stage, n0 + c0 + 32 * hh,
-                                ti.m_blk * kBlockM + 32 * q, grp);
+              ptx::tma_store_3d(dmap, stage, n0 + c0 + 16 * h, ti.m_blk * kBlockM + 32 * q, grp);
               ptx::bulk_commit_group();
-              ptx::bulk_wait_group_read0();  // staging tile free again
             }
-            __syncwarp();
+            ++f32_boxes;
           }
           continue;
         }
@@ -662,7 +728,7 @@ __global__ void __launch_bounds__(kThreads, MODE == 2 ? 2 : 1)
           const int n = n0 + c0 + 8 * sub;
           if (row_ok && n < p.N) {
             const size_t g_row = grow - lane + rr;  // the rows of a warp are consecutive
-            *reinterpret_cast<uint4*>(p.d + g_row * p.N + n) = *reinterpret_cast<const uint4*>(
+            *reinterpret_cast<uint4*>(p.d + g_row * p.ldd + n) = *reinterpret_cast<const uint4*>(
                 stage + rr * Shape::kEpiPitch + 16 * (sub ^ (rr % CPR)));
           }
         }
@@ -671,9 +737,45 @@ __global__ void __launch_bounds__(kThreads, MODE == 2 ? 2 : 1)
       if (split) ptx::fence_proxy_async_smem();  // parked rows are read by bulk copies
     }
   };
+  // A persistent CTA with a single accumulator (BLOCK_N 256) would hold its
+  // MMAs back for the whole epilogue.  Instead each epilogue thread reads its
+  // accumulator row into registers as packed BF16 pairs, releases the
+  // accumulator (the MMA warp starts the CTA's next tile), and only then
+  // stages and stores the row, overlapping the next tile's MMAs.
+  constexpr bool kEarlyRelease =
+      NUM_ACC == 1 && MODE == 0 && !OUT_F32 && Shape::kEpiCols == 64 && BLOCK_N % 64 == 0;
+  auto drain_release = [&](const Tile& ti, int a, int q, uint8_t* stage) {
+    bool valid;
+    size_t grow;
+    out_row(ti, q, true, valid, grow);
+    const uint32_t t_row = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + a * BLOCK_N;
+    const bool any = __any_sync(0xFFFFFFFFu, valid);
+    uint32_t pk[BLOCK_N / 2];
+    if (any) {
+#pragma unroll
+      for (int c = 0; c < BLOCK_N / 64; ++c) {
+        uint32_t r[64];
+        ptx::tc_ld_32x32b_x32(t_row + 64 * c, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+        ptx::tc_ld_32x32b_x32(t_row + 64 * c + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+        ptx::tc_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          pk[32 * c + j] = pack_bf16x2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
+      }
+    }
+    ptx::tc_fence_before_sync();
+    ptx::mbar_arrive(&acc_empty[a]);
+    if (!any) return;
+    const bool tma_store = KIND == kDense || __all_sync(0xFFFFFFFFu, valid);
+#pragma unroll
+    for (int c = 0; c < BLOCK_N / 64; ++c)
+      store_bf16_64(pk + 32 * c, stage, ti.n_blk * BLOCK_N, 64 * c, valid, grow, tma_store);
+  };
+
   // A single-tile CTA's warps 0-3 are idle once their roles end: they drain
   // the upper half of the columns while warps 4-7 drain the lower half.
-  const bool helpers = one_tile && !split && KIND != kMasked && BLOCK_N >= 2 * Shape::kEpiCols;
+  const bool helpers = one_tile && !split && KIND != kMasked && !OUT_F32 &&
+                       BLOCK_N >= 2 * Shape::kEpiCols && (BLOCK_N / 2) % Shape::kEpiCols == 0;
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer --
@@ -1145,12 +1247,17 @@ __global__ void __launch_bounds__(kThreads, MODE == 2 ? 2 : 1)
       if (!ok) break;
       ptx::tc_fence_after_sync();
 
-      const int split_col = helpers ? BLOCK_N / 2 : BLOCK_N;
-      // staging: in one_tile mode warp w owns tiles [w * NCH_ALL, (w + 1) * NCH_ALL)
-      drain_acc(ti, a, q, 0, split_col,
-                sEpi + (one_tile ? warp * NCH_ALL : q) * 32 * Shape::kEpiPitch, true);
-      ptx::tc_fence_before_sync();
-      ptx::mbar_arrive(&acc_empty[a]);
+      if (kEarlyRelease && !one_tile && !split) {
+        drain_release(ti, a, q, sEpi + q * kWarpEpiBytes);  // releases the buffer
+      } else {
+        const int split_col = helpers ? BLOCK_N / 2 : BLOCK_N;
+        // staging: in one_tile mode warp w owns tiles [w * NCH_ALL, (w + 1) * NCH_ALL)
+        drain_acc(ti, a, q, 0, split_col,
+                  sEpi + (one_tile ? warp * NCH_ALL * 32 * Shape::kEpiPitch : q * kWarpEpiBytes),
+                  true);
+        ptx::tc_fence_before_sync();
+        ptx::mbar_arrive(&acc_empty[a]);
+      }
       ++acc_it;
     }
     // this warp's TMA stores have read their staging tiles (the writes
@@ -1248,7 +1355,7 @@ __global__ void __launch_bounds__(kThreads, MODE == 2 ? 2 : 1)
         v.z = pack_bf16x2(hi.x, hi.y);
         v.w = pack_bf16x2(hi.z, hi.w);
         const size_t grow = (size_t)ti.m_blk * kBlockM + r0 + lr;
-        *reinterpret_cast<uint4*>(p.d + grow * p.N + n0 + c) = v;
+        *reinterpret_cast<uint4*>(p.d + grow * p.ldd + n0 + c) = v;
       }
     }
     if (threadIdx.x == 0) ptx::bulk_wait_group_read0();  // outgoing copies done reading

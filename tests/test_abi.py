@@ -179,6 +179,32 @@ def test_k_grouped_bad_arguments_rejected(dg):
     assert fn(FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, 0, 32, 128, 256, None) == 0     # no groups
 
 
+def test_last_wave_split_plan(dg):
+    """The dense form's last-wave split (host planning, no GPU): taken when
+    the tiles past the whole waves, as 128-column tiles split at least 2
+    ways, fit one wave and K is at least 4096 bytes, with the largest split
+    whose clusters fit one wave."""
+    q = dg.query_config
+    # 896 tiles = 6 waves + 8 tiles in one column: one rectangle, 16 tiles x 8
+    c = q(0, 4096, 7168, 16384)
+    assert (c["main_tiles"], c["tail_launches"], c["tail_split"]) == (888, 1, 8)
+    # 160 tiles = 1 wave + 12: two rectangles of 24 tiles, split 4
+    c = q(0, 1280, 4096, 4096)
+    assert (c["main_tiles"], c["tail_launches"], c["tail_split"]) == (148, 2, 4)
+    # no split: the last wave is more than half full (288 = 148 + 140), K is
+    # short, the problem fits one wave, the tiles divide into whole waves
+    # (4096 x 4096 x 7168: 3 waves + 68 tiles, 136 tail tiles, no split of 2 fits)
+    for shape in [(4096, 2112, 7168), (4096, 4096, 2048), (1024, 4096, 7168), (4736, 1024, 7168),
+                  (4096, 4096, 7168)]:
+        c = q(0, *shape)
+        assert (c["main_tiles"], c["tail_launches"], c["tail_split"]) == (0, 0, 0), shape
+    # the grouped forms never split their last wave
+    c = q(1, 10112, 4096, 7168, G=32)
+    assert c["tail_launches"] == 0
+    # fewer SMs: 512 tiles on 132 SMs = 3 waves + 116 (more than half): none
+    assert q(0, 4096, 4096, 7168, num_sms=132)["tail_launches"] == 0
+
+
 def test_query_rejects_bad_input(dg):
     with pytest.raises(dg.DgError):
         dg.query_config(4, 64, 128, 128)

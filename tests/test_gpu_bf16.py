@@ -74,7 +74,7 @@ def test_bf16_dense_integer_exact(dg):
 
 # (config, M): general variants (persistent, several tiles per CTA), decode
 # variants with split-K clusters, and a small variant (two CTAs per SM)
-FORCED = [("256:1", 300), ("128:1", 300), ("64:1", 300), ("32:1", 300), ("256:1:2:128:0", 300),
+FORCED = [("256:1:1:128:0", 300), ("128:1", 300), ("64:1", 300), ("32:1", 300),
           ("128:4:4:64:1", 64), ("64:2:2:128:1", 128), ("128:2:2:64:2", 48)]
 
 

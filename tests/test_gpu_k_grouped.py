@@ -112,3 +112,18 @@ def test_k_grouped_bad_group_sizes_write_nothing(dg):
         torch.cuda.synchronize()
         assert dg.get_last_device_error() == 0x203, bad
         assert torch.all(d == 7.0), bad
+
+
+@pytest.mark.parametrize("cfg", ["256:1", "128:1"])
+def test_k_grouped_each_fp32_output_variant(dg, cfg, monkeypatch):
+    """Both FP32-output variants (256 columns, one accumulator; 128 columns,
+    two), forced, on uneven groups with an empty one and an addend."""
+    monkeypatch.setenv("DG_FORCE_CONFIG", cfg)
+    ks, M, N = [128] * 3 + [1024, 0, 640], 384, 528
+    a, sfa, b, sfb, ks, c = make_case(11, ks, M, N)
+    d = dg.k_grouped_fp8_gemm_tn_contiguous(dev(a), dev(sfa), dev(b), dev(sfb), dev(ks), c=dev(c))
+    torch.cuda.synchronize()
+    assert dg.get_last_device_error() == 0
+    got = d.cpu().numpy()
+    assert np.array_equal(got[4], c[4])
+    check_f32(got, oracle.default().k_grouped_tn(a, sfa, b, sfb, ks, c), f"k-grouped forced {cfg}")

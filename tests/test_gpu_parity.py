@@ -108,7 +108,7 @@ def test_dense_scales_not_16_byte_aligned(dg):
 # Every general variant, forced, on one ragged shape with a random power-of-two
 # scale per A row and per B block (the picker would choose only some of them
 # for this shape).
-FORCED_GENERAL = ["256:1", "128:1", "64:1", "32:1", "256:1:2:128:0"]
+FORCED_GENERAL = ["256:1:1:128:0", "128:1", "64:1", "32:1"]
 
 
 @pytest.mark.parametrize("cfg", FORCED_GENERAL)
@@ -191,7 +191,8 @@ def test_dense_operand_layouts_prefill_sampled(dg, layout):
 # |ref| + rms(ref) (K/32 FP32 additions of exact products), and the global
 # 1 - 2 sum(xy) / sum(x^2 + y^2) within 1e-9.
 @pytest.mark.parametrize("mode", ["none", "c", "in_place"])
-@pytest.mark.parametrize("M,N,K", [(300, 400, 384), (64, 2112, 1024), (512, 256, 2048)])
+@pytest.mark.parametrize("M,N,K", [(300, 400, 384), (64, 2112, 1024), (512, 256, 2048),
+                                   (1040, 4864, 512)])   # the last: persistent, 171 tiles
 def test_dense_f32_output(dg, mode, M, N, K):
     rng = np.random.default_rng(M * 3 + N + K)
     p = workloads.dense_problem(M, N, K, seed=10)
