@@ -364,7 +364,8 @@ def time_workload(ctx: GpuContext, name: str, args, steps: int, per_gemm: bool, 
     dev, stream = ctx.dev, ctx.stream
     items = build_workload(name, seed=args.seed)
     # dense workloads: B is the weights, so the weight preload applies
-    preload = args.weight_preload == "on" and all(k in ("dense", "bf16_dense") for k, _ in items)
+    dense = all(k in ("dense", "bf16_dense") for k, _ in items)
+    preload = args.weight_preload == "on" and dense
     dg.set_weight_preload(preload)
     metric, unit, _ = workload_meta(name)
     set_bytes = sum(p.a.nbytes + p.b.nbytes + getattr(p, "sfa", p.a[:0]).nbytes
@@ -450,11 +451,11 @@ def time_workload(ctx: GpuContext, name: str, args, steps: int, per_gemm: bool, 
     if dg.get_last_device_error() != 0:
         raise RuntimeError(f"{name}: device error during the timed steps")
 
-    # the same steps with the weight preload off, for comparison (the dense
-    # workloads are timed with it on: B is the weights, written by no kernel)
-    ms_no_preload = None
-    if preload:
-        dg.set_weight_preload(False)
+    # the dense workloads: the same steps with the weight preload switched the
+    # other way, for comparison (B is the weights, written by no kernel)
+    ms_alt = None
+    if dense:
+        dg.set_weight_preload(not preload)
         plain = capture(R)
         plain_tail = capture(rem) if rem else None
         with torch.cuda.stream(stream):
@@ -472,8 +473,8 @@ def time_workload(ctx: GpuContext, name: str, args, steps: int, per_gemm: bool, 
             e1.record(stream)
         torch.cuda.synchronize(dev)
         ctx.barrier()
-        ms_no_preload = ctx.max_over_ranks(e0.elapsed_time(e1) / steps)
-        dg.set_weight_preload(True)
+        ms_alt = ctx.max_over_ranks(e0.elapsed_time(e1) / steps)
+        dg.set_weight_preload(preload)
         del plain, plain_tail
 
     # ---- per GEMM (second timed pass): R back-to-back launches of one shape ----
@@ -543,7 +544,7 @@ def time_workload(ctx: GpuContext, name: str, args, steps: int, per_gemm: bool, 
     dg.set_weight_preload(False)
     return {"items": items, "ms": ms, "R": R, "flush_note": flush_note, "kernel_ms": kernel_ms,
             "clocks": clocks.summary(), "e2e": e2e_res, "metric": metric, "unit": unit,
-            "preload": preload, "ms_no_preload": ms_no_preload}
+            "preload": preload, "ms_alt": ms_alt}
 
 
 def workload_record(name: str, t: dict, world: int, steps: int, warmup: int) -> dict:
@@ -596,9 +597,9 @@ def workload_record(name: str, t: dict, world: int, steps: int, warmup: int) -> 
             "per_gemm_us": [round(x * 1e3, 3) for x in t["kernel_ms"]],
         },
         "clocks": t["clocks"],
-        **({"value_without_weight_preload": round(
-            whole_job_value(step_units(items, unit), world, t["ms_no_preload"], unit), 3)}
-           if t["ms_no_preload"] else {}),
+        **({("value_without_weight_preload" if t["preload"] else "value_with_weight_preload"):
+            round(whole_job_value(step_units(items, unit), world, t["ms_alt"], unit), 3)}
+           if t["ms_alt"] else {}),
     }
 
 
@@ -632,8 +633,9 @@ def run_gpu(args):
         "roofline": rec["roofline"],
         "clocks": rec["clocks"],
     }
-    if "value_without_weight_preload" in rec:
-        res["value_without_weight_preload"] = rec["value_without_weight_preload"]
+    for key in ("value_without_weight_preload", "value_with_weight_preload"):
+        if key in rec:
+            res[key] = rec[key]
     cpu_ok = ctx.rank == 0 and ctx.world == 1 and not args.no_cpu_baseline
     if cpu_ok:
         res["cpu_baseline"] = run_oracle_sample(main["items"], main["unit"],
@@ -898,9 +900,10 @@ def main():
                     help="input copies rotated between steps (0: enough to exceed 3x L2)")
     ap.add_argument("--reference-budget-s", type=float, default=120.0,
                     help="reference arm: whole oracle steps if they fit in this time")
-    ap.add_argument("--weight-preload", choices=("on", "off"), default="on",
+    ap.add_argument("--weight-preload", choices=("on", "off"), default="off",
                     help="dense workloads: let each GEMM load B (the weights) before waiting "
-                         "on the previous kernel; the line also reports the value with it off")
+                         "on the previous kernel; the line also reports the value with the "
+                         "other setting")
     ap.add_argument("--measure-fp8-peak", action="store_true",
                     help="time the vendor library's dense E4M3 GEMM and print its TFLOP/s")
     ap.add_argument("--peak-size", type=int, default=8192)

@@ -158,9 +158,8 @@ inline PickedConfig pick_config(int kind, int rows, int N, int K, int G, int exp
   // 128 B; measured on B200 to bound these compute-bound tiles), so choose
   // the variant minimising waves x bytes per K block.  The FP32-output forms
   // are bound by writing their output instead: waves x output columns per
-  // tile, the variant with two accumulators (its epilogue overlaps the next
-  // tile) ahead by 5 % (measured on the K-grouped workload: 0.96 against
-  // 0.99 ms).
+  // tile (on a tie, the 256-column variant: 0.866 against 0.881 ms for the
+  // 128-column one with two accumulators on the K-grouped workload).
   int eff_rows = rows;
   int groups = 1;
   if (kind == 2) {
@@ -184,8 +183,7 @@ inline PickedConfig pick_config(int kind, int rows, int N, int K, int G, int exp
     const int n_tiles = ceil_div(N, bn);
     const long long tiles = static_cast<long long>(m_blocks) * n_tiles;
     const int waves = ceil_div(tiles, num_sms);
-    double cost = f32_out ? waves * bn * (var.num_acc > 1 ? 0.95 : 1.0)
-                          : waves * (tm / 8.0 + bn / 8.0);
+    double cost = f32_out ? static_cast<double>(waves) * bn : waves * (tm / 8.0 + bn / 8.0);
     if (cost < best_cost - 1e-9) {
       best_cost = cost;
       best.variant = v;

@@ -168,9 +168,9 @@ struct KernelShape {
   // their epilogue stages in the idle operand ring (no staging region of its
   // own) and they need no masked-group prefix.
   static constexpr bool kDecode = MODE != 0;
-  // (FP32-output forms: 8 KB per warp, four 2 KB output boxes in flight)
-  static constexpr int kF32Boxes = 4;
-  static constexpr int kEpiBytes = kDecode ? 0 : F32EPI ? 4 * kF32Boxes * 2048 : 4 * 32 * kEpiPitch;
+  // (FP32-output forms: 16 KB per warp, two halves of four 2 KB boxes)
+  static constexpr int kF32Bufs = 8;
+  static constexpr int kEpiBytes = kDecode ? 0 : F32EPI ? 4 * kF32Bufs * 2048 : 4 * 32 * kEpiPitch;
   // tmem slot, flags, and (grouped forms) the masked or K-group prefix
   static constexpr int kMiscBytes = 16 + (kDecode ? 0 : 4 * (kMaxMaskedGroups + 1));
   // A short A tile is read by the 128-row MMA past its end (rows that only
@@ -540,11 +540,14 @@ __global__ void __launch_bounds__(kThreads, MODE == 2 ? 2 : 1)
   // at stage0 to D, or (split-K) FP32 into the parked partial.
   constexpr int NCH_ALL = BLOCK_N / Shape::kEpiCols;
   const CUtensorMap* dmap = &tmap_d;
-  int f32_boxes = 0;  // FP32-output boxes this thread's warp has stored (its box buffer)
+  int f32_chunks = 0;  // FP32-output chunks this thread's warp has stored (its staging half)
   // staging bytes of one epilogue warp in the staging region (persistent CTAs)
   constexpr int kWarpEpiBytes = Shape::kEpiBytes / 4;
-  static_assert(!OUT_F32 || Shape::kEpiBytes == 4 * Shape::kF32Boxes * 2048,
-                "FP32 output: four 2 KB box buffers per epilogue warp");
+  static_assert(!OUT_F32 || (Shape::kEpiBytes == 4 * Shape::kF32Bufs * 2048 &&
+                             Shape::kEpiCols == 64 && Shape::kF32Bufs == 8),
+                "FP32 output: two halves of four 2 KB box buffers per epilogue warp");
+  static_assert(!OUT_F32 || STAGES * (A_BYTES + B_BYTES) >= Shape::kEpiBytes,
+                "FP32 output, one tile per CTA: the staging buffers fit in the operand ring");
   // The output row of accumulator row 32q + lane of tile `ti` (`grow`, the
   // row of D) and whether it is written; `report` flags a contiguous row of
   // another expert.
@@ -638,19 +641,23 @@ __global__ void __launch_bounds__(kThreads, MODE == 2 ? 2 : 1)
           ptx::tc_ld_32x32b_x32(t_row + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[CH - 32]));
         ptx::tc_wait_ld();
         if constexpr (OUT_F32) {
-          // FP32 output in boxes of 32 rows x 16 columns (64 bytes a row):
-          // each lane adds its row's C values if given (C may be D: every
-          // element is read by the thread that stages it, before its box is
-          // stored), stages the row's 64 bytes in one of the warp's four
-          // 2 KB box buffers (16-byte chunk j of row l at position
-          // j ^ ((l / 2) % 4): the 64-byte swizzle), and one TMA store writes
-          // the box; the tensor map is [groups][rows][N], so rows past a
-          // group's end and columns past N are clipped.  A buffer is reused
-          // once the store issued from it four boxes earlier has read it:
-          // the form is bound by writing its output, and three stores stay
-          // in flight while the next box is staged.
+          // FP32 output in boxes of 32 rows x 16 columns (64 bytes a row),
+          // four per 64-column chunk: each lane adds its row's C values if
+          // given (C may be D: every element is read by the thread that
+          // stages it, before its box is stored) and stages the row's 64
+          // bytes of each box (16-byte chunk j of row l at position
+          // j ^ ((l / 2) % 4): the 64-byte swizzle) in one half of the warp's
+          // staging buffers; then one fence, and four TMA stores committed as
+          // one bulk group (the tensor map is [groups][rows][N], so rows past
+          // a group's end and columns past N are clipped).  A half is reused
+          // once the group issued from it two chunks earlier has read it: the
+          // form is bound by writing its output, and one chunk's stores stay
+          // in flight while the next chunk is loaded from TMEM and staged.
           const int grp = (KIND == kKGrouped) ? ti.group : 0;
           const size_t off = grow * p.N + n0 + c0;
+          uint8_t* half = stage0 + (f32_chunks & 1) * (Shape::kF32Bufs / 2) * 2048;
+          if (lane == 0) ptx::bulk_wait_group_read<1>();
+          __syncwarp();
 #pragma unroll
           for (int h = 0; h < CH / 16; ++h) {
             float* v = reinterpret_cast<float*>(&r[16 * h]);
@@ -662,21 +669,21 @@ __global__ void __launch_bounds__(kThreads, MODE == 2 ? 2 : 1)
                 v[4 * j] += cv.x; v[4 * j + 1] += cv.y; v[4 * j + 2] += cv.z; v[4 * j + 3] += cv.w;
               }
             }
-            uint8_t* stage = stage0 + (f32_boxes % Shape::kF32Boxes) * 2048;
-            if (lane == 0) ptx::bulk_wait_group_read<Shape::kF32Boxes - 1>();
-            __syncwarp();
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-              *reinterpret_cast<float4*>(stage + lane * 64 + 16 * (j ^ ((lane >> 1) & 3))) =
+              *reinterpret_cast<float4*>(half + h * 2048 + lane * 64 + 16 * (j ^ ((lane >> 1) & 3))) =
                   make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-            ptx::fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-              ptx::tma_store_3d(dmap, stage, n0 + c0 + 16 * h, ti.m_blk * kBlockM + 32 * q, grp);
-              ptx::bulk_commit_group();
-            }
-            ++f32_boxes;
           }
+          ptx::fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+#pragma unroll
+            for (int h = 0; h < CH / 16; ++h)
+              ptx::tma_store_3d(dmap, half + h * 2048, n0 + c0 + 16 * h,
+                                ti.m_blk * kBlockM + 32 * q, grp);
+            ptx::bulk_commit_group();
+          }
+          ++f32_chunks;
           continue;
         }
         uint8_t* stage = one_tile ? stage0 + ((c0 - c_begin) / CH) * 32 * Shape::kEpiPitch : stage0;
@@ -1251,10 +1258,12 @@ __global__ void __launch_bounds__(kThreads, MODE == 2 ? 2 : 1)
         drain_release(ti, a, q, sEpi + q * kWarpEpiBytes);  // releases the buffer
       } else {
         const int split_col = helpers ? BLOCK_N / 2 : BLOCK_N;
-        // staging: in one_tile mode warp w owns tiles [w * NCH_ALL, (w + 1) * NCH_ALL)
-        drain_acc(ti, a, q, 0, split_col,
-                  sEpi + (one_tile ? warp * NCH_ALL * 32 * Shape::kEpiPitch : q * kWarpEpiBytes),
-                  true);
+        // staging: the warp's own slice of the staging region, or in one_tile
+        // mode of the idle operand ring (BF16: warp w owns tiles
+        // [w * NCH_ALL, (w + 1) * NCH_ALL); FP32: 16 KB per warp)
+        uint8_t* stage0 = (OUT_F32 || !one_tile) ? sEpi + q * kWarpEpiBytes
+                                                 : sEpi + warp * NCH_ALL * 32 * Shape::kEpiPitch;
+        drain_acc(ti, a, q, 0, split_col, stage0, true);
         ptx::tc_fence_before_sync();
         ptx::mbar_arrive(&acc_empty[a]);
       }
