@@ -24,9 +24,10 @@ from parity import check_close, d_bits, dev, sentinel_like
 pytestmark = pytest.mark.gpu
 
 # split-K decode shapes (cluster reduction in shared memory), a short one, a
-# ragged general one and a prefill-sized one (persistent CTAs, many tiles each)
+# ragged general one, a prefill-sized one (persistent CTAs, many tiles each)
+# and one whose last wave is split off (a first launch and two split-K tails)
 SHAPES = [(64, 2112, 7168), (128, 7168, 2048), (64, 512, 1024), (300, 384, 512),
-          (4096, 2112, 1024)]
+          (4096, 2112, 1024), (1280, 4096, 4096)]
 
 
 @pytest.fixture(scope="module")
