@@ -798,8 +798,10 @@ def run_oracle_sample(items, unit, budget_s: float):
         sample = f"{reps} whole steps back to back ({dt:.1f} s)"
     else:
         full_s = dt / (sum(done_frac) / len(done_frac))
-        sample = (f"first {100 * min(done_frac):.2f}%..{100 * max(done_frac):.2f}% of the output "
-                  f"rows of every GEMM of one step ({dt:.1f} s), scaled to the full step by rows")
+        lo, hi = 100 * min(done_frac), 100 * max(done_frac)
+        share = f"{lo:.2f}%" if f"{lo:.2f}" == f"{hi:.2f}" else f"{lo:.2f}%..{hi:.2f}%"
+        sample = (f"first {share} of the output rows of every GEMM of one step ({dt:.1f} s), "
+                  f"scaled to the full step by rows")
     return {"value": round(scale_units(units, unit, full_s), 4), "unit": unit,
             "cores": o.num_threads(), "kind": "oracle", "sample": sample}
 

@@ -39,6 +39,16 @@ def test_step_units_and_roofline_on_the_smoke_step():
     assert r["frac_time"] == pytest.approx(r["t_roof_s"] / 1e-6)
 
 
+def test_launches_per_step_count_the_tail_launches():
+    """gpu_launches counts every kernel launch of a step: one per GEMM, plus
+    the split-off last wave of a dense GEMM (the library's own plan)."""
+    assert bench.step_launches(bench.build_workload("decode")) == 6
+    # 4096 x 7168 x 16384 splits its last wave into one tail launch
+    assert bench.step_launches(bench.build_workload("prefill")) == 5
+    assert bench.step_launches(bench.build_workload("bf16-prefill")) == 5
+    assert bench.step_launches(bench.build_workload("masked")) == 1
+
+
 def test_bf16_problem_units():
     p = workloads.bf16_dense_problem(64, 256, 512, seed=0)
     assert p.a.dtype == np.uint16 and p.a.shape == (64, 512) and p.b.shape == (256, 512)
