@@ -433,12 +433,14 @@ def test_scale_contract_check(dg, M, N, K):
     assert dg.get_last_device_error() == 0
 
 
-@pytest.mark.parametrize("M,N,K", workloads.DECODE_SHAPES + [(300, 400, 1024), (4096, 2112, 1024)])
+@pytest.mark.parametrize("M,N,K", workloads.DECODE_SHAPES + [(300, 400, 1024), (4096, 2112, 1024),
+                                                              (1280, 4096, 4096)])
 def test_weight_preload_gives_the_same_results(dg, M, N, K):
     """With the weight preload on (B loaded before the wait on the previous
-    kernel), every decode shape (split-K clusters included) and persistent
-    tiles give bit-identical results to the preload off, and match the
-    oracle."""
+    kernel), every decode shape (split-K clusters included), persistent tiles
+    and a call whose last wave is split off into split-K tail launches (each
+    loading its B sub-block early) give bit-identical results to the preload
+    off, and match the oracle."""
     p = workloads.dense_problem(M, N, K, seed=15)
     try:
         dg.set_weight_preload(True)
