@@ -603,7 +603,7 @@ def workload_record(name: str, t: dict, world: int, steps: int, warmup: int) -> 
     }
 
 
-EXTRA_WORKLOADS = ("smoke", "prefill", "contiguous", "masked", "k-grouped")
+EXTRA_WORKLOADS = ("smoke", "prefill", "contiguous", "masked", "k-grouped", "bf16-decode", "bf16-prefill")
 
 
 def run_gpu(args):
