@@ -224,9 +224,17 @@ class ClockSampler:
     def summary(self):
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        idle = 0
         for line in self.lines:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 8:
+                continue
+            try:
+                active = int(parts[3], 16)
+            except ValueError:
+                active = 0
+            if active & 0x1:  # the GPU was idle at this sample (before the work started)
+                idle += 1
                 continue
             try:
                 sm.append(float(parts[0]))
@@ -237,9 +245,11 @@ class ClockSampler:
                 if val.lower() == "active":
                     reasons.add(name)
         if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0}
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0,
+                    "idle_samples": idle}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "idle_samples": idle,
+                "window": "the timed region and untimed replays of the same graphs just before it"}
 
 
 # ------------------------------------------------------------ rank logic --
@@ -433,11 +443,32 @@ def time_workload(ctx: GpuContext, name: str, args, steps: int, per_gemm: bool, 
         cycle.replay()
     torch.cuda.synchronize(dev)
 
+    # one rotation cycle's time, to size the clock soak below
+    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        c0.record(stream)
+        cycle.replay()
+        c1.record(stream)
+    torch.cuda.synchronize(dev)
+    cycle_s = max(c0.elapsed_time(c1) / 1e3, 1e-6)
+
     # ---- timed region: exactly `steps` steps ----
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ctx.barrier()
     torch.cuda.synchronize(dev)
     with ClockSampler(dev.index) as clocks:
+        # Clock soak: a timed region of a few milliseconds holds too few
+        # 50 ms clock samples, so the same graphs replay (untimed) for
+        # `clock_soak_s` first, under the same load, and the samples cover
+        # the soak and the timed region.
+        batch = max(1, int(0.05 / cycle_s))
+        for _ in range(max(0, int(math.ceil(args.clock_soak_s / (batch * cycle_s))))):
+            with torch.cuda.stream(stream):
+                for _ in range(batch):
+                    cycle.replay()
+            torch.cuda.synchronize(dev)
+        ctx.barrier()
+        torch.cuda.synchronize(dev)
         with torch.cuda.stream(stream):
             start.record(stream)
             for _ in range(steps // R):
@@ -902,6 +933,9 @@ def main():
                     help="input copies rotated between steps (0: enough to exceed 3x L2)")
     ap.add_argument("--reference-budget-s", type=float, default=120.0,
                     help="reference arm: whole oracle steps if they fit in this time")
+    ap.add_argument("--clock-soak-s", type=float, default=0.5,
+                    help="untimed replays of the same graphs just before the timed region, "
+                         "inside the clock-sampling window (seconds)")
     ap.add_argument("--weight-preload", choices=("on", "off"), default="off",
                     help="dense workloads: let each GEMM load B (the weights) before waiting "
                          "on the previous kernel; the line also reports the value with the "

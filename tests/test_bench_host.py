@@ -111,3 +111,19 @@ def test_warmup_below_three_is_refused(monkeypatch):
     monkeypatch.setattr(sys, "argv", ["bench.py", "--warmup", "2"])
     with pytest.raises(SystemExit):
         bench.main()
+
+
+def test_clock_summary_skips_idle_samples_and_reads_reasons():
+    """Samples taken while the GPU was idle (bit 0 of the active-reasons mask)
+    are left out of the median; throttle reasons are collected by name."""
+    c = bench.ClockSampler(0)
+    c.lines = [
+        "1072, 1965, 100.0, 0x0000000000000001, Not Active, Not Active, Not Active, Not Active",
+        "1965, 1965, 700.0, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "1900, 1965, 990.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "1965, 1965, 710.0, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+    ]
+    s = c.summary()
+    assert s["samples"] == 3 and s["idle_samples"] == 1
+    assert s["sm_mhz"] == 1965.0 and s["sm_max_mhz"] == 1965.0
+    assert s["reasons"] == ["sw_power_cap"]
