@@ -248,8 +248,7 @@ class ClockSampler:
             return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0,
                     "idle_samples": idle}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm), "idle_samples": idle,
-                "window": "the timed region and untimed replays of the same graphs just before it"}
+                "samples": len(sm), "idle_samples": idle}
 
 
 # ------------------------------------------------------------ rank logic --
@@ -273,20 +272,24 @@ def whole_job_value(units_per_step: float, world: int, ms_per_step: float, unit:
 
 # ---------------------------------------------------------------- GPU arm --
 
-def fp8_peak(peaks: dict):
+def fp8_peak(peaks: dict, sustained: bool = False):
     """Dense E4M3 tensor peak (TFLOP/s) and where it comes from: the measured
     figure of ``profiles/fp8_peak.md`` (a large FP8 library GEMM timed on this
-    pool's B200s; ``--measure-fp8-peak`` writes it), else 2 x the measured
-    BF16 figure (the nominal 4.5 : 2.25 FP8 : BF16 ratio)."""
+    pool's B200s, as a burst or back to back for seconds under the power cap;
+    ``--measure-fp8-peak`` writes both), else 2 x the measured BF16 figure
+    (the nominal 4.5 : 2.25 FP8 : BF16 ratio)."""
     path = os.path.join(ROOT, "profiles", "fp8_peak.md")
+    key = "fp8_tflops_sustained:" if sustained else "fp8_tflops:"
     try:
         with open(path) as f:
             for line in f:
-                if line.startswith("fp8_tflops:"):
-                    return float(line.split(":", 1)[1].strip()), "measured (fp8_peak.md, cuBLASLt E4M3)"
+                if line.startswith(key):
+                    return (float(line.split(":", 1)[1].strip()),
+                            f"measured (fp8_peak.md, cuBLASLt E4M3{', sustained' if sustained else ''})")
     except (OSError, ValueError):
         pass
-    bf16 = float(peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"]))
+    bf16 = float(peaks.get("bf16_tflops_sustained" if sustained else "bf16_tflops",
+                           PEAKS_FALLBACK["bf16_tflops"]))
     return 2.0 * bf16, "2 x bf16_tflops (nominal FP8:BF16 ratio)"
 
 
@@ -443,32 +446,11 @@ def time_workload(ctx: GpuContext, name: str, args, steps: int, per_gemm: bool, 
         cycle.replay()
     torch.cuda.synchronize(dev)
 
-    # one rotation cycle's time, to size the clock soak below
-    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        c0.record(stream)
-        cycle.replay()
-        c1.record(stream)
-    torch.cuda.synchronize(dev)
-    cycle_s = max(c0.elapsed_time(c1) / 1e3, 1e-6)
-
     # ---- timed region: exactly `steps` steps ----
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ctx.barrier()
     torch.cuda.synchronize(dev)
     with ClockSampler(dev.index) as clocks:
-        # Clock soak: a timed region of a few milliseconds holds too few
-        # 50 ms clock samples, so the same graphs replay (untimed) for
-        # `clock_soak_s` first, under the same load, and the samples cover
-        # the soak and the timed region.
-        batch = max(1, int(0.05 / cycle_s))
-        for _ in range(max(0, int(math.ceil(args.clock_soak_s / (batch * cycle_s))))):
-            with torch.cuda.stream(stream):
-                for _ in range(batch):
-                    cycle.replay()
-            torch.cuda.synchronize(dev)
-        ctx.barrier()
-        torch.cuda.synchronize(dev)
         with torch.cuda.stream(stream):
             start.record(stream)
             for _ in range(steps // R):
@@ -507,6 +489,40 @@ def time_workload(ctx: GpuContext, name: str, args, steps: int, per_gemm: bool, 
         ms_alt = ctx.max_over_ranks(e0.elapsed_time(e1) / steps)
         dg.set_weight_preload(preload)
         del plain, plain_tail
+
+    # ---- sustained pass: the same graphs back to back for `sustained_s`,
+    # long enough for the power cap to act; its own clock samples ----
+    sustained = None
+    if args.sustained_s > 0:
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            c0.record(stream)
+            cycle.replay()
+            c1.record(stream)
+        torch.cuda.synchronize(dev)
+        cycle_s = max(c0.elapsed_time(c1) / 1e3, 1e-6)
+        batch = max(1, int(0.05 / cycle_s))                    # ~50 ms per host sync
+        n_batches = max(1, int(math.ceil(args.sustained_s / (batch * cycle_s))))
+        ctx.barrier()
+        torch.cuda.synchronize(dev)
+        with ClockSampler(dev.index) as s_clocks:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                e0.record(stream)
+            for _ in range(n_batches):
+                with torch.cuda.stream(stream):
+                    for _ in range(batch):
+                        cycle.replay()
+                torch.cuda.synchronize(dev)
+            with torch.cuda.stream(stream):
+                e1.record(stream)
+            torch.cuda.synchronize(dev)
+        ctx.barrier()
+        n_steps = n_batches * batch * R
+        sustained = {"ms": ctx.max_over_ranks(e0.elapsed_time(e1) / n_steps), "steps": n_steps,
+                     "clocks": s_clocks.summary()}
+        if dg.get_last_device_error() != 0:
+            raise RuntimeError(f"{name}: device error during the sustained pass")
 
     # ---- per GEMM (second timed pass): R back-to-back launches of one shape ----
     kernel_ms = []
@@ -575,7 +591,28 @@ def time_workload(ctx: GpuContext, name: str, args, steps: int, per_gemm: bool, 
     dg.set_weight_preload(False)
     return {"items": items, "ms": ms, "R": R, "flush_note": flush_note, "kernel_ms": kernel_ms,
             "clocks": clocks.summary(), "e2e": e2e_res, "metric": metric, "unit": unit,
-            "preload": preload, "ms_alt": ms_alt}
+            "preload": preload, "ms_alt": ms_alt, "sustained": sustained}
+
+
+def sustained_record(name: str, t: dict, world: int, unit: str, bound: str, hbm_peak: float,
+                     peaks: dict) -> dict:
+    """The sustained pass: the same graphs back to back for seconds (the power
+    cap acts), its rate, clocks, and fraction of the sustained peak (HBM: the
+    same copy bandwidth; tensor: the sustained library GEMM rate)."""
+    items, su = t["items"], t["sustained"]
+    if bound == "hbm":
+        peak, src, r_unit = hbm_peak, "measured (hbm_gbs copy)", "GB/s"
+    elif is_bf16(name):
+        peak = float(peaks.get("bf16_tflops_sustained", PEAKS_FALLBACK["bf16_tflops"]))
+        src, r_unit = "measured (bf16_tflops_sustained)", "TFLOP/s"
+    else:
+        (peak, src), r_unit = fp8_peak(peaks, sustained=True), "TFLOP/s"
+    achieved = scale_units(step_units(items, r_unit), r_unit, su["ms"] / 1e3)
+    return {"value": round(whole_job_value(step_units(items, unit), world, su["ms"], unit), 3),
+            "ms_per_step": round(su["ms"], 6), "steps": su["steps"],
+            "roofline": {"achieved": round(achieved, 3), "peak": round(peak, 1), "unit": r_unit,
+                         "frac": round(achieved / peak, 4), "peak_source": src},
+            "clocks": su["clocks"]}
 
 
 def workload_record(name: str, t: dict, world: int, steps: int, warmup: int) -> dict:
@@ -628,6 +665,8 @@ def workload_record(name: str, t: dict, world: int, steps: int, warmup: int) -> 
             "per_gemm_us": [round(x * 1e3, 3) for x in t["kernel_ms"]],
         },
         "clocks": t["clocks"],
+        **({"sustained": sustained_record(name, t, world, unit, bound, hbm_peak, peaks)}
+           if t.get("sustained") else {}),
         **({("value_without_weight_preload" if t["preload"] else "value_with_weight_preload"):
             round(whole_job_value(step_units(items, unit), world, t["ms_alt"], unit), 3)}
            if t["ms_alt"] else {}),
@@ -664,7 +703,7 @@ def run_gpu(args):
         "roofline": rec["roofline"],
         "clocks": rec["clocks"],
     }
-    for key in ("value_without_weight_preload", "value_with_weight_preload"):
+    for key in ("value_without_weight_preload", "value_with_weight_preload", "sustained"):
         if key in rec:
             res[key] = rec[key]
     cpu_ok = ctx.rank == 0 and ctx.world == 1 and not args.no_cpu_baseline
@@ -933,9 +972,9 @@ def main():
                     help="input copies rotated between steps (0: enough to exceed 3x L2)")
     ap.add_argument("--reference-budget-s", type=float, default=120.0,
                     help="reference arm: whole oracle steps if they fit in this time")
-    ap.add_argument("--clock-soak-s", type=float, default=0.5,
-                    help="untimed replays of the same graphs just before the timed region, "
-                         "inside the clock-sampling window (seconds)")
+    ap.add_argument("--sustained-s", type=float, default=2.0,
+                    help="after the timed steps, replay the same graphs back to back for this "
+                         "long and report the sustained rate and its clocks (0: skip)")
     ap.add_argument("--weight-preload", choices=("on", "off"), default="off",
                     help="dense workloads: let each GEMM load B (the weights) before waiting "
                          "on the previous kernel; the line also reports the value with the "
