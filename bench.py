@@ -490,39 +490,6 @@ def time_workload(ctx: GpuContext, name: str, args, steps: int, per_gemm: bool, 
         dg.set_weight_preload(preload)
         del plain, plain_tail
 
-    # ---- sustained pass: the same graphs back to back for `sustained_s`,
-    # long enough for the power cap to act; its own clock samples ----
-    sustained = None
-    if args.sustained_s > 0:
-        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            c0.record(stream)
-            cycle.replay()
-            c1.record(stream)
-        torch.cuda.synchronize(dev)
-        cycle_s = max(c0.elapsed_time(c1) / 1e3, 1e-6)
-        batch = max(1, int(0.05 / cycle_s))                    # ~50 ms per host sync
-        n_batches = max(1, int(math.ceil(args.sustained_s / (batch * cycle_s))))
-        ctx.barrier()
-        torch.cuda.synchronize(dev)
-        with ClockSampler(dev.index) as s_clocks:
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            with torch.cuda.stream(stream):
-                e0.record(stream)
-            for _ in range(n_batches):
-                with torch.cuda.stream(stream):
-                    for _ in range(batch):
-                        cycle.replay()
-                torch.cuda.synchronize(dev)
-            with torch.cuda.stream(stream):
-                e1.record(stream)
-            torch.cuda.synchronize(dev)
-        ctx.barrier()
-        n_steps = n_batches * batch * R
-        sustained = {"ms": ctx.max_over_ranks(e0.elapsed_time(e1) / n_steps), "steps": n_steps,
-                     "clocks": s_clocks.summary()}
-        if dg.get_last_device_error() != 0:
-            raise RuntimeError(f"{name}: device error during the sustained pass")
 
     # ---- per GEMM (second timed pass): R back-to-back launches of one shape ----
     kernel_ms = []
@@ -587,7 +554,41 @@ def time_workload(ctx: GpuContext, name: str, args, steps: int, per_gemm: bool, 
         e2e_res = {"value": round(whole_job_value(step_units(items, unit), ctx.world, e2e_ms, unit), 3),
                    "unit": unit, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
+    # ---- sustained pass: the same graphs back to back for `sustained_s`,
+    # long enough for the power cap to act; its own clock samples ----
+    sustained = None
+    if args.sustained_s > 0:
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            c0.record(stream)
+            cycle.replay()
+            c1.record(stream)
+        torch.cuda.synchronize(dev)
+        cycle_s = max(c0.elapsed_time(c1) / 1e3, 1e-6)
+        batch = max(1, int(0.05 / cycle_s))                    # ~50 ms per host sync
+        n_batches = max(1, int(math.ceil(args.sustained_s / (batch * cycle_s))))
+        ctx.barrier()
+        torch.cuda.synchronize(dev)
+        with ClockSampler(dev.index) as s_clocks:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                e0.record(stream)
+            for _ in range(n_batches):
+                with torch.cuda.stream(stream):
+                    for _ in range(batch):
+                        cycle.replay()
+                torch.cuda.synchronize(dev)
+            with torch.cuda.stream(stream):
+                e1.record(stream)
+            torch.cuda.synchronize(dev)
+        ctx.barrier()
+        n_steps = n_batches * batch * R
+        sustained = {"ms": ctx.max_over_ranks(e0.elapsed_time(e1) / n_steps), "steps": n_steps,
+                     "clocks": s_clocks.summary()}
+        if dg.get_last_device_error() != 0:
+            raise RuntimeError(f"{name}: device error during the sustained pass")
     del cycle, tail
+
     dg.set_weight_preload(False)
     return {"items": items, "ms": ms, "R": R, "flush_note": flush_note, "kernel_ms": kernel_ms,
             "clocks": clocks.summary(), "e2e": e2e_res, "metric": metric, "unit": unit,
