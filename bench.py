@@ -76,6 +76,8 @@ def build_workload(name: str, seed: int = 0):
         return [("contiguous", workloads.contiguous_problem(**workloads.CONTIGUOUS_MOE, seed=seed))]
     if name == "masked":
         return [("masked", workloads.masked_problem(**workloads.MASKED_MOE, seed=seed))]
+    if name == "masked-decode":
+        return [("masked", workloads.masked_problem(**workloads.MASKED_DECODE_MOE, seed=seed))]
     if name == "k-grouped":
         return [("k_grouped", workloads.k_grouped_problem(**workloads.K_GROUPED_MOE, seed=seed))]
     if name == "bf16-decode":
@@ -384,7 +386,7 @@ def time_workload(ctx: GpuContext, name: str, args, steps: int, per_gemm: bool, 
     set_bytes = sum(p.a.nbytes + p.b.nbytes + getattr(p, "sfa", p.a[:0]).nbytes
                     + getattr(p, "sfb", p.a[:0]).nbytes for _, p in items)
     R = max(2, math.ceil(3 * L2_BYTES / max(set_bytes, 1)))
-    if name in ("prefill", "contiguous", "masked", "k-grouped", "bf16-prefill"):
+    if name in ("prefill", "contiguous", "masked", "masked-decode", "k-grouped", "bf16-prefill"):
         R = max(2, min(R, 4))
     if rotations > 0:
         R = rotations
@@ -674,7 +676,8 @@ def workload_record(name: str, t: dict, world: int, steps: int, warmup: int) -> 
     }
 
 
-EXTRA_WORKLOADS = ("smoke", "prefill", "contiguous", "masked", "k-grouped", "bf16-decode", "bf16-prefill")
+EXTRA_WORKLOADS = ("smoke", "prefill", "contiguous", "masked", "masked-decode", "k-grouped",
+                   "bf16-decode", "bf16-prefill")
 
 
 def run_gpu(args):
@@ -956,8 +959,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="decode",
-                    choices=("decode", "smoke", "prefill", "contiguous", "masked", "k-grouped",
-                             "bf16-decode", "bf16-prefill"))
+                    choices=("decode", "smoke", "prefill", "contiguous", "masked", "masked-decode",
+                             "k-grouped", "bf16-decode", "bf16-prefill"))
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--per-gemm-reps", type=int, default=20,

@@ -399,5 +399,7 @@ PREFILL_SHAPES = [(4096, n, k) for (n, k) in ((2112, 7168), (24576, 1536), (7168
                                               (4096, 7168))]
 CONTIGUOUS_MOE = dict(G=32, N=4096, K=7168, total_tokens=8192, zipf_s=1.1, align=128)
 MASKED_MOE = dict(G=32, max_m=256, N=4096, K=7168)
+# the masked layer in decode: few tokens per expert (masked_m uniform in [0, 64])
+MASKED_DECODE_MOE = dict(G=32, max_m=64, N=4096, K=7168)
 # the weight gradient of the contiguous MoE layer: dW[g] [4096, 7168] per expert
 K_GROUPED_MOE = dict(G=32, M=4096, N=7168, total_tokens=8192, zipf_s=1.1, align=128)
