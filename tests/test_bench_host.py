@@ -127,3 +127,16 @@ def test_clock_summary_skips_idle_samples_and_reads_reasons():
     assert s["samples"] == 3 and s["idle_samples"] == 1
     assert s["sm_mhz"] == 1965.0 and s["sm_max_mhz"] == 1965.0
     assert s["reasons"] == ["sw_power_cap"]
+
+
+def test_long_timed_regions_use_the_sustained_tensor_peak():
+    """20 prefill steps (15 ms) are held against the burst E4M3 peak; 2000
+    steps (1.5 s, the power cap acting) against the sustained one."""
+    items = bench.build_workload("prefill")
+    t = {"items": items, "ms": 0.77, "unit": "TFLOP/s", "metric": "m", "R": 2, "flush_note": "",
+         "preload": False, "clocks": {}, "kernel_ms": [], "ms_alt": None}
+    short = bench.workload_record("prefill", t, 1, 20, 5)["roofline"]
+    long = bench.workload_record("prefill", t, 1, 2000, 5)["roofline"]
+    assert "sustained" not in short["peak_source"] and "sustained" in long["peak_source"]
+    assert long["peak"] < short["peak"]
+    assert long["frac"] == pytest.approx(short["frac"] * short["peak"] / long["peak"], rel=1e-3)
