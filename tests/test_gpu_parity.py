@@ -378,6 +378,23 @@ def test_masked_small(dg):
             check_close(got[g, :v], ref[g, :v], f"masked group {g}")
 
 
+def test_masked_out_of_range_counts_are_clamped(dg):
+    """masked_m outside [0, max_m] is clamped on the device, as in the oracle:
+    a negative count writes no row of its group, one above max_m writes all
+    of them; the other rows keep the sentinel."""
+    p = workloads.masked_problem(G=4, max_m=128, N=272, K=384, seed=6,
+                                 masked_m=np.array([-7, 64, 300, 1]))
+    got = run_masked(dg, p)
+    assert dg.get_last_device_error() == 0
+    ref = np.full((p.G, p.max_m, p.N), workloads.SENTINEL_BF16, np.uint16)
+    oracle.default().grouped_masked(p.a, p.sfa, p.b, p.sfb, p.masked_m, d=ref)
+    for g, v in enumerate([0, 64, 128, 1]):
+        assert np.all(got[g, v:] == workloads.SENTINEL_BF16), f"group {g}: masked rows written"
+        assert np.all(ref[g, v:] == workloads.SENTINEL_BF16), f"oracle group {g}"
+        if v:
+            check_close(got[g, :v], ref[g, :v], f"clamped masked group {g}")
+
+
 def test_masked_full(dg):
     """The masked MoE workload (32 groups, masked_m uniform in [0, 256]),
     every valid row against the oracle and every masked row untouched."""
